@@ -1,0 +1,132 @@
+/*
+ * kda.h — C ABI of the Kimi Delta Attention (KDA) operator for NVIDIA B200 (sm_100a).
+ *
+ * KDA is the channel-wise gated delta rule
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,      o_t = S_t^T q_t
+ * ("Kimi Linear: An Expressive, Efficient Attention Architecture", paper-graph-ui walkthrough,
+ *  §3.4 "The KDA State Update Equation", Eq. 1 and the output read that follows it).
+ * S is d_k x d_v (rows indexed by key channels), alpha_t = exp(log_alpha_t) in (0,1]^{d_k},
+ * beta_t in [0,1]. No query scale is applied: o_t reads the updated state S_t.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. Nothing is allocated inside
+ *     the calls: prefill scratch is the caller's `workspace`.
+ *   - Calls are asynchronous and stream-ordered on `stream` (NULL = legacy default stream).
+ *     They return once the kernels are enqueued.
+ *   - Argument errors (null pointers, unsupported sizes, misaligned pointers, workspace too
+ *     small) are detected on the host before anything is launched; nothing is written then.
+ *   - Faults that only the device can see (a cu_seqlens array that is not monotone or that runs
+ *     past T) set a per-device status word; the kernels then skip their work and
+ *     kda_last_device_error() reports it.
+ *   - No C++ exception crosses this boundary.
+ *
+ * Layouts (row-major, innermost dimension last):
+ *   q, k          [B, T, H, Dk]   dtype = qkv_dtype (bf16 or fp32)
+ *   v, o          [B, T, H, Dv]   dtype = qkv_dtype
+ *   log_alpha     [B, T, H, Dk]   fp32, finite and <= 0 (log of the per-channel decay alpha)
+ *   beta          [B, T, H]       fp32
+ *   states        [N, H, Dk, Dv]  fp32 (N = number of sequences)
+ * For packed variable-length input, B = 1, T = total tokens and cu_seqlens holds N+1 offsets.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* null pointer, negative size, misalignment, bad cu_seqlens */
+  KDA_ERR_UNSUPPORTED = 2, /* a size or dtype combination this build has no kernel for */
+  KDA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch error, no device, ...) */
+  KDA_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up */
+  KDA_ERR_WORKSPACE = 5    /* workspace missing, too small or not 256-byte aligned */
+} kda_status_t;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
+
+/* Human-readable name of a status code. Never returns NULL. */
+const char* kda_status_string(kda_status_t status);
+
+/* Library version, "major.minor.patch". */
+const char* kda_version(void);
+
+/*
+ * kda_chunk_fwd_workspace_size — bytes of device scratch that kda_chunk_fwd needs.
+ *
+ * Chunkwise prefill keeps, per chunk and head, the UT-transform products of the walkthrough's
+ * §3.4 "Chunkwise Parallelization" (W, U, the decayed keys and queries, the causal
+ * query-key matrix and the chunk decay). The figure is an upper bound valid for any
+ * cu_seqlens with `num_seqs` sequences totalling B*T tokens.
+ *   B, T, H, Dk, Dv, chunk, num_seqs : as for kda_chunk_fwd; qkv_dtype selects the kernel path.
+ *   bytes (out, host pointer)         : required size, a multiple of 256.
+ * Returns KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED for sizes kda_chunk_fwd would reject.
+ */
+kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                          int32_t chunk, int32_t num_seqs, kda_dtype_t qkv_dtype,
+                                          size_t* bytes);
+
+/*
+ * kda_chunk_fwd — chunkwise-parallel prefill (the walkthrough's §3.4 "Chunkwise
+ * Parallelization": UT transform, chunk state update Eq. 8, chunk output Eq. 9).
+ *
+ *   q, k, v         device, layouts above, dtype qkv_dtype; 16-byte aligned.
+ *   log_alpha       device fp32 [B,T,H,Dk]; finite, <= 0. 16-byte aligned.
+ *   beta            device fp32 [B,T,H].
+ *   initial_state   device fp32 [N,H,Dk,Dv], or NULL for zero states. May alias final_state.
+ *   cu_seqlens      device int32 [N+1] with cu_seqlens[0] = 0, non-decreasing,
+ *                   cu_seqlens[N] <= B*T; or NULL, then the B rows are N = B sequences of T.
+ *                   When non-NULL, B must be 1. Sequences may be empty.
+ *   num_seqs        N (must equal B when cu_seqlens is NULL).
+ *   chunk           chunk length C: 64 on the bf16 path; 16, 32 or 64 on the fp32 path.
+ *   o               device [B,T,H,Dv], dtype qkv_dtype (rounded to nearest-even for bf16).
+ *   final_state     device fp32 [N,H,Dk,Dv], or NULL to skip it.
+ *   workspace       device scratch of at least kda_chunk_fwd_workspace_size() bytes,
+ *                   256-byte aligned; its contents on entry are ignored.
+ * Supported: qkv_dtype BF16 with Dk = Dv = 128, chunk = 64 (tensor-core path); qkv_dtype F32
+ * with 1 <= Dk, Dv <= 128 and Dv a multiple of 4 (CUDA-core fp32 path).
+ * Tokens past cu_seqlens[N] are neither read nor written.
+ */
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+                           const float* log_alpha, const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                           int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, void* o,
+                           float* final_state, void* workspace, size_t workspace_bytes,
+                           kda_stream_t stream);
+
+/*
+ * kda_recurrent_step — one decode token per sequence, state updated in place (the
+ * walkthrough's §3.4 "FLOPs Accounting and Inference Strategy": the recurrent kernel used for
+ * generation; the update is Eq. 1 in its online-gradient form of "Online Learning
+ * Interpretation": S' = Diag(alpha) S, S = S' - beta k (S'^T k - v)^T).
+ *
+ *   q, k            device [N,H,Dk], dtype qkv_dtype.
+ *   v               device [N,H,Dv], dtype qkv_dtype.
+ *   log_alpha       device fp32 [N,H,Dk]; beta device fp32 [N,H].
+ *   state           device fp32 [N,H,Dk,Dv], read and overwritten; 16-byte aligned.
+ *   o               device [N,H,Dv], dtype qkv_dtype: o = S_new^T q.
+ * Supported: 1 <= Dk <= 128, 4 <= Dv <= 128 with Dv a multiple of 4, either dtype.
+ * The state is streamed once from HBM and written once.
+ */
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+                                const float* log_alpha, const float* beta, float* state, void* o,
+                                int32_t N, int32_t H, int32_t Dk, int32_t Dv, kda_stream_t stream);
+
+/*
+ * kda_last_device_error — read and clear the per-device status word that the kernels set
+ * (KDA_ERR_INVALID_ARG for a bad cu_seqlens, KDA_ERR_TIMEOUT for a bounded wait that gave up).
+ * Synchronises `stream`. Returns KDA_OK when no kernel reported a fault.
+ */
+kda_status_t kda_last_device_error(kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

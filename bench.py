@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA operator on B200 — prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one chunkwise prefill (kda_chunk_fwd) of the standard prefill batch: B=2, T=4096, H=32,
+d_k = d_v = 128, C = 64, bf16 q/k/v, fp32 gates and states, initial state ~ N(0, 0.02^2).
+``value`` is prefill tokens/s over all ranks (each rank runs its own batch: weak scaling), with
+inputs resident in HBM; ``e2e`` is the same metric through the public API with pinned host
+inputs copied in and the outputs read back inside the timed region. Inputs rotate over four
+independently drawn sets (> 370 MB, above the 126 MB L2), so no step re-reads a cached input.
+
+Beside it the line carries the decode half of the metric (kda_recurrent_step on 256 sequences x
+32 heads with 128 x 128 fp32 states, 1024 steps, state GB/s), the long prefill (B=1, T=131072),
+the roofline of the dominant kernel (per-kernel CUDA-event times from the library's profiling
+hook), the SM clocks sampled during the timed region, and the fp64 CPU oracle timed on the
+host's cores as a reported baseline.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference implementation there is) on a
+bounded sample of the same workload per step and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s + % bf16 TC peak (H=32,d=128); decode state GB/s vs HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--decode-steps", type=int, default=1024)
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-long", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[4:8]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [x for x in sm if x >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------- helpers
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world, dev):
+    """W untimed warm-up steps, then K steps between a barrier + synchronize on both sides;
+    device time from CUDA events on the launching stream, max over ranks."""
+    import torch
+
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        fn(i)
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+
+# Algorithmic bytes one launch of each kernel must move (inputs read once, outputs written once);
+# the workspace records are the split design's intermediates, written by one kernel and read by
+# the next, and count for both.
+def prefill_kernel_bytes(name, spec, max_chunks, rec_bytes):
+    th = spec.token_heads()
+    qkv = 2 if spec.dtype == "bf16" else 4
+    inputs = th * ((2 * spec.Dk + spec.Dv) * qkv + 4 * spec.Dk + 4)
+    out_o = th * spec.Dv * qkv
+    states = spec.num_seqs * spec.H * spec.Dk * spec.Dv * 4
+    recs = max_chunks * spec.H * rec_bytes
+    if name.startswith("chunk_local"):
+        return inputs + recs
+    if name.startswith("chunk_state"):
+        return recs + out_o + states * (2 if spec.init_std > 0 else 1)
+    if name.startswith("chunk_map"):
+        return 8 * (spec.num_seqs + 1)
+    return None
+
+
+def profile_pass(fn, steps, dev):
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+
+    kda.kda_profile_read()  # drop stale records
+    kda.kda_profile_enable(True)
+    for i in range(steps):
+        fn(i)
+    torch.cuda.synchronize(dev)
+    kda.kda_profile_enable(False)
+    return kda.kda_profile_read()
+
+
+def chunk_count(spec):
+    C = spec.chunk
+    if spec.seqlens is None:
+        return spec.B * ((spec.T + C - 1) // C)
+    return sum((n + C - 1) // C for n in spec.seqlens)
+
+
+# ---------------------------------------------------------------------------------- arms
+def run_prefill(spec, seeds, dev, steps, warmup, world):
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+
+    sets = [kda_synth.prefill_inputs(spec, s, dev) for s in seeds]
+    o = torch.empty_like(sets[0]["v"])
+    fs = torch.empty((spec.num_seqs, spec.H, spec.Dk, spec.Dv), dtype=torch.float32, device=dev)
+    ws_bytes = kda.kda_chunk_fwd_workspace_size(spec.B, spec.T, spec.H, spec.Dk, spec.Dv,
+                                                spec.chunk, spec.num_seqs, sets[0]["q"].dtype)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        x = sets[i % len(sets)]
+        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                          initial_state=x["initial_state"], cu_seqlens=x["cu_seqlens"],
+                          chunk=spec.chunk, o=o, final_state=fs, workspace=ws)
+
+    ms = timed(step, steps, warmup, world, dev)
+    if kda.kda_last_device_error(dev) != kda.KDA_OK:
+        raise RuntimeError("device status word set during the prefill benchmark")
+    prof = profile_pass(step, steps, dev)
+    return dict(ms=ms, prof=prof, sets=sets, o=o, fs=fs, ws=ws, ws_bytes=ws_bytes, step=step)
+
+
+def run_prefill_e2e(spec, x, o, fs, ws, dev, steps, warmup, world):
+    """Public-API end to end: pinned host inputs -> device, kda_chunk_fwd, o and final state back
+    to pinned host memory, every step."""
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+
+    names = ["q", "k", "v", "log_alpha", "beta"] + \
+        (["initial_state"] if x["initial_state"] is not None else [])
+    host = {n: x[n].cpu().pin_memory() for n in names}
+    dbuf = {n: torch.empty_like(x[n]) for n in names}
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
+
+    def step(i):
+        for n in names:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        kda.kda_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
+                          initial_state=dbuf.get("initial_state"), chunk=spec.chunk, o=o,
+                          final_state=fs, workspace=ws)
+        ho.copy_(o, non_blocking=True)
+        hs.copy_(fs, non_blocking=True)
+
+    ms = timed(step, steps, warmup, world, dev)
+    return ms, h2d, d2h
+
+
+def run_decode(spec, n_steps, dev, warmup, world, rank):
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+
+    state = kda_synth.decode_state(spec, 2004 + 10 * rank, dev)
+    x = kda_synth.decode_step_inputs(spec, 2004 + 10 * rank, n_steps, dev)
+    o = torch.empty((spec.N, spec.H, spec.Dv), dtype=x["q"].dtype, device=dev)
+
+    def step(i):
+        s = i % n_steps
+        kda.kda_recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["log_alpha"][s], x["beta"][s],
+                               state, o=o)
+
+    ms = timed(step, n_steps, warmup, world, dev)
+    prof = profile_pass(step, min(n_steps, 64), dev)
+    del x
+    return ms, prof
+
+
+def cpu_baseline(spec, dev, budget_s):
+    """The fp64 oracle as it stands, on the host's cores, over whole sequences of the prefill
+    workload (all heads), repeated until ~budget_s of CPU work. Returns tokens/s."""
+    import kda_synth
+    import oracle
+
+    x = kda_synth.prefill_inputs(spec, 2001, "cpu")
+    done, t0 = 0, time.perf_counter()
+    n = 0
+    while True:
+        b = n % spec.B
+        s0 = None if x["initial_state"] is None else x["initial_state"][b:b + 1]
+        oracle.recurrent(x["q"][b], x["k"][b], x["v"][b], x["log_alpha"][b], x["beta"][b],
+                         initial_state=s0)
+        done += spec.T
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return dict(value=done / el, unit="tokens/s", cores=oracle.max_threads(), kind="oracle",
+                sample=f"{n} whole sequences of {spec.T} tokens x {spec.H} heads (fp64 "
+                       f"token-by-token recurrence, OpenMP over heads), {el:.1f} s")
+
+
+def reference_arm(args, world, rank):
+    """--impl reference: the fp64 CPU oracle on a bounded sample of the same workload per step."""
+    if rank != 0:
+        return
+    import kda_synth
+    import oracle
+
+    spec = kda_synth.STANDARD
+    x = kda_synth.prefill_inputs(spec, 2001, "cpu")
+    heads = 8  # per step: one sequence, 8 of the 32 heads, all 4096 tokens
+    sub = {n: x[n][0, :, :heads].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    s0 = x["initial_state"][0:1, :heads].contiguous()
+
+    def step():
+        oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"],
+                         initial_state=s0)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    tokens_per_s = args.steps * spec.T * heads / spec.H / el  # whole-head-equivalent tokens
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H, "d": spec.Dk,
+                   "chunk": spec.chunk},
+        "cpu_baseline": {"value": tokens_per_s, "unit": "tokens/s", "cores": oracle.max_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: 1 sequence x {heads} of {spec.H} heads x "
+                                   f"{spec.T} tokens, scaled to whole-head tokens"},
+        "e2e": {"value": tokens_per_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+    from gated_delta_rule_120_b200 import roofline
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.lib()
+    peaks, peak_src = load_peaks()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+
+    spec = kda_synth.STANDARD
+    seeds = [2001 + 10 * rank + r for r in range(4)]
+    with ClockSampler(uuid if rank == 0 else None) as clk:
+        pre = run_prefill(spec, seeds, dev, args.steps, args.warmup, world)
+    clocks = clk.summary() if rank == 0 else None
+    ms_step = pre["ms"] / args.steps
+    tokens = spec.total_tokens
+    value = world * tokens * args.steps / (pre["ms"] / 1e3)
+
+    # roofline of the dominant kernel
+    prof = pre["prof"]
+    launches_per_step = sum(p["launches"] for p in prof) / args.steps
+    rec_bytes = pre["ws_bytes"]  # placeholder, replaced below by the per-record size
+    n_chunks = chunk_count(spec)
+    top = prof[0]
+    ws_records = pre["ws_bytes"] - 256
+    rec_bytes = ws_records // max(1, n_chunks * spec.H)
+    top_bytes = prefill_kernel_bytes(top["name"], spec, n_chunks, rec_bytes)
+    top_ms = top["total_ms"] / top["launches"]
+    achieved = top_bytes / (top_ms / 1e3) / 1e9 if top_bytes else None
+    hbm_peak = peaks["hbm_gbs"]
+    roof = {"kernel": top["name"], "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+            "unit": "GB/s", "frac": (achieved / hbm_peak) if achieved else None, "traffic": None,
+            "peak_source": f"{peak_src} HBM copy bandwidth",
+            "launch_ms": top_ms,
+            "kernels": [{"name": p["name"], "launches_per_step": p["launches"] / args.steps,
+                         "ms_per_launch": p["total_ms"] / p["launches"],
+                         "share": p["total_ms"] / sum(q["total_ms"] for q in prof)}
+                        for p in prof]}
+    # path-level figures for the prefill step
+    min_bytes = roofline.prefill_min_bytes(spec.token_heads(), spec.num_seqs, spec.H, spec.Dk,
+                                           spec.Dv, 2, spec.init_std > 0, True)
+    eq13 = roofline.eq13_flops(spec.T, spec.chunk, spec.Dk) * spec.B * spec.H
+    tc_peak = peaks["bf16_tflops"]
+    path = {"min_bytes": min_bytes, "achieved_gbs": min_bytes / (ms_step / 1e3) / 1e9,
+            "frac_hbm": min_bytes / (ms_step / 1e3) / 1e9 / hbm_peak,
+            "eq13_flops": eq13, "eq13_tflops": eq13 / (ms_step / 1e3) / 1e12,
+            "frac_tc_peak_eq13": eq13 / (ms_step / 1e3) / 1e12 / tc_peak,
+            "issued_tile_tflops": roofline.issued_tile_flops(spec.T, spec.chunk, spec.Dk) *
+            spec.B * spec.H / (ms_step / 1e3) / 1e12,
+            "roofline_floor_ms": 1e3 * max(min_bytes / (hbm_peak * 1e9),
+                                           eq13 / (tc_peak * 1e12))}
+    path["frac_min_roofline"] = path["roofline_floor_ms"] / ms_step
+
+    # public-API end to end
+    e2e_ms, h2d, d2h = run_prefill_e2e(spec, pre["sets"][0], pre["o"], pre["fs"], pre["ws"], dev,
+                                       args.steps, args.warmup, world)
+    e2e = {"value": world * tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_ms / args.steps}
+    del pre
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if not args.no_long:
+        lspec = kda_synth.LONG
+        lp = run_prefill(lspec, [2002 + 10 * rank], dev, max(2, args.steps // 5), 1, world)
+        lms = lp["ms"] / max(2, args.steps // 5)
+        lmin = roofline.prefill_min_bytes(lspec.token_heads(), 1, lspec.H, lspec.Dk, lspec.Dv, 2,
+                                          False, True)
+        extra["long_prefill"] = {
+            "workload": lspec.name, "tokens_per_s": world * lspec.total_tokens / (lms / 1e3),
+            "ms_per_call": lms, "frac_hbm_min_bytes": lmin / (lms / 1e3) / 1e9 / hbm_peak,
+            "eq13_tflops": roofline.eq13_flops(lspec.T, 64, 128) * lspec.H / (lms / 1e3) / 1e12,
+            "kernels": [{"name": p["name"], "ms_per_launch": p["total_ms"] / p["launches"]}
+                        for p in lp["prof"]]}
+        del lp
+        torch.cuda.empty_cache()
+    if not args.no_decode:
+        dspec = kda_synth.DECODE
+        dms, dprof = run_decode(dspec, args.decode_steps, dev, 3, world, rank)
+        sbytes = roofline.decode_state_bytes(dspec.N, dspec.H, dspec.Dk, dspec.Dv)
+        tbytes = roofline.decode_total_bytes(dspec.N, dspec.H, dspec.Dk, dspec.Dv, 2)
+        per = dms / args.decode_steps
+        kms = dprof[0]["total_ms"] / dprof[0]["launches"]
+        extra["decode"] = {
+            "workload": dspec.name, "steps": args.decode_steps, "ms_per_step": per,
+            "state_gbs": world * sbytes / (per / 1e3) / 1e9,
+            "frac_hbm_state": sbytes / (per / 1e3) / 1e9 / hbm_peak,
+            "total_gbs": world * tbytes / (per / 1e3) / 1e9,
+            "kernel": {"name": dprof[0]["name"], "ms_per_launch": kms,
+                       "achieved_gbs": tbytes / (kms / 1e3) / 1e9,
+                       "frac": tbytes / (kms / 1e3) / 1e9 / hbm_peak}}
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec, dev, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
+                       "d_k": spec.Dk, "d_v": spec.Dv, "chunk": spec.chunk,
+                       "state": "fp32", "gates": "fp32",
+                       "l2": "4 rotating input sets (>370 MB) larger than the 126 MB L2",
+                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "roofline": roof, "prefill_path": path, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": clocks, **extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+"""Kimi Delta Attention (KDA) operator for NVIDIA B200 — Python binding of libkda.so.
+
+This module only marshals arguments: every step of the operator runs in the CUDA kernels of
+``libkda.so`` behind the C ABI declared in ``include/kda.h``. PyTorch supplies device memory and
+the current stream. There is no CPU fallback: without the built library every call raises.
+
+Entry points (same names as the C ABI):
+  kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk=64, ...)
+      chunkwise prefill -> (o, final_state)
+  kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None)
+      one decode token per sequence, ``state`` updated in place -> o
+  kda_chunk_fwd_workspace_size(...), kda_last_device_error(), kda_status_string(code)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import roofline  # noqa: F401  (work counts used by the benchmark)
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED = 0, 1, 2
+KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_WORKSPACE = 3, 4, 5
+KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+
+# every symbol include/kda.h declares
+ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
+               "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
+               "kda_profile_enable", "kda_profile_read")
+
+
+class ProfileEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
+                ("total_ms", ctypes.c_double)]
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {status_string(code)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkda.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"libkda.so not built at {LIB_PATH}; run "
+                                  "`python -m gated_delta_rule_120_b200._build` (or "
+                                  "__graft_entry__.build())")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+            L.kda_status_string.argtypes = [ctypes.c_int]
+            L.kda_status_string.restype = ctypes.c_char_p
+            L.kda_version.argtypes = []
+            L.kda_version.restype = ctypes.c_char_p
+            L.kda_chunk_fwd_workspace_size.argtypes = [i32] * 7 + [ctypes.c_int,
+                                                                   ctypes.POINTER(sz)]
+            L.kda_chunk_fwd_workspace_size.restype = ctypes.c_int
+            L.kda_chunk_fwd.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i32, i32,
+                                        i32, i32, i32, i32, vp, vp, vp, sz, vp]
+            L.kda_chunk_fwd.restype = ctypes.c_int
+            L.kda_recurrent_step.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i32,
+                                             i32, i32, vp]
+            L.kda_recurrent_step.restype = ctypes.c_int
+            L.kda_last_device_error.argtypes = [vp]
+            L.kda_last_device_error.restype = ctypes.c_int
+            L.kda_profile_enable.argtypes = [ctypes.c_int32]
+            L.kda_profile_enable.restype = ctypes.c_int
+            L.kda_profile_read.argtypes = [ctypes.POINTER(ProfileEntry), ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_int32)]
+            L.kda_profile_read.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().kda_status_string(int(code)).decode()
+
+
+kda_status_string = status_string
+
+
+def _check(code: int, where: str):
+    if code != KDA_OK:
+        raise KDAError(code, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"q/k/v dtype {t.dtype} not supported (bf16 or fp32)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, device, dtype=None):
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
+                                 num_seqs: int, dtype: torch.dtype) -> int:
+    out = ctypes.c_size_t(0)
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    _check(lib().kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, num_seqs, code,
+                                              ctypes.byref(out)), "kda_chunk_fwd_workspace_size")
+    return int(out.value)
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
+                  output_final_state: bool = True, o=None, final_state=None, workspace=None):
+    """Chunkwise KDA prefill.
+
+    q, k [B,T,H,Dk], v [B,T,H,Dv] (bf16 or fp32, same dtype); log_alpha [B,T,H,Dk] fp32;
+    beta [B,T,H] fp32; initial_state [N,H,Dk,Dv] fp32 or None; cu_seqlens int32 [N+1] on the
+    device or None (then N = B). Returns (o [B,T,H,Dv] in the input dtype, final_state or None).
+    """
+    dev = q.device
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, q.dtype)
+    _need(log_alpha, "log_alpha", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    if tuple(k.shape) != (B, T, H, Dk) or tuple(log_alpha.shape) != (B, T, H, Dk) or \
+            tuple(v.shape[:3]) != (B, T, H) or tuple(beta.shape) != (B, T, H):
+        raise ValueError("inconsistent q/k/v/log_alpha/beta shapes")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if initial_state is not None:
+        _need(initial_state, "initial_state", dev, torch.float32)
+        if tuple(initial_state.shape) != (N, H, Dk, Dv):
+            raise ValueError("initial_state must be [N,H,Dk,Dv]")
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
+    ws_bytes = kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, N, q.dtype)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    code = lib().kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+        _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
+        _ptr(final_state if output_final_state else None), _ptr(workspace),
+        workspace.numel(), _stream_handle(dev))
+    _check(code, "kda_chunk_fwd")
+    return o, (final_state if output_final_state else None)
+
+
+def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
+    """One decode token per sequence: q, k [N,H,Dk], v [N,H,Dv], log_alpha [N,H,Dk] fp32,
+    beta [N,H] fp32; ``state`` [N,H,Dk,Dv] fp32 is updated in place. Returns o [N,H,Dv]."""
+    dev = q.device
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, q.dtype)
+    _need(log_alpha, "log_alpha", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    _need(state, "state", dev, torch.float32)
+    if tuple(state.shape) != (N, H, Dk, Dv):
+        raise ValueError("state must be [N,H,Dk,Dv]")
+    if o is None:
+        o = torch.empty((N, H, Dv), dtype=q.dtype, device=dev)
+    code = lib().kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
+                                    _ptr(beta), _ptr(state), _ptr(o), N, H, Dk, Dv,
+                                    _stream_handle(dev))
+    _check(code, "kda_recurrent_step")
+    return o
+
+
+def kda_last_device_error(device=None) -> int:
+    """Read and clear the device status word (synchronises the current stream)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                        torch.cuda.current_device())
+    return int(lib().kda_last_device_error(_stream_handle(dev)))
+
+
+def kda_profile_enable(enable: bool = True) -> None:
+    """Bracket every kernel this library launches (from this thread) with CUDA events."""
+    _check(lib().kda_profile_enable(1 if enable else 0), "kda_profile_enable")
+
+
+def kda_profile_read() -> list[dict]:
+    """Per-kernel launches and summed device ms since the last read (synchronises the events)."""
+    cap = 64
+    arr = (ProfileEntry * cap)()
+    n = ctypes.c_int32(0)
+    _check(lib().kda_profile_read(arr, cap, ctypes.byref(n)), "kda_profile_read")
+    return [dict(name=arr[i].name.decode(), launches=int(arr[i].launches),
+                 total_ms=float(arr[i].total_ms)) for i in range(min(n.value, cap))]

@@ -1,0 +1,198 @@
+// kda_api.cu — the C ABI of the KDA library: argument validation, workspace layout, dispatch.
+// Every argument error is caught here, on the host, before anything is launched.
+#include <stdint.h>
+#include <string.h>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+namespace {
+
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Workspace layout of one prefill call:
+//   [0, 256)                 header: int32 `valid` flag written by the chunk-map kernel
+//   [256, 256 + off_bytes)   int32 chunk_off[N+1] (packed varlen batches only)
+//   [rec_base, ...)          per (chunk, head) records of the kernel path
+struct WsLayout {
+  size_t chunk_off_base;
+  size_t rec_base;
+  size_t rec_bytes;  // bytes of one record
+  long long max_chunks;
+  size_t total;
+};
+
+bool is_tc_path(kda_dtype_t dt) { return dt == KDA_DTYPE_BF16; }
+
+kda_status_t check_prefill_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                 int32_t C, int32_t N, kda_dtype_t dt, bool varlen) {
+  if (B < 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || N < 0 || C <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (varlen) {
+    if (B != 1 && !(B == 0 && T == 0)) return KDA_ERR_INVALID_ARG;
+  } else if (N != B) {
+    return KDA_ERR_INVALID_ARG;
+  }
+  if (dt == KDA_DTYPE_BF16) {
+    if (Dk != 128 || Dv != 128 || C != 64) return KDA_ERR_UNSUPPORTED;
+  } else {
+    if (Dk > 128 || Dv > 128) return KDA_ERR_UNSUPPORTED;
+    if (C != 16 && C != 32 && C != 64) return KDA_ERR_UNSUPPORTED;
+  }
+  const long long tokens = (long long)B * T;
+  const long long elems = tokens * H * (long long)(Dk > Dv ? Dk : Dv);
+  if (tokens > INT32_MAX || elems > (1LL << 40)) return KDA_ERR_UNSUPPORTED;
+  return KDA_OK;
+}
+
+WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv, int32_t C,
+                        int32_t N, bool varlen) {
+  WsLayout w;
+  const long long tokens = (long long)B * T;
+  w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
+  w.chunk_off_base = 256;
+  const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * ((size_t)N + 1), 256) : 0;
+  w.rec_base = w.chunk_off_base + off_bytes;
+  w.rec_bytes = SimtRecord::make(C, Dk, Dv).record_floats * sizeof(float);
+  w.total = w.rec_base + (size_t)w.max_chunks * H * w.rec_bytes;
+  return w;
+}
+
+kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_status_string(kda_status_t s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported size or dtype";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing, small or misaligned";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+const char* kda_version(void) { return "0.1.0"; }
+
+kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                          int32_t chunk, int32_t num_seqs, kda_dtype_t dt,
+                                          size_t* bytes) {
+  if (!bytes) return KDA_ERR_INVALID_ARG;
+  // the size query cannot know whether cu_seqlens will be passed: size for the larger (varlen)
+  // layout whenever B == 1, which also covers the fixed-length layout
+  const bool varlen = (B == 1);
+  kda_status_t st = check_prefill_shape(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, dt, varlen);
+  if (st != KDA_OK) return st;
+  *bytes = prefill_layout(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, varlen).total;
+  return KDA_OK;
+}
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                           const float* log_alpha, const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t N, int32_t B, int32_t T, int32_t H,
+                           int32_t Dk, int32_t Dv, int32_t C, void* o, float* final_state,
+                           void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+  const bool varlen = cu_seqlens != nullptr;
+  kda_status_t st = check_prefill_shape(B, T, H, Dk, Dv, C, N, dt, varlen);
+  if (st != KDA_OK) return st;
+  const long long tokens = (long long)B * T;
+  if (tokens > 0) {
+    if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(log_alpha, 16) || !aligned(beta, 4))
+      return KDA_ERR_INVALID_ARG;
+  }
+  if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+    return KDA_ERR_INVALID_ARG;
+  if (varlen && !aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+  if (N == 0) return KDA_OK;
+
+  const WsLayout lay = prefill_layout(B, T, H, Dk, Dv, C, N, varlen);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total)
+    return KDA_ERR_WORKSPACE;
+
+  cudaStream_t stream = (cudaStream_t)stream_;
+  char* ws = (char*)workspace;
+  int32_t* valid = (int32_t*)ws;
+  int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
+  if (varlen) {
+    st = from_cuda(launch_chunk_map(cu_seqlens, N, (int)tokens, C, chunk_off, valid, stream));
+    if (st != KDA_OK) return st;
+  }
+  SeqGeometry geo;
+  geo.cu_seqlens = cu_seqlens;
+  geo.chunk_off = chunk_off;
+  geo.valid = valid;
+  geo.N = N;
+  geo.T = T;
+  geo.C = C;
+
+  PrefillArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dtype = dt;
+  a.log_alpha = log_alpha;
+  a.beta = beta;
+  a.initial_state = initial_state;
+  a.cu_seqlens = cu_seqlens;
+  a.N = N;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.Dk = Dk;
+  a.Dv = Dv;
+  a.C = C;
+  a.o = o;
+  a.final_state = final_state;
+
+  const SimtRecord rec = SimtRecord::make(C, Dk, Dv);
+  return from_cuda(launch_prefill_simt(a, geo, (int)lay.max_chunks,
+                                       (float*)(ws + lay.rec_base), rec, stream));
+}
+
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                const float* log_alpha, const float* beta, float* state, void* o,
+                                int32_t N, int32_t H, int32_t Dk, int32_t Dv,
+                                kda_stream_t stream) {
+  if (N < 0 || H < 0 || Dk <= 0 || Dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H == 0) return KDA_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;  // q, k, v, o need element alignment only
+  if (!aligned(state, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
+      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+    return KDA_ERR_INVALID_ARG;
+  return from_cuda(launch_decode_step(q, k, v, dt, log_alpha, beta, state, o, N, H, Dk, Dv,
+                                      (cudaStream_t)stream));
+}
+
+kda_status_t kda_last_device_error(kda_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  unsigned int bits = 0;
+  e = cudaMemcpyFromSymbol(&bits, g_status, sizeof(bits));
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  if (bits) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  if (bits & kStatusTimeout) return KDA_ERR_TIMEOUT;
+  if (bits & kStatusBadSeqlens) return KDA_ERR_INVALID_ARG;
+  return KDA_OK;
+}
+
+}  // extern "C"

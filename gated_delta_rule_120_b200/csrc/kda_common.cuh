@@ -1,0 +1,101 @@
+// kda_common.cuh — shared device helpers of the KDA CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// ---------------------------------------------------------------------------------------------
+// Per-device status word. Kernels OR a kda_status_t bit pattern into it when they detect a fault
+// that the host could not see (bad cu_seqlens contents, a bounded wait that gave up); the host
+// reads and clears it in kda_last_device_error(). File-scope __device__ storage is instantiated
+// once per device context, so there is one word per GPU.
+// ---------------------------------------------------------------------------------------------
+__device__ unsigned int g_status = 0;  // one definition: the library is a single TU
+
+enum : unsigned int {
+  kStatusBadSeqlens = 1u << 0,
+  kStatusTimeout = 1u << 1,
+};
+
+__device__ __forceinline__ void raise_status(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// ---------------------------------------------------------------------------------------------
+// Element access for the two input dtypes.
+// ---------------------------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) {
+  return (x + a - 1) / a * a;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Sequence / chunk geometry of one prefill call.
+//   Without cu_seqlens: sequence n is batch row n, tokens [n*T, (n+1)*T), ceil(T/C) chunks each.
+//   With cu_seqlens: chunk_off[n] (device, in the workspace) is the index of the first chunk of
+//   sequence n; chunk_off[N] is the number of chunks. A global chunk index is mapped back to its
+//   sequence by binary search over chunk_off.
+// ---------------------------------------------------------------------------------------------
+struct SeqGeometry {
+  const int32_t* cu_seqlens;  // device, or nullptr
+  const int32_t* chunk_off;   // device [N+1], valid when cu_seqlens != nullptr
+  const int32_t* valid;       // device flag written by the chunk-map kernel (varlen only)
+  int32_t N;
+  int32_t T;  // tokens per sequence when cu_seqlens == nullptr
+  int32_t C;
+
+  __device__ __forceinline__ bool ok() const { return cu_seqlens == nullptr || *valid != 0; }
+
+  __device__ __forceinline__ int num_chunks_total() const {
+    return cu_seqlens ? chunk_off[N] : N * ceil_div(T, C);
+  }
+  __device__ __forceinline__ int seq_begin(int n) const {
+    return cu_seqlens ? cu_seqlens[n] : n * T;
+  }
+  __device__ __forceinline__ int seq_end(int n) const {
+    return cu_seqlens ? cu_seqlens[n + 1] : (n + 1) * T;
+  }
+  __device__ __forceinline__ int first_chunk(int n) const {
+    return cu_seqlens ? chunk_off[n] : n * ceil_div(T, C);
+  }
+  // Sequence that owns global chunk `c` (c < num_chunks_total()).
+  __device__ __forceinline__ int seq_of_chunk(int c) const {
+    if (!cu_seqlens) return c / ceil_div(T, C);
+    int lo = 0, hi = N - 1;  // largest n with chunk_off[n] <= c (skips empty sequences)
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (chunk_off[mid] <= c)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    return lo;
+  }
+};
+
+}  // namespace kda

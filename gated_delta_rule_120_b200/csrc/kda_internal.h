@@ -1,0 +1,83 @@
+// kda_internal.h — host-side declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+struct SeqGeometry;
+
+// RAII bracket of one kernel launch for kda_profile_* (no-op unless profiling is enabled).
+class ProfileScope {
+ public:
+  ProfileScope(const char* name, cudaStream_t stream);
+  ~ProfileScope();
+  ProfileScope(const ProfileScope&) = delete;
+  ProfileScope& operator=(const ProfileScope&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t stream_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+  bool active_ = false;
+};
+
+// Arguments of one kda_chunk_fwd call after host validation.
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  kda_dtype_t dtype;
+  const float* log_alpha;
+  const float* beta;
+  const float* initial_state;
+  const int32_t* cu_seqlens;
+  int N, B, T, H, Dk, Dv, C;
+  void* o;
+  float* final_state;
+};
+
+// Per (chunk, head) record of the fp32 CUDA-core path, in floats:
+//   W [C][Dk], U [C][Dv], Kt [C][Dk], Qt [C][Dk], A_qk [C][C], gamma_C [Dk]
+struct SimtRecord {
+  size_t record_floats;
+  size_t off_w, off_u, off_kt, off_qt, off_aqk, off_gam;
+
+  static SimtRecord make(int C, int Dk, int Dv) {
+    SimtRecord r;
+    size_t o = 0;
+    r.off_w = o;
+    o += (size_t)C * Dk;
+    r.off_u = o;
+    o += (size_t)C * Dv;
+    r.off_kt = o;
+    o += (size_t)C * Dk;
+    r.off_qt = o;
+    o += (size_t)C * Dk;
+    r.off_aqk = o;
+    o += (size_t)C * C;
+    r.off_gam = o;
+    o += (size_t)Dk;
+    r.record_floats = (o + 63) / 64 * 64;  // 256-byte records
+    return r;
+  }
+};
+
+cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                               const float* log_alpha, const float* beta, float* state, void* o,
+                               int N, int H, int Dk, int Dv, cudaStream_t stream);
+
+cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
+                             int32_t* valid, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
+                                float* records, const SimtRecord& rec, cudaStream_t stream);
+
+size_t simt_local_smem_bytes(int C, int Dk, int Dv);
+size_t simt_state_smem_bytes(int C, int Dk);
+
+}  // namespace kda

@@ -1,0 +1,7 @@
+// kda_lib.cu — single translation unit of libkda.so. The kernel files share one per-device
+// status word (defined in kda_api.cu), so they are compiled together rather than linked with
+// relocatable device code.
+#include "kda_api.cu"
+#include "kda_profile.cu"
+#include "kda_decode.cu"
+#include "kda_chunk_simt.cu"

@@ -34,6 +34,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -52,10 +58,10 @@ typedef enum {
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
 
 /* Human-readable name of a status code. Never returns NULL. */
-const char* kda_status_string(kda_status_t status);
+KDA_API const char* kda_status_string(kda_status_t status);
 
 /* Library version, "major.minor.patch". */
-const char* kda_version(void);
+KDA_API const char* kda_version(void);
 
 /*
  * kda_chunk_fwd_workspace_size — bytes of device scratch that kda_chunk_fwd needs.
@@ -68,7 +74,7 @@ const char* kda_version(void);
  *   bytes (out, host pointer)         : required size, a multiple of 256.
  * Returns KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED for sizes kda_chunk_fwd would reject.
  */
-kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+KDA_API kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
                                           int32_t chunk, int32_t num_seqs, kda_dtype_t qkv_dtype,
                                           size_t* bytes);
 
@@ -93,7 +99,7 @@ kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32
  * with 1 <= Dk, Dv <= 128 and Dv a multiple of 4 (CUDA-core fp32 path).
  * Tokens past cu_seqlens[N] are neither read nor written.
  */
-kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
                            const float* log_alpha, const float* beta, const float* initial_state,
                            const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                            int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, void* o,
@@ -111,10 +117,11 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtyp
  *   log_alpha       device fp32 [N,H,Dk]; beta device fp32 [N,H].
  *   state           device fp32 [N,H,Dk,Dv], read and overwritten; 16-byte aligned.
  *   o               device [N,H,Dv], dtype qkv_dtype: o = S_new^T q.
+ * q, k, v and o need the alignment of their element type; log_alpha and beta 4 bytes.
  * Supported: 1 <= Dk <= 128, 4 <= Dv <= 128 with Dv a multiple of 4, either dtype.
  * The state is streamed once from HBM and written once.
  */
-kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+KDA_API kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
                                 const float* log_alpha, const float* beta, float* state, void* o,
                                 int32_t N, int32_t H, int32_t Dk, int32_t Dv, kda_stream_t stream);
 
@@ -123,7 +130,24 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda
  * (KDA_ERR_INVALID_ARG for a bad cu_seqlens, KDA_ERR_TIMEOUT for a bounded wait that gave up).
  * Synchronises `stream`. Returns KDA_OK when no kernel reported a fault.
  */
-kda_status_t kda_last_device_error(kda_stream_t stream);
+KDA_API kda_status_t kda_last_device_error(kda_stream_t stream);
+
+/*
+ * Kernel-level timing (tracing). While enabled, every kernel the library launches on the calling
+ * host thread is bracketed by a pair of CUDA events recorded on its stream. kda_profile_read
+ * synchronises those events, returns per-kernel launch counts and summed device milliseconds
+ * (entries sorted by total time, descending) and forgets them. Events are host-side objects: no
+ * device memory is allocated. Disabled by default; enabling adds two event records per launch.
+ */
+typedef struct {
+  char name[48];
+  int32_t launches;
+  double total_ms;
+} kda_profile_entry_t;
+
+KDA_API kda_status_t kda_profile_enable(int32_t enable);
+KDA_API kda_status_t kda_profile_read(kda_profile_entry_t* entries, int32_t capacity,
+                                      int32_t* count);
 
 #ifdef __cplusplus
 }

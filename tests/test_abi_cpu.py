@@ -1,0 +1,127 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports every declared symbol,
+and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_120_b200 as kda
+from gated_delta_rule_120_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return kda.lib()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "kda.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    syms = declared_symbols()
+    assert len(syms) >= 6
+    assert set(syms) == set(kda.ABI_SYMBOLS)
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert kda.status_string(code).startswith("KDA_")
+    assert kda.status_string(99) == "KDA_ERR_UNKNOWN"
+    assert L.kda_version().decode().count(".") == 2
+
+
+def _ws(B, T, H, Dk, Dv, C, N, dt):
+    out = ctypes.c_size_t(0)
+    rc = kda.lib().kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, C, N, dt, ctypes.byref(out))
+    return rc, out.value
+
+
+def test_workspace_size_queries(L):
+    rc, n = _ws(2, 4096, 32, 128, 128, 64, 2, kda.KDA_DTYPE_BF16)
+    assert rc == kda.KDA_OK and n > 0 and n % 256 == 0
+    rc, n1 = _ws(1, 1000, 4, 32, 32, 64, 3, kda.KDA_DTYPE_F32)
+    assert rc == kda.KDA_OK
+    rc, n2 = _ws(1, 1000, 4, 32, 32, 64, 30, kda.KDA_DTYPE_F32)
+    assert rc == kda.KDA_OK and n2 >= n1  # more sequences => more partial chunks
+    assert _ws(1, 256, 1, 96, 128, 64, 1, kda.KDA_DTYPE_BF16)[0] == kda.KDA_ERR_UNSUPPORTED
+    assert _ws(1, 256, 1, 32, 32, 48, 1, kda.KDA_DTYPE_F32)[0] == kda.KDA_ERR_UNSUPPORTED
+    assert _ws(1, 256, 1, 256, 32, 64, 1, kda.KDA_DTYPE_F32)[0] == kda.KDA_ERR_UNSUPPORTED
+    assert _ws(1, -1, 1, 32, 32, 64, 1, kda.KDA_DTYPE_F32)[0] == kda.KDA_ERR_INVALID_ARG
+    assert _ws(1, 256, 0, 32, 32, 64, 1, kda.KDA_DTYPE_F32)[0] == kda.KDA_ERR_INVALID_ARG
+    assert _ws(1, 256, 1, 32, 32, 64, 1, 7)[0] == kda.KDA_ERR_INVALID_ARG
+    out = ctypes.c_size_t(0)
+    assert L.kda_chunk_fwd_workspace_size(1, 1, 1, 1, 1, 64, 1, 0, None) == kda.KDA_ERR_INVALID_ARG
+    del out
+
+
+FAKE = 1 << 20  # a 256-aligned non-null address: never dereferenced, the host rejects first
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=kda.KDA_DTYPE_BF16, la=FAKE, beta=FAKE, s0=None, cu=None,
+             N=1, B=1, T=64, H=1, Dk=128, Dv=128, C=64, o=FAKE, sT=None, ws=FAKE, wsb=1 << 40,
+             stream=None)
+    a.update(kw)
+    return kda.lib().kda_chunk_fwd(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"], a["s0"],
+                                   a["cu"], a["N"], a["B"], a["T"], a["H"], a["Dk"], a["Dv"],
+                                   a["C"], a["o"], a["sT"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_prefill_argument_errors_are_caught_on_host(L):
+    E = kda
+    assert _fwd(q=None) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(o=None) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(beta=None) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(q=FAKE + 8) == E.KDA_ERR_INVALID_ARG  # misaligned
+    assert _fwd(la=FAKE + 4) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(s0=FAKE + 4) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(Dk=64) == E.KDA_ERR_UNSUPPORTED  # bf16 path is 128 x 128, C = 64
+    assert _fwd(C=32) == E.KDA_ERR_UNSUPPORTED
+    assert _fwd(dt=kda.KDA_DTYPE_F32, C=48, Dk=32, Dv=32) == E.KDA_ERR_UNSUPPORTED
+    assert _fwd(N=2) == E.KDA_ERR_INVALID_ARG  # N must equal B without cu_seqlens
+    assert _fwd(cu=FAKE, B=2, N=2) == E.KDA_ERR_INVALID_ARG  # packed input needs B == 1
+    assert _fwd(T=-5) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(H=0) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(ws=None) == E.KDA_ERR_WORKSPACE
+    assert _fwd(ws=FAKE + 16) == E.KDA_ERR_WORKSPACE
+    assert _fwd(wsb=1024) == E.KDA_ERR_WORKSPACE
+    assert _fwd(dt=3) == E.KDA_ERR_INVALID_ARG
+    assert _fwd(N=0, B=0, T=0) == E.KDA_OK  # nothing to do, nothing launched
+
+
+def _step(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=kda.KDA_DTYPE_BF16, la=FAKE, beta=FAKE, S=FAKE, o=FAKE,
+             N=4, H=2, Dk=128, Dv=128, stream=None)
+    a.update(kw)
+    return kda.lib().kda_recurrent_step(a["q"], a["k"], a["v"], a["dt"], a["la"], a["beta"],
+                                        a["S"], a["o"], a["N"], a["H"], a["Dk"], a["Dv"],
+                                        a["stream"])
+
+
+def test_decode_argument_errors_are_caught_on_host(L):
+    E = kda
+    assert _step(S=None) == E.KDA_ERR_INVALID_ARG
+    assert _step(S=FAKE + 4) == E.KDA_ERR_INVALID_ARG
+    assert _step(q=None) == E.KDA_ERR_INVALID_ARG
+    assert _step(Dv=130) == E.KDA_ERR_UNSUPPORTED
+    assert _step(Dv=6) == E.KDA_ERR_UNSUPPORTED
+    assert _step(Dk=129) == E.KDA_ERR_UNSUPPORTED
+    assert _step(N=-1) == E.KDA_ERR_INVALID_ARG
+    assert _step(dt=9) == E.KDA_ERR_INVALID_ARG
+    assert _step(N=0) == E.KDA_OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(kda, "_lib", None)
+    with pytest.raises(ImportError):
+        kda.lib()

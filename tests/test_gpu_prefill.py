@@ -1,0 +1,210 @@
+"""GPU parity of kda_chunk_fwd (chunkwise prefill) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_120_b200 as kda
+import kda_synth
+import oracle
+from kda_synth import PrefillSpec
+from tests._parity import TOL_BF16_O, TOL_BF16_S, TOL_F32, cu_list, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, chunk, **kw):
+    o, s = kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                             initial_state=inp["initial_state"], cu_seqlens=inp["cu_seqlens"],
+                             chunk=chunk, **kw)
+    torch.cuda.synchronize()
+    assert kda.kda_last_device_error() == kda.KDA_OK
+    return o, s
+
+
+def _oracle(inp, B, T):
+    H = inp["q"].shape[2]
+    cu = inp["cu_seqlens"]
+    cu = cu_list(B, T) if cu is None else cu.cpu().numpy()
+    o, s = oracle.recurrent(*(inp[x].cpu() for x in ("q", "k", "v", "log_alpha", "beta")),
+                            initial_state=None if inp["initial_state"] is None
+                            else inp["initial_state"].cpu(), cu_seqlens=cu)
+    return o.reshape(B, T, H, -1), s
+
+
+def _check(spec: PrefillSpec, seed: int, dev, tol_o, tol_s):
+    inp = kda_synth.prefill_inputs(spec, seed, dev)
+    o, s = _run(inp, spec.chunk)
+    o_ref, s_ref = _oracle(inp, spec.B, spec.T)
+    eo, es = rel_err(o, o_ref), rel_err(s, s_ref)
+    assert eo <= tol_o, f"o error {eo:.3e} > {tol_o}"
+    assert es <= tol_s, f"state error {es:.3e} > {tol_s}"
+    return eo, es
+
+
+# ------------------------------------------------------------------ fp32 (CUDA-core) path
+def test_tiny_f32_workload(cuda_device):
+    """B=1, H=1, T=256, d=32, C=64, fp32, zero initial state."""
+    _check(kda_synth.TINY, 1000, cuda_device, TOL_F32, TOL_F32)
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 63, 130])
+def test_f32_chunks_and_ragged_tails(cuda_device, C, T):
+    spec = PrefillSpec("t", B=2, T=T, H=3, Dk=48, Dv=20, chunk=C, dtype="f32", decay="fast",
+                       init_std=0.02)
+    _check(spec, 11 + T + C, cuda_device, TOL_F32, TOL_F32)
+
+
+@pytest.mark.parametrize("dims", [(128, 128), (1, 4), (100, 128), (128, 36)])
+def test_f32_dims(cuda_device, dims):
+    Dk, Dv = dims
+    spec = PrefillSpec("t", B=1, T=200, H=2, Dk=Dk, Dv=Dv, chunk=64, dtype="f32", decay="slow",
+                       init_std=0.02)
+    _check(spec, 21, cuda_device, TOL_F32, TOL_F32)
+
+
+def test_f32_strong_decay(cuda_device):
+    """Per-token decays down to exp(-20): cumulative decays far below fp32's range inside a chunk;
+    the kernel never forms 1/Gamma, so nothing overflows."""
+    spec = PrefillSpec("t", B=1, T=192, H=2, Dk=32, Dv=32, chunk=64, dtype="f32", decay="fast",
+                       init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 5, cuda_device)
+    inp["log_alpha"] = inp["log_alpha"] * 40.0
+    o, s = _run(inp, 64)
+    o_ref, s_ref = _oracle(inp, 1, 192)
+    assert torch.isfinite(o).all() and torch.isfinite(s).all()
+    assert rel_err(o, o_ref) <= TOL_F32 and rel_err(s, s_ref) <= TOL_F32
+
+
+def test_f32_varlen_with_empty_sequences(cuda_device):
+    lens = [0, 5, 64, 0, 129, 1, 0]
+    spec = PrefillSpec("t", B=1, T=sum(lens), H=2, Dk=32, Dv=16, chunk=32, dtype="f32",
+                       decay="fast", init_std=0.02, seqlens=tuple(lens))
+    _check(spec, 31, cuda_device, TOL_F32, TOL_F32)
+
+
+# ------------------------------------------------------------------ bf16 path (d = 128, C = 64)
+def test_bf16_small_ragged(cuda_device):
+    spec = PrefillSpec("t", B=2, T=300, H=4, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.02)
+    _check(spec, 41, cuda_device, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_standard_prefill_workload(cuda_device):
+    """The standard prefill workload in full: B=2, T=4096, H=32, d=128, C=64, bf16 q/k/v, fp32
+    gates, initial state ~ N(0, 0.02^2); every output and final state against the oracle."""
+    _check(kda_synth.STANDARD, 1001, cuda_device, TOL_BF16_O, TOL_BF16_S)
+
+
+def test_bf16_varlen_small(cuda_device):
+    lens = [1, 64, 65, 0, 200, 127, 3]
+    spec = PrefillSpec("t", B=1, T=sum(lens), H=3, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.0, seqlens=tuple(lens))
+    _check(spec, 51, cuda_device, TOL_BF16_O, TOL_BF16_S)
+
+
+def _sampled_heads_check(spec, seed, dev, heads, seqs=None):
+    """Full-size run on the GPU; the oracle recomputes selected (sequence, head) pairs."""
+    inp = kda_synth.prefill_inputs(spec, seed, dev)
+    o, s = _run(inp, spec.chunk)
+    cu = inp["cu_seqlens"]
+    cu = cu_list(spec.B, spec.T) if cu is None else cu.cpu().numpy()
+    seqs = range(len(cu) - 1) if seqs is None else seqs
+    flat = {x: inp[x].reshape(-1, *inp[x].shape[2:]) for x in ("q", "k", "v", "log_alpha", "beta")}
+    o_flat = o.reshape(-1, *o.shape[2:])
+    worst_o = worst_s = 0.0
+    for n in seqs:
+        a, b = int(cu[n]), int(cu[n + 1])
+        if b == a:
+            continue
+        hs = torch.tensor(heads, device=dev)
+        sub = {x: flat[x][a:b].index_select(1, hs).cpu() for x in flat}
+        s0 = None if inp["initial_state"] is None else inp["initial_state"][n:n + 1][:, heads].cpu()
+        o_ref, s_ref = oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["log_alpha"],
+                                        sub["beta"], initial_state=s0)
+        worst_o = max(worst_o, rel_err(o_flat[a:b].index_select(1, hs), o_ref))
+        worst_s = max(worst_s, rel_err(s[n:n + 1][:, heads], s_ref))
+    assert worst_o <= TOL_BF16_O, worst_o
+    assert worst_s <= TOL_BF16_S, worst_s
+    return inp, o, s
+
+
+def test_bf16_long_prefill_sampled(cuda_device):
+    """B=1, T=131072, H=32: two heads recomputed by the oracle end to end (o and final state)."""
+    _sampled_heads_check(kda_synth.LONG, 1002, cuda_device, heads=[0, 17])
+
+
+def test_bf16_varlen_workload_sampled(cuda_device):
+    """16 packed sequences with log-uniform lengths in [256, 32768]: the shortest and the longest
+    sequence, two heads each, recomputed by the oracle."""
+    spec = kda_synth.varlen_spec(1003)
+    lens = np.asarray(spec.seqlens)
+    pick = [int(np.argmin(lens)), int(np.argmax(lens))]
+    _sampled_heads_check(spec, 1003, cuda_device, heads=[3, 30], seqs=pick)
+
+
+# ------------------------------------------------------------------ invariants and edge cases
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_state_handoff_between_calls(cuda_device, dtype):
+    """prefill(T) == prefill(T1) then prefill(T2) from its final state (the chunk boundary rule
+    at a call boundary), including a cut inside a chunk."""
+    D = 128 if dtype == "bf16" else 32
+    spec = PrefillSpec("t", B=1, T=400, H=2, Dk=D, Dv=D, chunk=64, dtype=dtype, decay="fast",
+                       init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 61, cuda_device)
+    o, s = _run(inp, 64)
+    for cut in (128, 173):
+        a = {x: (inp[x][:, :cut].contiguous() if x not in ("initial_state", "cu_seqlens")
+                 else inp[x]) for x in inp}
+        b = {x: (inp[x][:, cut:].contiguous() if x not in ("initial_state", "cu_seqlens")
+                 else inp[x]) for x in inp}
+        o1, s1 = _run(a, 64)
+        b["initial_state"] = s1
+        o2, s2 = _run(b, 64)
+        tol = TOL_BF16_S if dtype == "bf16" else TOL_F32
+        assert rel_err(torch.cat([o1, o2], 1), o) <= (TOL_BF16_O if dtype == "bf16" else TOL_F32)
+        assert rel_err(s2, s) <= tol
+
+
+def test_initial_state_may_alias_final_state(cuda_device):
+    spec = PrefillSpec("t", B=2, T=150, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 71, cuda_device)
+    _, s_ref = _run(inp, 64)
+    st = inp["initial_state"].clone()
+    inp["initial_state"] = st
+    _, s2 = _run(inp, 64, final_state=st)
+    assert s2.data_ptr() == st.data_ptr()
+    assert torch.equal(st, s_ref)
+
+
+def test_prefill_is_deterministic(cuda_device):
+    spec = PrefillSpec("t", B=1, T=700, H=4, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 81, cuda_device)
+    o1, s1 = _run(inp, 64)
+    o2, s2 = _run(inp, 64)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_empty_batch_copies_state(cuda_device):
+    spec = PrefillSpec("t", B=1, T=0, H=2, Dk=32, Dv=32, chunk=64, dtype="f32", decay="fast",
+                       init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 91, cuda_device)
+    o, s = _run(inp, 64)
+    assert o.numel() == 0 and torch.equal(s, inp["initial_state"])
+
+
+def test_bad_cu_seqlens_reported_not_crashing(cuda_device):
+    """A non-monotone cu_seqlens cannot be seen on the host (it lives on the device): the chunk
+    map flags it, every kernel skips its work, and the status word reports INVALID_ARG."""
+    spec = PrefillSpec("t", B=1, T=128, H=1, Dk=32, Dv=32, chunk=64, dtype="f32", decay="fast",
+                       init_std=0.0, seqlens=(64, 64))
+    inp = kda_synth.prefill_inputs(spec, 101, cuda_device)
+    inp["cu_seqlens"] = torch.tensor([0, 100, 64], dtype=torch.int32, device=cuda_device)
+    sentinel = torch.full((1, 128, 1, 32), 7.0, device=cuda_device)
+    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                      cu_seqlens=inp["cu_seqlens"], chunk=64, o=sentinel)
+    assert kda.kda_last_device_error() == kda.KDA_ERR_INVALID_ARG
+    assert torch.all(sentinel == 7.0)
+    assert kda.kda_last_device_error() == kda.KDA_OK  # reading clears the word

@@ -31,7 +31,7 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 # every symbol include/kda.h declares
 ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
-               "kda_profile_enable", "kda_profile_read")
+               "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc")
 
 
 class ProfileEntry(ctypes.Structure):
@@ -74,6 +74,9 @@ def lib() -> ctypes.CDLL:
             L.kda_recurrent_step.restype = ctypes.c_int
             L.kda_last_device_error.argtypes = [vp]
             L.kda_last_device_error.restype = ctypes.c_int
+            L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32,
+                                                i32, i32, i32, i32, i32, i32, vp, vp, vp]
+            L.kda_chunk_fwd_noalloc.restype = ctypes.c_int
             L.kda_profile_enable.argtypes = [ctypes.c_int32]
             L.kda_profile_enable.restype = ctypes.c_int
             L.kda_profile_read.argtypes = [ctypes.POINTER(ProfileEntry), ctypes.c_int32,
@@ -214,3 +217,28 @@ def kda_profile_read() -> list[dict]:
     _check(lib().kda_profile_read(arr, cap, ctypes.byref(n)), "kda_profile_read")
     return [dict(name=arr[i].name.decode(), launches=int(arr[i].launches),
                  total_ms=float(arr[i].total_ms)) for i in range(min(n.value, cap))]
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h
+
+
+def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                          chunk: int = 64, o=None, final_state=None):
+    """kda_chunk_fwd without a workspace, for callers that cannot allocate device scratch: the
+    library uses its own fixed array of NOALLOC_SCRATCH_BYTES per GPU. Calls that need more are
+    rejected (KDA_ERR_WORKSPACE); overlapping calls on one GPU race on the shared array. The
+    outputs ``o`` / ``final_state`` may be passed in so that nothing is allocated here either."""
+    dev = q.device
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
+    code = lib().kda_chunk_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+        _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
+        _ptr(final_state), _stream_handle(dev))
+    _check(code, "kda_chunk_fwd_noalloc")
+    return o, final_state

@@ -5,3 +5,4 @@
 #include "kda_profile.cu"
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
+#include "kda_noalloc.cu"

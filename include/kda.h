@@ -107,6 +107,38 @@ KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, 
                            kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc — kda_chunk_fwd for callers that must not allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists only for deployment. Some callers
+ * cannot hand the library a workspace: a serving engine that reserves nearly all of HBM for its
+ * caches up front and hands out no side buffers, a plugin whose host framework owns every
+ * device allocation, or a latency-critical loop that avoids cudaMalloc/cudaFree because they can
+ * synchronise the whole device. This variant takes the same arguments as kda_chunk_fwd minus the
+ * workspace and uses instead a scratch array of KDA_NOALLOC_SCRATCH_BYTES that lives in the
+ * library's own device image (every GPU that loads the library holds it until the process
+ * exits). It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Limit: a call whose workspace (kda_chunk_fwd_workspace_size) exceeds
+ *     KDA_NOALLOC_SCRATCH_BYTES is rejected with KDA_ERR_WORKSPACE before anything is launched.
+ *   - Set-up: the first call on a device looks up the device address of the scratch array (with
+ *     that device current), so make that first call before any stream capture; the current
+ *     device must be the one that owns the pointers.
+ *   - Sharing: all calls on a device share the one array and it keeps the last call's contents.
+ *     Nothing in it needs clearing (every byte a call reads was written earlier in that call),
+ *     but calls that overlap on the GPU (different streams, or different host threads) race on
+ *     it: serialise them.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+KDA_API kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                           kda_dtype_t qkv_dtype, const float* log_alpha,
+                                           const float* beta, const float* initial_state,
+                                           const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                                           int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                           int32_t chunk, void* o, float* final_state,
+                                           kda_stream_t stream);
+
+/*
  * kda_recurrent_step — one decode token per sequence, state updated in place (the
  * walkthrough's §3.4 "FLOPs Accounting and Inference Strategy": the recurrent kernel used for
  * generation; the update is Eq. 1 in its online-gradient form of "Online Learning

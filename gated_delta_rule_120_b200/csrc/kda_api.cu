@@ -49,14 +49,15 @@ kda_status_t check_prefill_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, in
 }
 
 WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv, int32_t C,
-                        int32_t N, bool varlen) {
+                        int32_t N, bool varlen, kda_dtype_t dt) {
   WsLayout w;
   const long long tokens = (long long)B * T;
   w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
   w.chunk_off_base = 256;
   const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * ((size_t)N + 1), 256) : 0;
   w.rec_base = w.chunk_off_base + off_bytes;
-  w.rec_bytes = SimtRecord::make(C, Dk, Dv).record_floats * sizeof(float);
+  w.rec_bytes = is_tc_path(dt) ? TcRecordBytes
+                               : SimtRecord::make(C, Dk, Dv).record_floats * sizeof(float);
   w.total = w.rec_base + (size_t)w.max_chunks * H * w.rec_bytes;
   return w;
 }
@@ -93,7 +94,7 @@ kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32
   const bool varlen = (B == 1);
   kda_status_t st = check_prefill_shape(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, dt, varlen);
   if (st != KDA_OK) return st;
-  *bytes = prefill_layout(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, varlen).total;
+  *bytes = prefill_layout(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, varlen, dt).total;
   return KDA_OK;
 }
 
@@ -117,7 +118,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtyp
   if (varlen && !aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
 
-  const WsLayout lay = prefill_layout(B, T, H, Dk, Dv, C, N, varlen);
+  const WsLayout lay = prefill_layout(B, T, H, Dk, Dv, C, N, varlen, dt);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total)
     return KDA_ERR_WORKSPACE;
 
@@ -156,6 +157,9 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtyp
   a.o = o;
   a.final_state = final_state;
 
+  if (is_tc_path(dt))
+    return from_cuda(launch_prefill_tc(a, geo, (int)lay.max_chunks, (uint8_t*)(ws + lay.rec_base),
+                                       stream));
   const SimtRecord rec = SimtRecord::make(C, Dk, Dv);
   return from_cuda(launch_prefill_simt(a, geo, (int)lay.max_chunks,
                                        (float*)(ws + lay.rec_base), rec, stream));

@@ -1,0 +1,696 @@
+// kda_chunk_tc.cu — tensor-core (tcgen05) chunkwise prefill of KDA for bf16 q/k/v, d = 128, C = 64.
+//
+// Same two-kernel structure as the fp32 CUDA-core path, following "Kimi Linear: An Expressive,
+// Efficient Attention Architecture" (paper-graph-ui walkthrough, §3.4 "Chunkwise
+// Parallelization"), with every dense chunk contraction on the fifth-generation tensor cores:
+//
+//   K1 chunk_local_tc  one CTA per (chunk, head):
+//        g = cumulative log decay (fp32); Kg = Gamma.K, Ki = K/Gamma, Qg = Gamma.Q (bf16 tiles)
+//        A_kk = Kg Ki^T, A_qk = Qg Ki^T                      (tcgen05, fp32 in TMEM)
+//        M = (I + StrictTril(Diag(beta) A_kk))^{-1} Diag(beta)  (blocked forward substitution, fp32)
+//        W = M Kg, U = M V                                   (tcgen05)
+//      and writes one bf16 record per (chunk, head): W, Qt = Qg, Kt = (gamma_C/gamma_i) k_i, the
+//      masked A_qk, U, gamma_C — every tile already in the tensor-core operand layout, so K2 moves
+//      it with plain bulk copies.
+//   K2 chunk_state_tc  one CTA per (sequence, head, 64-column half of d_v), sequential in chunks:
+//        D1 = W S, D2 = Qt S  ->  V' = U - D1  ->  D3 = Kt^T V', D2 += A_qk V'
+//        S = Diag(gamma_C) S + D3 (Eq. 8, fp32 in registers),  O = D2 (Eq. 9)
+//      Warp roles: a bulk-copy producer (double-buffered records), a single MMA-issuing thread,
+//      and four epilogue warps that hold the fp32 state slice (one row of S per thread).
+//
+// (K/Gamma) is formed as k * exp(-g) only when every channel's decay over the chunk stays above
+// exp(-60), so both factors of every product stay inside bf16/fp32 range; a chunk with stronger
+// decay takes an exact CUDA-core fallback for A_kk and A_qk (ratios exp(g_r - g_i) <= 1).
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "kda_sm100.cuh"
+
+namespace kda {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr float kFastDecayLimit = 60.f;  // |g_C| bound for the direct (K/Gamma) factorisation
+
+// record layout (bytes) of one (chunk, head)
+constexpr uint32_t kRecW = 0;
+constexpr uint32_t kRecQt = 16384;
+constexpr uint32_t kRecKt = 32768;
+constexpr uint32_t kRecAqk = 49152;
+constexpr uint32_t kRecU = 57344;
+constexpr uint32_t kRecGam = 73728;
+constexpr uint32_t kRecBytes = 74240;
+static_assert(kRecBytes == TcRecordBytes, "record size mismatch");
+
+// ============================================================================================
+// K1
+// ============================================================================================
+constexpr int kK1Threads = 256;
+
+// shared-memory map of K1 (offsets from a 1024-aligned base)
+constexpr uint32_t kS1Kg = 0;          // [64 x 128] bf16 tile
+constexpr uint32_t kS1Ki = 16384;      // [64 x 128]
+constexpr uint32_t kS1Qg = 32768;      // [64 x 128]
+constexpr uint32_t kS1V = 49152;       // [64 x 128]
+constexpr uint32_t kS1M = 65536;       // [64 x 64]
+constexpr uint32_t kS1A = 73728;       // fp32 [64][65] (the scan partials alias it)
+constexpr uint32_t kS1T = 90368;       // fp32 [64][65]
+constexpr uint32_t kS1X = 107008;      // fp32 [3][16][17] level products
+constexpr uint32_t kS1Beta = 110272;   // fp32 [64]
+constexpr uint32_t kS1GC = 110528;     // fp32 [128]
+constexpr uint32_t kS1Bar = 111040;    // mbarrier
+constexpr uint32_t kS1Tmem = 111048;   // TMEM base address
+constexpr uint32_t kS1Bytes = 111056;
+constexpr int kLdA = 65;  // padded row stride of the fp32 A / T matrices
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
+  float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                    pack_bf16(f[6], f[7]));
+}
+
+__global__ void __launch_bounds__(kK1Threads, 2)
+    chunk_local_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                          const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
+                          const float* __restrict__ beta, SeqGeometry geo, int H,
+                          uint8_t* __restrict__ ws_records) {
+  extern __shared__ uint8_t smem_raw[];
+  if (!geo.ok()) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= geo.num_chunks_total()) return;
+
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sb = smem_u32(sm);
+  float* sA = reinterpret_cast<float*>(sm + kS1A);
+  float* sT = reinterpret_cast<float*>(sm + kS1T);
+  float* sX = reinterpret_cast<float*>(sm + kS1X);
+  float* sBeta = reinterpret_cast<float*>(sm + kS1Beta);
+  float* sGC = reinterpret_cast<float*>(sm + kS1GC);
+  float* sScan = sA;  // [16][128], used before A exists
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kS1Bar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS1Tmem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = geo.seq_of_chunk(c);
+  const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * kC;
+  const int L = min(kC, geo.seq_end(n) - t0);
+  uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)c * H + h);
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+
+  // ---- phase 1: loads (thread = 8 channels x 4 rows) and the cumulative decay ----------------
+  const int cg = tid & 15, rg = tid >> 4;
+  uint4 kr[4], qr[4], vr[4];
+  float g[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rg * 4 + i;
+    if (r < L) {
+      const size_t row = (size_t)(t0 + r) * H + h;
+      const uint4* kp = reinterpret_cast<const uint4*>(k + row * kD) + cg;
+      const uint4* qp = reinterpret_cast<const uint4*>(q + row * kD) + cg;
+      const uint4* vp = reinterpret_cast<const uint4*>(v + row * kD) + cg;
+      const float4* lp = reinterpret_cast<const float4*>(log_alpha + row * kD) + 2 * cg;
+      kr[i] = __ldg(kp);
+      qr[i] = __ldg(qp);
+      vr[i] = __ldg(vp);
+      const float4 a0 = __ldg(lp), a1 = __ldg(lp + 1);
+      g[i][0] = a0.x; g[i][1] = a0.y; g[i][2] = a0.z; g[i][3] = a0.w;
+      g[i][4] = a1.x; g[i][5] = a1.y; g[i][6] = a1.z; g[i][7] = a1.w;
+    } else {
+      kr[i] = qr[i] = vr[i] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[i][j] = 0.f;
+    }
+  }
+  if (tid < kC) sBeta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+#pragma unroll
+  for (int i = 1; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[i][j] += g[i - 1][j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sScan[rg * kD + cg * 8 + j] = g[3][j];
+  __syncthreads();
+  {
+    float pre[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pre[j] = 0.f;
+    for (int r2 = 0; r2 < rg; ++r2)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pre[j] += sScan[r2 * kD + cg * 8 + j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) g[i][j] += pre[j];
+  }
+  if (rg == 15)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sGC[cg * 8 + j] = g[3][j];
+  __syncthreads();
+  float gc[8];
+  bool ok = true;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    gc[j] = sGC[cg * 8 + j];
+    ok = ok && (gc[j] >= -kFastDecayLimit);
+  }
+  const bool fast = __syncthreads_and(ok) != 0;
+
+  // ---- phase 2: scaled operand tiles (smem) and the Qt / Kt record tiles (global) ------------
+  {
+    float egc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) egc[j] = expf(gc[j]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rg * 4 + i;
+      float kf[8], qf[8], kg[8], ki[8], qg[8], kt[8];
+      unpack8(kr[i], kf);
+      unpack8(qr[i], qf);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float e = __expf(g[i][j]);
+        kg[j] = kf[j] * e;
+        qg[j] = qf[j] * e;
+        if (fast) {
+          ki[j] = kf[j] * __expf(-g[i][j]);
+          kt[j] = ki[j] * egc[j];
+        } else {
+          ki[j] = 0.f;
+          kt[j] = kf[j] * __expf(gc[j] - g[i][j]);
+        }
+      }
+      const uint32_t off = tile_chunk_off(r, cg, 8192);
+      const uint4 qgv = pack8(qg), ktv = pack8(kt);
+      st_shared_v4(sb + kS1Kg + off, pack8(kg));
+      st_shared_v4(sb + kS1Ki + off, pack8(ki));
+      st_shared_v4(sb + kS1Qg + off, qgv);
+      st_shared_v4(sb + kS1V + off, vr[i]);
+      *reinterpret_cast<uint4*>(rec + kRecQt + off) = qgv;
+      *reinterpret_cast<uint4*>(rec + kRecKt + off) = ktv;
+    }
+  }
+  if (!fast) {
+    // exact fallback: keep the cumulative decay in this record's W/U area (overwritten later)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rg * 4 + i;
+      float* gp = reinterpret_cast<float*>(rec + (r < 32 ? kRecW + r * 512 : kRecU + (r - 32) * 512));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gp[cg * 8 + j] = g[i][j];
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- phase 3: A_kk = Kg Ki^T (cols 0..63), A_qk = Qg Ki^T (cols 64..127) -------------------
+  bool alive = true;
+  if (fast) {
+    if (tid == 0) {
+      const uint32_t id = idesc_bf16_f32(64, 64, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+        const uint64_t bdesc = smem_desc_sw128(sb + kS1Ki + koff, 16, 1024);
+        mma_bf16(tmem + 0, smem_desc_sw128(sb + kS1Kg + koff, 16, 1024), bdesc, id, kk > 0);
+        mma_bf16(tmem + 64, smem_desc_sw128(sb + kS1Qg + koff, 16, 1024), bdesc, id, kk > 0);
+      }
+      mma_commit(bar);
+    }
+    alive = __syncthreads_and(mbar_wait(bar, 0)) != 0;
+    tc_fence_after();
+    const int sp = warp & 3, half = warp >> 2;
+    const int r = sp * 16 + (lane & 15);
+    float va[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      tmem_ld32(tmem_at(tmem, sp * 32, half * 64 + part * 32), va);
+      tmem_ld_wait();
+      if (lane < 16) {
+        if (half == 0) {
+          const float br = sBeta[r];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int i = part * 32 + j;
+            sA[r * kLdA + i] = (i < r) ? br * va[j] : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int i = part * 32 + c8 * 8 + j;
+              f[j] = (i <= r) ? va[c8 * 8 + j] : 0.f;
+            }
+            *reinterpret_cast<uint4*>(rec + kRecAqk + tile_chunk_off(r, part * 4 + c8, 8192)) =
+                pack8(f);
+          }
+        }
+      }
+    }
+  } else {
+    // exact fallback: one warp per (r, i) pair, ratios exp(g_r - g_i) <= 1, fp32
+    __threadfence_block();
+    for (int p = warp; p < kC * (kC + 1) / 2; p += kK1Threads / 32) {
+      int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+      while ((r + 1) * (r + 2) / 2 <= p) ++r;
+      while (r * (r + 1) / 2 > p) --r;
+      const int i = p - r * (r + 1) / 2;
+      float akk = 0.f, aqk = 0.f;
+      if (r < L) {
+        const float* gr = reinterpret_cast<const float*>(rec + (r < 32 ? kRecW + r * 512 : kRecU + (r - 32) * 512));
+        const float* gi = reinterpret_cast<const float*>(rec + (i < 32 ? kRecW + i * 512 : kRecU + (i - 32) * 512));
+        const size_t rowr = (size_t)(t0 + r) * H + h, rowi = (size_t)(t0 + i) * H + h;
+        for (int cc = lane; cc < kD; cc += 32) {
+          const float f = __expf(gr[cc] - gi[cc]);
+          const float kk = __bfloat162float(k[rowi * kD + cc]) * f;
+          akk += __bfloat162float(k[rowr * kD + cc]) * kk;
+          aqk += __bfloat162float(q[rowr * kD + cc]) * kk;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        akk += __shfl_xor_sync(0xffffffffu, akk, off);
+        aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
+      }
+      if (lane == 0) {
+        sA[r * kLdA + i] = (i < r) ? sBeta[r] * akk : 0.f;
+        reinterpret_cast<__nv_bfloat16*>(rec + kRecAqk + tile_off(r, i, 8192))[0] =
+            __float2bfloat16_rn(aqk);
+      }
+    }
+    for (int idx = tid; idx < kC * kC; idx += kK1Threads) {
+      const int r = idx >> 6, i = idx & 63;
+      if (i > r) {
+        sA[r * kLdA + i] = 0.f;
+        reinterpret_cast<__nv_bfloat16*>(rec + kRecAqk + tile_off(r, i, 8192))[0] =
+            __float2bfloat16_rn(0.f);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- phase 4: T = (I + A)^{-1}, 16 x 16 blocks --------------------------------------------
+  for (int idx = tid; idx < kC * kLdA; idx += kK1Threads) sT[idx] = 0.f;
+  __syncthreads();
+  if (warp < 4 && lane < 16) {  // diagonal blocks: lane = column of T_bb
+    const int b = warp, cidx = lane;
+    float col[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float val = (i == cidx) ? 1.f : 0.f;
+#pragma unroll
+      for (int j = 0; j < i; ++j)
+        if (j >= cidx) val -= sA[(16 * b + i) * kLdA + 16 * b + j] * col[j];
+      col[i] = (i >= cidx) ? val : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sT[(16 * b + i) * kLdA + 16 * b + cidx] = col[i];
+  }
+  __syncthreads();
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;  // blocks (R, R-d), R = d..3
+    // X_R = sum_{J=R-d}^{R-1} A_RJ T_J,R-d
+    for (int e = tid; e < nb * 256; e += kK1Threads) {
+      const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      const int R = d + bi, I = R - d;
+      float acc = 0.f;
+      for (int J = I; J < R; ++J)
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          acc += sA[(16 * R + rr) * kLdA + 16 * J + m] * sT[(16 * J + m) * kLdA + 16 * I + cc];
+      sX[bi * 272 + rr * 17 + cc] = acc;
+    }
+    __syncthreads();
+    // T_R,R-d = -T_RR X_R
+    for (int e = tid; e < nb * 256; e += kK1Threads) {
+      const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+      const int R = d + bi, I = R - d;
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        acc += sT[(16 * R + rr) * kLdA + 16 * R + m] * sX[bi * 272 + m * 17 + cc];
+      sT[(16 * R + rr) * kLdA + 16 * I + cc] = -acc;
+    }
+    __syncthreads();
+  }
+  // M = T Diag(beta) -> bf16 operand tile
+  for (int e = tid; e < kC * 8; e += kK1Threads) {
+    const int r = e >> 3, c8 = e & 7;
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = c8 * 8 + j;
+      f[j] = (i <= r) ? sT[r * kLdA + i] * sBeta[i] : 0.f;
+    }
+    st_shared_v4(sb + kS1M + tile_chunk_off(r, c8, 8192), pack8(f));
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---- phase 5: W = M Kg (cols 0..127), U = M V (cols 128..255) -----------------------------
+  if (alive) {
+    if (tid == 0) {
+      const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t adesc = smem_desc_sw128(sb + kS1M + kk * 32, 16, 1024);
+        mma_bf16(tmem + 0, adesc, smem_desc_sw128(sb + kS1Kg + kk * 2048, 8192, 1024), id, kk > 0);
+        mma_bf16(tmem + 128, adesc, smem_desc_sw128(sb + kS1V + kk * 2048, 8192, 1024), id,
+                 kk > 0);
+      }
+      mma_commit(bar);
+    }
+    alive = __syncthreads_and(mbar_wait(bar, fast ? 1 : 0)) != 0;
+    tc_fence_after();
+    const int sp = warp & 3, half = warp >> 2;
+    const int r = sp * 16 + (lane & 15);
+    uint8_t* dst = rec + (half == 0 ? kRecW : kRecU);
+    float va[32];
+#pragma unroll
+    for (int part = 0; part < 4; ++part) {
+      tmem_ld32(tmem_at(tmem, sp * 32, half * 128 + part * 32), va);
+      tmem_ld_wait();
+      if (lane < 16 && alive) {
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float f[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = va[c8 * 8 + j];
+          *reinterpret_cast<uint4*>(dst + tile_chunk_off(r, part * 4 + c8, 8192)) = pack8(f);
+        }
+      }
+    }
+  }
+  if (tid < kD) reinterpret_cast<float*>(rec + kRecGam)[tid] = expf(sGC[tid]);
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ============================================================================================
+// K2
+// ============================================================================================
+constexpr int kK2Threads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 epilogue
+constexpr uint32_t kStW = 0, kStQt = 16384, kStKt = 32768, kStAqk = 49152, kStU = 57344,
+                   kStGam = 65536;
+constexpr uint32_t kStageBytes = 66560;  // 65 KiB (keeps every stage 1024-aligned)
+constexpr uint32_t kStageTx = 16384 * 3 + 8192 + 8192 + 512;
+constexpr uint32_t kS2Stage0 = 0;
+constexpr uint32_t kS2S = 2 * kStageBytes;         // [128 x 64] bf16 state tile
+constexpr uint32_t kS2Vp = kS2S + 16384;           // [64 x 64] bf16 pseudo-value tile
+constexpr uint32_t kS2Bar = kS2Vp + 8192;          // 8 mbarriers
+constexpr uint32_t kS2Tmem = kS2Bar + 64;
+constexpr uint32_t kS2Flags = kS2Tmem + 4;
+constexpr uint32_t kS2Bytes = kS2Flags + 12;
+// TMEM columns: D1 [0,64), D3 [64,128), D2 double buffer [128,192) / [192,256)
+constexpr uint32_t kTmD1 = 0, kTmD3 = 64, kTmD2 = 128;
+
+__global__ void __launch_bounds__(kK2Threads, 1)
+    chunk_state_tc_kernel(const uint8_t* __restrict__ ws_records, SeqGeometry geo, int H,
+                          const float* __restrict__ initial_state, float* __restrict__ final_state,
+                          __nv_bfloat16* __restrict__ o) {
+  extern __shared__ uint8_t smem_raw[];
+  if (!geo.ok()) return;
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sb = smem_u32(sm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kS2Bar);
+  uint64_t* full = bars + 0;   // [2]
+  uint64_t* empty = bars + 2;  // [2]
+  uint64_t* d12 = bars + 4;
+  uint64_t* d3 = bars + 5;
+  uint64_t* vp_ready = bars + 6;
+  uint64_t* s_ready = bars + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS2Tmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kS2Flags);
+
+  const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * 64;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
+  const int nchunks = te > tb ? ceil_div(te - tb, kC) : 0;
+  const int c_first = geo.first_chunk(n);
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    mbar_init(d12, 1);
+    mbar_init(d3, 1);
+    mbar_init(vp_ready, 128);
+    mbar_init(s_ready, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int ci = 0; ci < nchunks; ++ci) {
+        const int st = ci & 1;
+        if (ci >= 2 && !mbar_wait(empty + st, ((ci >> 1) - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
+        uint8_t* stage = sm + kS2Stage0 + st * kStageBytes;
+        mbar_arrive_expect_tx(full + st, kStageTx);
+        bulk_g2s(stage + kStW, rec + kRecW, 16384, full + st);
+        bulk_g2s(stage + kStQt, rec + kRecQt, 16384, full + st);
+        bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
+        bulk_g2s(stage + kStAqk, rec + kRecAqk, 8192, full + st);
+        bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
+        bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
+      }
+      // drain: the last copies must land before the CTA may exit
+      const int issued = nchunks;
+      for (int ci = issued > 2 ? issued - 2 : 0; ci < issued; ++ci)
+        mbar_wait(full + (ci & 1), (ci >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_64 = idesc_bf16_f32(64, 64, 0, 1);     // K-major A, MN-major B
+      const uint32_t id_128 = idesc_bf16_f32(128, 64, 1, 1);   // MN-major A and B
+      for (int ci = 0; ci < nchunks; ++ci) {
+        const int st = ci & 1;
+        const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
+        if (!mbar_wait(full + st, (ci >> 1) & 1) || !mbar_wait(s_ready, ci & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d2 = tmem + kTmD2 + (ci & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+          const uint64_t bdesc = smem_desc_sw128(sb + kS2S + kk * 2048, 8192, 1024);
+          mma_bf16(tmem + kTmD1, smem_desc_sw128(stage + kStW + koff, 16, 1024), bdesc, id_64,
+                   kk > 0);
+          mma_bf16(d2, smem_desc_sw128(stage + kStQt + koff, 16, 1024), bdesc, id_64, kk > 0);
+        }
+        mma_commit(d12);
+        if (!mbar_wait(vp_ready, ci & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024);
+          mma_bf16(tmem + kTmD3, smem_desc_sw128(stage + kStKt + kk * 2048, 8192, 1024), bdesc,
+                   id_128, kk > 0);
+          mma_bf16(d2, smem_desc_sw128(stage + kStAqk + kk * 32, 16, 1024), bdesc, id_64, true);
+        }
+        mma_commit(d3);
+        mma_commit(empty + st);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (4 warps)
+    const int sp = warp & 3;
+    const int crow = sp * 32 + lane;       // state row (key channel) owned by this thread
+    const int r = sp * 16 + (lane & 15);   // chunk row of the M = 64 accumulators
+    const bool rowlane = lane < 16;
+    float S[64];
+    const size_t sbase = (((size_t)n * H + h) * kD + crow) * kD + j0;
+    if (initial_state) {
+      const float4* src = reinterpret_cast<const float4*>(initial_state + sbase);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 x = src[j];
+        S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) S[j] = 0.f;
+    }
+    auto write_state_tile = [&]() {
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = S[c8 * 8 + j];
+        st_shared_v4(sb + kS2S + tile_chunk_off(crow, c8, 16384), pack8(f));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(s_ready);
+    };
+    write_state_tile();
+
+    float va[32], vb[32];
+    for (int ci = 0; ci < nchunks; ++ci) {
+      const int st = ci & 1;
+      const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
+      const int t0 = tb + ci * kC;
+      const int L = min(kC, te - t0);
+      // the staged U and gamma_C are read below: wait for their copy, then for W S / Qt S
+      bool ok = !*abort_flag && mbar_wait(full + st, (ci >> 1) & 1) && mbar_wait(d12, ci & 1);
+      if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform exit: tcgen05.ld is warp-collective
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[crow];
+      // V' = U - W S  (rows r of the M = 64 accumulator live in lanes 0..15)
+      tmem_ld32(tmem_at(tmem, sp * 32, kTmD1), va);
+      tmem_ld32(tmem_at(tmem, sp * 32, kTmD1 + 32), vb);
+      tmem_ld_wait();
+      if (rowlane) {
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint32_t off = tile_chunk_off(r, c8, 8192);
+          float u[8], f[8];
+          unpack8(ld_shared_v4(stage + kStU + off), u);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int col = c8 * 8 + j;
+            f[j] = u[j] - (col < 32 ? va[col] : vb[col - 32]);
+          }
+          st_shared_v4(sb + kS2Vp + off, pack8(f));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(vp_ready);
+      // S = Diag(gamma_C) S + Kt^T V'
+      ok = mbar_wait(d3, ci & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      tmem_ld32(tmem_at(tmem, sp * 32, kTmD3), va);
+      tmem_ld32(tmem_at(tmem, sp * 32, kTmD3 + 32), vb);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        S[j] = fmaf(gam, S[j], va[j]);
+        S[32 + j] = fmaf(gam, S[32 + j], vb[j]);
+      }
+      // O = Qt S + A_qk V' (read before this thread lets the next chunk's MMAs start)
+      const uint32_t d2 = kTmD2 + (ci & 1) * 64;
+      tmem_ld32(tmem_at(tmem, sp * 32, d2), va);
+      tmem_ld32(tmem_at(tmem, sp * 32, d2 + 32), vb);
+      tmem_ld_wait();
+      write_state_tile();
+      if (rowlane && r < L) {
+        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0);
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float f[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int col = c8 * 8 + j;
+            f[j] = col < 32 ? va[col] : vb[col - 32];
+          }
+          dst[c8] = pack8(f);
+        }
+      }
+    }
+    if (final_state && !*abort_flag) {
+      float4* dst = reinterpret_cast<float4*>(final_state + sbase);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace tc
+
+size_t tc_local_smem_bytes() { return tc::kS1Bytes + 1024; }
+size_t tc_state_smem_bytes() { return tc::kS2Bytes + 1024; }
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
+                              uint8_t* records, cudaStream_t stream) {
+  const int sm1 = (int)tc_local_smem_bytes(), sm2 = (int)tc_state_smem_bytes();
+  cudaError_t err = cudaFuncSetAttribute(tc::chunk_local_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(tc::chunk_state_tc_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
+  if (err != cudaSuccess) return err;
+  if (max_chunks > 0) {
+    ProfileScope prof("chunk_local_tc", stream);
+    tc::chunk_local_tc_kernel<<<dim3(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
+        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
+        a.log_alpha, a.beta, geo, a.H, records);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  ProfileScope prof("chunk_state_tc", stream);
+  tc::chunk_state_tc_kernel<<<dim3(a.N, a.H, 2), tc::kK2Threads, sm2, stream>>>(
+      records, geo, a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

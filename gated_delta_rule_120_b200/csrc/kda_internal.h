@@ -67,6 +67,14 @@ struct SimtRecord {
   }
 };
 
+// bytes of one (chunk, head) record of the bf16 tensor-core path (d = 128, C = 64)
+constexpr size_t TcRecordBytes = 74240;
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
+                              uint8_t* records, cudaStream_t stream);
+size_t tc_local_smem_bytes();
+size_t tc_state_smem_bytes();
+
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                const float* log_alpha, const float* beta, float* state, void* o,
                                int N, int H, int Dk, int Dv, cudaStream_t stream);

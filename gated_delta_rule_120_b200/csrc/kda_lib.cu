@@ -5,4 +5,5 @@
 #include "kda_profile.cu"
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
+#include "kda_chunk_tc.cu"
 #include "kda_noalloc.cu"

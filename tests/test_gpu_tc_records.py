@@ -1,0 +1,91 @@
+"""The bf16 tensor-core path's per-chunk records, decoded from the workspace and checked against the
+chunk formulas of "Kimi Linear: An Expressive, Efficient Attention Architecture" (paper-graph-ui
+walkthrough, §3.4 "Chunkwise Parallelization") evaluated here in fp64 from the same inputs.
+
+This localises a failure of the end-to-end parity tests to the chunk-local kernel (records wrong)
+or to the state kernel (records right, outputs wrong). Record layout per (chunk, head), bf16
+tiles in the 128-byte-swizzled operand layout: W, Qt, Kt [64 x 128], A_qk [64 x 64], U [64 x 128],
+then gamma_C as 128 fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_120_b200 as kda
+import kda_synth
+from kda_synth import PrefillSpec
+from tests._parity import to_np
+
+pytestmark = pytest.mark.gpu
+
+REC = dict(W=0, Qt=16384, Kt=32768, Aqk=49152, U=57344, gam=73728, size=74240)
+
+
+def tile_index(rows, cols):
+    """Element offsets (in bf16 units) of a [rows x cols] tile in the swizzled operand layout."""
+    r = np.arange(rows)[:, None]
+    c = np.arange(cols)[None, :]
+    block = rows * 128
+    off = (c // 64) * block + (r // 8) * 1024 + (r % 8) * 128 + (((c % 64) // 8) ^ (r % 8)) * 16 \
+        + (c % 8) * 2
+    return off // 2
+
+
+def decode_tile(buf_u8: np.ndarray, base: int, rows: int, cols: int) -> np.ndarray:
+    bf = buf_u8[base:base + rows * cols * 2].view(np.uint16).astype(np.uint32) << 16
+    vals = bf.view(np.float32)
+    return vals[tile_index(rows, cols)].astype(np.float64)
+
+
+def chunk_reference(k, q, v, la, beta, L):
+    """fp64 W, Qt, Kt, A_qk, U, gamma_C of one chunk (rows >= L are identity padding)."""
+    C = 64
+    K = np.zeros((C, 128)); Q = np.zeros((C, 128)); V = np.zeros((C, 128))
+    G = np.zeros((C, 128)); b = np.zeros(C)
+    K[:L], Q[:L], V[:L], G[:L], b[:L] = k, q, v, la, beta
+    g = np.cumsum(G, axis=0)
+    ratio = np.exp(g[:, None, :] - g[None, :, :])  # [r, i, c] = gamma_r / gamma_i
+    akk = np.einsum("rc,ic,ric->ri", K, K, np.where(np.arange(C)[:, None, None] >=
+                                                    np.arange(C)[None, :, None], ratio, 0.0))
+    aqk = np.einsum("rc,ic,ric->ri", Q, K, np.where(np.arange(C)[:, None, None] >=
+                                                    np.arange(C)[None, :, None], ratio, 0.0))
+    A = np.tril(b[:, None] * akk, -1)
+    M = np.linalg.inv(np.eye(C) + A) * b[None, :]
+    W = M @ (np.exp(g) * K)
+    U = M @ V
+    return dict(W=W, Qt=np.exp(g) * Q, Kt=np.exp(g[-1] - g) * K, Aqk=np.tril(aqk), U=U,
+                gam=np.exp(g[-1]))
+
+
+@pytest.mark.parametrize("T", [64, 150])
+def test_chunk_records_match_formulas(cuda_device, T):
+    spec = PrefillSpec("t", B=1, T=T, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16", decay="fast",
+                       init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 500 + T, cuda_device)
+    nbytes = kda.kda_chunk_fwd_workspace_size(1, T, 2, 128, 128, 64, 1, torch.bfloat16)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda_device)
+    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                      initial_state=inp["initial_state"], chunk=64, workspace=ws)
+    torch.cuda.synchronize()
+    assert kda.kda_last_device_error() == kda.KDA_OK
+    buf = ws.cpu().numpy()
+    x = {n: to_np(inp[n][0]) for n in ("q", "k", "v", "log_alpha", "beta")}
+    nchunks = (T + 63) // 64
+    for c in range(nchunks):
+        t0 = 64 * c
+        L = min(64, T - t0)
+        for h in range(2):
+            ref = chunk_reference(x["k"][t0:t0 + L, h], x["q"][t0:t0 + L, h],
+                                  x["v"][t0:t0 + L, h], x["log_alpha"][t0:t0 + L, h],
+                                  x["beta"][t0:t0 + L, h], L)
+            base = 256 + REC["size"] * (c * 2 + h)
+            got = dict(W=decode_tile(buf, base + REC["W"], 64, 128),
+                       Qt=decode_tile(buf, base + REC["Qt"], 64, 128),
+                       Kt=decode_tile(buf, base + REC["Kt"], 64, 128),
+                       Aqk=decode_tile(buf, base + REC["Aqk"], 64, 64),
+                       U=decode_tile(buf, base + REC["U"], 64, 128),
+                       gam=buf[base + REC["gam"]:base + REC["gam"] + 512].view(np.float32))
+            for name in ("Qt", "Kt", "Aqk", "W", "U", "gam"):
+                r, gval = ref[name], np.asarray(got[name], dtype=np.float64)
+                err = np.abs(gval - r).max() / max(np.abs(r).max(), 1e-30)
+                assert err <= 2e-2, f"chunk {c} head {h} {name}: rel err {err:.3e}"

@@ -62,8 +62,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(cuda_device):
 
 
 def test_noalloc_refuses_calls_beyond_its_scratch(cuda_device):
-    # 114 chunks x 4 heads of fp32 records need more than the 64 MiB array: refused on the host
-    spec = PrefillSpec("big", B=1, T=64 * 114, H=4, Dk=128, Dv=128, chunk=64, dtype="bf16",
+    # 256 chunks x 4 heads of records need more than the 64 MiB array: refused on the host
+    spec = PrefillSpec("big", B=1, T=64 * 256, H=4, Dk=128, Dv=128, chunk=64, dtype="bf16",
                        decay="fast", init_std=0.0)
     need = kda.kda_chunk_fwd_workspace_size(spec.B, spec.T, spec.H, 128, 128, 64, 1,
                                             torch.bfloat16)

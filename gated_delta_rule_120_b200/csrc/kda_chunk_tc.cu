@@ -48,22 +48,30 @@ static_assert(kRecBytes == TcRecordBytes, "record size mismatch");
 // K1
 // ============================================================================================
 constexpr int kK1Threads = 256;
+constexpr int kK1Tmem = 128;  // A_kk | A_qk, then W, then U
 
-// shared-memory map of K1 (offsets from a 1024-aligned base)
-constexpr uint32_t kS1Kg = 0;          // [64 x 128] bf16 tile
-constexpr uint32_t kS1Ki = 16384;      // [64 x 128]
-constexpr uint32_t kS1Qg = 32768;      // [64 x 128]
-constexpr uint32_t kS1V = 49152;       // [64 x 128]
-constexpr uint32_t kS1M = 65536;       // [64 x 64]
-constexpr uint32_t kS1A = 73728;       // fp32 [64][65] (the scan partials alias it)
-constexpr uint32_t kS1T = 90368;       // fp32 [64][65]
-constexpr uint32_t kS1X = 107008;      // fp32 [3][16][17] level products
-constexpr uint32_t kS1Beta = 110272;   // fp32 [64]
-constexpr uint32_t kS1GC = 110528;     // fp32 [128]
-constexpr uint32_t kS1Bar = 111040;    // mbarrier
-constexpr uint32_t kS1Tmem = 111048;   // TMEM base address
-constexpr uint32_t kS1Bytes = 111056;
-constexpr int kLdA = 65;  // padded row stride of the fp32 A / T matrices
+// shared-memory map of K1 (offsets from a 1024-aligned base). Three CTAs fit on an SM.
+constexpr uint32_t kS1Kg = 0;         // [64 x 128] bf16: raw k, then Gamma.K
+constexpr uint32_t kS1Ki = 16384;     // [64 x 128] bf16: scan partials, then K/Gamma, then fp32 A
+constexpr uint32_t kS1Qg = 32768;     // [64 x 128] bf16: raw q, then Gamma.Q, then fp32 T
+constexpr uint32_t kS1V = 49152;      // [64 x 128] bf16 v
+constexpr uint32_t kS1M = 65536;      // [64 x 64] bf16 M (the level products X alias it first)
+constexpr uint32_t kS1Beta = 73728;   // fp32 [64]
+constexpr uint32_t kS1GC = 73984;     // fp32 [128]
+constexpr uint32_t kS1Bar = 74496;    // mbarrier
+constexpr uint32_t kS1Tmem = 74504;   // TMEM base address
+constexpr uint32_t kS1Bytes = 74512;
+
+// fp32 64 x 64 matrices (A, T) are stored row-major with column bits 2..5 XOR-ed by (row % 16):
+// groups of four consecutive columns stay contiguous (128-bit accesses) while sixteen consecutive
+// rows of one column group spread over the banks.
+__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + (c ^ ((r & 15) << 2)); }
+__device__ __forceinline__ float4 lds4(const float* base, int r, int c4) {  // cols 4*c4 .. +3
+  return *reinterpret_cast<const float4*>(base + sidx(r, 4 * c4));
+}
+__device__ __forceinline__ void sts4(float* base, int r, int c4, float4 v) {
+  *reinterpret_cast<float4*>(base + sidx(r, 4 * c4)) = v;
+}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
@@ -74,8 +82,15 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
+               : "r"(addr)
+               : "memory");
   return v;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
@@ -87,7 +102,31 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
                     pack_bf16(f[6], f[7]));
 }
 
-__global__ void __launch_bounds__(kK1Threads, 2)
+// TMEM [0, 128) of an M = 64 accumulator -> bf16 record tile rows (lanes 0..15 of each warp of
+// warps 0..3 own rows 16*warp + lane; warps 4..7 take the upper 64 columns).
+__device__ __forceinline__ void readout_rows_bf16(uint32_t tmem, int warp, int lane,
+                                                  uint8_t* dst_tile) {
+  const int sp = warp & 3, half = warp >> 2;
+  const int r = sp * 16 + (lane & 15);
+  float va[32];
+#pragma unroll
+  for (int part = 0; part < 2; ++part) {
+    const int col0 = half * 64 + part * 32;
+    tmem_ld32(tmem_at(tmem, sp * 32, col0), va);
+    tmem_ld_wait();
+    if (lane < 16) {
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = va[c8 * 8 + j];
+        *reinterpret_cast<uint4*>(dst_tile + tile_chunk_off(r, (col0 >> 3) + c8, 8192)) = pack8(f);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kK1Threads, 3)
     chunk_local_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                           const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
                           const float* __restrict__ beta, SeqGeometry geo, int H,
@@ -99,12 +138,12 @@ __global__ void __launch_bounds__(kK1Threads, 2)
 
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(sm);
-  float* sA = reinterpret_cast<float*>(sm + kS1A);
-  float* sT = reinterpret_cast<float*>(sm + kS1T);
-  float* sX = reinterpret_cast<float*>(sm + kS1X);
+  float* sA = reinterpret_cast<float*>(sm + kS1Ki);
+  float* sT = reinterpret_cast<float*>(sm + kS1Qg);
+  float* sX = reinterpret_cast<float*>(sm + kS1M);
   float* sBeta = reinterpret_cast<float*>(sm + kS1Beta);
   float* sGC = reinterpret_cast<float*>(sm + kS1GC);
-  float* sScan = sA;  // [16][128], used before A exists
+  float* sScan = reinterpret_cast<float*>(sm + kS1Ki);  // [16][128], before K/Gamma exists
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kS1Bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS1Tmem);
 
@@ -115,7 +154,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
   uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)c * H + h);
 
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kK1Tmem);
     tmem_relinquish();
     tc_fence_before();
   }
@@ -124,27 +163,27 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     fence_mbar_init();
   }
 
-  // ---- phase 1: loads (thread = 8 channels x 4 rows) and the cumulative decay ----------------
-  const int cg = tid & 15, rg = tid >> 4;
-  uint4 kr[4], qr[4], vr[4];
+  // ---- phase 1: raw k, q, v straight into their operand tiles; log decay into registers ------
+  const int cg = tid & 15, rg = tid >> 4;  // thread = 8 channels (one 16-byte chunk) x 4 rows
   float g[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = rg * 4 + i;
+    const uint32_t off = tile_chunk_off(r, cg, 8192);
     if (r < L) {
       const size_t row = (size_t)(t0 + r) * H + h;
-      const uint4* kp = reinterpret_cast<const uint4*>(k + row * kD) + cg;
-      const uint4* qp = reinterpret_cast<const uint4*>(q + row * kD) + cg;
-      const uint4* vp = reinterpret_cast<const uint4*>(v + row * kD) + cg;
+      cp_async16(sb + kS1Kg + off, reinterpret_cast<const uint4*>(k + row * kD) + cg);
+      cp_async16(sb + kS1Qg + off, reinterpret_cast<const uint4*>(q + row * kD) + cg);
+      cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
       const float4* lp = reinterpret_cast<const float4*>(log_alpha + row * kD) + 2 * cg;
-      kr[i] = __ldg(kp);
-      qr[i] = __ldg(qp);
-      vr[i] = __ldg(vp);
       const float4 a0 = __ldg(lp), a1 = __ldg(lp + 1);
       g[i][0] = a0.x; g[i][1] = a0.y; g[i][2] = a0.z; g[i][3] = a0.w;
       g[i][4] = a1.x; g[i][5] = a1.y; g[i][6] = a1.z; g[i][7] = a1.w;
-    } else {
-      kr[i] = qr[i] = vr[i] = make_uint4(0, 0, 0, 0);
+    } else {  // identity padding: log alpha = 0, k = q = v = 0
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      st_shared_v4(sb + kS1Kg + off, z);
+      st_shared_v4(sb + kS1Qg + off, z);
+      st_shared_v4(sb + kS1V + off, z);
 #pragma unroll
       for (int j = 0; j < 8; ++j) g[i][j] = 0.f;
     }
@@ -172,55 +211,47 @@ __global__ void __launch_bounds__(kK1Threads, 2)
   if (rg == 15)
 #pragma unroll
     for (int j = 0; j < 8; ++j) sGC[cg * 8 + j] = g[3][j];
+  cp_async_wait_all();
   __syncthreads();
-  float gc[8];
+  float egc[8];
   bool ok = true;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    gc[j] = sGC[cg * 8 + j];
-    ok = ok && (gc[j] >= -kFastDecayLimit);
+    const float gcj = sGC[cg * 8 + j];
+    ok = ok && (gcj >= -kFastDecayLimit);
+    egc[j] = expf(gcj);
   }
   const bool fast = __syncthreads_and(ok) != 0;
 
-  // ---- phase 2: scaled operand tiles (smem) and the Qt / Kt record tiles (global) ------------
-  {
-    float egc[8];
+  // ---- phase 2: scale in place (each thread rewrites only the chunks it staged) --------------
 #pragma unroll
-    for (int j = 0; j < 8; ++j) egc[j] = expf(gc[j]);
+  for (int i = 0; i < 4; ++i) {
+    const int r = rg * 4 + i;
+    const uint32_t off = tile_chunk_off(r, cg, 8192);
+    float kf[8], qf[8];
+    unpack8(ld_shared_v4(sb + kS1Kg + off), kf);
+    unpack8(ld_shared_v4(sb + kS1Qg + off), qf);
+    float kg[8], ki[8], kt[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rg * 4 + i;
-      float kf[8], qf[8], kg[8], ki[8], qg[8], kt[8];
-      unpack8(kr[i], kf);
-      unpack8(qr[i], qf);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float e = __expf(g[i][j]);
-        kg[j] = kf[j] * e;
-        qg[j] = qf[j] * e;
-        if (fast) {
-          ki[j] = kf[j] * __expf(-g[i][j]);
-          kt[j] = ki[j] * egc[j];
-        } else {
-          ki[j] = 0.f;
-          kt[j] = kf[j] * __expf(gc[j] - g[i][j]);
-        }
+    for (int j = 0; j < 8; ++j) {
+      const float e = __expf(g[i][j]);
+      kg[j] = kf[j] * e;
+      qf[j] *= e;
+      if (fast) {
+        ki[j] = kf[j] * __expf(-g[i][j]);
+        kt[j] = ki[j] * egc[j];
+      } else {
+        ki[j] = 0.f;
+        kt[j] = kf[j] * __expf(sGC[cg * 8 + j] - g[i][j]);
       }
-      const uint32_t off = tile_chunk_off(r, cg, 8192);
-      const uint4 qgv = pack8(qg), ktv = pack8(kt);
-      st_shared_v4(sb + kS1Kg + off, pack8(kg));
-      st_shared_v4(sb + kS1Ki + off, pack8(ki));
-      st_shared_v4(sb + kS1Qg + off, qgv);
-      st_shared_v4(sb + kS1V + off, vr[i]);
-      *reinterpret_cast<uint4*>(rec + kRecQt + off) = qgv;
-      *reinterpret_cast<uint4*>(rec + kRecKt + off) = ktv;
     }
-  }
-  if (!fast) {
-    // exact fallback: keep the cumulative decay in this record's W/U area (overwritten later)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rg * 4 + i;
+    const uint4 qgv = pack8(qf);
+    st_shared_v4(sb + kS1Kg + off, pack8(kg));
+    st_shared_v4(sb + kS1Ki + off, pack8(ki));
+    st_shared_v4(sb + kS1Qg + off, qgv);
+    *reinterpret_cast<uint4*>(rec + kRecQt + off) = qgv;
+    *reinterpret_cast<uint4*>(rec + kRecKt + off) = pack8(kt);
+    if (!fast) {  // exact fallback keeps the cumulative decay in this record's W/U area
       float* gp = reinterpret_cast<float*>(rec + (r < 32 ? kRecW + r * 512 : kRecU + (r - 32) * 512));
 #pragma unroll
       for (int j = 0; j < 8; ++j) gp[cg * 8 + j] = g[i][j];
@@ -247,6 +278,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     }
     alive = __syncthreads_and(mbar_wait(bar, 0)) != 0;
     tc_fence_after();
+    // K/Gamma and Gamma.Q are dead from here: A (fp32) takes the K/Gamma area
     const int sp = warp & 3, half = warp >> 2;
     const int r = sp * 16 + (lane & 15);
     float va[32];
@@ -258,9 +290,12 @@ __global__ void __launch_bounds__(kK1Threads, 2)
         if (half == 0) {
           const float br = sBeta[r];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int i = part * 32 + j;
-            sA[r * kLdA + i] = (i < r) ? br * va[j] : 0.f;
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const int i = part * 32 + j4 * 4;
+            sts4(sA, r, i >> 2,
+                 make_float4(i < r ? br * va[4 * j4] : 0.f, i + 1 < r ? br * va[4 * j4 + 1] : 0.f,
+                             i + 2 < r ? br * va[4 * j4 + 2] : 0.f,
+                             i + 3 < r ? br * va[4 * j4 + 3] : 0.f));
           }
         } else {
 #pragma unroll
@@ -279,7 +314,6 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     }
   } else {
     // exact fallback: one warp per (r, i) pair, ratios exp(g_r - g_i) <= 1, fp32
-    __threadfence_block();
     for (int p = warp; p < kC * (kC + 1) / 2; p += kK1Threads / 32) {
       int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
       while ((r + 1) * (r + 2) / 2 <= p) ++r;
@@ -303,7 +337,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
         aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
       }
       if (lane == 0) {
-        sA[r * kLdA + i] = (i < r) ? sBeta[r] * akk : 0.f;
+        sA[sidx(r, i)] = (i < r) ? sBeta[r] * akk : 0.f;
         reinterpret_cast<__nv_bfloat16*>(rec + kRecAqk + tile_off(r, i, 8192))[0] =
             __float2bfloat16_rn(aqk);
       }
@@ -311,7 +345,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     for (int idx = tid; idx < kC * kC; idx += kK1Threads) {
       const int r = idx >> 6, i = idx & 63;
       if (i > r) {
-        sA[r * kLdA + i] = 0.f;
+        sA[sidx(r, i)] = 0.f;
         reinterpret_cast<__nv_bfloat16*>(rec + kRecAqk + tile_off(r, i, 8192))[0] =
             __float2bfloat16_rn(0.f);
       }
@@ -320,98 +354,105 @@ __global__ void __launch_bounds__(kK1Threads, 2)
   tc_fence_before();
   __syncthreads();
 
-  // ---- phase 4: T = (I + A)^{-1}, 16 x 16 blocks --------------------------------------------
-  for (int idx = tid; idx < kC * kLdA; idx += kK1Threads) sT[idx] = 0.f;
-  __syncthreads();
-  if (warp < 4 && lane < 16) {  // diagonal blocks: lane = column of T_bb
+  // ---- phase 4: T = (I + A)^{-1} in fp32 (16 x 16 blocks), T in the Gamma.Q area ------------
+  // Only the lower triangle of T is ever read (the M build masks the rest), so T is not cleared.
+  if (warp < 4 && lane < 16) {  // diagonal blocks by forward substitution: lane = column of T_bb
     const int b = warp, cidx = lane;
-    float col[16];
+    float col[16];  // col[i] = T_bb[i][cidx]; entries above the diagonal come out as 0
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float val = (i == cidx) ? 1.f : 0.f;
 #pragma unroll
-      for (int j = 0; j < i; ++j)
-        if (j >= cidx) val -= sA[(16 * b + i) * kLdA + 16 * b + j] * col[j];
-      col[i] = (i >= cidx) ? val : 0.f;
+      for (int j4 = 0; j4 < 4; ++j4) {
+        if (4 * j4 < i) {
+          const float4 a = lds4(sA, 16 * b + i, 4 * b + j4);
+          if (4 * j4 + 0 < i) val -= a.x * col[4 * j4 + 0];
+          if (4 * j4 + 1 < i) val -= a.y * col[4 * j4 + 1];
+          if (4 * j4 + 2 < i) val -= a.z * col[4 * j4 + 2];
+          if (4 * j4 + 3 < i) val -= a.w * col[4 * j4 + 3];
+        }
+      }
+      col[i] = val;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) sT[(16 * b + i) * kLdA + 16 * b + cidx] = col[i];
+    for (int i = 0; i < 16; ++i) sT[sidx(16 * b + i, 16 * b + cidx)] = col[i];
   }
   __syncthreads();
+  // off-diagonal blocks, one block-diagonal at a time:  T_R,I = -T_RR sum_{J=I}^{R-1} A_RJ T_JI
+  // (d = R - I). A thread owns a 1 x 4 strip (row rr, columns 4cq..4cq+3) of one block.
   for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;  // blocks (R, R-d), R = d..3
-    // X_R = sum_{J=R-d}^{R-1} A_RJ T_J,R-d
-    for (int e = tid; e < nb * 256; e += kK1Threads) {
-      const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      const int R = d + bi, I = R - d;
-      float acc = 0.f;
-      for (int J = I; J < R; ++J)
-#pragma unroll
-        for (int m = 0; m < 16; ++m)
-          acc += sA[(16 * R + rr) * kLdA + 16 * J + m] * sT[(16 * J + m) * kLdA + 16 * I + cc];
-      sX[bi * 272 + rr * 17 + cc] = acc;
+    const int nstrips = (4 - d) * 64;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int bi = 0, rr = 0, cq = 0, R = 0, I = 0;
+    const bool act = tid < nstrips;
+    if (act) {
+      bi = tid >> 6; rr = (tid >> 2) & 15; cq = tid & 3;
+      R = d + bi; I = R - d;
+      for (int k4 = 4 * I; k4 < 4 * R; ++k4) {
+        const float4 a = lds4(sA, 16 * R + rr, k4);
+        const float4 t0 = lds4(sT, 4 * k4 + 0, 4 * I + cq), t1 = lds4(sT, 4 * k4 + 1, 4 * I + cq);
+        const float4 t2 = lds4(sT, 4 * k4 + 2, 4 * I + cq), t3 = lds4(sT, 4 * k4 + 3, 4 * I + cq);
+        acc.x += a.x * t0.x + a.y * t1.x + a.z * t2.x + a.w * t3.x;
+        acc.y += a.x * t0.y + a.y * t1.y + a.z * t2.y + a.w * t3.y;
+        acc.z += a.x * t0.z + a.y * t1.z + a.z * t2.z + a.w * t3.z;
+        acc.w += a.x * t0.w + a.y * t1.w + a.z * t2.w + a.w * t3.w;
+      }
+      *reinterpret_cast<float4*>(sX + bi * 256 + rr * 16 + 4 * cq) = acc;
     }
     __syncthreads();
-    // T_R,R-d = -T_RR X_R
-    for (int e = tid; e < nb * 256; e += kK1Threads) {
-      const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-      const int R = d + bi, I = R - d;
-      float acc = 0.f;
+    if (act) {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int m = 0; m < 16; ++m)
-        acc += sT[(16 * R + rr) * kLdA + 16 * R + m] * sX[bi * 272 + m * 17 + cc];
-      sT[(16 * R + rr) * kLdA + 16 * I + cc] = -acc;
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const float4 a = lds4(sT, 16 * R + rr, 4 * R + m4);
+        const float4* xr = reinterpret_cast<const float4*>(sX + bi * 256 + (4 * m4) * 16 + 4 * cq);
+        const float4 x0 = xr[0], x1 = xr[4], x2 = xr[8], x3 = xr[12];
+        t.x += a.x * x0.x + a.y * x1.x + a.z * x2.x + a.w * x3.x;
+        t.y += a.x * x0.y + a.y * x1.y + a.z * x2.y + a.w * x3.y;
+        t.z += a.x * x0.z + a.y * x1.z + a.z * x2.z + a.w * x3.z;
+        t.w += a.x * x0.w + a.y * x1.w + a.z * x2.w + a.w * x3.w;
+      }
+      sts4(sT, 16 * R + rr, 4 * I + cq, make_float4(-t.x, -t.y, -t.z, -t.w));
     }
     __syncthreads();
   }
-  // M = T Diag(beta) -> bf16 operand tile
+  // M = T Diag(beta) -> bf16 operand tile (the level products are dead)
   for (int e = tid; e < kC * 8; e += kK1Threads) {
     const int r = e >> 3, c8 = e & 7;
-    float f[8];
+    const float4 ta = lds4(sT, r, 2 * c8), tb = lds4(sT, r, 2 * c8 + 1);
+    const float4 ba = *reinterpret_cast<const float4*>(sBeta + 8 * c8);
+    const float4 bb = *reinterpret_cast<const float4*>(sBeta + 8 * c8 + 4);
+    const int i0 = 8 * c8;
+    float f[8] = {ta.x * ba.x, ta.y * ba.y, ta.z * ba.z, ta.w * ba.w,
+                  tb.x * bb.x, tb.y * bb.y, tb.z * bb.z, tb.w * bb.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = c8 * 8 + j;
-      f[j] = (i <= r) ? sT[r * kLdA + i] * sBeta[i] : 0.f;
-    }
+    for (int j = 0; j < 8; ++j) f[j] = (i0 + j <= r) ? f[j] : 0.f;
     st_shared_v4(sb + kS1M + tile_chunk_off(r, c8, 8192), pack8(f));
   }
   fence_proxy_async_smem();
   __syncthreads();
   tc_fence_after();
 
-  // ---- phase 5: W = M Kg (cols 0..127), U = M V (cols 128..255) -----------------------------
-  if (alive) {
+  // ---- phase 5: W = M Kg, then U = M V, through TMEM [0, 128) -------------------------------
+  uint32_t phase = fast ? 1 : 0;
+#pragma unroll 1
+  for (int which = 0; which < 2 && alive; ++which) {
     if (tid == 0) {
       const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
+      const uint32_t src = which == 0 ? kS1Kg : kS1V;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t adesc = smem_desc_sw128(sb + kS1M + kk * 32, 16, 1024);
-        mma_bf16(tmem + 0, adesc, smem_desc_sw128(sb + kS1Kg + kk * 2048, 8192, 1024), id, kk > 0);
-        mma_bf16(tmem + 128, adesc, smem_desc_sw128(sb + kS1V + kk * 2048, 8192, 1024), id,
-                 kk > 0);
-      }
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem, smem_desc_sw128(sb + kS1M + kk * 32, 16, 1024),
+                 smem_desc_sw128(sb + src + kk * 2048, 8192, 1024), id, kk > 0);
       mma_commit(bar);
     }
-    alive = __syncthreads_and(mbar_wait(bar, fast ? 1 : 0)) != 0;
+    alive = __syncthreads_and(mbar_wait(bar, phase)) != 0;
+    phase ^= 1;
     tc_fence_after();
-    const int sp = warp & 3, half = warp >> 2;
-    const int r = sp * 16 + (lane & 15);
-    uint8_t* dst = rec + (half == 0 ? kRecW : kRecU);
-    float va[32];
-#pragma unroll
-    for (int part = 0; part < 4; ++part) {
-      tmem_ld32(tmem_at(tmem, sp * 32, half * 128 + part * 32), va);
-      tmem_ld_wait();
-      if (lane < 16 && alive) {
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          float f[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] = va[c8 * 8 + j];
-          *reinterpret_cast<uint4*>(dst + tile_chunk_off(r, part * 4 + c8, 8192)) = pack8(f);
-        }
-      }
-    }
+    readout_rows_bf16(tmem, warp, lane, rec + (which == 0 ? kRecW : kRecU));
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
   }
   if (tid < kD) reinterpret_cast<float*>(rec + kRecGam)[tid] = expf(sGC[tid]);
 
@@ -419,7 +460,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kK1Tmem);
   }
 }
 
@@ -431,11 +472,12 @@ constexpr uint32_t kStW = 0, kStQt = 16384, kStKt = 32768, kStAqk = 49152, kStU 
                    kStGam = 65536;
 constexpr uint32_t kStageBytes = 66560;  // 65 KiB (keeps every stage 1024-aligned)
 constexpr uint32_t kStageTx = 16384 * 3 + 8192 + 8192 + 512;
+constexpr int kStages = 3;                          // records in flight per CTA
 constexpr uint32_t kS2Stage0 = 0;
-constexpr uint32_t kS2S = 2 * kStageBytes;         // [128 x 64] bf16 state tile
+constexpr uint32_t kS2S = kStages * kStageBytes;   // [128 x 64] bf16 state tile
 constexpr uint32_t kS2Vp = kS2S + 16384;           // [64 x 64] bf16 pseudo-value tile
-constexpr uint32_t kS2Bar = kS2Vp + 8192;          // 8 mbarriers
-constexpr uint32_t kS2Tmem = kS2Bar + 64;
+constexpr uint32_t kS2Bar = kS2Vp + 8192;          // 2 * kStages + 4 mbarriers
+constexpr uint32_t kS2Tmem = kS2Bar + 8 * (2 * kStages + 4);
 constexpr uint32_t kS2Flags = kS2Tmem + 4;
 constexpr uint32_t kS2Bytes = kS2Flags + 12;
 // TMEM columns: D1 [0,64), D3 [64,128), D2 double buffer [128,192) / [192,256)
@@ -450,12 +492,12 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(sm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kS2Bar);
-  uint64_t* full = bars + 0;   // [2]
-  uint64_t* empty = bars + 2;  // [2]
-  uint64_t* d12 = bars + 4;
-  uint64_t* d3 = bars + 5;
-  uint64_t* vp_ready = bars + 6;
-  uint64_t* s_ready = bars + 7;
+  uint64_t* full = bars + 0;         // [kStages]
+  uint64_t* empty = bars + kStages;  // [kStages]
+  uint64_t* d12 = bars + 2 * kStages;
+  uint64_t* d3 = d12 + 1;
+  uint64_t* vp_ready = d12 + 2;
+  uint64_t* s_ready = d12 + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS2Tmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kS2Flags);
 
@@ -470,7 +512,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 2 * kStages; ++i) mbar_init(bars + i, 1);
     mbar_init(d12, 1);
     mbar_init(d3, 1);
     mbar_init(vp_ready, 128);
@@ -487,8 +529,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       for (int ci = 0; ci < nchunks; ++ci) {
-        const int st = ci & 1;
-        if (ci >= 2 && !mbar_wait(empty + st, ((ci >> 1) - 1) & 1)) {
+        const int st = ci % kStages;
+        if (ci >= kStages && !mbar_wait(empty + st, ((ci / kStages) - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -505,8 +547,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
       }
       // drain: the last copies must land before the CTA may exit
       const int issued = nchunks;
-      for (int ci = issued > 2 ? issued - 2 : 0; ci < issued; ++ci)
-        mbar_wait(full + (ci & 1), (ci >> 1) & 1);
+      for (int ci = issued > kStages ? issued - kStages : 0; ci < issued; ++ci)
+        mbar_wait(full + ci % kStages, (ci / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -514,9 +556,9 @@ __global__ void __launch_bounds__(kK2Threads, 1)
       const uint32_t id_64 = idesc_bf16_f32(64, 64, 0, 1);     // K-major A, MN-major B
       const uint32_t id_128 = idesc_bf16_f32(128, 64, 1, 1);   // MN-major A and B
       for (int ci = 0; ci < nchunks; ++ci) {
-        const int st = ci & 1;
+        const int st = ci % kStages;
         const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
-        if (!mbar_wait(full + st, (ci >> 1) & 1) || !mbar_wait(s_ready, ci & 1)) {
+        if (!mbar_wait(full + st, (ci / kStages) & 1) || !mbar_wait(s_ready, ci & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -582,12 +624,12 @@ __global__ void __launch_bounds__(kK2Threads, 1)
 
     float va[32], vb[32];
     for (int ci = 0; ci < nchunks; ++ci) {
-      const int st = ci & 1;
+      const int st = ci % kStages;
       const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
       const int t0 = tb + ci * kC;
       const int L = min(kC, te - t0);
       // the staged U and gamma_C are read below: wait for their copy, then for W S / Qt S
-      bool ok = !*abort_flag && mbar_wait(full + st, (ci >> 1) & 1) && mbar_wait(d12, ci & 1);
+      bool ok = !*abort_flag && mbar_wait(full + st, (ci / kStages) & 1) && mbar_wait(d12, ci & 1);
       if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform exit: tcgen05.ld is warp-collective
         *abort_flag = 1;
         break;

@@ -90,6 +90,22 @@ def test_bf16_small_ragged(cuda_device):
     _check(spec, 41, cuda_device, TOL_BF16_O, TOL_BF16_S)
 
 
+def test_bf16_strong_decay_chunks(cuda_device):
+    """Chunks whose per-channel decay over 64 tokens goes far below exp(-60) take the exact
+    fallback for A_kk / A_qk; the neighbouring ordinary chunks keep the tensor-core path."""
+    spec = PrefillSpec("t", B=1, T=256, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 43, cuda_device)
+    la = inp["log_alpha"].clone()
+    la[:, 64:128] *= 40.0  # the second chunk only
+    inp["log_alpha"] = la
+    o, s = _run(inp, 64)
+    o_ref, s_ref = _oracle(inp, 1, 256)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(s).all()
+    assert rel_err(o, o_ref) <= TOL_BF16_O
+    assert rel_err(s, s_ref) <= TOL_BF16_S
+
+
 def test_bf16_standard_prefill_workload(cuda_device):
     """The standard prefill workload in full: B=2, T=4096, H=32, d=128, C=64, bf16 q/k/v, fp32
     gates, initial state ~ N(0, 0.02^2); every output and final state against the oracle."""

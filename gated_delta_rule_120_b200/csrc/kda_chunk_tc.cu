@@ -34,14 +34,25 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr float kFastDecayLimit = 60.f;  // |g_C| bound for the direct (K/Gamma) factorisation
 
-// record layout (bytes) of one (chunk, head)
-constexpr uint32_t kRecW = 0;
-constexpr uint32_t kRecQt = 16384;
+// record layout (bytes) of one (chunk, head). QW is a [128 x 128] tile (64-column blocks
+// 16 KiB apart): rows 0..63 hold Qt = Gamma.Q, rows 64..127 hold W, so one M = 128 MMA
+// computes [Qt; W] S.
+constexpr uint32_t kRecQW = 0;
 constexpr uint32_t kRecKt = 32768;
 constexpr uint32_t kRecAqk = 49152;
 constexpr uint32_t kRecU = 57344;
 constexpr uint32_t kRecGam = 73728;
 constexpr uint32_t kRecBytes = 74240;
+__device__ __forceinline__ uint32_t qw_chunk_off(int row128, int c8) {
+  return tile_chunk_off(row128, c8, 16384);
+}
+// exact-fallback scratch for the cumulative decay g (fp32 [64][128]) inside the record: the W
+// half of QW (rows 0..31) and U (rows 32..63), both written only after g is consumed
+__device__ __forceinline__ uint32_t g_scratch_off(int r) {
+  return r < 16 ? kRecQW + 8192u + (uint32_t)r * 512u
+                : (r < 32 ? kRecQW + 24576u + (uint32_t)(r - 16) * 512u
+                          : kRecU + (uint32_t)(r - 32) * 512u);
+}
 static_assert(kRecBytes == TcRecordBytes, "record size mismatch");
 
 // ============================================================================================
@@ -105,7 +116,8 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 // TMEM [0, 128) of an M = 64 accumulator -> bf16 record tile rows (lanes 0..15 of each warp of
 // warps 0..3 own rows 16*warp + lane; warps 4..7 take the upper 64 columns).
 __device__ __forceinline__ void readout_rows_bf16(uint32_t tmem, int warp, int lane,
-                                                  uint8_t* dst_tile) {
+                                                  uint8_t* dst_tile, int row_off,
+                                                  uint32_t block_bytes) {
   const int sp = warp & 3, half = warp >> 2;
   const int r = sp * 16 + (lane & 15);
   float va[32];
@@ -120,7 +132,9 @@ __device__ __forceinline__ void readout_rows_bf16(uint32_t tmem, int warp, int l
         float f[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) f[j] = va[c8 * 8 + j];
-        *reinterpret_cast<uint4*>(dst_tile + tile_chunk_off(r, (col0 >> 3) + c8, 8192)) = pack8(f);
+        *reinterpret_cast<uint4*>(dst_tile +
+                                  tile_chunk_off(r + row_off, (col0 >> 3) + c8, block_bytes)) =
+            pack8(f);
       }
     }
   }
@@ -249,10 +263,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     st_shared_v4(sb + kS1Kg + off, pack8(kg));
     st_shared_v4(sb + kS1Ki + off, pack8(ki));
     st_shared_v4(sb + kS1Qg + off, qgv);
-    *reinterpret_cast<uint4*>(rec + kRecQt + off) = qgv;
+    *reinterpret_cast<uint4*>(rec + kRecQW + qw_chunk_off(r, cg)) = qgv;
     *reinterpret_cast<uint4*>(rec + kRecKt + off) = pack8(kt);
     if (!fast) {  // exact fallback keeps the cumulative decay in this record's W/U area
-      float* gp = reinterpret_cast<float*>(rec + (r < 32 ? kRecW + r * 512 : kRecU + (r - 32) * 512));
+      float* gp = reinterpret_cast<float*>(rec + g_scratch_off(r));
 #pragma unroll
       for (int j = 0; j < 8; ++j) gp[cg * 8 + j] = g[i][j];
     }
@@ -321,8 +335,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       const int i = p - r * (r + 1) / 2;
       float akk = 0.f, aqk = 0.f;
       if (r < L) {
-        const float* gr = reinterpret_cast<const float*>(rec + (r < 32 ? kRecW + r * 512 : kRecU + (r - 32) * 512));
-        const float* gi = reinterpret_cast<const float*>(rec + (i < 32 ? kRecW + i * 512 : kRecU + (i - 32) * 512));
+        const float* gr = reinterpret_cast<const float*>(rec + g_scratch_off(r));
+        const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i));
         const size_t rowr = (size_t)(t0 + r) * H + h, rowi = (size_t)(t0 + i) * H + h;
         for (int cc = lane; cc < kD; cc += 32) {
           const float f = __expf(gr[cc] - gi[cc]);
@@ -449,7 +463,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     alive = __syncthreads_and(mbar_wait(bar, phase)) != 0;
     phase ^= 1;
     tc_fence_after();
-    readout_rows_bf16(tmem, warp, lane, rec + (which == 0 ? kRecW : kRecU));
+    if (which == 0)
+      readout_rows_bf16(tmem, warp, lane, rec + kRecQW, 64, 16384);  // W: rows 64..127 of QW
+    else
+      readout_rows_bf16(tmem, warp, lane, rec + kRecU, 0, 8192);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -468,20 +485,22 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 // K2
 // ============================================================================================
 constexpr int kK2Threads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 epilogue
-constexpr uint32_t kStW = 0, kStQt = 16384, kStKt = 32768, kStAqk = 49152, kStU = 57344,
-                   kStGam = 65536;
-constexpr uint32_t kStageBytes = 66560;  // 65 KiB (keeps every stage 1024-aligned)
-constexpr uint32_t kStageTx = 16384 * 3 + 8192 + 8192 + 512;
-constexpr int kStages = 3;                          // records in flight per CTA
+// stage: QW [128 x 128] | AZ [128 x 64] = A_qk rows 0..63, zero rows 64..127 | Kt [64 x 128] |
+//        U (this CTA's 64-column block) [64 x 64] | gamma_C fp32 [128]
+constexpr uint32_t kStQW = 0, kStAZ = 32768, kStKt = 49152, kStU = 65536, kStGam = 73728;
+constexpr uint32_t kStageBytes = 74752;  // 73 KiB, keeps every stage 1024-aligned
+constexpr uint32_t kStageTx = 32768 + 8192 + 16384 + 8192 + 512;
+constexpr int kStages = 2;
 constexpr uint32_t kS2Stage0 = 0;
-constexpr uint32_t kS2S = kStages * kStageBytes;   // [128 x 64] bf16 state tile
+constexpr uint32_t kS2S = kStages * kStageBytes;   // [128 x 64] bf16 state tile (B operand)
 constexpr uint32_t kS2Vp = kS2S + 16384;           // [64 x 64] bf16 pseudo-value tile
-constexpr uint32_t kS2Bar = kS2Vp + 8192;          // 2 * kStages + 4 mbarriers
-constexpr uint32_t kS2Tmem = kS2Bar + 8 * (2 * kStages + 4);
+constexpr uint32_t kS2Bar = kS2Vp + 8192;
+constexpr int kNumBars2 = 2 * kStages + 5;
+constexpr uint32_t kS2Tmem = kS2Bar + 8 * kNumBars2;
 constexpr uint32_t kS2Flags = kS2Tmem + 4;
 constexpr uint32_t kS2Bytes = kS2Flags + 12;
-// TMEM columns: D1 [0,64), D3 [64,128), D2 double buffer [128,192) / [192,256)
-constexpr uint32_t kTmD1 = 0, kTmD3 = 64, kTmD2 = 128;
+// TMEM columns: [Qt; W] S accumulators (double buffer) [0,64) / [64,128); Kt^T V' [128,192)
+constexpr uint32_t kTmD12 = 0, kTmD3 = 128;
 
 __global__ void __launch_bounds__(kK2Threads, 1)
     chunk_state_tc_kernel(const uint8_t* __restrict__ ws_records, SeqGeometry geo, int H,
@@ -492,12 +511,13 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(sm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kS2Bar);
-  uint64_t* full = bars + 0;         // [kStages]
-  uint64_t* empty = bars + kStages;  // [kStages]
-  uint64_t* d12 = bars + 2 * kStages;
-  uint64_t* d3 = d12 + 1;
-  uint64_t* vp_ready = d12 + 2;
-  uint64_t* s_ready = d12 + 3;
+  uint64_t* full = bars + 0;         // [kStages] record copied
+  uint64_t* empty = bars + kStages;  // [kStages] record consumed by the tensor cores
+  uint64_t* d12 = bars + 2 * kStages;  // [Qt; W] S done
+  uint64_t* d3 = d12 + 1;              // Kt^T V' done (state update can proceed)
+  uint64_t* d2done = d12 + 2;          // A_qk V' accumulated (output can be read)
+  uint64_t* vp_ready = d12 + 3;        // V' tile written (128 arrivals)
+  uint64_t* s_ready = d12 + 4;         // state tile written (128 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS2Tmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kS2Flags);
 
@@ -510,11 +530,13 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   if (warp == 0) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
+    tc_fence_before();
   }
   if (tid == 0) {
     for (int i = 0; i < 2 * kStages; ++i) mbar_init(bars + i, 1);
     mbar_init(d12, 1);
     mbar_init(d3, 1);
+    mbar_init(d2done, 1);
     mbar_init(vp_ready, 128);
     mbar_init(s_ready, 128);
     *abort_flag = 0;
@@ -538,23 +560,21 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
         uint8_t* stage = sm + kS2Stage0 + st * kStageBytes;
         mbar_arrive_expect_tx(full + st, kStageTx);
-        bulk_g2s(stage + kStW, rec + kRecW, 16384, full + st);
-        bulk_g2s(stage + kStQt, rec + kRecQt, 16384, full + st);
+        bulk_g2s(stage + kStQW, rec + kRecQW, 32768, full + st);
+        bulk_g2s(stage + kStAZ, rec + kRecAqk, 8192, full + st);
         bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
-        bulk_g2s(stage + kStAqk, rec + kRecAqk, 8192, full + st);
         bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
         bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
       }
-      // drain: the last copies must land before the CTA may exit
-      const int issued = nchunks;
-      for (int ci = issued > kStages ? issued - kStages : 0; ci < issued; ++ci)
+      // the last copies must land before the CTA may exit
+      for (int ci = nchunks > kStages ? nchunks - kStages : 0; ci < nchunks; ++ci)
         mbar_wait(full + ci % kStages, (ci / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_64 = idesc_bf16_f32(64, 64, 0, 1);     // K-major A, MN-major B
-      const uint32_t id_128 = idesc_bf16_f32(128, 64, 1, 1);   // MN-major A and B
+      const uint32_t id_qw = idesc_bf16_f32(128, 64, 0, 1);  // K-major A, MN-major B
+      const uint32_t id_kt = idesc_bf16_f32(128, 64, 1, 1);  // MN-major A and B
       for (int ci = 0; ci < nchunks; ++ci) {
         const int st = ci % kStages;
         const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
@@ -563,15 +583,12 @@ __global__ void __launch_bounds__(kK2Threads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d2 = tmem + kTmD2 + (ci & 1) * 64;
+        const uint32_t d12t = tmem + kTmD12 + (ci & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
-          const uint64_t bdesc = smem_desc_sw128(sb + kS2S + kk * 2048, 8192, 1024);
-          mma_bf16(tmem + kTmD1, smem_desc_sw128(stage + kStW + koff, 16, 1024), bdesc, id_64,
-                   kk > 0);
-          mma_bf16(d2, smem_desc_sw128(stage + kStQt + koff, 16, 1024), bdesc, id_64, kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)  // [Qt; W] S
+          mma_bf16(d12t,
+                   smem_desc_sw128(stage + kStQW + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                   smem_desc_sw128(sb + kS2S + kk * 2048, 8192, 1024), id_qw, kk > 0);
         mma_commit(d12);
         if (!mbar_wait(vp_ready, ci & 1)) {
           *abort_flag = 1;
@@ -579,24 +596,33 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024);
-          mma_bf16(tmem + kTmD3, smem_desc_sw128(stage + kStKt + kk * 2048, 8192, 1024), bdesc,
-                   id_128, kk > 0);
-          mma_bf16(d2, smem_desc_sw128(stage + kStAqk + kk * 32, 16, 1024), bdesc, id_64, true);
-        }
+        for (int kk = 0; kk < 4; ++kk)  // Kt^T V'
+          mma_bf16(tmem + kTmD3, smem_desc_sw128(stage + kStKt + kk * 2048, 8192, 1024),
+                   smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024), id_kt, kk > 0);
         mma_commit(d3);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // [A_qk; 0] V' accumulated onto the output rows
+          mma_bf16(d12t, smem_desc_sw128(stage + kStAZ + kk * 32, 16, 1024),
+                   smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024), id_qw, true);
+        mma_commit(d2done);
         mma_commit(empty + st);
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue (4 warps)
+    // thread = TMEM lane = row: rows 0..63 of D12 are the chunk output O, rows 64..127 are W S;
+    // every row is a row of the state slice for D3.
     const int sp = warp & 3;
-    const int crow = sp * 32 + lane;       // state row (key channel) owned by this thread
-    const int r = sp * 16 + (lane & 15);   // chunk row of the M = 64 accumulators
-    const bool rowlane = lane < 16;
+    const int row = sp * 32 + lane;
+    const bool out_warp = sp < 2;   // reads O (rows 0..63)
+    const int r = row & 63;         // chunk row for O (out warps) or W S (the other two)
+    // the zero rows of every stage's [A_qk; 0] operand
+    for (int st = 0; st < kStages; ++st)
+      for (int i = tid - 64; i < 512; i += 128)
+        st_shared_v4(sb + kS2Stage0 + st * kStageBytes + kStAZ + 8192 + i * 16,
+                     make_uint4(0, 0, 0, 0));
     float S[64];
-    const size_t sbase = (((size_t)n * H + h) * kD + crow) * kD + j0;
+    const size_t sbase = (((size_t)n * H + h) * kD + row) * kD + j0;
     if (initial_state) {
       const float4* src = reinterpret_cast<const float4*>(initial_state + sbase);
 #pragma unroll
@@ -614,7 +640,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         float f[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) f[j] = S[c8 * 8 + j];
-        st_shared_v4(sb + kS2S + tile_chunk_off(crow, c8, 16384), pack8(f));
+        st_shared_v4(sb + kS2S + tile_chunk_off(row, c8, 16384), pack8(f));
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -628,34 +654,40 @@ __global__ void __launch_bounds__(kK2Threads, 1)
       const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
       const int t0 = tb + ci * kC;
       const int L = min(kC, te - t0);
-      // the staged U and gamma_C are read below: wait for their copy, then for W S / Qt S
-      bool ok = !*abort_flag && mbar_wait(full + st, (ci / kStages) & 1) && mbar_wait(d12, ci & 1);
+      const uint32_t d12c = kTmD12 + (ci & 1) * 64;
+      bool ok = !*abort_flag && mbar_wait(full + st, (ci / kStages) & 1);
       if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform exit: tcgen05.ld is warp-collective
         *abort_flag = 1;
         break;
       }
-      tc_fence_after();
-      const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[crow];
-      // V' = U - W S  (rows r of the M = 64 accumulator live in lanes 0..15)
-      tmem_ld32(tmem_at(tmem, sp * 32, kTmD1), va);
-      tmem_ld32(tmem_at(tmem, sp * 32, kTmD1 + 32), vb);
-      tmem_ld_wait();
-      if (rowlane) {
+      const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[row];
+      if (!out_warp) {  // V' = U - W S for chunk row r
+        uint4 u4[8];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) u4[c8] = ld_shared_v4(stage + kStU + tile_chunk_off(r, c8, 8192));
+        ok = mbar_wait(d12, ci & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        tmem_ld32(tmem_at(tmem, sp * 32, d12c), va);
+        tmem_ld32(tmem_at(tmem, sp * 32, d12c + 32), vb);
+        tmem_ld_wait();
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          const uint32_t off = tile_chunk_off(r, c8, 8192);
           float u[8], f[8];
-          unpack8(ld_shared_v4(stage + kStU + off), u);
+          unpack8(u4[c8], u);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int col = c8 * 8 + j;
             f[j] = u[j] - (col < 32 ? va[col] : vb[col - 32]);
           }
-          st_shared_v4(sb + kS2Vp + off, pack8(f));
+          st_shared_v4(sb + kS2Vp + tile_chunk_off(r, c8, 8192), pack8(f));
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
       mbar_arrive(vp_ready);
       // S = Diag(gamma_C) S + Kt^T V'
       ok = mbar_wait(d3, ci & 1);
@@ -672,23 +704,29 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         S[j] = fmaf(gam, S[j], va[j]);
         S[32 + j] = fmaf(gam, S[32 + j], vb[j]);
       }
-      // O = Qt S + A_qk V' (read before this thread lets the next chunk's MMAs start)
-      const uint32_t d2 = kTmD2 + (ci & 1) * 64;
-      tmem_ld32(tmem_at(tmem, sp * 32, d2), va);
-      tmem_ld32(tmem_at(tmem, sp * 32, d2 + 32), vb);
-      tmem_ld_wait();
       write_state_tile();
-      if (rowlane && r < L) {
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0);
+      if (out_warp) {  // O = Qt S + A_qk V' (Eq. 9), off the state chain
+        ok = mbar_wait(d2done, ci & 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        tmem_ld32(tmem_at(tmem, sp * 32, d12c), va);
+        tmem_ld32(tmem_at(tmem, sp * 32, d12c + 32), vb);
+        tmem_ld_wait();
+        if (r < L) {
+          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float f[8];
+          for (int c8 = 0; c8 < 8; ++c8) {
+            float f[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = c8 * 8 + j;
-            f[j] = col < 32 ? va[col] : vb[col - 32];
+            for (int j = 0; j < 8; ++j) {
+              const int col = c8 * 8 + j;
+              f[j] = col < 32 ? va[col] : vb[col - 32];
+            }
+            dst[c8] = pack8(f);
           }
-          dst[c8] = pack8(f);
         }
       }
     }

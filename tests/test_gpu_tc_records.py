@@ -4,8 +4,9 @@ walkthrough, §3.4 "Chunkwise Parallelization") evaluated here in fp64 from the 
 
 This localises a failure of the end-to-end parity tests to the chunk-local kernel (records wrong)
 or to the state kernel (records right, outputs wrong). Record layout per (chunk, head), bf16
-tiles in the 128-byte-swizzled operand layout: W, Qt, Kt [64 x 128], A_qk [64 x 64], U [64 x 128],
-then gamma_C as 128 fp32.
+tiles in the 128-byte-swizzled operand layout: [Qt; W] [128 x 128], Kt [64 x 128], A_qk [64 x 64],
+U [64 x 128],
+then gamma_C as 128 fp32. Qt and W share one [128 x 128] tile (Qt rows 0..63, W rows 64..127).
 """
 import numpy as np
 import pytest
@@ -18,7 +19,7 @@ from tests._parity import to_np
 
 pytestmark = pytest.mark.gpu
 
-REC = dict(W=0, Qt=16384, Kt=32768, Aqk=49152, U=57344, gam=73728, size=74240)
+REC = dict(QW=0, Kt=32768, Aqk=49152, U=57344, gam=73728, size=74240)
 
 
 def tile_index(rows, cols):
@@ -79,8 +80,8 @@ def test_chunk_records_match_formulas(cuda_device, T):
                                   x["v"][t0:t0 + L, h], x["log_alpha"][t0:t0 + L, h],
                                   x["beta"][t0:t0 + L, h], L)
             base = 256 + REC["size"] * (c * 2 + h)
-            got = dict(W=decode_tile(buf, base + REC["W"], 64, 128),
-                       Qt=decode_tile(buf, base + REC["Qt"], 64, 128),
+            qw = decode_tile(buf, base + REC["QW"], 128, 128)
+            got = dict(W=qw[64:], Qt=qw[:64],
                        Kt=decode_tile(buf, base + REC["Kt"], 64, 128),
                        Aqk=decode_tile(buf, base + REC["Aqk"], 64, 64),
                        U=decode_tile(buf, base + REC["U"], 64, 128),

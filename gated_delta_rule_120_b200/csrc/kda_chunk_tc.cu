@@ -484,7 +484,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 // ============================================================================================
 // K2
 // ============================================================================================
-constexpr int kK2Threads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEpiWarps = 8;                       // two per TMEM sub-partition, 32 columns each
+constexpr int kK2Threads = 64 + 32 * kEpiWarps;    // warp 0 producer, warp 1 MMA, then epilogue
 // stage: QW [128 x 128] | AZ [128 x 64] = A_qk rows 0..63, zero rows 64..127 | Kt [64 x 128] |
 //        U (this CTA's 64-column block) [64 x 64] | gamma_C fp32 [128]
 constexpr uint32_t kStQW = 0, kStAZ = 32768, kStKt = 49152, kStU = 65536, kStGam = 73728;
@@ -511,13 +512,13 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(sm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kS2Bar);
-  uint64_t* full = bars + 0;         // [kStages] record copied
-  uint64_t* empty = bars + kStages;  // [kStages] record consumed by the tensor cores
+  uint64_t* full = bars + 0;           // [kStages] record copied
+  uint64_t* empty = bars + kStages;    // [kStages] record consumed by the tensor cores
   uint64_t* d12 = bars + 2 * kStages;  // [Qt; W] S done
   uint64_t* d3 = d12 + 1;              // Kt^T V' done (state update can proceed)
   uint64_t* d2done = d12 + 2;          // A_qk V' accumulated (output can be read)
-  uint64_t* vp_ready = d12 + 3;        // V' tile written (128 arrivals)
-  uint64_t* s_ready = d12 + 4;         // state tile written (128 arrivals)
+  uint64_t* vp_ready = d12 + 3;        // V' tile written (one arrival per epilogue warp)
+  uint64_t* s_ready = d12 + 4;         // state tile written (one arrival per epilogue warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS2Tmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kS2Flags);
 
@@ -537,8 +538,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     mbar_init(d12, 1);
     mbar_init(d3, 1);
     mbar_init(d2done, 1);
-    mbar_init(vp_ready, 128);
-    mbar_init(s_ready, 128);
+    mbar_init(vp_ready, kEpiWarps);
+    mbar_init(s_ready, kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -575,20 +576,27 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     if (lane == 0) {
       const uint32_t id_qw = idesc_bf16_f32(128, 64, 0, 1);  // K-major A, MN-major B
       const uint32_t id_kt = idesc_bf16_f32(128, 64, 1, 1);  // MN-major A and B
+      // descriptors are built once; the start-address field (bits 0..13, >> 4) is advanced by
+      // plain addition, which never carries out of the field inside shared memory
+      const uint64_t dqw = smem_desc_sw128(sb + kS2Stage0 + kStQW, 16, 1024);
+      const uint64_t daz = smem_desc_sw128(sb + kS2Stage0 + kStAZ, 16, 1024);
+      const uint64_t dkt = smem_desc_sw128(sb + kS2Stage0 + kStKt, 8192, 1024);
+      const uint64_t ds = smem_desc_sw128(sb + kS2S, 8192, 1024);
+      const uint64_t dvp = smem_desc_sw128(sb + kS2Vp, 8192, 1024);
       for (int ci = 0; ci < nchunks; ++ci) {
         const int st = ci % kStages;
-        const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
         if (!mbar_wait(full + st, (ci / kStages) & 1) || !mbar_wait(s_ready, ci & 1)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
         const uint32_t d12t = tmem + kTmD12 + (ci & 1) * 64;
+        const uint64_t soff = (uint64_t)((st * kStageBytes) >> 4);
+        const uint64_t aqw = dqw + soff, aaz = daz + soff, akt = dkt + soff;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // [Qt; W] S
-          mma_bf16(d12t,
-                   smem_desc_sw128(stage + kStQW + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                   smem_desc_sw128(sb + kS2S + kk * 2048, 8192, 1024), id_qw, kk > 0);
+          mma_bf16(d12t, aqw + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                   ds + (uint64_t)((kk * 2048) >> 4), id_qw, kk > 0);
         mma_commit(d12);
         if (!mbar_wait(vp_ready, ci & 1)) {
           *abort_flag = 1;
@@ -597,74 +605,82 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // Kt^T V'
-          mma_bf16(tmem + kTmD3, smem_desc_sw128(stage + kStKt + kk * 2048, 8192, 1024),
-                   smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024), id_kt, kk > 0);
+          mma_bf16(tmem + kTmD3, akt + (uint64_t)((kk * 2048) >> 4),
+                   dvp + (uint64_t)((kk * 2048) >> 4), id_kt, kk > 0);
         mma_commit(d3);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // [A_qk; 0] V' accumulated onto the output rows
-          mma_bf16(d12t, smem_desc_sw128(stage + kStAZ + kk * 32, 16, 1024),
-                   smem_desc_sw128(sb + kS2Vp + kk * 2048, 8192, 1024), id_qw, true);
+          mma_bf16(d12t, aaz + (uint64_t)((kk * 32) >> 4), dvp + (uint64_t)((kk * 2048) >> 4),
+                   id_qw, true);
         mma_commit(d2done);
         mma_commit(empty + st);
       }
     }
   } else {
-    // ------------------------------------------------------------------ epilogue (4 warps)
-    // thread = TMEM lane = row: rows 0..63 of D12 are the chunk output O, rows 64..127 are W S;
-    // every row is a row of the state slice for D3.
+    // ------------------------------------------------------------------ epilogue (8 warps)
+    // thread = TMEM lane = row, warp pair = column half: rows 0..63 of D12 are the chunk output
+    // O, rows 64..127 are W S; every row is a row of the state slice for D3.
+    const int ew = warp - 2;
     const int sp = warp & 3;
+    const int chalf = ew >> 2;       // columns [32 chalf, 32 chalf + 32) of the 64-column slice
     const int row = sp * 32 + lane;
-    const bool out_warp = sp < 2;   // reads O (rows 0..63)
-    const int r = row & 63;         // chunk row for O (out warps) or W S (the other two)
+    const bool out_warp = sp < 2;    // reads O (rows 0..63); the others compute V'
+    const int r = row & 63;
     // the zero rows of every stage's [A_qk; 0] operand
     for (int st = 0; st < kStages; ++st)
-      for (int i = tid - 64; i < 512; i += 128)
+      for (int i = tid - 64; i < 512; i += 32 * kEpiWarps)
         st_shared_v4(sb + kS2Stage0 + st * kStageBytes + kStAZ + 8192 + i * 16,
                      make_uint4(0, 0, 0, 0));
-    float S[64];
-    const size_t sbase = (((size_t)n * H + h) * kD + row) * kD + j0;
+    float S[32];
+    const size_t sbase = (((size_t)n * H + h) * kD + row) * kD + j0 + 32 * chalf;
     if (initial_state) {
       const float4* src = reinterpret_cast<const float4*>(initial_state + sbase);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const float4 x = src[j];
         S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) S[j] = 0.f;
+      for (int j = 0; j < 32; ++j) S[j] = 0.f;
     }
     auto write_state_tile = [&]() {
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
+      for (int q8 = 0; q8 < 4; ++q8) {
         float f[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = S[c8 * 8 + j];
-        st_shared_v4(sb + kS2S + tile_chunk_off(row, c8, 16384), pack8(f));
+        for (int j = 0; j < 8; ++j) f[j] = S[q8 * 8 + j];
+        st_shared_v4(sb + kS2S + tile_chunk_off(row, 4 * chalf + q8, 16384), pack8(f));
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(s_ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_ready);
     };
     write_state_tile();
 
-    float va[32], vb[32];
+    float va[32];
     for (int ci = 0; ci < nchunks; ++ci) {
       const int st = ci % kStages;
       const uint32_t stage = sb + kS2Stage0 + st * kStageBytes;
       const int t0 = tb + ci * kC;
       const int L = min(kC, te - t0);
-      const uint32_t d12c = kTmD12 + (ci & 1) * 64;
+      const uint32_t d12c = kTmD12 + (ci & 1) * 64 + 32 * chalf;
       bool ok = !*abort_flag && mbar_wait(full + st, (ci / kStages) & 1);
       if (!__all_sync(0xffffffffu, ok)) {  // warp-uniform exit: tcgen05.ld is warp-collective
         *abort_flag = 1;
         break;
       }
       const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[row];
-      if (!out_warp) {  // V' = U - W S for chunk row r
-        uint4 u4[8];
+      if (!out_warp) {  // V' = U - W S for chunk row r, this warp's 32 columns
+        float u[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) u4[c8] = ld_shared_v4(stage + kStU + tile_chunk_off(r, c8, 8192));
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float f[8];
+          unpack8(ld_shared_v4(stage + kStU + tile_chunk_off(r, 4 * chalf + q8, 8192)), f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) u[q8 * 8 + j] = f[j];
+        }
         ok = mbar_wait(d12, ci & 1);
         if (!__all_sync(0xffffffffu, ok)) {
           *abort_flag = 1;
@@ -672,23 +688,19 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         }
         tc_fence_after();
         tmem_ld32(tmem_at(tmem, sp * 32, d12c), va);
-        tmem_ld32(tmem_at(tmem, sp * 32, d12c + 32), vb);
         tmem_ld_wait();
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float u[8], f[8];
-          unpack8(u4[c8], u);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float f[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = c8 * 8 + j;
-            f[j] = u[j] - (col < 32 ? va[col] : vb[col - 32]);
-          }
-          st_shared_v4(sb + kS2Vp + tile_chunk_off(r, c8, 8192), pack8(f));
+          for (int j = 0; j < 8; ++j) f[j] = u[q8 * 8 + j] - va[q8 * 8 + j];
+          st_shared_v4(sb + kS2Vp + tile_chunk_off(r, 4 * chalf + q8, 8192), pack8(f));
         }
         fence_proxy_async_smem();
         tc_fence_before();
       }
-      mbar_arrive(vp_ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(vp_ready);
       // S = Diag(gamma_C) S + Kt^T V'
       ok = mbar_wait(d3, ci & 1);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -696,14 +708,10 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         break;
       }
       tc_fence_after();
-      tmem_ld32(tmem_at(tmem, sp * 32, kTmD3), va);
-      tmem_ld32(tmem_at(tmem, sp * 32, kTmD3 + 32), vb);
+      tmem_ld32(tmem_at(tmem, sp * 32, kTmD3 + 32 * chalf), va);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        S[j] = fmaf(gam, S[j], va[j]);
-        S[32 + j] = fmaf(gam, S[32 + j], vb[j]);
-      }
+      for (int j = 0; j < 32; ++j) S[j] = fmaf(gam, S[j], va[j]);
       write_state_tile();
       if (out_warp) {  // O = Qt S + A_qk V' (Eq. 9), off the state chain
         ok = mbar_wait(d2done, ci & 1);
@@ -713,19 +721,16 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         }
         tc_fence_after();
         tmem_ld32(tmem_at(tmem, sp * 32, d12c), va);
-        tmem_ld32(tmem_at(tmem, sp * 32, d12c + 32), vb);
         tmem_ld_wait();
         if (r < L) {
-          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0);
+          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0 +
+                                                32 * chalf);
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
+          for (int q8 = 0; q8 < 4; ++q8) {
             float f[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int col = c8 * 8 + j;
-              f[j] = col < 32 ? va[col] : vb[col - 32];
-            }
-            dst[c8] = pack8(f);
+            for (int j = 0; j < 8; ++j) f[j] = va[q8 * 8 + j];
+            dst[q8] = pack8(f);
           }
         }
       }
@@ -733,7 +738,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     if (final_state && !*abort_flag) {
       float4* dst = reinterpret_cast<float4*>(final_state + sbase);
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
+      for (int j = 0; j < 8; ++j)
         dst[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
     }
   }

@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   for (int j = 0; j < 8; ++j) {
     const float gcj = sGC[cg * 8 + j];
     ok = ok && (gcj >= -kFastDecayLimit);
-    egc[j] = expf(gcj);
+    egc[j] = __expf(gcj);  // only scales a bf16 operand; the carried gamma_C uses expf
   }
   const bool fast = __syncthreads_and(ok) != 0;
 
@@ -392,41 +392,82 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     for (int i = 0; i < 16; ++i) sT[sidx(16 * b + i, 16 * b + cidx)] = col[i];
   }
   __syncthreads();
-  // off-diagonal blocks, one block-diagonal at a time:  T_R,I = -T_RR sum_{J=I}^{R-1} A_RJ T_JI
-  // (d = R - I). A thread owns a 1 x 4 strip (row rr, columns 4cq..4cq+3) of one block.
-  for (int d = 1; d < 4; ++d) {
-    const int nstrips = (4 - d) * 64;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int bi = 0, rr = 0, cq = 0, R = 0, I = 0;
-    const bool act = tid < nstrips;
-    if (act) {
-      bi = tid >> 6; rr = (tid >> 2) & 15; cq = tid & 3;
-      R = d + bi; I = R - d;
-      for (int k4 = 4 * I; k4 < 4 * R; ++k4) {
-        const float4 a = lds4(sA, 16 * R + rr, k4);
-        const float4 t0 = lds4(sT, 4 * k4 + 0, 4 * I + cq), t1 = lds4(sT, 4 * k4 + 1, 4 * I + cq);
-        const float4 t2 = lds4(sT, 4 * k4 + 2, 4 * I + cq), t3 = lds4(sT, 4 * k4 + 3, 4 * I + cq);
+  // Off-diagonal blocks by the 2 x 2 block rule (I + A)^{-1} = [[T11, 0], [-T22 A21 T11, T22]]:
+  //   32 x 32 halves first (t_{b+1,b} = -t_{b+1} a_{b+1,b} t_b for b = 0, 2), then the lower-left
+  //   32 x 32 block T21 = -T22 (A21 T11). Threads own 1 x 4 strips; entries of T above the
+  //   diagonal outside the diagonal blocks are never read.
+  {
+    // stage 2: X_b = a_{b+1,b} t_b for b = 0, 2 (two 16 x 16 products, 128 strips)
+    const int b2 = (tid >> 6) & 1, rr = (tid >> 2) & 15, cq = tid & 3;
+    const int bb = 2 * b2;  // b = 0 or 2
+    if (tid < 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        if (k4 < cq) continue;  // t_b[k][c] = 0 for k < c
+        const float4 a = lds4(sA, 16 * (bb + 1) + rr, 4 * bb + k4);
+        const float4 t0 = lds4(sT, 16 * bb + 4 * k4 + 0, 4 * bb + cq);
+        const float4 t1 = lds4(sT, 16 * bb + 4 * k4 + 1, 4 * bb + cq);
+        const float4 t2 = lds4(sT, 16 * bb + 4 * k4 + 2, 4 * bb + cq);
+        const float4 t3 = lds4(sT, 16 * bb + 4 * k4 + 3, 4 * bb + cq);
         acc.x += a.x * t0.x + a.y * t1.x + a.z * t2.x + a.w * t3.x;
         acc.y += a.x * t0.y + a.y * t1.y + a.z * t2.y + a.w * t3.y;
         acc.z += a.x * t0.z + a.y * t1.z + a.z * t2.z + a.w * t3.z;
         acc.w += a.x * t0.w + a.y * t1.w + a.z * t2.w + a.w * t3.w;
       }
-      *reinterpret_cast<float4*>(sX + bi * 256 + rr * 16 + 4 * cq) = acc;
+      *reinterpret_cast<float4*>(sX + b2 * 256 + rr * 16 + 4 * cq) = acc;
     }
     __syncthreads();
-    if (act) {
+    // t_{b+1,b} = -t_{b+1} X_b
+    if (tid < 128) {
       float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int m4 = 0; m4 < 4; ++m4) {
-        const float4 a = lds4(sT, 16 * R + rr, 4 * R + m4);
-        const float4* xr = reinterpret_cast<const float4*>(sX + bi * 256 + (4 * m4) * 16 + 4 * cq);
+        if (4 * m4 > rr) continue;  // t_{b+1}[rr][m] = 0 for m > rr
+        const float4 a = lds4(sT, 16 * (bb + 1) + rr, 4 * (bb + 1) + m4);
+        const float4* xr = reinterpret_cast<const float4*>(sX + b2 * 256 + (4 * m4) * 16 + 4 * cq);
         const float4 x0 = xr[0], x1 = xr[4], x2 = xr[8], x3 = xr[12];
         t.x += a.x * x0.x + a.y * x1.x + a.z * x2.x + a.w * x3.x;
         t.y += a.x * x0.y + a.y * x1.y + a.z * x2.y + a.w * x3.y;
         t.z += a.x * x0.z + a.y * x1.z + a.z * x2.z + a.w * x3.z;
         t.w += a.x * x0.w + a.y * x1.w + a.z * x2.w + a.w * x3.w;
       }
-      sts4(sT, 16 * R + rr, 4 * I + cq, make_float4(-t.x, -t.y, -t.z, -t.w));
+      sts4(sT, 16 * (bb + 1) + rr, 4 * bb + cq, make_float4(-t.x, -t.y, -t.z, -t.w));
+    }
+    __syncthreads();
+    // stage 3: Y = A21 T11 (32 x 32, K over k >= c), one strip per thread
+    const int r3 = tid >> 3, c3 = tid & 7;  // row 0..31, column group 0..7
+    {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        if (k4 < c3) continue;
+        const float4 a = lds4(sA, 32 + r3, k4);
+        const float4 t0 = lds4(sT, 4 * k4 + 0, c3), t1 = lds4(sT, 4 * k4 + 1, c3);
+        const float4 t2 = lds4(sT, 4 * k4 + 2, c3), t3 = lds4(sT, 4 * k4 + 3, c3);
+        acc.x += a.x * t0.x + a.y * t1.x + a.z * t2.x + a.w * t3.x;
+        acc.y += a.x * t0.y + a.y * t1.y + a.z * t2.y + a.w * t3.y;
+        acc.z += a.x * t0.z + a.y * t1.z + a.z * t2.z + a.w * t3.z;
+        acc.w += a.x * t0.w + a.y * t1.w + a.z * t2.w + a.w * t3.w;
+      }
+      *reinterpret_cast<float4*>(sX + r3 * 32 + 4 * c3) = acc;
+    }
+    __syncthreads();
+    // T21 = -T22 Y (K over k <= r)
+    {
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        if (4 * k4 > r3) continue;
+        const float4 a = lds4(sT, 32 + r3, 8 + k4);
+        const float4* yr = reinterpret_cast<const float4*>(sX + (4 * k4) * 32 + 4 * c3);
+        const float4 y0 = yr[0], y1 = yr[8], y2 = yr[16], y3 = yr[24];
+        t.x += a.x * y0.x + a.y * y1.x + a.z * y2.x + a.w * y3.x;
+        t.y += a.x * y0.y + a.y * y1.y + a.z * y2.y + a.w * y3.y;
+        t.z += a.x * y0.z + a.y * y1.z + a.z * y2.z + a.w * y3.z;
+        t.w += a.x * y0.w + a.y * y1.w + a.z * y2.w + a.w * y3.w;
+      }
+      sts4(sT, 32 + r3, c3, make_float4(-t.x, -t.y, -t.z, -t.w));
     }
     __syncthreads();
   }

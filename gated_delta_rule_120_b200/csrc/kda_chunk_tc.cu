@@ -207,31 +207,46 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   for (int i = 1; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) g[i][j] += g[i - 1][j];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) sScan[rg * kD + cg * 8 + j] = g[3][j];
+  {  // 128-bit accesses: eight lanes of a row segment cover all 32 banks once
+    float4* sc = reinterpret_cast<float4*>(sScan + rg * kD + cg * 8);
+    sc[0] = make_float4(g[3][0], g[3][1], g[3][2], g[3][3]);
+    sc[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
+  }
   __syncthreads();
   {
     float pre[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) pre[j] = 0.f;
-    for (int r2 = 0; r2 < rg; ++r2)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) pre[j] += sScan[r2 * kD + cg * 8 + j];
+    for (int r2 = 0; r2 < rg; ++r2) {
+      const float4* sc = reinterpret_cast<const float4*>(sScan + r2 * kD + cg * 8);
+      const float4 a = sc[0], b = sc[1];
+      pre[0] += a.x; pre[1] += a.y; pre[2] += a.z; pre[3] += a.w;
+      pre[4] += b.x; pre[5] += b.y; pre[6] += b.z; pre[7] += b.w;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 8; ++j) g[i][j] += pre[j];
   }
-  if (rg == 15)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sGC[cg * 8 + j] = g[3][j];
+  if (rg == 15) {
+    float4* gcp = reinterpret_cast<float4*>(sGC + cg * 8);
+    gcp[0] = make_float4(g[3][0], g[3][1], g[3][2], g[3][3]);
+    gcp[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
+  }
   cp_async_wait_all();
   __syncthreads();
   float egc[8];
   bool ok = true;
+  float gcv[8];
+  {
+    const float4* gcp = reinterpret_cast<const float4*>(sGC + cg * 8);
+    const float4 a = gcp[0], b = gcp[1];
+    gcv[0] = a.x; gcv[1] = a.y; gcv[2] = a.z; gcv[3] = a.w;
+    gcv[4] = b.x; gcv[5] = b.y; gcv[6] = b.z; gcv[7] = b.w;
+  }
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float gcj = sGC[cg * 8 + j];
+    const float gcj = gcv[j];
     ok = ok && (gcj >= -kFastDecayLimit);
     egc[j] = __expf(gcj);  // only scales a bf16 operand; the carried gamma_C uses expf
   }

@@ -17,6 +17,7 @@
 // than L2 and is not reused within the step.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_sm100.cuh"
 
 namespace kda {
 
@@ -143,11 +144,243 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Streaming variant (used whenever the per-head vectors allow 16-byte bulk copies): one
+// persistent CTA per SM walks its heads through a three-stage shared-memory ring. A producer warp
+// bulk-loads a head's whole state plus its q, k, v and log-decay vectors ahead of use and bulk-
+// stores the updated state back, so HBM reads of later heads overlap the compute and the write
+// of earlier ones; eight compute warps do the same one-pass update as above on the staged copy.
+// ---------------------------------------------------------------------------------------------
+constexpr int kDsStages = 3;
+constexpr int kDsCompute = 256;                // 8 compute warps
+constexpr int kDsThreads = kDsCompute + 32;    // + producer warp
+
+struct DsLayout {
+  uint32_t state_bytes, la_off, q_off, k_off, v_off, stage_bytes, vec_tx;
+};
+
+__host__ __device__ inline uint32_t align16u(uint32_t x) { return (x + 15u) & ~15u; }
+
+static DsLayout make_ds_layout(int Dk, int Dv, int es) {
+  DsLayout L;
+  L.state_bytes = (uint32_t)Dk * Dv * 4;
+  L.la_off = L.state_bytes;
+  L.q_off = L.la_off + align16u((uint32_t)Dk * 4);
+  L.k_off = L.q_off + align16u((uint32_t)Dk * es);
+  L.v_off = L.k_off + align16u((uint32_t)Dk * es);
+  L.stage_bytes = (L.v_off + align16u((uint32_t)Dv * es) + 127u) & ~127u;
+  L.vec_tx = (uint32_t)Dk * 4 + 2u * Dk * es + (uint32_t)Dv * es;
+  return L;
+}
+
+__device__ __forceinline__ bool block_all(bool pred, uint32_t bar_id, uint32_t nthreads) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(bar_id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kDsThreads, 1)
+    decode_stream_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                         const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                         const float* __restrict__ beta, float* __restrict__ state,
+                         Tin* __restrict__ o, int NH, int Dk, int Dv, DsLayout lay) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((128 - (sm100::smem_u32(smem_raw) & 127)) & 127);
+  uint8_t* stages = sm;
+  float4* s_e = reinterpret_cast<float4*>(sm + kDsStages * lay.stage_bytes);  // [8][32]
+  float4* s_p = s_e + 8 * 32;                                                 // [8][32]
+  float* s_kq = reinterpret_cast<float*>(s_p + 8 * 32);                        // [8]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_kq + 8);                      // [kDsStages]
+  uint64_t* computed = full + kDsStages;                                       // [kDsStages]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int first = blockIdx.x, stride = gridDim.x;
+  const int count = first < NH ? (NH - first + stride - 1) / stride : 0;
+  const uint32_t es = sizeof(Tin);
+
+  if (tid == 0) {
+    for (int i = 0; i < kDsStages; ++i) {
+      sm100::mbar_init(full + i, 1);
+      sm100::mbar_init(computed + i, 1);
+    }
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kDsCompute / 32) {
+    // ---------------------------------------------------------------- producer warp
+    if (lane == 0) {
+      auto issue_load = [&](int it) {
+        const int s = it % kDsStages;
+        const size_t head = (size_t)first + (size_t)it * stride;
+        uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+        sm100::mbar_arrive_expect_tx(full + s, lay.state_bytes + lay.vec_tx);
+        sm100::bulk_g2s(st, state + head * Dk * Dv, lay.state_bytes, full + s);
+        sm100::bulk_g2s(st + lay.la_off, log_alpha + head * Dk, Dk * 4, full + s);
+        sm100::bulk_g2s(st + lay.q_off, q + head * Dk, Dk * es, full + s);
+        sm100::bulk_g2s(st + lay.k_off, k + head * Dk, Dk * es, full + s);
+        sm100::bulk_g2s(st + lay.v_off, v + head * Dv, Dv * es, full + s);
+      };
+      for (int it = 0; it < count && it < kDsStages; ++it) issue_load(it);
+      for (int it = 0; it < count; ++it) {
+        const int s = it % kDsStages;
+        if (!sm100::mbar_wait(computed + s, (it / kDsStages) & 1)) break;
+        const size_t head = (size_t)first + (size_t)it * stride;
+        sm100::bulk_s2g(state + head * Dk * Dv, stages + (size_t)s * lay.stage_bytes,
+                        lay.state_bytes);
+        sm100::bulk_commit();
+        if (it + kDsStages < count) {
+          sm100::bulk_wait_read_all();  // the stage is free once its store has read it
+          issue_load(it + kDsStages);
+        }
+      }
+      sm100::bulk_wait_all();
+      // loads that were issued but never consumed (only after a timeout) must land first
+      for (int it = 0; it < count && it < kDsStages; ++it) {
+        const int last = count - 1 - it;
+        if (last >= 0) sm100::mbar_wait(full + last % kDsStages, (last / kDsStages) & 1, 100000000ull);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    const int col = lane * 4;
+    const bool col_ok = col < Dv;
+    const int row0 = warp * kDecRowsPerWarp;
+    float b_next = count > 0 ? beta[first] : 0.f;
+    for (int it = 0; it < count; ++it) {
+      const int s = it % kDsStages;
+      const size_t head = (size_t)first + (size_t)it * stride;
+      const float b = b_next;
+      if (it + 1 < count) b_next = beta[head + stride];
+      const bool ok = sm100::mbar_wait(full + s, (it / kDsStages) & 1);
+      if (!block_all(ok, 1, kDsCompute)) break;
+      uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+      const float* la = reinterpret_cast<const float*>(st + lay.la_off);
+      const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off);
+      const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off);
+      const Tin* vv = reinterpret_cast<const Tin*>(st + lay.v_off);
+      // decay of this warp's 16 rows: lanes 0..15 evaluate one each, shuffled to the warp
+      const int rl = row0 + (lane & 15);
+      const float a_mine = (rl < Dk) ? expf(la[rl]) : 1.f;
+      float4* Srow = reinterpret_cast<float4*>(st) + (col >> 2);
+      const int vstride = Dv >> 2;
+      float4 sreg[kDecRowsPerWarp];
+#pragma unroll
+      for (int i = 0; i < kDecRowsPerWarp; ++i) {
+        const int r = row0 + i;
+        sreg[i] = (col_ok && r < Dk) ? Srow[r * vstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
+      float kq = 0.f;
+      float kr_[kDecRowsPerWarp];
+#pragma unroll
+      for (int i = 0; i < kDecRowsPerWarp; ++i) {
+        const int r = row0 + i;
+        const float a = __shfl_sync(0xffffffffu, a_mine, i);
+        const float kr = (r < Dk) ? to_f32(kv[r]) : 0.f;
+        const float qr = (r < Dk) ? to_f32(qv[r]) : 0.f;
+        kr_[i] = kr;
+        kq += kr * qr;
+        sreg[i].x *= a; sreg[i].y *= a; sreg[i].z *= a; sreg[i].w *= a;
+        e.x += sreg[i].x * kr; e.y += sreg[i].y * kr; e.z += sreg[i].z * kr; e.w += sreg[i].w * kr;
+        p.x += sreg[i].x * qr; p.y += sreg[i].y * qr; p.z += sreg[i].z * qr; p.w += sreg[i].w * qr;
+      }
+      s_e[warp * 32 + lane] = e;
+      s_p[warp * 32 + lane] = p;
+      if (lane == 0) s_kq[warp] = kq;
+      sm100::named_barrier_sync(1, kDsCompute);
+      e = make_float4(0.f, 0.f, 0.f, 0.f);
+      p = e;
+      kq = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float4 ew = s_e[w * 32 + lane], pw = s_p[w * 32 + lane];
+        e.x += ew.x; e.y += ew.y; e.z += ew.z; e.w += ew.w;
+        p.x += pw.x; p.y += pw.y; p.z += pw.z; p.w += pw.w;
+        kq += s_kq[w];
+      }
+      float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (col_ok) {
+        u.x = b * (to_f32(vv[col]) - e.x);
+        u.y = b * (to_f32(vv[col + 1]) - e.y);
+        u.z = b * (to_f32(vv[col + 2]) - e.z);
+        u.w = b * (to_f32(vv[col + 3]) - e.w);
+      }
+#pragma unroll
+      for (int i = 0; i < kDecRowsPerWarp; ++i) {
+        const int r = row0 + i;
+        if (col_ok && r < Dk) {
+          float4 t = sreg[i];
+          t.x += kr_[i] * u.x; t.y += kr_[i] * u.y; t.z += kr_[i] * u.z; t.w += kr_[i] * u.w;
+          Srow[r * vstride] = t;
+        }
+      }
+      if (warp == 0 && col_ok) {
+        Tin* op = o + head * Dv + col;
+        op[0] = from_f32<Tin>(p.x + kq * u.x);
+        op[1] = from_f32<Tin>(p.y + kq * u.y);
+        op[2] = from_f32<Tin>(p.z + kq * u.z);
+        op[3] = from_f32<Tin>(p.w + kq * u.w);
+      }
+      sm100::fence_proxy_async_smem();
+      sm100::named_barrier_sync(1, kDsCompute);
+      if (tid == 0) sm100::mbar_arrive(computed + s);
+    }
+  }
+  __syncthreads();
+}
+
+static int g_num_sms[64] = {0};
+
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                const float* log_alpha, const float* beta, float* state, void* o,
                                int N, int H, int Dk, int Dv, cudaStream_t stream) {
   const long long heads = (long long)N * H;
   if (heads == 0) return cudaSuccess;
+  const int es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  const bool streamable = (Dk * es) % 16 == 0 && (Dv * es) % 16 == 0 && (Dk * 4) % 16 == 0 &&
+                          al16(q) && al16(k) && al16(v) && al16(log_alpha) && al16(state);
+  if (streamable) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    int nsm = (dev >= 0 && dev < 64) ? g_num_sms[dev] : 0;
+    if (nsm == 0) {
+      err = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      if (err != cudaSuccess) return err;
+      if (dev >= 0 && dev < 64) g_num_sms[dev] = nsm;
+    }
+    const DsLayout lay = make_ds_layout(Dk, Dv, es);
+    const size_t smem = (size_t)kDsStages * lay.stage_bytes + 2 * 8 * 32 * sizeof(float4) +
+                        8 * sizeof(float) + 2 * kDsStages * sizeof(uint64_t) + 128;
+    const int grid = (int)(heads < nsm ? heads : nsm);
+    ProfileScope prof("decode_stream", stream);
+    if (dt == KDA_DTYPE_BF16) {
+      err = cudaFuncSetAttribute(decode_stream_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      decode_stream_kernel<__nv_bfloat16><<<grid, kDsThreads, smem, stream>>>(
+          (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha,
+          beta, state, (__nv_bfloat16*)o, (int)heads, Dk, Dv, lay);
+    } else {
+      err = cudaFuncSetAttribute(decode_stream_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+      decode_stream_kernel<float><<<grid, kDsThreads, smem, stream>>>(
+          (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, state, (float*)o,
+          (int)heads, Dk, Dv, lay);
+    }
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)heads), block(kDecThreads);
   ProfileScope prof("decode_step", stream);
   if (dt == KDA_DTYPE_BF16) {

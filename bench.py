@@ -149,6 +149,7 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int, dev) -> float:
+    """The slowest rank's time (every rank gets it). Works with NCCL (cuda `dev`) and gloo (cpu)."""
     if world == 1:
         return x
     import torch
@@ -157,6 +158,12 @@ def max_over_ranks(x: float, world: int, dev) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank processes `units_per_rank`; the job's rate is all units over the
+    slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 def timed(fn, steps, warmup, world, dev):
@@ -390,7 +397,7 @@ def main():
     clocks = clk.summary() if rank == 0 else None
     ms_step = pre["ms"] / args.steps
     tokens = spec.total_tokens
-    value = world * tokens * args.steps / (pre["ms"] / 1e3)
+    value = whole_job_rate(tokens * args.steps, world, pre["ms"])
 
     # roofline of the dominant kernel
     prof = pre["prof"]

@@ -31,7 +31,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 # every symbol include/kda.h declares
 ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
-               "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc")
+               "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
+               "kda_recurrent_fwd")
 
 
 class ProfileEntry(ctypes.Structure):
@@ -72,6 +73,9 @@ def lib() -> ctypes.CDLL:
             L.kda_recurrent_step.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i32,
                                              i32, i32, vp]
             L.kda_recurrent_step.restype = ctypes.c_int
+            L.kda_recurrent_fwd.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, i32,
+                                            i32, i32, i32, i32, i32, vp]
+            L.kda_recurrent_fwd.restype = ctypes.c_int
             L.kda_last_device_error.argtypes = [vp]
             L.kda_last_device_error.restype = ctypes.c_int
             L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32,
@@ -194,6 +198,36 @@ def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
                                     _ptr(beta), _ptr(state), _ptr(o), N, H, Dk, Dv,
                                     _stream_handle(dev))
     _check(code, "kda_recurrent_step")
+    return o
+
+
+def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, o=None):
+    """Token-by-token KDA over short sequences with states from a pool (serving-cache layout).
+
+    q, k [N,T,H,Dk], v [N,T,H,Dv] (bf16 or fp32); log_alpha [N,T,H,Dk] fp32; beta [N,T,H] fp32;
+    state_pool [P,H,Dk,Dv] fp32 updated in place; state_indices int32 [N] on the device (negative
+    entries skip their sequence) or None for pool rows 0..N-1. Returns o [N,T,H,Dv]."""
+    dev = q.device
+    N, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, q.dtype)
+    _need(log_alpha, "log_alpha", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    _need(state_pool, "state_pool", dev, torch.float32)
+    P = state_pool.shape[0]
+    if tuple(state_pool.shape[1:]) != (H, Dk, Dv):
+        raise ValueError("state_pool must be [P,H,Dk,Dv]")
+    if state_indices is not None:
+        _need(state_indices, "state_indices", dev, torch.int32)
+        if state_indices.numel() != N:
+            raise ValueError("state_indices must have N entries")
+    if o is None:
+        o = torch.empty((N, T, H, Dv), dtype=q.dtype, device=dev)
+    code = lib().kda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
+                                   _ptr(beta), _ptr(state_pool), _ptr(state_indices), _ptr(o), N,
+                                   T, H, Dk, Dv, P, _stream_handle(dev))
+    _check(code, "kda_recurrent_fwd")
     return o
 
 

@@ -183,6 +183,28 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda
                                       (cudaStream_t)stream));
 }
 
+kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                               const float* log_alpha, const float* beta, float* pool,
+                               const int32_t* state_indices, void* o, int32_t N, int32_t T,
+                               int32_t H, int32_t Dk, int32_t Dv, int32_t P,
+                               kda_stream_t stream) {
+  if (N < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0 || P < 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > INT32_MAX || (long long)N * T * H * (Dk > Dv ? Dk : Dv) > (1LL << 40))
+    return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H * T == 0) return KDA_OK;
+  if (!state_indices && P < N) return KDA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !log_alpha || !beta || !pool || !o) return KDA_ERR_INVALID_ARG;
+  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+  if (!aligned(pool, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
+      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
+      (state_indices && !aligned(state_indices, 4)))
+    return KDA_ERR_INVALID_ARG;
+  return from_cuda(launch_recurrent_multi(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N,
+                                          T, H, Dk, Dv, P, (cudaStream_t)stream));
+}
+
 kda_status_t kda_last_device_error(kda_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return KDA_ERR_CUDA;

@@ -18,7 +18,7 @@ namespace kda {
 __device__ unsigned int g_status = 0;  // one definition: the library is a single TU
 
 enum : unsigned int {
-  kStatusBadSeqlens = 1u << 0,
+  kStatusBadSeqlens = 1u << 0,  // also: a state index beyond the pool
   kStatusTimeout = 1u << 1,
 };
 

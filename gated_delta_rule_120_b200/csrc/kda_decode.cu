@@ -145,6 +145,141 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Multi-token recurrent variant: one CTA per (sequence, head) applies T tokens to a state that
+// stays in registers (same thread layout as above); the next token's vectors are fetched while
+// the current one is processed. Two block-wide barriers per token (cross-warp reductions).
+// ---------------------------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    recurrent_multi_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                           const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                           const float* __restrict__ beta, float* __restrict__ pool,
+                           const int32_t* __restrict__ state_indices, Tin* __restrict__ o, int T,
+                           int H, int Dk, int Dv, int P) {
+  __shared__ float s_a[128], s_k[128], s_q[128];
+  __shared__ float4 s_e[8][32], s_p[8][32];
+  __shared__ float s_kq[4];
+
+  const int nh = blockIdx.x;
+  const int n = nh / H, h = nh - n * H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int slot = state_indices ? state_indices[n] : n;
+  if (slot < 0) return;  // padding entry of the batch
+  if (slot >= P) {
+    if (tid == 0) raise_status(kStatusBadSeqlens);
+    return;
+  }
+
+  const int col = lane * 4;
+  const bool col_ok = col < Dv;
+  float4* Srow = reinterpret_cast<float4*>(pool + ((size_t)slot * H + h) * Dk * Dv) + (col >> 2);
+  const int row0 = warp * kDecRowsPerWarp;
+  const int vstride = Dv >> 2;
+  float4 s[kDecRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kDecRowsPerWarp; ++i) {
+    const int r = row0 + i;
+    s[i] = (col_ok && r < Dk) ? Srow[(size_t)r * vstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  // per-token vectors: threads 0..127 hold one key channel, lanes hold 4 value columns
+  auto vec_base = [&](int t) { return (((size_t)n * T + t) * H + h); };
+  float la_n = 0.f, k_n = 0.f, q_n = 0.f, b_n = 0.f;
+  float4 v_n = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto fetch = [&](int t) {
+    const size_t base = vec_base(t);
+    if (tid < Dk) {
+      la_n = log_alpha[base * Dk + tid];
+      k_n = to_f32(k[base * Dk + tid]);
+      q_n = to_f32(q[base * Dk + tid]);
+    }
+    if (col_ok) {
+      const Tin* vp = v + base * Dv + col;
+      v_n = make_float4(to_f32(vp[0]), to_f32(vp[1]), to_f32(vp[2]), to_f32(vp[3]));
+    }
+    b_n = beta[base];
+  };
+  if (T > 0) fetch(0);
+  for (int t = 0; t < T; ++t) {
+    const float la_c = la_n, k_c = k_n, q_c = q_n, b = b_n;
+    const float4 vc = v_n;
+    if (tid < 128) {
+      const bool in = tid < Dk;
+      s_a[tid] = in ? expf(la_c) : 1.f;
+      s_k[tid] = in ? k_c : 0.f;
+      s_q[tid] = in ? q_c : 0.f;
+      float kq = in ? k_c * q_c : 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      if (lane == 0) s_kq[warp] = kq;
+    }
+    if (t + 1 < T) fetch(t + 1);  // in flight while this token is processed
+    __syncthreads();
+    float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
+#pragma unroll
+    for (int i = 0; i < kDecRowsPerWarp; ++i) {
+      const int r = row0 + i;
+      const float a = s_a[r], kr = s_k[r], qr = s_q[r];
+      s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+      e.x += s[i].x * kr; e.y += s[i].y * kr; e.z += s[i].z * kr; e.w += s[i].w * kr;
+      p.x += s[i].x * qr; p.y += s[i].y * qr; p.z += s[i].z * qr; p.w += s[i].w * qr;
+    }
+    s_e[warp][lane] = e;
+    s_p[warp][lane] = p;
+    __syncthreads();
+    e = make_float4(0.f, 0.f, 0.f, 0.f);
+    p = e;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float4 ew = s_e[w][lane], pw = s_p[w][lane];
+      e.x += ew.x; e.y += ew.y; e.z += ew.z; e.w += ew.w;
+      p.x += pw.x; p.y += pw.y; p.z += pw.z; p.w += pw.w;
+    }
+    const float kq = s_kq[0] + s_kq[1] + s_kq[2] + s_kq[3];
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (col_ok) {
+      u.x = b * (vc.x - e.x); u.y = b * (vc.y - e.y); u.z = b * (vc.z - e.z); u.w = b * (vc.w - e.w);
+    }
+#pragma unroll
+    for (int i = 0; i < kDecRowsPerWarp; ++i) {
+      const float kr = s_k[row0 + i];
+      s[i].x += kr * u.x; s[i].y += kr * u.y; s[i].z += kr * u.z; s[i].w += kr * u.w;
+    }
+    if (warp == 0 && col_ok) {
+      Tin* op = o + vec_base(t) * Dv + col;
+      op[0] = from_f32<Tin>(p.x + kq * u.x);
+      op[1] = from_f32<Tin>(p.y + kq * u.y);
+      op[2] = from_f32<Tin>(p.z + kq * u.z);
+      op[3] = from_f32<Tin>(p.w + kq * u.w);
+    }
+    __syncthreads();  // s_a / s_k / s_q / s_e / s_p are rewritten by the next token
+  }
+#pragma unroll
+  for (int i = 0; i < kDecRowsPerWarp; ++i) {
+    const int r = row0 + i;
+    if (col_ok && r < Dk) Srow[(size_t)r * vstride] = s[i];
+  }
+}
+
+cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                   const float* log_alpha, const float* beta, float* pool,
+                                   const int32_t* idx, void* o, int N, int T, int H, int Dk,
+                                   int Dv, int P, cudaStream_t stream) {
+  const long long heads = (long long)N * H;
+  if (heads == 0 || T == 0) return cudaSuccess;
+  ProfileScope prof("recurrent_multi", stream);
+  if (dt == KDA_DTYPE_BF16)
+    recurrent_multi_kernel<__nv_bfloat16><<<(unsigned)heads, kDecThreads, 0, stream>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha, beta,
+        pool, idx, (__nv_bfloat16*)o, T, H, Dk, Dv, P);
+  else
+    recurrent_multi_kernel<float><<<(unsigned)heads, kDecThreads, 0, stream>>>(
+        (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, pool, idx, (float*)o,
+        T, H, Dk, Dv, P);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------------
 // Streaming variant (used whenever the per-head vectors allow 16-byte bulk copies): one
 // persistent CTA per SM walks its heads through a three-stage shared-memory ring. A producer warp
 // bulk-loads a head's whole state plus its q, k, v and log-decay vectors ahead of use and bulk-

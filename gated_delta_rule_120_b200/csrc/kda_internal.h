@@ -79,6 +79,11 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_
                                const float* log_alpha, const float* beta, float* state, void* o,
                                int N, int H, int Dk, int Dv, cudaStream_t stream);
 
+cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                   const float* log_alpha, const float* beta, float* pool,
+                                   const int32_t* idx, void* o, int N, int T, int H, int Dk,
+                                   int Dv, int P, cudaStream_t stream);
+
 cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
                              int32_t* valid, cudaStream_t stream);
 

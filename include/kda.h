@@ -158,6 +158,31 @@ KDA_API kda_status_t kda_recurrent_step(const void* q, const void* k, const void
                                 int32_t N, int32_t H, int32_t Dk, int32_t Dv, kda_stream_t stream);
 
 /*
+ * kda_recurrent_fwd — token-by-token KDA over short sequences (the recurrent mode the walkthrough's
+ * §3.4 "FLOPs Accounting and Inference Strategy" uses for generation; the model card's code picks
+ * it for query lengths up to 64) with states taken from a pool, as a serving cache holds them.
+ * For each sequence n the T tokens are applied in order to state pool[state_indices[n]] (Eq. 1,
+ * o_t = S_t^T q_t); that state is read once, kept on chip for all T tokens and written once.
+ *
+ *   q, k            device [N, T, H, Dk], dtype qkv_dtype.
+ *   v, o            device [N, T, H, Dv], dtype qkv_dtype.
+ *   log_alpha       device fp32 [N, T, H, Dk]; beta device fp32 [N, T, H].
+ *   state_pool      device fp32 [P, H, Dk, Dv], updated in place; 16-byte aligned.
+ *   state_indices   device int32 [N]: pool row of sequence n. A negative entry skips the sequence
+ *                   (no state update, its o is left untouched). Entries must be distinct; an
+ *                   entry >= P is skipped too and reported as KDA_ERR_INVALID_ARG through
+ *                   kda_last_device_error(). NULL means pool row n (then P >= N is required).
+ * Supported: as kda_recurrent_step (1 <= Dk <= 128, 4 <= Dv <= 128, Dv % 4 == 0), T >= 0.
+ * For longer sequences kda_chunk_fwd is the faster path.
+ */
+KDA_API kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void* v,
+                                       kda_dtype_t qkv_dtype, const float* log_alpha,
+                                       const float* beta, float* state_pool,
+                                       const int32_t* state_indices, void* o, int32_t N, int32_t T,
+                                       int32_t H, int32_t Dk, int32_t Dv, int32_t P,
+                                       kda_stream_t stream);
+
+/*
  * kda_last_device_error — read and clear the per-device status word that the kernels set
  * (KDA_ERR_INVALID_ARG for a bad cu_seqlens, KDA_ERR_TIMEOUT for a bounded wait that gave up).
  * Synchronises `stream`. Returns KDA_OK when no kernel reported a fault.

@@ -32,7 +32,13 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
                "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
-               "kda_recurrent_fwd")
+               "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused")
+
+
+class Fusion(ctypes.Structure):
+    """kda_fusion_t: in-kernel q/k L2 normalisation and the fused log-space decay gate."""
+    _fields_ = [("qk_l2norm", ctypes.c_int32), ("qk_l2norm_eps", ctypes.c_float),
+                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
 
 
 class ProfileEntry(ctypes.Structure):
@@ -76,6 +82,14 @@ def lib() -> ctypes.CDLL:
             L.kda_recurrent_fwd.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, i32,
                                             i32, i32, i32, i32, i32, vp]
             L.kda_recurrent_fwd.restype = ctypes.c_int
+            L.kda_chunk_fwd_fused.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i32,
+                                              i32, i32, i32, i32, i32, vp, vp, vp, sz,
+                                              ctypes.POINTER(Fusion), vp]
+            L.kda_chunk_fwd_fused.restype = ctypes.c_int
+            L.kda_recurrent_fwd_fused.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp,
+                                                  i32, i32, i32, i32, i32, i32,
+                                                  ctypes.POINTER(Fusion), vp]
+            L.kda_recurrent_fwd_fused.restype = ctypes.c_int
             L.kda_last_device_error.argtypes = [vp]
             L.kda_last_device_error.restype = ctypes.c_int
             L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32,
@@ -136,13 +150,34 @@ def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, chunk
     return int(out.value)
 
 
+def _fusion(fusion, dev, H, Dk):
+    """dict(qk_l2norm=bool, eps=float, A_log=[H] fp32, dt_bias=[H,Dk] fp32) -> kda_fusion_t."""
+    if fusion is None:
+        return None
+    A_log, dt_bias = fusion.get("A_log"), fusion.get("dt_bias")
+    if A_log is not None:
+        _need(A_log, "A_log", dev, torch.float32)
+        if A_log.numel() != H:
+            raise ValueError("A_log must have H entries")
+    if dt_bias is not None:
+        _need(dt_bias, "dt_bias", dev, torch.float32)
+        if dt_bias.numel() != H * Dk:
+            raise ValueError("dt_bias must be [H, Dk]")
+    return Fusion(1 if fusion.get("qk_l2norm") else 0, float(fusion.get("eps", 1e-6)),
+                  None if A_log is None else A_log.data_ptr(),
+                  None if dt_bias is None else dt_bias.data_ptr())
+
+
 def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
-                  output_final_state: bool = True, o=None, final_state=None, workspace=None):
+                  output_final_state: bool = True, o=None, final_state=None, workspace=None,
+                  fusion=None):
     """Chunkwise KDA prefill.
 
     q, k [B,T,H,Dk], v [B,T,H,Dv] (bf16 or fp32, same dtype); log_alpha [B,T,H,Dk] fp32;
     beta [B,T,H] fp32; initial_state [N,H,Dk,Dv] fp32 or None; cu_seqlens int32 [N+1] on the
     device or None (then N = B). Returns (o [B,T,H,Dv] in the input dtype, final_state or None).
+    ``fusion`` (dict, optional): qk_l2norm / eps normalise q and k in-kernel; A_log [H] and
+    dt_bias [H,Dk] turn ``log_alpha`` (then the raw gate) into -exp(A_log) * softplus(g + dt_bias).
     """
     dev = q.device
     B, T, H, Dk = q.shape
@@ -170,11 +205,14 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     ws_bytes = kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, N, q.dtype)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    code = lib().kda_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
-        _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
-        _ptr(final_state if output_final_state else None), _ptr(workspace),
-        workspace.numel(), _stream_handle(dev))
+    fz = _fusion(fusion, dev, H, Dk)
+    args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+            _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
+            _ptr(final_state if output_final_state else None), _ptr(workspace), workspace.numel())
+    if fz is None:
+        code = lib().kda_chunk_fwd(*args, _stream_handle(dev))
+    else:
+        code = lib().kda_chunk_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_chunk_fwd")
     return o, (final_state if output_final_state else None)
 
@@ -201,7 +239,8 @@ def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
     return o
 
 
-def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, o=None):
+def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, o=None,
+                      fusion=None):
     """Token-by-token KDA over short sequences with states from a pool (serving-cache layout).
 
     q, k [N,T,H,Dk], v [N,T,H,Dv] (bf16 or fp32); log_alpha [N,T,H,Dk] fp32; beta [N,T,H] fp32;
@@ -224,9 +263,13 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, 
             raise ValueError("state_indices must have N entries")
     if o is None:
         o = torch.empty((N, T, H, Dv), dtype=q.dtype, device=dev)
-    code = lib().kda_recurrent_fwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
-                                   _ptr(beta), _ptr(state_pool), _ptr(state_indices), _ptr(o), N,
-                                   T, H, Dk, Dv, P, _stream_handle(dev))
+    fz = _fusion(fusion, dev, H, Dk)
+    args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+            _ptr(state_pool), _ptr(state_indices), _ptr(o), N, T, H, Dk, Dv, P)
+    if fz is None:
+        code = lib().kda_recurrent_fwd(*args, _stream_handle(dev))
+    else:
+        code = lib().kda_recurrent_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_recurrent_fwd")
     return o
 

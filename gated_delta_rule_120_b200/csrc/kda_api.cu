@@ -98,11 +98,31 @@ kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32
   return KDA_OK;
 }
 
-kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t dt,
-                           const float* log_alpha, const float* beta, const float* initial_state,
-                           const int32_t* cu_seqlens, int32_t N, int32_t B, int32_t T, int32_t H,
-                           int32_t Dk, int32_t Dv, int32_t C, void* o, float* final_state,
-                           void* workspace, size_t workspace_bytes, kda_stream_t stream_) {
+}  // extern "C"
+
+namespace kda {
+namespace {
+
+// Validates a fusion descriptor (NULL = no fusion) and converts it.
+kda_status_t to_fusion(const kda_fusion_t* f, Fusion* out) {
+  *out = Fusion();
+  if (!f) return KDA_OK;
+  if (f->qk_l2norm && !(f->qk_l2norm_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+  if ((f->A_log && !aligned(f->A_log, 4)) || (f->dt_bias && !aligned(f->dt_bias, 4)))
+    return KDA_ERR_INVALID_ARG;
+  out->l2 = f->qk_l2norm ? 1 : 0;
+  out->eps = f->qk_l2norm_eps;
+  out->A_log = f->A_log;
+  out->dt_bias = f->A_log ? f->dt_bias : nullptr;
+  return KDA_OK;
+}
+
+kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                            const float* log_alpha, const float* beta, const float* initial_state,
+                            const int32_t* cu_seqlens, int32_t N, int32_t B, int32_t T, int32_t H,
+                            int32_t Dk, int32_t Dv, int32_t C, void* o, float* final_state,
+                            void* workspace, size_t workspace_bytes, const Fusion& fz,
+                            kda_stream_t stream_) {
   const bool varlen = cu_seqlens != nullptr;
   kda_status_t st = check_prefill_shape(B, T, H, Dk, Dv, C, N, dt, varlen);
   if (st != KDA_OK) return st;
@@ -156,6 +176,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtyp
   a.C = C;
   a.o = o;
   a.final_state = final_state;
+  a.fz = fz;
 
   if (is_tc_path(dt))
     return from_cuda(launch_prefill_tc(a, geo, (int)lay.max_chunks, (uint8_t*)(ws + lay.rec_base),
@@ -163,6 +184,56 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtyp
   const SimtRecord rec = SimtRecord::make(C, Dk, Dv);
   return from_cuda(launch_prefill_simt(a, geo, (int)lay.max_chunks,
                                        (float*)(ws + lay.rec_base), rec, stream));
+}
+
+kda_status_t recurrent_fwd_impl(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                const float* log_alpha, const float* beta, float* pool,
+                                const int32_t* state_indices, void* o, int32_t N, int32_t T,
+                                int32_t H, int32_t Dk, int32_t Dv, int32_t P, const Fusion& fz,
+                                kda_stream_t stream) {
+  if (N < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0 || P < 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > INT32_MAX || (long long)N * T * H * (Dk > Dv ? Dk : Dv) > (1LL << 40))
+    return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H * T == 0) return KDA_OK;
+  if (!state_indices && P < N) return KDA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !log_alpha || !beta || !pool || !o) return KDA_ERR_INVALID_ARG;
+  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+  if (!aligned(pool, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
+      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
+      (state_indices && !aligned(state_indices, 4)))
+    return KDA_ERR_INVALID_ARG;
+  return from_cuda(launch_recurrent_multi(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N,
+                                          T, H, Dk, Dv, P, fz, (cudaStream_t)stream));
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                           const float* log_alpha, const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t N, int32_t B, int32_t T, int32_t H,
+                           int32_t Dk, int32_t Dv, int32_t C, void* o, float* final_state,
+                           void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  return chunk_fwd_impl(q, k, v, dt, log_alpha, beta, initial_state, cu_seqlens, N, B, T, H, Dk,
+                        Dv, C, o, final_state, workspace, workspace_bytes, Fusion(), stream);
+}
+
+kda_status_t kda_chunk_fwd_fused(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                 const float* log_alpha_or_gate, const float* beta,
+                                 const float* initial_state, const int32_t* cu_seqlens, int32_t N,
+                                 int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                 int32_t C, void* o, float* final_state, void* workspace,
+                                 size_t workspace_bytes, const kda_fusion_t* fusion,
+                                 kda_stream_t stream) {
+  Fusion fz;
+  const kda_status_t st = to_fusion(fusion, &fz);
+  if (st != KDA_OK) return st;
+  return chunk_fwd_impl(q, k, v, dt, log_alpha_or_gate, beta, initial_state, cu_seqlens, N, B, T,
+                        H, Dk, Dv, C, o, final_state, workspace, workspace_bytes, fz, stream);
 }
 
 kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
@@ -188,21 +259,20 @@ kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void* v, kda_
                                const int32_t* state_indices, void* o, int32_t N, int32_t T,
                                int32_t H, int32_t Dk, int32_t Dv, int32_t P,
                                kda_stream_t stream) {
-  if (N < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0 || P < 0) return KDA_ERR_INVALID_ARG;
-  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
-  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
-  if ((long long)N * H > INT32_MAX || (long long)N * T * H * (Dk > Dv ? Dk : Dv) > (1LL << 40))
-    return KDA_ERR_UNSUPPORTED;
-  if ((long long)N * H * T == 0) return KDA_OK;
-  if (!state_indices && P < N) return KDA_ERR_INVALID_ARG;
-  if (!q || !k || !v || !log_alpha || !beta || !pool || !o) return KDA_ERR_INVALID_ARG;
-  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
-  if (!aligned(pool, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
-      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
-      (state_indices && !aligned(state_indices, 4)))
-    return KDA_ERR_INVALID_ARG;
-  return from_cuda(launch_recurrent_multi(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N,
-                                          T, H, Dk, Dv, P, (cudaStream_t)stream));
+  return recurrent_fwd_impl(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N, T, H, Dk, Dv,
+                            P, Fusion(), stream);
+}
+
+kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                     const float* log_alpha_or_gate, const float* beta,
+                                     float* pool, const int32_t* state_indices, void* o,
+                                     int32_t N, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                     int32_t P, const kda_fusion_t* fusion, kda_stream_t stream) {
+  Fusion fz;
+  const kda_status_t st = to_fusion(fusion, &fz);
+  if (st != KDA_OK) return st;
+  return recurrent_fwd_impl(q, k, v, dt, log_alpha_or_gate, beta, pool, state_indices, o, N, T, H,
+                            Dk, Dv, P, fz, stream);
 }
 
 kda_status_t kda_last_device_error(kda_stream_t stream) {

@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     chunk_local_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                             const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                             const float* __restrict__ beta, SeqGeometry geo, int H, int Dk, int Dv,
-                            float* __restrict__ ws, SimtRecord rec) {
+                            float* __restrict__ ws, SimtRecord rec, Fusion fz) {
   extern __shared__ float smem[];
   const int C = geo.C;
   float* sk = smem;            // [C][Dk]  k, later Gamma.K
@@ -105,13 +105,17 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
   float* out = ws + rec.record_floats * ((size_t)c * H + h);
 
+  const float neg_a = fz.A_log ? -expf(fz.A_log[h]) : 0.f;
   for (int idx = tid; idx < C * Dk; idx += nt) {
     const int r = idx / Dk, cc = idx - r * Dk;
     const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + cc;
     const bool in = r < L;
     sk[idx] = in ? to_f32(k[gi]) : 0.f;
     sq[idx] = in ? to_f32(q[gi]) : 0.f;
-    sg[idx] = in ? log_alpha[gi] : 0.f;
+    float la = in ? log_alpha[gi] : 0.f;
+    if (fz.A_log && in)  // fused gate: raw gate -> log decay
+      la = neg_a * softplus_f(la + (fz.dt_bias ? fz.dt_bias[h * Dk + cc] : 0.f));
+    sg[idx] = la;
   }
   for (int idx = tid; idx < C * Dv; idx += nt) {
     const int r = idx / Dv, cc = idx - r * Dv;
@@ -119,6 +123,26 @@ __global__ void __launch_bounds__(kSimtThreads)
   }
   for (int r = tid; r < C; r += nt) sb[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
   __syncthreads();
+  if (fz.l2) {  // fused L2 norm of q and k rows (one warp per row)
+    for (int r = warp; r < C; r += nt / 32) {
+      float ssk = 0.f, ssq = 0.f;
+      for (int cc = lane; cc < Dk; cc += 32) {
+        ssk += sk[r * Dk + cc] * sk[r * Dk + cc];
+        ssq += sq[r * Dk + cc] * sq[r * Dk + cc];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+      }
+      const float ik = rsqrtf(ssk + fz.eps), iq = rsqrtf(ssq + fz.eps);
+      for (int cc = lane; cc < Dk; cc += 32) {
+        sk[r * Dk + cc] *= ik;
+        sq[r * Dk + cc] *= iq;
+      }
+    }
+    __syncthreads();
+  }
 
   // g_r = sum_{j<=r} log alpha_j, per key channel
   for (int cc = tid; cc < Dk; cc += nt) {
@@ -332,7 +356,7 @@ static cudaError_t launch_simt_typed(const PrefillArgs& a, const SeqGeometry& ge
     ProfileScope prof("chunk_local_simt", stream);
     chunk_local_simt_kernel<Tin><<<g1, kSimtThreads, sm1, stream>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
-        a.Dv, records, rec);
+        a.Dv, records, rec, a.fz);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     chunk_local_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                           const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
                           const float* __restrict__ beta, SeqGeometry geo, int H,
-                          uint8_t* __restrict__ ws_records) {
+                          uint8_t* __restrict__ ws_records, Fusion fz) {
   extern __shared__ uint8_t smem_raw[];
   if (!geo.ok()) return;
   const int c = blockIdx.x, h = blockIdx.y;
@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   float* sBeta = reinterpret_cast<float*>(sm + kS1Beta);
   float* sGC = reinterpret_cast<float*>(sm + kS1GC);
   float* sScan = reinterpret_cast<float*>(sm + kS1Ki);  // [16][128], before K/Gamma exists
+  float* sInv = reinterpret_cast<float*>(sm + kS1M);   // [2][64] inverse norms, until phase 4
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kS1Bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS1Tmem);
 
@@ -203,6 +204,17 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     }
   }
   if (tid < kC) sBeta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+  if (fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log decays
+    const float neg_a = -expf(fz.A_log[h]);
+    float bias[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) bias[j] = fz.dt_bias ? fz.dt_bias[h * kD + cg * 8 + j] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (rg * 4 + i < L)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g[i][j] = neg_a * softplus_f(g[i][j] + bias[j]);
+  }
 #pragma unroll
   for (int i = 1; i < 4; ++i)
 #pragma unroll
@@ -260,6 +272,29 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     float kf[8], qf[8];
     unpack8(ld_shared_v4(sb + kS1Kg + off), kf);
     unpack8(ld_shared_v4(sb + kS1Qg + off), qf);
+    if (fz.l2) {  // fused L2 norm: the 16 lanes holding this row reduce its sums of squares
+      float ssk = 0.f, ssq = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ssk += kf[j] * kf[j];
+        ssq += qf[j] * qf[j];
+      }
+#pragma unroll
+      for (int off2 = 1; off2 < 16; off2 <<= 1) {
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, off2);
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, off2);
+      }
+      const float ik = rsqrtf(ssk + fz.eps), iq = rsqrtf(ssq + fz.eps);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        kf[j] *= ik;
+        qf[j] *= iq;
+      }
+      if (cg == 0) {  // for the exact fallback, which re-reads k and q from global memory
+        sInv[r] = ik;
+        sInv[64 + r] = iq;
+      }
+    }
     float kg[8], ki[8], kt[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -364,6 +399,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       for (int off = 16; off > 0; off >>= 1) {
         akk += __shfl_xor_sync(0xffffffffu, akk, off);
         aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
+      }
+      if (fz.l2) {
+        akk *= sInv[r] * sInv[i];
+        aqk *= sInv[64 + r] * sInv[i];
       }
       if (lane == 0) {
         sA[sidx(r, i)] = (i < r) ? sBeta[r] * akk : 0.f;
@@ -824,7 +863,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
     ProfileScope prof("chunk_local_tc", stream);
     tc::chunk_local_tc_kernel<<<dim3(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-        a.log_alpha, a.beta, geo, a.H, records);
+        a.log_alpha, a.beta, geo, a.H, records, a.fz);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

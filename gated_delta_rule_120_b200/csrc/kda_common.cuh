@@ -50,6 +50,9 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// log(1 + exp(x)) without overflow.
+__device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
 __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) {
   return (x + a - 1) / a * a;
 }

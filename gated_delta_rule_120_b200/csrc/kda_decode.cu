@@ -155,10 +155,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                            const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                            const float* __restrict__ beta, float* __restrict__ pool,
                            const int32_t* __restrict__ state_indices, Tin* __restrict__ o, int T,
-                           int H, int Dk, int Dv, int P) {
+                           int H, int Dk, int Dv, int P, Fusion fz) {
   __shared__ float s_a[128], s_k[128], s_q[128];
   __shared__ float4 s_e[8][32], s_p[8][32];
-  __shared__ float s_kq[4];
+  __shared__ float s_kq[4], s_ssk[4], s_ssq[4];
 
   const int nh = blockIdx.x;
   const int n = nh / H, h = nh - n * H;
@@ -186,10 +186,13 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   auto vec_base = [&](int t) { return (((size_t)n * T + t) * H + h); };
   float la_n = 0.f, k_n = 0.f, q_n = 0.f, b_n = 0.f;
   float4 v_n = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float neg_a = fz.A_log ? -expf(fz.A_log[h]) : 0.f;
+  const float bias_c = (fz.A_log && fz.dt_bias && tid < Dk) ? fz.dt_bias[h * Dk + tid] : 0.f;
   auto fetch = [&](int t) {
     const size_t base = vec_base(t);
     if (tid < Dk) {
       la_n = log_alpha[base * Dk + tid];
+      if (fz.A_log) la_n = neg_a * softplus_f(la_n + bias_c);  // fused gate
       k_n = to_f32(k[base * Dk + tid]);
       q_n = to_f32(q[base * Dk + tid]);
     }
@@ -209,9 +212,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       s_k[tid] = in ? k_c : 0.f;
       s_q[tid] = in ? q_c : 0.f;
       float kq = in ? k_c * q_c : 0.f;
+      float ssk = in ? k_c * k_c : 0.f, ssq = in ? q_c * q_c : 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-      if (lane == 0) s_kq[warp] = kq;
+      for (int off = 16; off > 0; off >>= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+        ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+      }
+      if (lane == 0) {
+        s_kq[warp] = kq;
+        s_ssk[warp] = ssk;
+        s_ssq[warp] = ssq;
+      }
     }
     if (t + 1 < T) fetch(t + 1);  // in flight while this token is processed
     __syncthreads();
@@ -235,14 +247,22 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       e.x += ew.x; e.y += ew.y; e.z += ew.z; e.w += ew.w;
       p.x += pw.x; p.y += pw.y; p.z += pw.z; p.w += pw.w;
     }
-    const float kq = s_kq[0] + s_kq[1] + s_kq[2] + s_kq[3];
+    float kq = s_kq[0] + s_kq[1] + s_kq[2] + s_kq[3];
+    float ik = 1.f;
+    if (fz.l2) {  // fused L2 norm, applied to the reductions rather than to the state pass
+      ik = rsqrtf(s_ssk[0] + s_ssk[1] + s_ssk[2] + s_ssk[3] + fz.eps);
+      const float iq = rsqrtf(s_ssq[0] + s_ssq[1] + s_ssq[2] + s_ssq[3] + fz.eps);
+      e.x *= ik; e.y *= ik; e.z *= ik; e.w *= ik;
+      p.x *= iq; p.y *= iq; p.z *= iq; p.w *= iq;
+      kq *= ik * iq;
+    }
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
     if (col_ok) {
       u.x = b * (vc.x - e.x); u.y = b * (vc.y - e.y); u.z = b * (vc.z - e.z); u.w = b * (vc.w - e.w);
     }
 #pragma unroll
     for (int i = 0; i < kDecRowsPerWarp; ++i) {
-      const float kr = s_k[row0 + i];
+      const float kr = s_k[row0 + i] * ik;
       s[i].x += kr * u.x; s[i].y += kr * u.y; s[i].z += kr * u.z; s[i].w += kr * u.w;
     }
     if (warp == 0 && col_ok) {
@@ -264,18 +284,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                    const float* log_alpha, const float* beta, float* pool,
                                    const int32_t* idx, void* o, int N, int T, int H, int Dk,
-                                   int Dv, int P, cudaStream_t stream) {
+                                   int Dv, int P, const Fusion& fz, cudaStream_t stream) {
   const long long heads = (long long)N * H;
   if (heads == 0 || T == 0) return cudaSuccess;
   ProfileScope prof("recurrent_multi", stream);
   if (dt == KDA_DTYPE_BF16)
     recurrent_multi_kernel<__nv_bfloat16><<<(unsigned)heads, kDecThreads, 0, stream>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha, beta,
-        pool, idx, (__nv_bfloat16*)o, T, H, Dk, Dv, P);
+        pool, idx, (__nv_bfloat16*)o, T, H, Dk, Dv, P, fz);
   else
     recurrent_multi_kernel<float><<<(unsigned)heads, kDecThreads, 0, stream>>>(
         (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, pool, idx, (float*)o,
-        T, H, Dk, Dv, P);
+        T, H, Dk, Dv, P, fz);
   return cudaGetLastError();
 }
 

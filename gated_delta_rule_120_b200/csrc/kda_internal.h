@@ -26,6 +26,14 @@ class ProfileScope {
   bool active_ = false;
 };
 
+// Prologue fusion (see kda_fusion_t): in-kernel q/k L2 normalisation and the log-space gate.
+struct Fusion {
+  int l2 = 0;
+  float eps = 0.f;
+  const float* A_log = nullptr;    // [H]; non-null: the decay input is the raw gate
+  const float* dt_bias = nullptr;  // [H, Dk] or null
+};
+
 // Arguments of one kda_chunk_fwd call after host validation.
 struct PrefillArgs {
   const void* q;
@@ -39,6 +47,7 @@ struct PrefillArgs {
   int N, B, T, H, Dk, Dv, C;
   void* o;
   float* final_state;
+  Fusion fz;
 };
 
 // Per (chunk, head) record of the fp32 CUDA-core path, in floats:
@@ -82,7 +91,7 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_
 cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                    const float* log_alpha, const float* beta, float* pool,
                                    const int32_t* idx, void* o, int N, int T, int H, int Dk,
-                                   int Dv, int P, cudaStream_t stream);
+                                   int Dv, int P, const Fusion& fz, cudaStream_t stream);
 
 cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
                              int32_t* valid, cudaStream_t stream);

@@ -183,6 +183,43 @@ KDA_API kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void*
                                        kda_stream_t stream);
 
 /*
+ * Prologue fusion for the two steps that precede the operator in the model ("Kimi Linear: An
+ * Expressive, Efficient Attention Architecture", paper-graph-ui walkthrough, §3.4 "Neural
+ * Parameterization": q, k = L2Norm(...) and alpha = f(low-rank gate); the L2 Deep Distill page's
+ * implementation notes: L2 normalisation of q and k inside the kernel, and the decay gate fused
+ * with A_log and a bias). The pages leave f unspecified beyond "similar to GDN and Mamba2, in log
+ * space"; this library reads it as
+ *     log alpha[t, h, c] = -exp(A_log[h]) * softplus(g[t, h, c] + dt_bias[h, c]).
+ */
+typedef struct {
+  int32_t qk_l2norm;     /* nonzero: q and k are divided by sqrt(sum x^2 + qk_l2norm_eps) per
+                            (token, head) inside the kernels */
+  float qk_l2norm_eps;   /* e.g. 1e-6 */
+  const float* A_log;    /* device fp32 [H], or NULL. Non-NULL: the log_alpha argument holds the
+                            raw gate g (same layout) and the decay is computed as above */
+  const float* dt_bias;  /* device fp32 [H, Dk], or NULL for a zero bias; used only with A_log */
+} kda_fusion_t;
+
+/* kda_chunk_fwd with the prologue fusion above; fusion == NULL is exactly kda_chunk_fwd. */
+KDA_API kda_status_t kda_chunk_fwd_fused(const void* q, const void* k, const void* v,
+                                         kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,
+                                         const float* beta, const float* initial_state,
+                                         const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                                         int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                         int32_t chunk, void* o, float* final_state,
+                                         void* workspace, size_t workspace_bytes,
+                                         const kda_fusion_t* fusion, kda_stream_t stream);
+
+/* kda_recurrent_fwd with the prologue fusion above; fusion == NULL is exactly kda_recurrent_fwd. */
+KDA_API kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const void* v,
+                                             kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,
+                                             const float* beta, float* state_pool,
+                                             const int32_t* state_indices, void* o, int32_t N,
+                                             int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                             int32_t P, const kda_fusion_t* fusion,
+                                             kda_stream_t stream);
+
+/*
  * kda_last_device_error — read and clear the per-device status word that the kernels set
  * (KDA_ERR_INVALID_ARG for a bad cu_seqlens, KDA_ERR_TIMEOUT for a bounded wait that gave up).
  * Synchronises `stream`. Returns KDA_OK when no kernel reported a fault.

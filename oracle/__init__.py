@@ -13,6 +13,10 @@ Functions
   chunked(...)             the chunkwise WY/UT evaluation of §3.4 "Chunkwise Parallelization"
                            (Eq. 8, Eq. 9), fp64; pins the chunk algebra against ``recurrent``.
   unit_lower_inverse(A)    (I + A)^{-1} by forward substitution (the UT transform's inverse).
+  prologue(...)            the fused input steps: L2-normalised q, k and the log-space decay gate
+                           log alpha = -exp(A_log[h]) * softplus(g + dt_bias[h, c]) (walkthrough
+                           §3.4 "Neural Parameterization"; the L2 Deep Distill page's
+                           implementation notes on the in-kernel L2 norm and the fused gate).
 
 All inputs follow the packed layout [T_total, H, D] with int64 ``cu_seqlens`` [N+1]; a batch of B
 equal-length sequences is the same memory as [B, T, H, D] with cu_seqlens = [0, T, 2T, ...].
@@ -158,3 +162,24 @@ def unit_lower_inverse(A) -> np.ndarray:
     X = np.zeros((C, C), dtype=np.float64)
     _load().kda_oracle_unit_lower_inverse(_ptr(A), C, _ptr(X))
     return X
+
+
+def _softplus(x: np.ndarray) -> np.ndarray:
+    """log(1 + exp(x)), evaluated without overflow for large x."""
+    return np.where(x > 30.0, x, np.log1p(np.exp(np.minimum(x, 30.0))))
+
+
+def prologue(q, k, log_alpha_or_gate, A_log=None, dt_bias=None, qk_l2norm=False, eps=1e-6):
+    """fp64 (q', k', log_alpha') after the optional in-kernel steps: q, k divided by
+    sqrt(sum x^2 + eps) over the key channels of each (token, head); and, when A_log is given,
+    log_alpha' = -exp(A_log[h]) * softplus(g + dt_bias[h, c]) with g = log_alpha_or_gate.
+    Arrays keep their shapes (..., H, Dk)."""
+    q, k, g = _f64(q), _f64(k), _f64(log_alpha_or_gate)
+    if qk_l2norm:
+        q = q / np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + eps)
+        k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + eps)
+    if A_log is not None:
+        a = np.exp(_f64(A_log))  # [H]
+        b = np.zeros(g.shape[-2:]) if dt_bias is None else _f64(dt_bias).reshape(g.shape[-2:])
+        g = -a[:, None] * _softplus(g + b)
+    return q, k, g

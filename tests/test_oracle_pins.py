@@ -293,3 +293,37 @@ def test_eq13_flops_golden():
     assert abs(sum(terms.values()) - total) == 0
     assert abs(total - gold["printed_total_approx"]) <= 0.01 * total
     assert 128 * 128 == gold["state_elements_per_head"]
+
+
+# --- fused prologue: in-kernel L2 norm and the log-space decay gate ---------------------------
+def test_prologue_gate_closed_forms():
+    """softplus(0) = ln 2: with g = -dt_bias the decay is exactly -exp(A_log) * ln 2; a very
+    negative pre-activation gives no decay; a large one gives log alpha ~ -exp(A_log) * x."""
+    H, Dk = 3, 5
+    A_log = np.log(np.array([1.0, 4.0, 16.0]))
+    bias = np.linspace(-1, 1, H * Dk).reshape(H, Dk)
+    q = np.ones((2, H, Dk))
+    _, _, la = oracle.prologue(q, q, -bias[None].repeat(2, 0), A_log=A_log, dt_bias=bias)
+    np.testing.assert_allclose(la, -np.exp(A_log)[None, :, None] * np.log(2.0) * np.ones_like(la),
+                               rtol=1e-14)
+    _, _, la = oracle.prologue(q, q, np.full((1, H, Dk), -60.0), A_log=A_log)
+    assert np.all(la <= 0) and np.abs(la).max() < 1e-20
+    _, _, la = oracle.prologue(q, q, np.full((1, H, Dk), 50.0), A_log=A_log)
+    np.testing.assert_allclose(la, -np.exp(A_log)[None, :, None] * 50.0 * np.ones_like(la),
+                               rtol=1e-12)
+
+
+def test_prologue_l2norm_makes_the_operator_scale_invariant():
+    """With in-kernel normalisation, positive rescaling of a token's q or k changes nothing, and
+    the normalised keys have unit norm (up to eps)."""
+    rng = np.random.default_rng(31)
+    T, H, Dk, Dv = 12, 2, 8, 4
+    q, k, v, la, beta = _rand_inputs(rng, T, H, Dk, Dv, unit_keys=False)
+    s = rng.uniform(0.1, 10.0, size=(T, H, 1))
+    q1, k1, _ = oracle.prologue(q, k, la, qk_l2norm=True, eps=0.0)
+    q2, k2, _ = oracle.prologue(q * s, k * s[::-1], la, qk_l2norm=True, eps=0.0)
+    np.testing.assert_allclose(np.linalg.norm(k1, axis=-1), 1.0, rtol=1e-14)
+    o1, S1 = oracle.recurrent(q1, k1, v, la, beta)
+    o2, S2 = oracle.recurrent(q2, k2, v, la, beta)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S1, rtol=1e-12, atol=1e-13)

@@ -304,6 +304,58 @@ def run_decode(spec, n_steps, dev, warmup, world, rank):
     return ms, prof
 
 
+def run_fused_prefill(spec, seed, dev, steps, warmup, world):
+    """Standard prefill through kda_chunk_fwd with the fused prologue: raw (un-normalised) q, k and
+    raw decay gates turned into log decays in-kernel from A_log and dt_bias."""
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+
+    x = kda_synth.prefill_inputs(spec, seed, dev)
+    g = torch.Generator(device=dev).manual_seed(seed + 7)
+    q = (x["q"].float() * 3.0).to(x["q"].dtype)
+    k = (x["k"].float() * 3.0).to(x["k"].dtype)
+    gate = torch.randn(x["log_alpha"].shape, generator=g, device=dev) - 1.0
+    fusion = dict(qk_l2norm=True, eps=1e-6,
+                  A_log=torch.log(torch.rand((spec.H,), generator=g, device=dev) * 15 + 1) - 2.0,
+                  dt_bias=torch.randn((spec.H, spec.Dk), generator=g, device=dev) * 0.5)
+    o = torch.empty_like(x["v"])
+    fs = torch.empty((spec.num_seqs, spec.H, spec.Dk, spec.Dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.kda_chunk_fwd_workspace_size(spec.B, spec.T, spec.H, spec.Dk, spec.Dv,
+                                                      spec.chunk, spec.num_seqs, q.dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        kda.kda_chunk_fwd(q, k, x["v"], gate, x["beta"], initial_state=x["initial_state"],
+                          chunk=spec.chunk, o=o, final_state=fs, workspace=ws, fusion=fusion)
+
+    return timed(step, steps, warmup, world, dev)
+
+
+def run_recurrent_mode(N, T, H, D, dev, steps, warmup, world, seed):
+    """Multi-token recurrent mode (kda_recurrent_fwd): N sequences x T tokens applied to states
+    gathered from a pool by index (serving-cache layout); bf16 q/k/v, fp32 gates and states."""
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+
+    spec = kda_synth.PrefillSpec("recurrent", B=N, T=T, H=H, Dk=D, Dv=D, chunk=64, dtype="bf16",
+                                 decay="slow", init_std=0.0)
+    x = kda_synth.prefill_inputs(spec, seed, dev)
+    g = torch.Generator(device=dev).manual_seed(seed + 1)
+    P = 2 * N
+    pool = torch.randn((P, H, D, D), generator=g, device=dev) * 0.02
+    idx = torch.randperm(P, generator=g, device=dev)[:N].to(torch.int32)
+    o = torch.empty_like(x["v"])
+
+    def step(i):
+        kda.kda_recurrent_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool, idx, o=o)
+
+    return timed(step, steps, warmup, world, dev)
+
+
 def cpu_baseline(spec, dev, budget_s):
     """The fp64 oracle as it stands, on the host's cores, over whole sequences of the prefill
     workload (all heads), repeated until ~budget_s of CPU work. Returns tokens/s."""
@@ -458,6 +510,27 @@ def main():
                         for p in lp["prof"]]}
         del lp
         torch.cuda.empty_cache()
+    # the fused prologue on the standard workload
+    fms = run_fused_prefill(spec, 2001 + 10 * rank, dev, args.steps, args.warmup, world)
+    extra["fused_prologue_prefill"] = {
+        "workload": spec.name + "_raw_qk_and_gates",
+        "tokens_per_s": whole_job_rate(tokens * args.steps, world, fms),
+        "ms_per_call": fms / args.steps,
+        "overhead_vs_plain": (fms / args.steps) / ms_step - 1.0}
+    # the multi-token recurrent mode: 256 sequences x 16 tokens x 32 heads, states from a pool
+    rN, rT = 256, 16
+    rsteps = max(3, args.steps // 2)
+    rms = run_recurrent_mode(rN, rT, 32, 128, dev, rsteps, 2, world, 2005 + 10 * rank)
+    per = rms / rsteps
+    rstate = roofline.decode_state_bytes(rN, 32, 128, 128)
+    rtotal = rstate + rN * 32 * rT * ((3 * 128) * 2 + 4 * 128 + 4 + 128 * 2)
+    extra["recurrent_mode"] = {
+        "workload": f"recurrent_N{rN}_T{rT}_H32_d128_pool",
+        "tokens_per_s": whole_job_rate(rN * rT, world, per),
+        "ms_per_call": per,
+        "achieved_gbs": rtotal / (per / 1e3) / 1e9,
+        "frac_hbm": rtotal / (per / 1e3) / 1e9 / hbm_peak}
+    torch.cuda.empty_cache()
     if not args.no_decode:
         dspec = kda_synth.DECODE
         dms, dprof = run_decode(dspec, args.decode_steps, dev, 3, world, rank)

@@ -18,9 +18,16 @@
 //      Warp roles: a bulk-copy producer (double-buffered records), a single MMA-issuing thread,
 //      and four epilogue warps that hold the fp32 state slice (one row of S per thread).
 //
-// (K/Gamma) is formed as k * exp(-g) only when every channel's decay over the chunk stays above
-// exp(-60), so both factors of every product stay inside bf16/fp32 range; a chunk with stronger
-// decay takes an exact CUDA-core fallback for A_kk and A_qk (ratios exp(g_r - g_i) <= 1).
+// The ratio exp(g_r - g_i) inside A_kk and A_qk is split into two bf16 factors around a reference
+// log decay, and each factor must stay inside bf16 range. Three cases per (chunk, head):
+//   fast   every channel decays by less than exp(-60) over the chunk: one reference (the chunk
+//          start), K/Gamma = k * exp(-g), one pair of MMAs;
+//   blocks some channel decays harder, but none by more than exp(-60) within any 16-row block:
+//          row block R takes the reference g at the end of block R-1, so the row factor
+//          k_r exp(g_r - ref_R) is <= 1 and the column factor k_i exp(ref_R - g_i) is <= 1 for
+//          earlier blocks and <= exp(60) inside block R; three rounds of MMAs cover the four row
+//          blocks (the column tile is rebuilt per reference);
+//   exact  otherwise: a CUDA-core evaluation of every product with ratios exp(g_r - g_i) <= 1.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -32,7 +39,8 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr float kFastDecayLimit = 60.f;  // |g_C| bound for the direct (K/Gamma) factorisation
+constexpr float kFastDecayLimit = 60.f;  // log-decay range bound for one bf16 factorisation
+constexpr int kModeFast = 0, kModeBlocks = 1, kModeExact = 2;
 
 // record layout (bytes) of one (chunk, head). QW is a [128 x 128] tile (64-column blocks
 // 16 KiB apart): rows 0..63 hold Qt = Gamma.Q, rows 64..127 hold W, so one M = 128 MMA
@@ -67,11 +75,12 @@ constexpr uint32_t kS1Ki = 16384;     // [64 x 128] bf16: scan partials, then K/
 constexpr uint32_t kS1Qg = 32768;     // [64 x 128] bf16: raw q, then Gamma.Q, then fp32 T
 constexpr uint32_t kS1V = 49152;      // [64 x 128] bf16 v
 constexpr uint32_t kS1M = 65536;      // [64 x 64] bf16 M (the level products X alias it first)
+constexpr uint32_t kS1Inv = kS1M;     // fp32 [2][64] inverse norms of k and q, until phase 4
+constexpr uint32_t kS1Ref = kS1M + 1024;  // fp32 [4][128] g at rows 15, 31, 47, 63 (row 3 = g_C)
 constexpr uint32_t kS1Beta = 73728;   // fp32 [64]
-constexpr uint32_t kS1GC = 73984;     // fp32 [128]
-constexpr uint32_t kS1Bar = 74496;    // mbarrier
-constexpr uint32_t kS1Tmem = 74504;   // TMEM base address
-constexpr uint32_t kS1Bytes = 74512;
+constexpr uint32_t kS1Bar = 73984;    // mbarrier
+constexpr uint32_t kS1Tmem = 73992;   // TMEM base address
+constexpr uint32_t kS1Bytes = 74000;
 
 // fp32 64 x 64 matrices (A, T) are stored row-major with column bits 2..5 XOR-ed by (row % 16):
 // groups of four consecutive columns stay contiguous (128-bit accesses) while sixteen consecutive
@@ -156,9 +165,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   float* sT = reinterpret_cast<float*>(sm + kS1Qg);
   float* sX = reinterpret_cast<float*>(sm + kS1M);
   float* sBeta = reinterpret_cast<float*>(sm + kS1Beta);
-  float* sGC = reinterpret_cast<float*>(sm + kS1GC);
   float* sScan = reinterpret_cast<float*>(sm + kS1Ki);  // [16][128], before K/Gamma exists
-  float* sInv = reinterpret_cast<float*>(sm + kS1M);   // [2][64] inverse norms, until phase 4
+  float* sInv = reinterpret_cast<float*>(sm + kS1Inv);
+  float* sRef = reinterpret_cast<float*>(sm + kS1Ref);
+  const float* sGC = sRef + 3 * kD;  // the chunk's cumulative log decay g_C
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kS1Bar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS1Tmem);
 
@@ -240,8 +250,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 #pragma unroll
       for (int j = 0; j < 8; ++j) g[i][j] += pre[j];
   }
-  if (rg == 15) {
-    float4* gcp = reinterpret_cast<float4*>(sGC + cg * 8);
+  if ((rg & 3) == 3) {  // the last row of each 16-row block: the block references and g_C
+    float4* gcp = reinterpret_cast<float4*>(sRef + (rg >> 2) * kD + cg * 8);
     gcp[0] = make_float4(g[3][0], g[3][1], g[3][2], g[3][3]);
     gcp[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
   }
@@ -262,7 +272,21 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     ok = ok && (gcj >= -kFastDecayLimit);
     egc[j] = __expf(gcj);  // only scales a bf16 operand; the carried gamma_C uses expf
   }
-  const bool fast = __syncthreads_and(ok) != 0;
+  int mode = kModeFast;
+  if (!__syncthreads_and(ok)) {
+    bool blocks_ok = true;  // every channel's decay within every 16-row block
+    if (tid < kD) {
+      float prev = 0.f;
+#pragma unroll
+      for (int R = 0; R < 4; ++R) {
+        const float next = sRef[R * kD + tid];
+        blocks_ok = blocks_ok && (prev - next <= kFastDecayLimit);
+        prev = next;
+      }
+    }
+    mode = __syncthreads_and(blocks_ok) ? kModeBlocks : kModeExact;
+  }
+  if (tid < kD) reinterpret_cast<float*>(rec + kRecGam)[tid] = expf(sGC[tid]);
 
   // ---- phase 2: scale in place (each thread rewrites only the chunks it staged) --------------
 #pragma unroll
@@ -295,30 +319,52 @@ __global__ void __launch_bounds__(kK1Threads, 3)
         sInv[64 + r] = iq;
       }
     }
-    float kg[8], ki[8], kt[8];
+    if (mode == kModeFast) {
+      float kg[8], ki[8], kt[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float e = __expf(g[i][j]);
-      kg[j] = kf[j] * e;
-      qf[j] *= e;
-      if (fast) {
+      for (int j = 0; j < 8; ++j) {
+        const float e = __expf(g[i][j]);
+        kg[j] = kf[j] * e;
+        qf[j] *= e;
         ki[j] = kf[j] * __expf(-g[i][j]);
         kt[j] = ki[j] * egc[j];
-      } else {
-        ki[j] = 0.f;
-        kt[j] = kf[j] * __expf(sGC[cg * 8 + j] - g[i][j]);
       }
-    }
-    const uint4 qgv = pack8(qf);
-    st_shared_v4(sb + kS1Kg + off, pack8(kg));
-    st_shared_v4(sb + kS1Ki + off, pack8(ki));
-    st_shared_v4(sb + kS1Qg + off, qgv);
-    *reinterpret_cast<uint4*>(rec + kRecQW + qw_chunk_off(r, cg)) = qgv;
-    *reinterpret_cast<uint4*>(rec + kRecKt + off) = pack8(kt);
-    if (!fast) {  // exact fallback keeps the cumulative decay in this record's W/U area
-      float* gp = reinterpret_cast<float*>(rec + g_scratch_off(r));
+      const uint4 qgv = pack8(qf);
+      st_shared_v4(sb + kS1Kg + off, pack8(kg));
+      st_shared_v4(sb + kS1Ki + off, pack8(ki));
+      st_shared_v4(sb + kS1Qg + off, qgv);
+      *reinterpret_cast<uint4*>(rec + kRecQW + qw_chunk_off(r, cg)) = qgv;
+      *reinterpret_cast<uint4*>(rec + kRecKt + off) = pack8(kt);
+    } else {
+      const int R = rg >> 2;
+      {
+        float kt[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) gp[cg * 8 + j] = g[i][j];
+        for (int j = 0; j < 8; ++j) kt[j] = kf[j] * __expf(sGC[cg * 8 + j] - g[i][j]);
+        *reinterpret_cast<uint4*>(rec + kRecKt + off) = pack8(kt);
+      }
+      if (mode == kModeBlocks) {
+        float qr[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float er = R > 0 ? __expf(g[i][j] - sRef[(R - 1) * kD + cg * 8 + j]) : __expf(g[i][j]);
+          kf[j] *= er;
+          qr[j] = qf[j] * er;
+        }
+        st_shared_v4(sb + kS1Kg + off, pack8(kf));
+        st_shared_v4(sb + kS1Qg + off, pack8(qr));
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float e = __expf(g[i][j]);
+        if (mode != kModeBlocks) kf[j] *= e;
+        qf[j] *= e;
+      }
+      if (mode != kModeBlocks) st_shared_v4(sb + kS1Kg + off, pack8(kf));
+      *reinterpret_cast<uint4*>(rec + kRecQW + qw_chunk_off(r, cg)) = pack8(qf);
+      float* gp = reinterpret_cast<float*>(rec + g_scratch_off(r));
+      *reinterpret_cast<float4*>(gp + cg * 8) = make_float4(g[i][0], g[i][1], g[i][2], g[i][3]);
+      *reinterpret_cast<float4*>(gp + cg * 8 + 4) = make_float4(g[i][4], g[i][5], g[i][6], g[i][7]);
     }
   }
   fence_proxy_async_smem();
@@ -328,7 +374,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 
   // ---- phase 3: A_kk = Kg Ki^T (cols 0..63), A_qk = Qg Ki^T (cols 64..127) -------------------
   bool alive = true;
-  if (fast) {
+  uint32_t nwait = 0;  // completed phases of `bar`
+  if (mode == kModeFast) {
     if (tid == 0) {
       const uint32_t id = idesc_bf16_f32(64, 64, 0, 0);
 #pragma unroll
@@ -341,6 +388,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       mma_commit(bar);
     }
     alive = __syncthreads_and(mbar_wait(bar, 0)) != 0;
+    nwait = 1;
     tc_fence_after();
     // K/Gamma and Gamma.Q are dead from here: A (fp32) takes the K/Gamma area
     const int sp = warp & 3, half = warp >> 2;
@@ -374,6 +422,135 @@ __global__ void __launch_bounds__(kK1Threads, 3)
                 pack8(f);
           }
         }
+      }
+    }
+  } else if (mode == kModeBlocks) {
+    // Three rounds; round `rho` serves row blocks {3}, {2, 0}, {1}. A piece (R, ts) puts the
+    // column tile of row block R (rows i < 16R + 16, factor k_i exp(ref_R - g_i)) at rows
+    // [ts, ts + 16R + 16) of the v area and its products at TMEM columns [ts, ...) (A_kk) and
+    // [64 + ts, ...) (A_qk); only the 16 rows of block R (lanes 0..15 of TMEM sub-partition R)
+    // are read back. The K/Gamma area receives A (fp32) row block by row block.
+#pragma unroll 1
+    for (int rho = 0; rho < 3 && alive; ++rho) {
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) {
+        const int t = rg * 4 + ii;
+        const bool second = (rho == 1 && t >= 48);
+        const int R = rho == 0 ? 3 : (rho == 1 ? (second ? 0 : 2) : 1);
+        const int i = second ? t - 48 : t;
+        if (i >= 16 * R + 16) continue;
+        float kc[8];
+        if (i < L) {
+          unpack8(*(reinterpret_cast<const uint4*>(k + ((size_t)(t0 + i) * H + h) * kD) + cg), kc);
+          const float sc = fz.l2 ? sInv[i] : 1.f;
+          const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i)) + cg * 8;
+          const float4 ga = *reinterpret_cast<const float4*>(gi);
+          const float4 gb = *reinterpret_cast<const float4*>(gi + 4);
+          const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float ref = R > 0 ? sRef[(R - 1) * kD + cg * 8 + j] : 0.f;
+            kc[j] = kc[j] * sc * __expf(ref - gv[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) kc[j] = 0.f;
+        }
+        st_shared_v4(sb + kS1V + tile_chunk_off(t, cg, 8192), pack8(kc));
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+      tc_fence_after();
+      const int npieces = rho == 1 ? 2 : 1;
+      if (tid == 0) {
+        for (int pc = 0; pc < npieces; ++pc) {
+          const int R = rho == 0 ? 3 : (rho == 1 ? (pc == 0 ? 2 : 0) : 1);
+          const int ts = pc == 1 ? 48 : 0;
+          const uint32_t id = idesc_bf16_f32(64, 16 * R + 16, 0, 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+            const uint64_t bdesc = smem_desc_sw128(sb + kS1V + koff + ts * 128, 16, 1024);
+            mma_bf16(tmem + ts, smem_desc_sw128(sb + kS1Kg + koff, 16, 1024), bdesc, id, kk > 0);
+            mma_bf16(tmem + 64 + ts, smem_desc_sw128(sb + kS1Qg + koff, 16, 1024), bdesc, id,
+                     kk > 0);
+          }
+        }
+        mma_commit(bar);
+      }
+      alive = __syncthreads_and(mbar_wait(bar, nwait & 1)) != 0;
+      ++nwait;
+      tc_fence_after();
+      {
+        const int R = warp & 3, half = warp >> 2;
+        const bool mine = rho == 0 ? R == 3 : (rho == 1 ? (R == 2 || R == 0) : R == 1);
+        if (mine) {
+          const int ts = (rho == 1 && R == 0) ? 48 : 0, N = 16 * R + 16;
+          const int r = 16 * R + (lane & 15);
+          const float br = sBeta[r];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float va[16];
+            if (16 * u < N) {
+              tmem_ld16(tmem_at(tmem, 32 * R, half * 64 + ts + 16 * u), va);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) va[j] = 0.f;
+            }
+            if (lane < 16) {
+              if (half == 0) {
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                  const int i = 16 * u + 4 * j4;
+                  sts4(sA, r, i >> 2,
+                       make_float4(i < r ? br * va[4 * j4] : 0.f,
+                                   i + 1 < r ? br * va[4 * j4 + 1] : 0.f,
+                                   i + 2 < r ? br * va[4 * j4 + 2] : 0.f,
+                                   i + 3 < r ? br * va[4 * j4 + 3] : 0.f));
+                }
+              } else {
+#pragma unroll
+                for (int c8 = 0; c8 < 2; ++c8) {
+                  float f[8];
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) {
+                    const int i = 16 * u + 8 * c8 + j;
+                    f[j] = (i <= r) ? va[8 * c8 + j] : 0.f;
+                  }
+                  *reinterpret_cast<uint4*>(rec + kRecAqk +
+                                            tile_chunk_off(r, 2 * u + c8, 8192)) = pack8(f);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();  // TMEM read and the v area free before the next round
+    }
+    // the row tiles and column tiles are dead: Gamma.K back into its area for W, v reloaded
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+      const int r = rg * 4 + ii;
+      const uint32_t off = tile_chunk_off(r, cg, 8192);
+      if (r < L) {
+        const size_t row = (size_t)(t0 + r) * H + h;
+        cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
+        float kf[8];
+        unpack8(*(reinterpret_cast<const uint4*>(k + row * kD) + cg), kf);
+        const float sc = fz.l2 ? sInv[r] : 1.f;
+        const float* gr = reinterpret_cast<const float*>(rec + g_scratch_off(r)) + cg * 8;
+        const float4 ga = *reinterpret_cast<const float4*>(gr);
+        const float4 gb = *reinterpret_cast<const float4*>(gr + 4);
+        const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kf[j] = kf[j] * sc * __expf(gv[j]);
+        st_shared_v4(sb + kS1Kg + off, pack8(kf));
+      } else {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        st_shared_v4(sb + kS1V + off, z);
+        st_shared_v4(sb + kS1Kg + off, z);
       }
     }
   } else {
@@ -538,12 +715,13 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     for (int j = 0; j < 8; ++j) f[j] = (i0 + j <= r) ? f[j] : 0.f;
     st_shared_v4(sb + kS1M + tile_chunk_off(r, c8, 8192), pack8(f));
   }
+  cp_async_wait_all();  // the reloaded v of the block mode
   fence_proxy_async_smem();
   __syncthreads();
   tc_fence_after();
 
   // ---- phase 5: W = M Kg, then U = M V, through TMEM [0, 128) -------------------------------
-  uint32_t phase = fast ? 1 : 0;
+  uint32_t phase = nwait & 1;
 #pragma unroll 1
   for (int which = 0; which < 2 && alive; ++which) {
     if (tid == 0) {
@@ -566,7 +744,6 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     __syncthreads();
     tc_fence_after();
   }
-  if (tid < kD) reinterpret_cast<float*>(rec + kRecGam)[tid] = expf(sGC[tid]);
 
   tc_fence_before();
   __syncthreads();

@@ -106,6 +106,26 @@ def test_bf16_strong_decay_chunks(cuda_device):
     assert rel_err(s, s_ref) <= TOL_BF16_S
 
 
+def test_bf16_block_reference_chunks(cuda_device):
+    """Per-token decays of about exp(-1.6) (over 64 tokens far below exp(-60), within 16 tokens
+    above it) take the block-reference tensor-core evaluation of A_kk / A_qk: on every channel of
+    every chunk, on 32 channels of some chunks (mixed with ordinary channels), and on one chunk
+    strong enough for the exact fallback; ragged last chunk."""
+    spec = PrefillSpec("t", B=2, T=250, H=3, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.02)
+    inp = kda_synth.prefill_inputs(spec, 47, cuda_device)
+    la = inp["log_alpha"].clone()
+    la[0] *= 4.0
+    la[1, :, :, :32] *= 4.0
+    la[1, 128:192] *= 10.0
+    inp["log_alpha"] = la
+    o, s = _run(inp, 64)
+    o_ref, s_ref = _oracle(inp, 2, 250)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(s).all()
+    assert rel_err(o, o_ref) <= TOL_BF16_O
+    assert rel_err(s, s_ref) <= TOL_BF16_S
+
+
 def test_bf16_standard_prefill_workload(cuda_device):
     """The standard prefill workload in full: B=2, T=4096, H=32, d=128, C=64, bf16 q/k/v, fp32
     gates, initial state ~ N(0, 0.02^2); every output and final state against the oracle."""

@@ -58,11 +58,36 @@ def chunk_reference(k, q, v, la, beta, L):
                 gam=np.exp(g[-1]))
 
 
-@pytest.mark.parametrize("T", [64, 150])
-def test_chunk_records_match_formulas(cuda_device, T):
+def chunk_mode(la_chunk: np.ndarray) -> str:
+    """Which evaluation of A_kk / A_qk the kernel picks for one chunk of one head: "fast" when
+    every channel decays by at most exp(-60) over the chunk, "blocks" when it does so within
+    every 16-row block, "exact" otherwise."""
+    g = np.concatenate([np.zeros((1, la_chunk.shape[1])), np.cumsum(la_chunk, axis=0)])
+    if g[-1].min() >= -60:
+        return "fast"
+    ends = [min(16 * (R + 1), la_chunk.shape[0]) for R in range(4)]
+    starts = [min(16 * R, la_chunk.shape[0]) for R in range(4)]
+    drops = [(g[s] - g[e]).max() for s, e in zip(starts, ends)]
+    return "blocks" if max(drops) <= 60 else "exact"
+
+
+# per-chunk decay scalings: (channels scaled, factor); 1 = the plain recipe
+MIXED_MODES = [(slice(None), 1.0), (slice(None), 4.0), (slice(None), 40.0), (slice(0, 32), 4.0)]
+
+
+@pytest.mark.parametrize("T,mixed", [(64, False), (150, False), (250, True)])
+def test_chunk_records_match_formulas(cuda_device, T, mixed):
     spec = PrefillSpec("t", B=1, T=T, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16", decay="fast",
                        init_std=0.02)
     inp = kda_synth.prefill_inputs(spec, 500 + T, cuda_device)
+    if mixed:  # one chunk in each mode, the block mode twice (all channels / 32 of them, ragged)
+        la = inp["log_alpha"].clone()
+        for c, (chs, f) in enumerate(MIXED_MODES):
+            la[:, 64 * c:64 * c + 64, :, chs] *= f
+        inp["log_alpha"] = la
+        modes = [chunk_mode(to_np(la[0, 64 * c:64 * c + 64, h])) for c in range(4)
+                 for h in range(2)]
+        assert modes == ["fast"] * 2 + ["blocks"] * 2 + ["exact"] * 2 + ["blocks"] * 2, modes
     nbytes = kda.kda_chunk_fwd_workspace_size(1, T, 2, 128, 128, 64, 1, torch.bfloat16)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda_device)
     kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],

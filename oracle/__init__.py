@@ -17,6 +17,11 @@ Functions
                            log alpha = -exp(A_log[h]) * softplus(g + dt_bias[h, c]) (walkthrough
                            §3.4 "Neural Parameterization"; the L2 Deep Distill page's
                            implementation notes on the in-kernel L2 norm and the fused gate).
+  output_norm_gate(...)    the output epilogue y = sigmoid(gate) * weight * o / RMS(o), the RMS
+                           taken over the value channels of each (token, head) (walkthrough §3.4
+                           "Neural Parameterization", the output-gate equation; the L2 Deep
+                           Distill page's module table: FusedRMSNormGated, sigmoid gate inside the
+                           RMSNorm).
 
 All inputs follow the packed layout [T_total, H, D] with int64 ``cu_seqlens`` [N+1]; a batch of B
 equal-length sequences is the same memory as [B, T, H, D] with cu_seqlens = [0, T, 2T, ...].
@@ -183,3 +188,23 @@ def prologue(q, k, log_alpha_or_gate, A_log=None, dt_bias=None, qk_l2norm=False,
         b = np.zeros(g.shape[-2:]) if dt_bias is None else _f64(dt_bias).reshape(g.shape[-2:])
         g = -a[:, None] * _softplus(g + b)
     return q, k, g
+
+
+def _sigmoid(x: np.ndarray) -> np.ndarray:
+    """1 / (1 + exp(-x)), evaluated without overflow for either sign."""
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def output_norm_gate(o, gate=None, weight=None, eps=1e-6):
+    """fp64 y = sigmoid(gate) * weight * o / sqrt(mean_c(o_c^2) + eps) over the last axis (the
+    value channels of one (token, head)); gate None means no gate, weight None means ones.
+    ``o`` and ``gate`` share a shape (..., Dv); ``weight`` is [Dv]."""
+    o = _f64(o)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    y = o / rms
+    if weight is not None:
+        y = y * _f64(weight).reshape(-1)
+    if gate is not None:
+        y = y * _sigmoid(_f64(gate).reshape(o.shape))
+    return y

@@ -327,3 +327,40 @@ def test_prologue_l2norm_makes_the_operator_scale_invariant():
     o2, S2 = oracle.recurrent(q2, k2, v, la, beta)
     np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(S2, S1, rtol=1e-12, atol=1e-13)
+
+
+def test_output_norm_gate_worked_example():
+    """o = (3, 4): mean square 12.5, RMS 5/sqrt(2) = 3.5355339..., so the normalised row is
+    (0.8485281374, 1.1313708499) (= 3 sqrt(2)/5, 4 sqrt(2)/5); a zero gate halves it (sigmoid(0) =
+    1/2) and the weight scales channel by channel."""
+    y = oracle.output_norm_gate(np.array([[3.0, 4.0]]), eps=0.0)
+    np.testing.assert_allclose(y, [[0.8485281374238570, 1.1313708498984760]], rtol=1e-14)
+    y = oracle.output_norm_gate(np.array([[3.0, 4.0]]), gate=np.zeros((1, 2)),
+                                weight=np.array([2.0, -1.0]), eps=0.0)
+    np.testing.assert_allclose(y, [[0.8485281374238570, -0.5656854249492380]], rtol=1e-14)
+    # eps enters under the square root: o = (1, 1), eps = 3 -> 1 / sqrt(1 + 3) = 1/2
+    y = oracle.output_norm_gate(np.array([[1.0, 1.0]]), eps=3.0)
+    np.testing.assert_allclose(y, [[0.5, 0.5]], rtol=1e-15)
+
+
+def test_output_norm_gate_structure():
+    """The RMS is per (token, head) row over the value channels: every row of the ungated output
+    has unit RMS, positive rescaling of a row changes nothing, rows do not mix; a saturated gate
+    passes the row through and a very negative one closes it."""
+    rng = np.random.default_rng(41)
+    o = rng.normal(size=(5, 3, 16)) * rng.uniform(0.01, 100.0, size=(5, 3, 1))
+    y = oracle.output_norm_gate(o, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-13)
+    s = rng.uniform(0.1, 10.0, size=(5, 3, 1))
+    np.testing.assert_allclose(oracle.output_norm_gate(o * s, eps=0.0), y, rtol=1e-13)
+    o2 = o.copy()
+    o2[2, 1] *= -7.0
+    y2 = oracle.output_norm_gate(o2, eps=0.0)
+    mask = np.ones((5, 3), bool)
+    mask[2, 1] = False
+    np.testing.assert_array_equal(y2[mask], y[mask])
+    np.testing.assert_allclose(y2[2, 1], -y[2, 1], rtol=1e-13)
+    g_open = oracle.output_norm_gate(o, gate=np.full(o.shape, 40.0), eps=0.0)
+    np.testing.assert_allclose(g_open, y, rtol=1e-15)
+    g_shut = oracle.output_norm_gate(o, gate=np.full(o.shape, -800.0), eps=0.0)
+    assert np.all(np.abs(g_shut) < 1e-300)

@@ -304,9 +304,10 @@ def run_decode(spec, n_steps, dev, warmup, world, rank):
     return ms, prof
 
 
-def run_fused_prefill(spec, seed, dev, steps, warmup, world):
+def run_fused_prefill(spec, seed, dev, steps, warmup, world, epilogue=False):
     """Standard prefill through kda_chunk_fwd with the fused prologue: raw (un-normalised) q, k and
-    raw decay gates turned into log decays in-kernel from A_log and dt_bias."""
+    raw decay gates turned into log decays in-kernel from A_log and dt_bias; with ``epilogue`` the
+    output is also normalised head-wise and gated (RMSNorm x sigmoid) before the store."""
     import torch
 
     import gated_delta_rule_120_b200 as kda
@@ -320,6 +321,10 @@ def run_fused_prefill(spec, seed, dev, steps, warmup, world):
     fusion = dict(qk_l2norm=True, eps=1e-6,
                   A_log=torch.log(torch.rand((spec.H,), generator=g, device=dev) * 15 + 1) - 2.0,
                   dt_bias=torch.randn((spec.H, spec.Dk), generator=g, device=dev) * 0.5)
+    if epilogue:
+        fusion.update(out_norm=True, out_norm_eps=1e-5,
+                      out_norm_weight=torch.rand((spec.Dv,), generator=g, device=dev) + 0.5,
+                      out_gate=torch.randn(x["v"].shape, generator=g, device=dev).to(x["v"].dtype))
     o = torch.empty_like(x["v"])
     fs = torch.empty((spec.num_seqs, spec.H, spec.Dk, spec.Dv), dtype=torch.float32, device=dev)
     ws = torch.empty(kda.kda_chunk_fwd_workspace_size(spec.B, spec.T, spec.H, spec.Dk, spec.Dv,
@@ -517,6 +522,14 @@ def main():
         "tokens_per_s": whole_job_rate(tokens * args.steps, world, fms),
         "ms_per_call": fms / args.steps,
         "overhead_vs_plain": (fms / args.steps) / ms_step - 1.0}
+    # prologue + output epilogue (head-wise RMSNorm x sigmoid gate fused into the state kernel)
+    lms = run_fused_prefill(spec, 2001 + 10 * rank, dev, args.steps, args.warmup, world,
+                            epilogue=True)
+    extra["fused_layer_prefill"] = {
+        "workload": spec.name + "_raw_qk_gates_and_output_gate",
+        "tokens_per_s": whole_job_rate(tokens * args.steps, world, lms),
+        "ms_per_call": lms / args.steps,
+        "overhead_vs_plain": (lms / args.steps) / ms_step - 1.0}
     # the multi-token recurrent mode: 256 sequences x 16 tokens x 32 heads, states from a pool
     rN, rT = 256, 16
     rsteps = max(3, args.steps // 2)

@@ -36,9 +36,12 @@ ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size
 
 
 class Fusion(ctypes.Structure):
-    """kda_fusion_t: in-kernel q/k L2 normalisation and the fused log-space decay gate."""
+    """kda_fusion_t: in-kernel q/k L2 normalisation, the fused log-space decay gate, and the output
+    epilogue (head-wise RMSNorm x sigmoid gate)."""
     _fields_ = [("qk_l2norm", ctypes.c_int32), ("qk_l2norm_eps", ctypes.c_float),
-                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
+                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("out_norm", ctypes.c_int32), ("out_norm_eps", ctypes.c_float),
+                ("out_norm_weight", ctypes.c_void_p), ("out_gate", ctypes.c_void_p)]
 
 
 class ProfileEntry(ctypes.Structure):
@@ -150,10 +153,23 @@ def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, chunk
     return int(out.value)
 
 
-def _fusion(fusion, dev, H, Dk):
-    """dict(qk_l2norm=bool, eps=float, A_log=[H] fp32, dt_bias=[H,Dk] fp32) -> kda_fusion_t."""
+def _fusion(fusion, dev, H, Dk, o_like=None):
+    """dict(qk_l2norm=bool, eps=float, A_log=[H] fp32, dt_bias=[H,Dk] fp32, out_norm=bool,
+    out_norm_eps=float, out_norm_weight=[Dv] fp32, out_gate=o-shaped) -> kda_fusion_t."""
     if fusion is None:
         return None
+    w, og = fusion.get("out_norm_weight"), fusion.get("out_gate")
+    if fusion.get("out_norm"):
+        if w is not None:
+            _need(w, "out_norm_weight", dev, torch.float32)
+            if o_like is not None and w.numel() != o_like.shape[-1]:
+                raise ValueError("out_norm_weight must have Dv entries")
+        if og is not None:
+            _need(og, "out_gate", dev, o_like.dtype if o_like is not None else None)
+            if o_like is not None and tuple(og.shape) != tuple(o_like.shape):
+                raise ValueError("out_gate must have o's shape")
+    else:
+        w = og = None
     A_log, dt_bias = fusion.get("A_log"), fusion.get("dt_bias")
     if A_log is not None:
         _need(A_log, "A_log", dev, torch.float32)
@@ -165,7 +181,9 @@ def _fusion(fusion, dev, H, Dk):
             raise ValueError("dt_bias must be [H, Dk]")
     return Fusion(1 if fusion.get("qk_l2norm") else 0, float(fusion.get("eps", 1e-6)),
                   None if A_log is None else A_log.data_ptr(),
-                  None if dt_bias is None else dt_bias.data_ptr())
+                  None if dt_bias is None else dt_bias.data_ptr(),
+                  1 if fusion.get("out_norm") else 0, float(fusion.get("out_norm_eps", 1e-5)),
+                  None if w is None else w.data_ptr(), None if og is None else og.data_ptr())
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
@@ -177,7 +195,9 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     beta [B,T,H] fp32; initial_state [N,H,Dk,Dv] fp32 or None; cu_seqlens int32 [N+1] on the
     device or None (then N = B). Returns (o [B,T,H,Dv] in the input dtype, final_state or None).
     ``fusion`` (dict, optional): qk_l2norm / eps normalise q and k in-kernel; A_log [H] and
-    dt_bias [H,Dk] turn ``log_alpha`` (then the raw gate) into -exp(A_log) * softplus(g + dt_bias).
+    dt_bias [H,Dk] turn ``log_alpha`` (then the raw gate) into -exp(A_log) * softplus(g + dt_bias);
+    out_norm / out_norm_eps / out_norm_weight [Dv] fp32 / out_gate (o's shape and dtype) make the
+    stored output sigmoid(out_gate) * weight * o / sqrt(mean(o^2) + eps) per (token, head).
     """
     dev = q.device
     B, T, H, Dk = q.shape
@@ -205,7 +225,7 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     ws_bytes = kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, N, q.dtype)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    fz = _fusion(fusion, dev, H, Dk)
+    fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
             _ptr(final_state if output_final_state else None), _ptr(workspace), workspace.numel())
@@ -263,7 +283,7 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, 
             raise ValueError("state_indices must have N entries")
     if o is None:
         o = torch.empty((N, T, H, Dv), dtype=q.dtype, device=dev)
-    fz = _fusion(fusion, dev, H, Dk)
+    fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(state_pool), _ptr(state_indices), _ptr(o), N, T, H, Dk, Dv, P)
     if fz is None:

@@ -83,7 +83,7 @@ const char* kda_status_string(kda_status_t s) {
   return "KDA_ERR_UNKNOWN";
 }
 
-const char* kda_version(void) { return "0.1.0"; }
+const char* kda_version(void) { return "0.2.0"; }
 
 kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
                                           int32_t chunk, int32_t num_seqs, kda_dtype_t dt,
@@ -114,6 +114,14 @@ kda_status_t to_fusion(const kda_fusion_t* f, Fusion* out) {
   out->eps = f->qk_l2norm_eps;
   out->A_log = f->A_log;
   out->dt_bias = f->A_log ? f->dt_bias : nullptr;
+  if (f->out_norm) {
+    if (!(f->out_norm_eps >= 0.f) || (f->out_norm_weight && !aligned(f->out_norm_weight, 4)))
+      return KDA_ERR_INVALID_ARG;
+    out->onorm = 1;
+    out->oeps = f->out_norm_eps;
+    out->ow = f->out_norm_weight;
+    out->og = f->out_gate;
+  }
   return KDA_OK;
 }
 
@@ -136,6 +144,7 @@ kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, kda_dty
   if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
     return KDA_ERR_INVALID_ARG;
   if (varlen && !aligned(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+  if (fz.onorm && fz.og && tokens > 0 && !aligned(fz.og, 16)) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
 
   const WsLayout lay = prefill_layout(B, T, H, Dk, Dv, C, N, varlen, dt);
@@ -202,7 +211,8 @@ kda_status_t recurrent_fwd_impl(const void* q, const void* k, const void* v, kda
   const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
   if (!aligned(pool, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
       !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4) ||
-      (state_indices && !aligned(state_indices, 4)))
+      (state_indices && !aligned(state_indices, 4)) || (fz.onorm && fz.og && !aligned(fz.og, es)) ||
+      (fz.onorm && fz.ow && !aligned(fz.ow, 16)))
     return KDA_ERR_INVALID_ARG;
   return from_cuda(launch_recurrent_multi(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N,
                                           T, H, Dk, Dv, P, fz, (cudaStream_t)stream));

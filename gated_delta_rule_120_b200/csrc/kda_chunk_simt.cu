@@ -364,7 +364,10 @@ static cudaError_t launch_simt_typed(const PrefillArgs& a, const SeqGeometry& ge
   ProfileScope prof("chunk_state_simt", stream);
   chunk_state_simt_kernel<Tin><<<g2, kSimtThreads, sm2, stream>>>(
       records, rec, geo, a.H, a.Dk, a.Dv, a.initial_state, a.final_state, (Tin*)a.o);
-  return cudaGetLastError();
+  err = cudaGetLastError();
+  if (err != cudaSuccess || !a.fz.onorm) return err;
+  return launch_output_norm_gate(a.o, a.dtype, a.fz, (long long)a.B * a.T * a.H, a.H, a.Dv,
+                                 a.cu_seqlens ? a.cu_seqlens + a.N : nullptr, stream);
 }
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,

@@ -760,30 +760,50 @@ constexpr int kEpiWarps = 8;                       // two per TMEM sub-partition
 constexpr int kK2Threads = 64 + 32 * kEpiWarps;    // warp 0 producer, warp 1 MMA, then epilogue
 // stage: QW [128 x 128] | AZ [128 x 64] = A_qk rows 0..63, zero rows 64..127 | Kt [64 x 128] |
 //        U (this CTA's 64-column block) [64 x 64] | gamma_C fp32 [128]
+//        (+ with the output epilogue: the output-gate rows of this CTA's columns [64 x 64] bf16,
+//        row-major)
 constexpr uint32_t kStQW = 0, kStAZ = 32768, kStKt = 49152, kStU = 65536, kStGam = 73728;
-constexpr uint32_t kStageBytes = 74752;  // 73 KiB, keeps every stage 1024-aligned
+constexpr uint32_t kStGate = 74752;
 constexpr uint32_t kStageTx = 32768 + 8192 + 16384 + 8192 + 512;
 constexpr int kStages = 2;
 constexpr uint32_t kS2Stage0 = 0;
-constexpr uint32_t kS2S = kStages * kStageBytes;   // [128 x 64] bf16 state tile (B operand)
-constexpr uint32_t kS2Vp = kS2S + 16384;           // [64 x 64] bf16 pseudo-value tile
-constexpr uint32_t kS2Bar = kS2Vp + 8192;
 constexpr int kNumBars2 = 2 * kStages + 5;
-constexpr uint32_t kS2Tmem = kS2Bar + 8 * kNumBars2;
-constexpr uint32_t kS2Flags = kS2Tmem + 4;
-constexpr uint32_t kS2Bytes = kS2Flags + 12;
+constexpr int kOutWarps = 4;
+
+// shared-memory map of K2; the output epilogue (head-wise RMSNorm x sigmoid gate) adds a gate
+// tile to every stage, and, because the two column halves of one (sequence, head) run as a
+// cluster of two CTAs that exchange per-row sums of squares of their 64 columns, the exchange
+// buffers
+template <bool kNorm>
+struct K2Smem {
+  static constexpr uint32_t stage = kNorm ? 74752 + 8192 : 74752;  // 1024-aligned stages
+  static constexpr uint32_t S = kStages * stage;   // [128 x 64] bf16 state tile (B operand)
+  static constexpr uint32_t Vp = S + 16384;        // [64 x 64] bf16 pseudo-value tile
+  static constexpr uint32_t Bar = Vp + 8192;
+  static constexpr uint32_t Tmem = Bar + 8 * kNumBars2;
+  static constexpr uint32_t Flags = Tmem + 4;
+  static constexpr uint32_t Part = (Flags + 12 + 15) & ~15u;  // fp32 [2 parity][2 half][64 rows]
+  static constexpr uint32_t Peer = Part + 1024;    // fp32 [2 parity][64]: the peer's row sums
+  static constexpr uint32_t W = Peer + 512;        // fp32 [64] norm weight of this CTA's columns
+  static constexpr uint32_t NBar = W + 256;        // mbarriers: part (local), norm[2] (peer)
+  static constexpr uint32_t bytes = kNorm ? NBar + 24 : Flags + 12;
+};
 // TMEM columns: [Qt; W] S accumulators (double buffer) [0,64) / [64,128); Kt^T V' [128,192)
 constexpr uint32_t kTmD12 = 0, kTmD3 = 128;
 
+template <bool kNorm>
 __global__ void __launch_bounds__(kK2Threads, 1)
     chunk_state_tc_kernel(const uint8_t* __restrict__ ws_records, SeqGeometry geo, int H,
                           const float* __restrict__ initial_state, float* __restrict__ final_state,
-                          __nv_bfloat16* __restrict__ o) {
+                          __nv_bfloat16* __restrict__ o, Fusion fz) {
   extern __shared__ uint8_t smem_raw[];
   if (!geo.ok()) return;
+  using SM = K2Smem<kNorm>;
+  constexpr uint32_t kStageBytes = SM::stage;
+  constexpr uint32_t kS2S = SM::S, kS2Vp = SM::Vp;
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(sm);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kS2Bar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::Bar);
   uint64_t* full = bars + 0;           // [kStages] record copied
   uint64_t* empty = bars + kStages;    // [kStages] record consumed by the tensor cores
   uint64_t* d12 = bars + 2 * kStages;  // [Qt; W] S done
@@ -791,8 +811,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   uint64_t* d2done = d12 + 2;          // A_qk V' accumulated (output can be read)
   uint64_t* vp_ready = d12 + 3;        // V' tile written (one arrival per epilogue warp)
   uint64_t* s_ready = d12 + 4;         // state tile written (one arrival per epilogue warp)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kS2Tmem);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kS2Flags);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::Tmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM::Flags);
 
   const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * 64;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -813,35 +833,60 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     mbar_init(vp_ready, kEpiWarps);
     mbar_init(s_ready, kEpiWarps);
     *abort_flag = 0;
+    if (kNorm) {
+      uint64_t* nb = reinterpret_cast<uint64_t*>(sm + SM::NBar);
+      mbar_init(nb, kOutWarps);  // this CTA's out warps wrote their partial sums
+      mbar_init(nb + 1, 1);      // the peer's 64 row sums landed (256 transaction bytes), even
+      mbar_init(nb + 2, 1);      // chunk index / odd; the one arrival is this CTA's expect_tx
+    }
     fence_mbar_init();
   }
+  if (kNorm && tid < 64)
+    reinterpret_cast<float*>(sm + SM::W)[tid] = fz.ow ? fz.ow[j0 + tid] : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (kNorm) cluster_sync();  // the peer's barriers are initialised before any remote arrival
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
+    // lane 0 copies the record; with the gated output epilogue the whole warp also copies the
+    // chunk's gate rows (128 bytes of this CTA's columns per row)
+    const bool gate_rows = kNorm && fz.og != nullptr;
+    if (lane == 0 || gate_rows) {
       for (int ci = 0; ci < nchunks; ++ci) {
         const int st = ci % kStages;
-        if (ci >= kStages && !mbar_wait(empty + st, ((ci / kStages) - 1) & 1)) {
+        bool ok = (ci < kStages || mbar_wait(empty + st, ((ci / kStages) - 1) & 1)) &&
+                  !*abort_flag;
+        if (gate_rows) ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
           *abort_flag = 1;
           break;
         }
-        if (*abort_flag) break;
-        const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
         uint8_t* stage = sm + kS2Stage0 + st * kStageBytes;
-        mbar_arrive_expect_tx(full + st, kStageTx);
-        bulk_g2s(stage + kStQW, rec + kRecQW, 32768, full + st);
-        bulk_g2s(stage + kStAZ, rec + kRecAqk, 8192, full + st);
-        bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
-        bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
-        bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
+        const int t0 = tb + ci * kC;
+        const int L = min(kC, te - t0);
+        if (lane == 0) {
+          const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
+          mbar_arrive_expect_tx(full + st, kStageTx + (gate_rows ? (uint32_t)L * 128u : 0u));
+          bulk_g2s(stage + kStQW, rec + kRecQW, 32768, full + st);
+          bulk_g2s(stage + kStAZ, rec + kRecAqk, 8192, full + st);
+          bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
+          bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
+          bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
+        }
+        if (gate_rows) {
+          const __nv_bfloat16* g0 = reinterpret_cast<const __nv_bfloat16*>(fz.og);
+          for (int rr = lane; rr < L; rr += 32)
+            bulk_g2s(stage + kStGate + rr * 128, g0 + ((size_t)(t0 + rr) * H + h) * kD + j0, 128,
+                     full + st);
+        }
       }
       // the last copies must land before the CTA may exit
-      for (int ci = nchunks > kStages ? nchunks - kStages : 0; ci < nchunks; ++ci)
-        mbar_wait(full + ci % kStages, (ci / kStages) & 1);
+      if (lane == 0)
+        for (int ci = nchunks > kStages ? nchunks - kStages : 0; ci < nchunks; ++ci)
+          mbar_wait(full + ci % kStages, (ci / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -944,6 +989,13 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         break;
       }
       const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[row];
+      // the output gate row leaves the stage now: the stage is released once V' is in
+      uint4 graw[4];
+      if (kNorm && out_warp && fz.og && r < L) {
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          graw[q8] = ld_shared_v4(stage + kStGate + r * 128 + chalf * 64 + q8 * 16);
+      }
       if (!out_warp) {  // V' = U - W S for chunk row r, this warp's 32 columns
         float u[32];
 #pragma unroll
@@ -994,6 +1046,49 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         tc_fence_after();
         tmem_ld32(tmem_at(tmem, sp * 32, d12c), va);
         tmem_ld_wait();
+        if (kNorm) {  // y = sigmoid(gate) * weight * O / RMS over all 128 columns of the row
+          const int b = ci & 1;
+          float* sPart = reinterpret_cast<float*>(sm + SM::Part) + b * 128;
+          const float* sPeer = reinterpret_cast<const float*>(sm + SM::Peer) + b * 64;
+          uint64_t* nb = reinterpret_cast<uint64_t*>(sm + SM::NBar);
+          const bool gated = fz.og && r < L;
+          float ss = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = fmaf(va[j], va[j], ss);
+          sPart[chalf * 64 + r] = ss;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(nb);
+          ok = mbar_wait(nb, ci & 1);
+          if (ok && chalf == 0) {  // send this CTA's 64-column sum of the row to the peer
+            const uint32_t peer = cluster_ctarank() ^ 1u;
+            if (sp == 0 && lane == 0) mbar_arrive_expect_tx(nb + 1 + b, 64 * 4);
+            st_async_remote_f32(mapa_shared(smem_u32(sPeer + r), peer), ss + sPart[64 + r],
+                                mapa_shared(smem_u32(nb + 1 + b), peer));
+          }
+          ok = ok && mbar_wait(nb + 1 + b, (ci >> 1) & 1);
+          if (!__all_sync(0xffffffffu, ok)) {
+            *abort_flag = 1;
+            break;
+          }
+          const float inv =
+              rsqrtf((sPart[r] + sPart[64 + r] + sPeer[r]) * (1.f / kD) + fz.oeps);
+          const float* sW = reinterpret_cast<const float*>(sm + SM::W) + 32 * chalf;
+          float gt[32];
+          if (gated) {  // the gate row staged by the producer: 32 columns of row r
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float f[8];
+              unpack8(graw[q8], f);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) gt[q8 * 8 + j] = __fdividef(1.f, 1.f + __expf(-f[j]));
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) gt[j] = 1.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) va[j] = va[j] * inv * sW[j] * gt[j];
+        }
         if (r < L) {
           uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0 +
                                                 32 * chalf);
@@ -1020,20 +1115,24 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+  if (kNorm) cluster_sync();  // no CTA leaves while its peer may still write into it
 }
 
 }  // namespace tc
 
 size_t tc_local_smem_bytes() { return tc::kS1Bytes + 1024; }
-size_t tc_state_smem_bytes() { return tc::kS2Bytes + 1024; }
+size_t tc_state_smem_bytes() { return tc::K2Smem<false>::bytes + 1024; }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
                               uint8_t* records, cudaStream_t stream) {
-  const int sm1 = (int)tc_local_smem_bytes(), sm2 = (int)tc_state_smem_bytes();
+  const bool norm = a.fz.onorm != 0;
+  const int sm1 = (int)tc_local_smem_bytes();
+  const int sm2 = (int)(norm ? tc::K2Smem<true>::bytes + 1024 : tc_state_smem_bytes());
   cudaError_t err = cudaFuncSetAttribute(tc::chunk_local_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(tc::chunk_state_tc_kernel,
+  err = cudaFuncSetAttribute(norm ? tc::chunk_state_tc_kernel<true>
+                                  : tc::chunk_state_tc_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
   if (err != cudaSuccess) return err;
   if (max_chunks > 0) {
@@ -1044,10 +1143,28 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  ProfileScope prof("chunk_state_tc", stream);
-  tc::chunk_state_tc_kernel<<<dim3(a.N, a.H, 2), tc::kK2Threads, sm2, stream>>>(
-      records, geo, a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o);
-  return cudaGetLastError();
+  if (!norm) {
+    ProfileScope prof("chunk_state_tc", stream);
+    tc::chunk_state_tc_kernel<false><<<dim3(a.N, a.H, 2), tc::kK2Threads, sm2, stream>>>(
+        records, geo, a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o, a.fz);
+    return cudaGetLastError();
+  }
+  // the two column halves of a (sequence, head) form one cluster
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.N, a.H, 2);
+  cfg.blockDim = dim3(tc::kK2Threads);
+  cfg.dynamicSmemBytes = (size_t)sm2;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 2;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfileScope prof("chunk_state_tc_norm", stream);
+  return cudaLaunchKernelEx(&cfg, tc::chunk_state_tc_kernel<true>, (const uint8_t*)records, geo,
+                            (int)a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o, a.fz);
 }
 
 }  // namespace kda

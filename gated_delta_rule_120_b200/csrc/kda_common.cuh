@@ -53,6 +53,8 @@ __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b -
 
 // log(1 + exp(x)) without overflow.
 __device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+// 1 / (1 + exp(-x)); exp(-x) = inf for very negative x gives exactly 0.
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
 __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) {
   return (x + a - 1) / a * a;
 }

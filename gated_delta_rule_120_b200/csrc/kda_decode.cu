@@ -265,12 +265,33 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const float kr = s_k[row0 + i] * ik;
       s[i].x += kr * u.x; s[i].y += kr * u.y; s[i].z += kr * u.z; s[i].w += kr * u.w;
     }
-    if (warp == 0 && col_ok) {
-      Tin* op = o + vec_base(t) * Dv + col;
-      op[0] = from_f32<Tin>(p.x + kq * u.x);
-      op[1] = from_f32<Tin>(p.y + kq * u.y);
-      op[2] = from_f32<Tin>(p.z + kq * u.z);
-      op[3] = from_f32<Tin>(p.w + kq * u.w);
+    if (warp == 0) {
+      float4 y = make_float4(p.x + kq * u.x, p.y + kq * u.y, p.z + kq * u.z, p.w + kq * u.w);
+      if (fz.onorm) {  // output epilogue: head-wise RMSNorm x sigmoid gate over the Dv columns
+        float ss = col_ok ? y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w : 0.f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
+        if (col_ok) {
+          float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+          if (fz.og) {
+            const Tin* gp = reinterpret_cast<const Tin*>(fz.og) + vec_base(t) * Dv + col;
+            wv.x *= sigmoid_f(to_f32(gp[0]));
+            wv.y *= sigmoid_f(to_f32(gp[1]));
+            wv.z *= sigmoid_f(to_f32(gp[2]));
+            wv.w *= sigmoid_f(to_f32(gp[3]));
+          }
+          y = make_float4(y.x * inv * wv.x, y.y * inv * wv.y, y.z * inv * wv.z, y.w * inv * wv.w);
+        }
+      }
+      if (col_ok) {
+        Tin* op = o + vec_base(t) * Dv + col;
+        op[0] = from_f32<Tin>(y.x);
+        op[1] = from_f32<Tin>(y.y);
+        op[2] = from_f32<Tin>(y.z);
+        op[3] = from_f32<Tin>(y.w);
+      }
     }
     __syncthreads();  // s_a / s_k / s_q / s_e / s_p are rewritten by the next token
   }

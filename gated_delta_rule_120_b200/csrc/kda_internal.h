@@ -32,6 +32,10 @@ struct Fusion {
   float eps = 0.f;
   const float* A_log = nullptr;    // [H]; non-null: the decay input is the raw gate
   const float* dt_bias = nullptr;  // [H, Dk] or null
+  int onorm = 0;                   // output epilogue: head-wise RMSNorm x sigmoid gate
+  float oeps = 0.f;
+  const float* ow = nullptr;       // [Dv] norm weight or null (ones)
+  const void* og = nullptr;        // gate in o's layout and dtype, or null
 };
 
 // Arguments of one kda_chunk_fwd call after host validation.
@@ -100,6 +104,11 @@ cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, in
                                 float* records, const SimtRecord& rec, cudaStream_t stream);
 
 size_t simt_local_smem_bytes(int C, int Dk, int Dv);
+
+// The output epilogue as its own in-place pass over o (rows = token-head pairs); cu_end (device,
+// may be null) bounds the rows to cu_seqlens[N] * H.
+cudaError_t launch_output_norm_gate(void* o, kda_dtype_t dt, const Fusion& fz, long long rows,
+                                    int H, int Dv, const int32_t* cu_end, cudaStream_t stream);
 size_t simt_state_smem_bytes(int C, int Dk);
 
 }  // namespace kda

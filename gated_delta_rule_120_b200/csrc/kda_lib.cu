@@ -6,4 +6,5 @@
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
 #include "kda_chunk_tc.cu"
+#include "kda_epilogue.cu"
 #include "kda_noalloc.cu"

@@ -183,13 +183,23 @@ KDA_API kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void*
                                        kda_stream_t stream);
 
 /*
- * Prologue fusion for the two steps that precede the operator in the model ("Kimi Linear: An
- * Expressive, Efficient Attention Architecture", paper-graph-ui walkthrough, §3.4 "Neural
- * Parameterization": q, k = L2Norm(...) and alpha = f(low-rank gate); the L2 Deep Distill page's
- * implementation notes: L2 normalisation of q and k inside the kernel, and the decay gate fused
- * with A_log and a bias). The pages leave f unspecified beyond "similar to GDN and Mamba2, in log
- * space"; this library reads it as
+ * Fusion of the steps around the operator in the model ("Kimi Linear: An Expressive, Efficient
+ * Attention Architecture", paper-graph-ui walkthrough, §3.4 "Neural Parameterization").
+ *
+ * Prologue: q, k = L2Norm(...) and alpha = f(low-rank gate); the L2 Deep Distill page's
+ * implementation notes put the L2 normalisation of q and k inside the kernel and fuse the decay
+ * gate with A_log and a bias. The pages leave f unspecified beyond "similar to GDN and Mamba2, in
+ * log space"; this library reads it as
  *     log alpha[t, h, c] = -exp(A_log[h]) * softplus(g[t, h, c] + dt_bias[h, c]).
+ *
+ * Epilogue: the output-gate equation of the same section applies, per (token, head), a head-wise
+ * RMSNorm and a sigmoid gate to the operator's output (the module table of the L2 Deep Distill
+ * page names it FusedRMSNormGated: the sigmoid gate inside the RMSNorm). With out_norm set the
+ * library stores, instead of o,
+ *     y[t, h, c] = sigmoid(out_gate[t, h, c]) * out_norm_weight[c] * o[t, h, c]
+ *                  / sqrt(mean_c' o[t, h, c']^2 + out_norm_eps)
+ * where o is the fp32 result before rounding. The output projection W_o that follows is a plain
+ * GEMM and stays with the caller.
  */
 typedef struct {
   int32_t qk_l2norm;     /* nonzero: q and k are divided by sqrt(sum x^2 + qk_l2norm_eps) per
@@ -198,9 +208,16 @@ typedef struct {
   const float* A_log;    /* device fp32 [H], or NULL. Non-NULL: the log_alpha argument holds the
                             raw gate g (same layout) and the decay is computed as above */
   const float* dt_bias;  /* device fp32 [H, Dk], or NULL for a zero bias; used only with A_log */
+  int32_t out_norm;      /* nonzero: the output epilogue above replaces o by y */
+  float out_norm_eps;    /* e.g. 1e-5; must be >= 0 */
+  const float* out_norm_weight; /* device fp32 [Dv] (16-byte aligned), or NULL for ones */
+  const void* out_gate;  /* device, o's layout and dtype ([B,T,H,Dv] / [N,T,H,Dv]), or NULL for
+                            no gate; used only with out_norm. 16-byte aligned for bf16 prefill */
 } kda_fusion_t;
 
-/* kda_chunk_fwd with the prologue fusion above; fusion == NULL is exactly kda_chunk_fwd. */
+/* kda_chunk_fwd with the fusion above; fusion == NULL is exactly kda_chunk_fwd. With out_norm on
+ * the bf16 path, the state kernel runs as clusters of two CTAs (the two column halves of one
+ * (sequence, head)) that exchange per-row sums of squares through distributed shared memory. */
 KDA_API kda_status_t kda_chunk_fwd_fused(const void* q, const void* k, const void* v,
                                          kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,
                                          const float* beta, const float* initial_state,
@@ -210,7 +227,7 @@ KDA_API kda_status_t kda_chunk_fwd_fused(const void* q, const void* k, const voi
                                          void* workspace, size_t workspace_bytes,
                                          const kda_fusion_t* fusion, kda_stream_t stream);
 
-/* kda_recurrent_fwd with the prologue fusion above; fusion == NULL is exactly kda_recurrent_fwd. */
+/* kda_recurrent_fwd with the fusion above; fusion == NULL is exactly kda_recurrent_fwd. */
 KDA_API kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const void* v,
                                              kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,
                                              const float* beta, float* state_pool,

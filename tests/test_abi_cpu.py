@@ -125,3 +125,25 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(kda, "_lib", None)
     with pytest.raises(ImportError):
         kda.lib()
+
+
+def test_fusion_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes mirror of kda_fusion_t has the C compiler's size and offsets."""
+    import ctypes
+    import subprocess
+
+    import gated_delta_rule_120_b200 as kda
+
+    src = tmp_path / "layout.c"
+    fields = [f[0] for f in kda.Fusion._fields_]
+    body = "".join(f'  printf("%zu\\n", offsetof(kda_fusion_t, {f}));\n' for f in fields)
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "kda.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(kda_fusion_t));\n' + body + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(root, "include"), "-o", str(exe),
+                    str(src)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    want = [ctypes.sizeof(kda.Fusion)] + [getattr(kda.Fusion, f).offset for f in fields]
+    assert got == want

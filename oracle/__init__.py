@@ -13,6 +13,8 @@ Functions
   chunked(...)             the chunkwise WY/UT evaluation of §3.4 "Chunkwise Parallelization"
                            (Eq. 8, Eq. 9), fp64; pins the chunk algebra against ``recurrent``.
   unit_lower_inverse(A)    (I + A)^{-1} by forward substitution (the UT transform's inverse).
+  recurrent_bwd(...)       reverse-mode derivative of ``recurrent`` (the backward pass): gradients
+                           of <d_o, o> + <d_final, S_T> with respect to every input.
   prologue(...)            the fused input steps: L2-normalised q, k and the log-space decay gate
                            log alpha = -exp(A_log[h]) * softplus(g + dt_bias[h, c]) (walkthrough
                            §3.4 "Neural Parameterization"; the L2 Deep Distill page's
@@ -71,6 +73,9 @@ def _load():
             lib.kda_oracle_chunked.restype = ctypes.c_int
             lib.kda_oracle_unit_lower_inverse.argtypes = [_dp, ctypes.c_int64, _dp]
             lib.kda_oracle_unit_lower_inverse.restype = None
+            lib.kda_oracle_recurrent_bwd.argtypes = sig + [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                                            ctypes.c_int]
+            lib.kda_oracle_recurrent_bwd.restype = ctypes.c_int
             lib.kda_oracle_max_threads.argtypes = []
             lib.kda_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -208,3 +213,24 @@ def output_norm_gate(o, gate=None, weight=None, eps=1e-6):
     if gate is not None:
         y = y * _sigmoid(_f64(gate).reshape(o.shape))
     return y
+
+
+def recurrent_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final=None,
+                  cu_seqlens=None, nthreads: int = 0):
+    """fp64 gradients (d_q, d_k, d_v, d_log_alpha, d_beta, d_initial) of
+    L = <d_o, o> + <d_final, final_state> for the recurrence of :func:`recurrent` (same input
+    conventions; d_o has o's shape, d_final the state's)."""
+    q, k, v, la, b, s0, cu, N, H, Dk, Dv = _prep(q, k, v, log_alpha, beta, initial_state,
+                                                 cu_seqlens)
+    T = q.shape[0]
+    do = _f64(d_o).reshape(T, H, Dv)
+    dfin = None if d_final is None else _f64(d_final).reshape(N, H, Dk, Dv)
+    dq = np.zeros((T, H, Dk)); dk = np.zeros((T, H, Dk)); dla = np.zeros((T, H, Dk))
+    dv = np.zeros((T, H, Dv)); db = np.zeros((T, H)); ds0 = np.zeros((N, H, Dk, Dv))
+    rc = _load().kda_oracle_recurrent_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0),
+                                          cu.ctypes.data_as(_i64p), N, H, Dk, Dv, _ptr(do),
+                                          _ptr(dfin), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla),
+                                          _ptr(db), _ptr(ds0), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle: kda_oracle_recurrent_bwd failed")
+    return dq, dk, dv, dla, db, ds0

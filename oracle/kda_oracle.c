@@ -274,3 +274,165 @@ int kda_oracle_chunked(const double* q, const double* k, const double* v, const 
   }
   return bad;
 }
+
+/*
+ * Reverse-mode derivative of kda_oracle_recurrent (the backward pass of the operator; the pages
+ * motivate it through training: [W] §3.4 "Chunkwise Parallelization" calls the UT transform
+ * central to training, and "FLOPs Accounting and Inference Strategy" counts training FLOPs).
+ *
+ * Given the output cotangent d_o [T_total, H, Dv] and the final-state cotangent d_final
+ * [N, H, Dk, Dv] (NULL = 0), returns the gradients of L = <d_o, o> + <d_final, S_T> with respect
+ * to q, k (d_q, d_k [T_total, H, Dk]), v (d_v), log_alpha (d_log_alpha), beta (d_beta [T_total,
+ * H]) and the initial state (d_initial [N, H, Dk, Dv]; may be NULL). Tokens outside every
+ * sequence get zero gradients.
+ *
+ * The forward step, with S' = Diag(alpha) S_{t-1}, e = S'^T k, u = beta (v - e),
+ * S_t = S' + k u^T, o_t = S_t^T q, is walked backwards with the running cotangent dS of S_t:
+ *     dS   += q d_o^T              d_q = S_t d_o
+ *     du    = dS^T k               d_k = dS u
+ *     d_beta = du . (v - e)        d_v = beta du            de = -beta du
+ *     dS'   = dS + k de^T          d_k += S' de
+ *     d_log_alpha[a] = sum_j dS'[a, j] S'[a, j]             dS_{t-1} = Diag(alpha) dS'
+ * The states of each sequence are recomputed forward from checkpoints every `seg` tokens.
+ */
+int kda_oracle_recurrent_bwd(const double* q, const double* k, const double* v,
+                             const double* log_alpha, const double* beta,
+                             const double* initial_state, const int64_t* cu_seqlens, int64_t N,
+                             int64_t H, int64_t Dk, int64_t Dv, const double* d_o,
+                             const double* d_final, double* d_q, double* d_k, double* d_v,
+                             double* d_log_alpha, double* d_beta, double* d_initial,
+                             int nthreads) {
+  if (!q || !k || !v || !log_alpha || !beta || !cu_seqlens || !d_o || !d_q || !d_k || !d_v ||
+      !d_log_alpha || !d_beta)
+    return 1;
+  if (N < 0 || H <= 0 || Dk <= 0 || Dv <= 0) return 1;
+  const int64_t T_total = cu_seqlens[N];
+  memset(d_q, 0, sizeof(double) * T_total * H * Dk);
+  memset(d_k, 0, sizeof(double) * T_total * H * Dk);
+  memset(d_log_alpha, 0, sizeof(double) * T_total * H * Dk);
+  memset(d_v, 0, sizeof(double) * T_total * H * Dv);
+  memset(d_beta, 0, sizeof(double) * T_total * H);
+  set_threads(nthreads);
+  const int64_t seg = 32;
+  const int64_t SS = Dk * Dv;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t nh = 0; nh < N * H; ++nh) {
+    const int64_t n = nh / H, h = nh % H;
+    const int64_t t_begin = cu_seqlens[n], len = cu_seqlens[n + 1] - cu_seqlens[n];
+    const int64_t nseg = (len + seg - 1) / seg;
+    /* checkpoints: state before each segment; states: S_{t0 - 1}, ..., S_{t0 + seg - 1} */
+    double* ckpt = (double*)malloc(sizeof(double) * SS * (nseg + 1));
+    double* S = (double*)malloc(sizeof(double) * SS);
+    double* states = (double*)malloc(sizeof(double) * SS * (seg + 1));
+    double* dS = (double*)malloc(sizeof(double) * SS);
+    double* Sp = (double*)malloc(sizeof(double) * SS);
+    double* e = (double*)malloc(sizeof(double) * Dv);
+    double* u = (double*)malloc(sizeof(double) * Dv);
+    double* du = (double*)malloc(sizeof(double) * Dv);
+    double* de = (double*)malloc(sizeof(double) * Dv);
+    if (!ckpt || !S || !states || !dS || !Sp || !e || !u || !du || !de) {
+      bad |= 1;
+      free(ckpt); free(S); free(states); free(dS); free(Sp); free(e); free(u); free(du); free(de);
+      continue;
+    }
+    /* forward pass over the sequence, keeping the state before every segment */
+    for (int64_t x = 0; x < SS; ++x) S[x] = initial_state ? initial_state[nh * SS + x] : 0.0;
+    for (int64_t t = 0; t < len; ++t) {
+      if (t % seg == 0) memcpy(ckpt + (t / seg) * SS, S, sizeof(double) * SS);
+      const int64_t tt = t_begin + t;
+      for (int64_t a = 0; a < Dk; ++a) {
+        const double al = exp(log_alpha[IDX3(tt, h, a, H, Dk)]);
+        for (int64_t j = 0; j < Dv; ++j) S[a * Dv + j] *= al;
+      }
+      for (int64_t j = 0; j < Dv; ++j) {
+        double acc = 0.0;
+        for (int64_t a = 0; a < Dk; ++a) acc += S[a * Dv + j] * k[IDX3(tt, h, a, H, Dk)];
+        u[j] = beta[tt * H + h] * (v[IDX3(tt, h, j, H, Dv)] - acc);
+      }
+      for (int64_t a = 0; a < Dk; ++a)
+        for (int64_t j = 0; j < Dv; ++j) S[a * Dv + j] += k[IDX3(tt, h, a, H, Dk)] * u[j];
+    }
+    for (int64_t x = 0; x < SS; ++x) dS[x] = d_final ? d_final[nh * SS + x] : 0.0;
+    for (int64_t sg = nseg - 1; sg >= 0; --sg) {
+      const int64_t s0 = sg * seg, s1 = (s0 + seg < len) ? s0 + seg : len;
+      /* recompute S_{s0-1} .. S_{s1-1} into states[0 .. s1-s0] */
+      memcpy(states, ckpt + sg * SS, sizeof(double) * SS);
+      for (int64_t t = s0; t < s1; ++t) {
+        const int64_t tt = t_begin + t;
+        const double* P = states + (t - s0) * SS;
+        double* Q = states + (t - s0 + 1) * SS;
+        for (int64_t a = 0; a < Dk; ++a) {
+          const double al = exp(log_alpha[IDX3(tt, h, a, H, Dk)]);
+          for (int64_t j = 0; j < Dv; ++j) Q[a * Dv + j] = al * P[a * Dv + j];
+        }
+        for (int64_t j = 0; j < Dv; ++j) {
+          double acc = 0.0;
+          for (int64_t a = 0; a < Dk; ++a) acc += Q[a * Dv + j] * k[IDX3(tt, h, a, H, Dk)];
+          u[j] = beta[tt * H + h] * (v[IDX3(tt, h, j, H, Dv)] - acc);
+        }
+        for (int64_t a = 0; a < Dk; ++a)
+          for (int64_t j = 0; j < Dv; ++j) Q[a * Dv + j] += k[IDX3(tt, h, a, H, Dk)] * u[j];
+      }
+      /* reverse steps */
+      for (int64_t t = s1 - 1; t >= s0; --t) {
+        const int64_t tt = t_begin + t;
+        const double* Sprev = states + (t - s0) * SS;
+        const double* Scur = states + (t - s0 + 1) * SS;
+        const double b = beta[tt * H + h];
+        for (int64_t a = 0; a < Dk; ++a) {
+          const double al = exp(log_alpha[IDX3(tt, h, a, H, Dk)]);
+          for (int64_t j = 0; j < Dv; ++j) Sp[a * Dv + j] = al * Sprev[a * Dv + j];
+        }
+        for (int64_t j = 0; j < Dv; ++j) {
+          double acc = 0.0;
+          for (int64_t a = 0; a < Dk; ++a) acc += Sp[a * Dv + j] * k[IDX3(tt, h, a, H, Dk)];
+          e[j] = acc;
+          u[j] = b * (v[IDX3(tt, h, j, H, Dv)] - acc);
+        }
+        /* o_t = S_t^T q_t */
+        for (int64_t a = 0; a < Dk; ++a) {
+          double acc = 0.0;
+          for (int64_t j = 0; j < Dv; ++j) {
+            dS[a * Dv + j] += q[IDX3(tt, h, a, H, Dk)] * d_o[IDX3(tt, h, j, H, Dv)];
+            acc += Scur[a * Dv + j] * d_o[IDX3(tt, h, j, H, Dv)];
+          }
+          d_q[IDX3(tt, h, a, H, Dk)] = acc;
+        }
+        /* S_t = S' + k u^T */
+        for (int64_t j = 0; j < Dv; ++j) {
+          double acc = 0.0;
+          for (int64_t a = 0; a < Dk; ++a) acc += dS[a * Dv + j] * k[IDX3(tt, h, a, H, Dk)];
+          du[j] = acc;
+        }
+        double db = 0.0;
+        for (int64_t j = 0; j < Dv; ++j) {
+          db += du[j] * (v[IDX3(tt, h, j, H, Dv)] - e[j]);
+          d_v[IDX3(tt, h, j, H, Dv)] = b * du[j];
+          de[j] = -b * du[j];
+        }
+        d_beta[tt * H + h] = db;
+        for (int64_t a = 0; a < Dk; ++a) {
+          double acc = 0.0;
+          for (int64_t j = 0; j < Dv; ++j) acc += dS[a * Dv + j] * u[j] + Sp[a * Dv + j] * de[j];
+          d_k[IDX3(tt, h, a, H, Dk)] = acc;
+        }
+        /* e = S'^T k: dS' = dS + k de^T; S' = Diag(alpha) S_{t-1} */
+        for (int64_t a = 0; a < Dk; ++a) {
+          const double ka = k[IDX3(tt, h, a, H, Dk)];
+          const double al = exp(log_alpha[IDX3(tt, h, a, H, Dk)]);
+          double acc = 0.0;
+          for (int64_t j = 0; j < Dv; ++j) {
+            const double dsp = dS[a * Dv + j] + ka * de[j];
+            acc += dsp * Sp[a * Dv + j];
+            dS[a * Dv + j] = al * dsp;
+          }
+          d_log_alpha[IDX3(tt, h, a, H, Dk)] = acc;
+        }
+      }
+    }
+    if (d_initial) memcpy(d_initial + nh * SS, dS, sizeof(double) * SS);
+    free(ckpt); free(S); free(states); free(dS); free(Sp); free(e); free(u); free(du); free(de);
+  }
+  return bad ? 1 : 0;
+}

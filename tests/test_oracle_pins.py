@@ -364,3 +364,78 @@ def test_output_norm_gate_structure():
     np.testing.assert_allclose(g_open, y, rtol=1e-15)
     g_shut = oracle.output_norm_gate(o, gate=np.full(o.shape, -800.0), eps=0.0)
     assert np.all(np.abs(g_shut) < 1e-300)
+
+
+# --- backward pass: reverse-mode derivative of the recurrence ---------------------------------
+def _loss(x, cu, d_o, d_fin):
+    o, S = oracle.recurrent(x["q"], x["k"], x["v"], x["la"], x["beta"], x["s0"], cu_seqlens=cu)
+    return float(np.sum(o * d_o) + np.sum(S * d_fin))
+
+
+def _bwd_case(seed, lens, H, Dk, Dv):
+    rng = np.random.default_rng(seed)
+    T = sum(lens)
+    q, k, v, la, beta = _rand_inputs(rng, T, H, Dk, Dv, unit_keys=False)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    s0 = rng.standard_normal((len(lens), H, Dk, Dv))
+    x = dict(q=q, k=k, v=v, la=la, beta=beta, s0=s0)
+    d_o = rng.standard_normal((T, H, Dv))
+    d_fin = rng.standard_normal((len(lens), H, Dk, Dv))
+    g = oracle.recurrent_bwd(q, k, v, la, beta, d_o, initial_state=s0, d_final=d_fin,
+                             cu_seqlens=cu)
+    return x, cu, d_o, d_fin, dict(zip(("q", "k", "v", "la", "beta", "s0"), g))
+
+
+def _central_difference(x, cu, d_o, d_fin, name, idx, h=1e-6):
+    xp = {n: a.copy() for n, a in x.items()}
+    xp[name][idx] += h
+    lp = _loss(xp, cu, d_o, d_fin)
+    xp[name][idx] -= 2 * h
+    lm = _loss(xp, cu, d_o, d_fin)
+    return (lp - lm) / (2 * h)
+
+
+def test_backward_matches_finite_differences_everywhere():
+    """Every partial derivative of <d_o, o> + <d_final, S_T> (q, k, v, log alpha, beta, S_0) on
+    two short sequences equals its central finite difference; Dk != Dv catches transposes."""
+    x, cu, d_o, d_fin, g = _bwd_case(51, [4, 3], 2, 3, 2)
+    for name in ("q", "k", "v", "la", "beta", "s0"):
+        for idx in np.ndindex(*x[name].shape):
+            fd = _central_difference(x, cu, d_o, d_fin, name, idx)
+            assert abs(fd - g[name][idx]) <= 1e-7 * max(1.0, abs(fd)), (name, idx, fd,
+                                                                        g[name][idx])
+
+
+def test_backward_across_recompute_segments():
+    """A 75-token sequence crosses the oracle's 32-token recompute segments; sampled partial
+    derivatives in every segment equal their finite differences."""
+    x, cu, d_o, d_fin, g = _bwd_case(52, [75], 1, 4, 3)
+    rng = np.random.default_rng(53)
+    for name in ("q", "k", "v", "la", "beta"):
+        for t in (0, 5, 31, 32, 33, 63, 64, 74):
+            idx = (t, 0) if name == "beta" else (t, 0, int(rng.integers(x[name].shape[-1])))
+            fd = _central_difference(x, cu, d_o, d_fin, name, idx)
+            assert abs(fd - g[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx)
+    for idx in ((0, 0, 0, 0), (0, 0, 3, 2)):
+        fd = _central_difference(x, cu, d_o, d_fin, "s0", idx)
+        assert abs(fd - g["s0"][idx]) <= 1e-6 * max(1.0, abs(fd))
+
+
+def test_backward_closed_form_without_writes():
+    """beta = 0: S_t = Gamma_t S_0 (pure decay), so d_q_t = S_t d_o_t, d_v = d_k = 0 and
+    d_S_0 = sum_t Gamma_t q_t d_o_t^T + Gamma_T d_final (written out, no recurrence)."""
+    rng = np.random.default_rng(54)
+    T, H, Dk, Dv = 6, 1, 3, 2
+    q, k, v, la, _ = _rand_inputs(rng, T, H, Dk, Dv)
+    beta = np.zeros((T, H))
+    s0 = rng.standard_normal((1, H, Dk, Dv))
+    d_o = rng.standard_normal((T, H, Dv))
+    d_fin = rng.standard_normal((1, H, Dk, Dv))
+    dq, dk, dv, dla, db, ds0 = oracle.recurrent_bwd(q, k, v, la, beta, d_o, initial_state=s0,
+                                                    d_final=d_fin)
+    gam = np.exp(np.cumsum(la[:, 0], axis=0))  # [T, Dk]
+    S_t = gam[:, :, None] * s0[0, 0][None]
+    np.testing.assert_allclose(dq[:, 0], np.einsum("tkv,tv->tk", S_t, d_o[:, 0]), rtol=1e-13)
+    assert np.all(dv == 0) and np.all(dk == 0)
+    want = np.einsum("tk,tk,tv->kv", gam, q[:, 0], d_o[:, 0]) + gam[-1][:, None] * d_fin[0, 0]
+    np.testing.assert_allclose(ds0[0, 0], want, rtol=1e-13)

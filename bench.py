@@ -361,6 +361,31 @@ def run_recurrent_mode(N, T, H, D, dev, steps, warmup, world, seed):
     return timed(step, steps, warmup, world, dev)
 
 
+def run_backward(spec, seed, dev, steps, warmup, world):
+    """The backward pass (kda_chunk_bwd) of the standard prefill: gradients of every input for a
+    random output cotangent and final-state cotangent. Returns (ms over `steps`, profile)."""
+    import torch
+
+    import gated_delta_rule_120_b200 as kda
+    import kda_synth
+
+    x = kda_synth.prefill_inputs(spec, seed, dev)
+    g = torch.Generator(device=dev).manual_seed(seed + 3)
+    d_o = torch.randn(x["v"].shape, generator=g, device=dev).to(x["v"].dtype)
+    d_fin = torch.randn((spec.num_seqs, spec.H, spec.Dk, spec.Dv), generator=g, device=dev)
+    ws = torch.empty(kda.kda_chunk_bwd_workspace_size(spec.B, spec.T, spec.H, spec.Dk, spec.Dv,
+                                                      spec.num_seqs, x["q"].dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        kda.kda_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o,
+                          initial_state=x["initial_state"], d_final_state=d_fin, workspace=ws)
+
+    ms = timed(step, steps, warmup, world, dev)
+    prof = profile_pass(step, 2, dev)
+    return ms, prof
+
+
 def cpu_baseline(spec, dev, budget_s):
     """The fp64 oracle as it stands, on the host's cores, over whole sequences of the prefill
     workload (all heads), repeated until ~budget_s of CPU work. Returns tokens/s."""
@@ -543,6 +568,17 @@ def main():
         "ms_per_call": per,
         "achieved_gbs": rtotal / (per / 1e3) / 1e9,
         "frac_hbm": rtotal / (per / 1e3) / 1e9 / hbm_peak}
+    torch.cuda.empty_cache()
+    # the backward pass of the standard prefill
+    bsteps = max(3, args.steps // 4)
+    bms, bprof = run_backward(spec, 2007 + 10 * rank, dev, bsteps, 2, world)
+    extra["backward"] = {
+        "workload": spec.name + "_backward",
+        "tokens_per_s": whole_job_rate(tokens * bsteps, world, bms),
+        "ms_per_call": bms / bsteps,
+        "vs_forward": (bms / bsteps) / ms_step,
+        "kernels": [{"name": p["name"], "ms_per_launch": p["total_ms"] / p["launches"]}
+                    for p in bprof]}
     torch.cuda.empty_cache()
     if not args.no_decode:
         dspec = kda_synth.DECODE

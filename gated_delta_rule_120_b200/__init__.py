@@ -32,7 +32,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
                "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
-               "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused")
+               "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused",
+               "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
 
 
 class Fusion(ctypes.Structure):
@@ -93,6 +94,12 @@ def lib() -> ctypes.CDLL:
                                                   i32, i32, i32, i32, i32, i32,
                                                   ctypes.POINTER(Fusion), vp]
             L.kda_recurrent_fwd_fused.restype = ctypes.c_int
+            L.kda_chunk_bwd_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int,
+                                                                   ctypes.POINTER(sz)]
+            L.kda_chunk_bwd_workspace_size.restype = ctypes.c_int
+            L.kda_chunk_bwd.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32, i32, i32,
+                                        i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            L.kda_chunk_bwd.restype = ctypes.c_int
             L.kda_last_device_error.argtypes = [vp]
             L.kda_last_device_error.restype = ctypes.c_int
             L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32,
@@ -235,6 +242,58 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         code = lib().kda_chunk_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_chunk_fwd")
     return o, (final_state if output_final_state else None)
+
+
+def kda_chunk_bwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, num_seqs: int,
+                                 dtype: torch.dtype) -> int:
+    out = ctypes.c_size_t(0)
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    _check(lib().kda_chunk_bwd_workspace_size(B, T, H, Dk, Dv, num_seqs, code, ctypes.byref(out)),
+           "kda_chunk_bwd_workspace_size")
+    return int(out.value)
+
+
+def kda_chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None,
+                  cu_seqlens=None, need_d_initial: bool = True, workspace=None):
+    """Backward pass of :func:`kda_chunk_fwd` (same inputs, no fusion): gradients of
+    <d_o, o> + <d_final_state, final_state>. Returns (dq, dk, dv in q's dtype, dlog_alpha and
+    dbeta fp32, d_initial_state [N,H,Dk,Dv] fp32 or None)."""
+    dev = q.device
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
+        _need(t, n, dev, q.dtype)
+    _need(log_alpha, "log_alpha", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    if tuple(k.shape) != (B, T, H, Dk) or tuple(log_alpha.shape) != (B, T, H, Dk) or \
+            tuple(v.shape[:3]) != (B, T, H) or tuple(beta.shape) != (B, T, H) or \
+            tuple(d_o.shape) != tuple(v.shape):
+        raise ValueError("inconsistent q/k/v/log_alpha/beta/d_o shapes")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
+        if t is not None:
+            _need(t, n, dev, torch.float32)
+            if tuple(t.shape) != (N, H, Dk, Dv):
+                raise ValueError(f"{n} must be [N,H,Dk,Dv]")
+    dq, dk = torch.zeros_like(q), torch.zeros_like(k)
+    dv = torch.zeros_like(v)
+    dla = torch.zeros_like(log_alpha)
+    db = torch.zeros_like(beta)
+    ds0 = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev) if need_d_initial else None
+    ws_bytes = kda_chunk_bwd_workspace_size(B, T, H, Dk, Dv, N, q.dtype)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    code = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
+                               _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk,
+                               Dv, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(dla), _ptr(db), _ptr(ds0), _ptr(workspace), workspace.numel(),
+                               _stream_handle(dev))
+    _check(code, "kda_chunk_bwd")
+    return dq, dk, dv, dla, db, ds0
 
 
 def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):

@@ -64,6 +64,51 @@ WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
 
 kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// Backward pass: chunk of 32 tokens, fp32 arithmetic for both input dtypes.
+constexpr int32_t kBwdChunk = 32;
+
+kda_status_t check_backward_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                  int32_t N, kda_dtype_t dt, bool varlen) {
+  if (B < 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || N < 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (varlen) {
+    if (B != 1 && !(B == 0 && T == 0)) return KDA_ERR_INVALID_ARG;
+  } else if (N != B) {
+    return KDA_ERR_INVALID_ARG;
+  }
+  if (Dk > 128 || Dv > 128) return KDA_ERR_UNSUPPORTED;
+  const long long tokens = (long long)B * T;
+  const long long elems = tokens * H * (long long)(Dk > Dv ? Dk : Dv);
+  if (tokens > INT32_MAX || elems > (1LL << 40)) return KDA_ERR_UNSUPPORTED;
+  return KDA_OK;
+}
+
+// Workspace layout of one backward call:
+//   header | chunk_off | fp32 records (with T and B) | states entering every chunk |
+//   cotangents of the states leaving every chunk | dV' [B*T, H, Dv]
+struct BwdLayout {
+  size_t chunk_off_base, rec_base, states_base, dstates_base, dvp_base, total;
+  long long max_chunks;
+};
+
+BwdLayout backward_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv, int32_t N,
+                          bool varlen) {
+  BwdLayout w;
+  const int32_t C = kBwdChunk;
+  const long long tokens = (long long)B * T;
+  w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
+  w.chunk_off_base = 256;
+  const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * ((size_t)N + 1), 256) : 0;
+  w.rec_base = w.chunk_off_base + off_bytes;
+  const size_t rec_bytes = SimtRecord::make(C, Dk, Dv, true).record_floats * sizeof(float);
+  const size_t state_bytes = (size_t)Dk * Dv * sizeof(float);
+  w.states_base = w.rec_base + (size_t)w.max_chunks * H * rec_bytes;
+  w.dstates_base = align_up(w.states_base + (size_t)w.max_chunks * H * state_bytes, 256);
+  w.dvp_base = align_up(w.dstates_base + (size_t)w.max_chunks * H * state_bytes, 256);
+  w.total = align_up(w.dvp_base + (size_t)tokens * H * Dv * sizeof(float), 256);
+  return w;
+}
+
 }  // namespace
 }  // namespace kda
 
@@ -96,6 +141,97 @@ kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32
   if (st != KDA_OK) return st;
   *bytes = prefill_layout(B, T, H, Dk, Dv, chunk, varlen ? num_seqs : B, varlen, dt).total;
   return KDA_OK;
+}
+
+kda_status_t kda_chunk_bwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                                          int32_t num_seqs, kda_dtype_t dt, size_t* bytes) {
+  if (!bytes) return KDA_ERR_INVALID_ARG;
+  const bool varlen = (B == 1);
+  kda_status_t st = check_backward_shape(B, T, H, Dk, Dv, varlen ? num_seqs : B, dt, varlen);
+  if (st != KDA_OK) return st;
+  *bytes = backward_layout(B, T, H, Dk, Dv, varlen ? num_seqs : B, varlen).total;
+  return KDA_OK;
+}
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                           const float* log_alpha, const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t N, int32_t B, int32_t T, int32_t H,
+                           int32_t Dk, int32_t Dv, const void* d_o, const float* d_final_state,
+                           void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
+                           float* d_initial_state, void* workspace, size_t workspace_bytes,
+                           kda_stream_t stream_) {
+  const bool varlen = cu_seqlens != nullptr;
+  kda_status_t st = check_backward_shape(B, T, H, Dk, Dv, N, dt, varlen);
+  if (st != KDA_OK) return st;
+  const long long tokens = (long long)B * T;
+  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+  if (tokens > 0) {
+    if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk || !dv || !dlog_alpha ||
+        !dbeta)
+      return KDA_ERR_INVALID_ARG;
+    if (!aligned(q, es) || !aligned(k, es) || !aligned(v, es) || !aligned(d_o, es) ||
+        !aligned(dq, es) || !aligned(dk, es) || !aligned(dv, es) || !aligned(log_alpha, 4) ||
+        !aligned(beta, 4) || !aligned(dlog_alpha, 4) || !aligned(dbeta, 4))
+      return KDA_ERR_INVALID_ARG;
+  }
+  if ((initial_state && !aligned(initial_state, 4)) ||
+      (d_final_state && !aligned(d_final_state, 4)) ||
+      (d_initial_state && !aligned(d_initial_state, 4)) || (varlen && !aligned(cu_seqlens, 4)))
+    return KDA_ERR_INVALID_ARG;
+  if (N == 0) return KDA_OK;
+  const BwdLayout lay = backward_layout(B, T, H, Dk, Dv, N, varlen);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < lay.total)
+    return KDA_ERR_WORKSPACE;
+
+  cudaStream_t stream = (cudaStream_t)stream_;
+  char* ws = (char*)workspace;
+  int32_t* valid = (int32_t*)ws;
+  int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
+  if (varlen) {
+    st = from_cuda(
+        launch_chunk_map(cu_seqlens, N, (int)tokens, kBwdChunk, chunk_off, valid, stream));
+    if (st != KDA_OK) return st;
+  }
+  SeqGeometry geo;
+  geo.cu_seqlens = cu_seqlens;
+  geo.chunk_off = chunk_off;
+  geo.valid = valid;
+  geo.N = N;
+  geo.T = T;
+  geo.C = kBwdChunk;
+
+  BackwardArgs b;
+  PrefillArgs& a = b.fwd;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dtype = dt;
+  a.log_alpha = log_alpha;
+  a.beta = beta;
+  a.initial_state = initial_state;
+  a.cu_seqlens = cu_seqlens;
+  a.N = N;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.Dk = Dk;
+  a.Dv = Dv;
+  a.C = kBwdChunk;
+  a.o = nullptr;
+  a.final_state = nullptr;
+  b.d_o = d_o;
+  b.d_final = d_final_state;
+  b.dq = dq;
+  b.dk = dk;
+  b.dv = dv;
+  b.dlog_alpha = dlog_alpha;
+  b.dbeta = dbeta;
+  b.d_initial = d_initial_state;
+  const SimtRecord rec = SimtRecord::make(kBwdChunk, Dk, Dv, true);
+  return from_cuda(launch_chunk_bwd(b, geo, (int)lay.max_chunks, (float*)(ws + lay.rec_base), rec,
+                                    (float*)(ws + lay.states_base),
+                                    (float*)(ws + lay.dstates_base), (float*)(ws + lay.dvp_base),
+                                    stream));
 }
 
 }  // extern "C"

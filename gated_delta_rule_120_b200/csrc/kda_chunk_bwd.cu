@@ -1,0 +1,475 @@
+// kda_chunk_bwd.cu — backward pass of the chunkwise KDA operator (fp32 arithmetic, CUDA cores).
+//
+// Reverse-mode derivative of the chunk form of "Kimi Linear: An Expressive, Efficient Attention
+// Architecture" (paper-graph-ui walkthrough, §3.4 "Chunkwise Parallelization": the UT transform,
+// Eq. 8 and Eq. 9), for gradients of L = <dO, O> + <dS_T, S_T>. Per chunk, with the chunk-start
+// state S, the notation of the forward kernels (g cumulative log decay, Qt = Gamma.Q,
+// Kt = (gamma_C / gamma_i) k_i, P = Tril((Gamma.Q)(K/Gamma)^T), A = StrictTril(Diag(beta) B),
+// B = (Gamma.K)(K/Gamma)^T, T = (I + A)^{-1}, M = T Diag(beta), W = M Gamma.K, U = M V,
+// V' = U - W S) and dS' the cotangent of the state leaving the chunk:
+//
+//   state pass, sequential over chunks backwards (chunk_state_bwd):
+//       dV' = P^T dO + Kt dS'          dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV'
+//   chunk-local pass, all chunks in parallel (chunk_local_bwd):
+//       dQt = dO S^T    dW = -dV' S^T    dKt = V' dS'^T    dgamma_C = rowsum(dS' . S)
+//       dP = Tril(dO V'^T)               dM = Tril(dW (Gamma.K)^T + dV' V^T)
+//       dbeta += colsum(dM . T)          dT = dM Diag(beta)     dA = -StrictTril(T^T dT T^T)
+//       dbeta += rowsum(dA . B)          d(Gamma.K) = M^T dW     dV = M^T dV'
+//   and the products through A and P are differentiated in ratio form, exp(g_r - g_i) <= 1 for
+//   i <= r, so no factor overflows for any decay:
+//       dk_r += sum_i dA_ri beta_r k_i e_ri      dk_i += sum_r (dA_ri beta_r k_r + dP_ri q_r) e_ri
+//       dq_r += sum_i dP_ri k_i e_ri             dg_r += s_ri,  dg_i -= s_ri,
+//       s_ri = (dA_ri beta_r k_r + dP_ri q_r) k_i e_ri     (per key channel, elementwise)
+//   then the elementwise maps of Qt, Gamma.K, Kt, gamma_C onto q, k, g, and d log_alpha as the
+//   reverse cumulative sum of dg inside the chunk.
+//
+// The forward quantities come from the fp32 chunk kernels run first (records with T and B, and
+// the state entering every chunk). The backward pass uses chunks of 32 tokens whatever the
+// forward pass used (the result does not depend on the chunk size).
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwSlice = 32;  // value columns per CTA of the state pass
+
+// ----------------------------------------------------------------------------------------------
+// state pass: one CTA per (sequence, head, 32-column slice of d_v), chunks in reverse order
+// ----------------------------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(kBwdThreads)
+    chunk_state_bwd_kernel(const float* __restrict__ ws, SimtRecord rec, SeqGeometry geo, int H,
+                           int Dk, int Dv, const Tin* __restrict__ d_o,
+                           const float* __restrict__ d_final, float* __restrict__ d_initial,
+                           float* __restrict__ dstates, float* __restrict__ dvp) {
+  extern __shared__ float smem[];
+  const int C = geo.C;
+  float* sdS = smem;                 // [Dk][32] cotangent of the state leaving the chunk
+  float* sW = sdS + Dk * kBwSlice;   // [C][Dk]
+  float* sKt = sW + C * Dk;          // [C][Dk]
+  float* sQt = sKt + C * Dk;         // [C][Dk]
+  float* sP = sQt + C * Dk;          // [C][C]
+  float* sGam = sP + C * C;          // [Dk]
+  float* sdO = sGam + Dk;            // [C][32]
+  float* sdV = sdO + C * kBwSlice;   // [C][32]
+
+  if (!geo.ok()) return;
+  const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kBwSlice;
+  const int NV = min(kBwSlice, Dv - j0);
+  const int tid = threadIdx.x, nt = blockDim.x, j = tid & 31, rg = tid >> 5, ng = nt >> 5;
+  const size_t sbase = ((size_t)n * H + h) * Dk * Dv;
+
+  for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
+    const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
+    sdS[idx] = (d_final && jj < NV) ? d_final[sbase + (size_t)a * Dv + j0 + jj] : 0.f;
+  }
+  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
+  const int c_first = geo.first_chunk(n);
+  const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
+  for (int ci = nchunks - 1; ci >= 0; --ci) {
+    const int c = c_first + ci;
+    const int t0 = tb + ci * C;
+    const int L = min(C, te - t0);
+    const float* r_ = ws + rec.record_floats * ((size_t)c * H + h);
+    __syncthreads();  // the previous chunk is done with the staging buffers
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      sW[idx] = r_[rec.off_w + idx];
+      sKt[idx] = r_[rec.off_kt + idx];
+      sQt[idx] = r_[rec.off_qt + idx];
+    }
+    for (int idx = tid; idx < C * C; idx += nt) sP[idx] = r_[rec.off_aqk + idx];
+    for (int a = tid; a < Dk; a += nt) sGam[a] = r_[rec.off_gam + a];
+    for (int idx = tid; idx < C * kBwSlice; idx += nt) {
+      const int r = idx / kBwSlice, jj = idx - r * kBwSlice;
+      sdO[idx] = (r < L && jj < NV) ? to_f32(d_o[((size_t)(t0 + r) * H + h) * Dv + j0 + jj]) : 0.f;
+    }
+    {  // the cotangent entering from the right of this chunk, for the chunk-local pass
+      float* dst = dstates + ((size_t)c * H + h) * Dk * Dv;
+      for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
+        const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
+        if (jj < NV) dst[(size_t)a * Dv + j0 + jj] = sdS[idx];
+      }
+    }
+    __syncthreads();
+    // dV'[i][j] = sum_{r >= i} P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j]
+    for (int i = rg; i < C; i += ng) {
+      float acc = 0.f;
+      for (int r = i; r < C; ++r) acc += sP[r * C + i] * sdO[r * kBwSlice + j];
+      for (int a = 0; a < Dk; ++a) acc += sKt[i * Dk + a] * sdS[a * kBwSlice + j];
+      sdV[i * kBwSlice + j] = acc;
+      if (i < L && j < NV) dvp[((size_t)(t0 + i) * H + h) * Dv + j0 + j] = acc;
+    }
+    __syncthreads();
+    // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV'  (each thread owns its (a, j) elements)
+    for (int a = rg; a < Dk; a += ng) {
+      float acc = sGam[a] * sdS[a * kBwSlice + j];
+      for (int r = 0; r < C; ++r)
+        acc += sQt[r * Dk + a] * sdO[r * kBwSlice + j] - sW[r * Dk + a] * sdV[r * kBwSlice + j];
+      sdS[a * kBwSlice + j] = acc;
+    }
+  }
+  __syncthreads();
+  if (d_initial) {
+    for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
+      const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
+      if (jj < NV) d_initial[sbase + (size_t)a * Dv + j0 + jj] = sdS[idx];
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------------------
+// chunk-local pass: one CTA per (chunk, head); chunk = 32 tokens
+// ----------------------------------------------------------------------------------------------
+constexpr int kBwdC = 32;
+
+struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
+  int K, Q, G, V, dO, dV, X1, X2, X3, X4, Y1, Y2, T, P, B, dP, dM, X, beta, dgam, db, total;
+  __host__ __device__ static BwdSmem make(int Dk, int Dv) {
+    const int C = kBwdC, Dm = Dk > Dv ? Dk : Dv;
+    BwdSmem s;
+    int o = 0;
+    s.K = o; o += C * Dk;
+    s.Q = o; o += C * Dk;
+    s.G = o; o += C * Dk;
+    s.V = o; o += C * Dv;
+    s.dO = o; o += C * Dv;
+    s.dV = o; o += C * Dv;
+    s.X1 = o; o += C * Dm;   // V', then dg
+    s.X2 = o; o += C * Dk;   // dQt, then dq
+    s.X3 = o; o += C * Dk;   // dW, then dk
+    s.X4 = o; o += C * Dk;   // W, then dKt
+    s.Y1 = o; o += C * Dm;   // chunk-start state rows, then Gamma.K
+    s.Y2 = o; o += C * Dm;   // cotangent rows, then d(Gamma.K)
+    s.T = o; o += C * C;
+    s.P = o; o += C * C;
+    s.B = o; o += C * C;
+    s.dP = o; o += C * C;
+    s.dM = o; o += C * C;    // dM, then dT, then dA
+    s.X = o; o += C * C;
+    s.beta = o; o += C;
+    s.dgam = o; o += Dk;
+    s.db = o; o += C;
+    s.total = o;
+    return s;
+  }
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kBwdThreads)
+    chunk_local_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                           const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                           const float* __restrict__ beta, SeqGeometry geo, int H, int Dk, int Dv,
+                           const float* __restrict__ ws, SimtRecord rec,
+                           const float* __restrict__ states, const float* __restrict__ dstates,
+                           const float* __restrict__ dvp, const Tin* __restrict__ d_o,
+                           Tin* __restrict__ dq, Tin* __restrict__ dk, Tin* __restrict__ dv,
+                           float* __restrict__ dla, float* __restrict__ dbeta) {
+  extern __shared__ float smem[];
+  constexpr int C = kBwdC;
+  const BwdSmem L_ = BwdSmem::make(Dk, Dv);
+  float* sK = smem + L_.K;
+  float* sQ = smem + L_.Q;
+  float* sG = smem + L_.G;
+  float* sV = smem + L_.V;
+  float* sdO = smem + L_.dO;
+  float* sdV = smem + L_.dV;
+  float* X1 = smem + L_.X1;
+  float* X2 = smem + L_.X2;
+  float* X3 = smem + L_.X3;
+  float* X4 = smem + L_.X4;
+  float* Y1 = smem + L_.Y1;
+  float* Y2 = smem + L_.Y2;
+  float* sT = smem + L_.T;
+  float* sP = smem + L_.P;
+  float* sB = smem + L_.B;
+  float* sdP = smem + L_.dP;
+  float* sdM = smem + L_.dM;
+  float* sX = smem + L_.X;
+  float* sbeta = smem + L_.beta;
+  float* sdgam = smem + L_.dgam;
+  float* sdb = smem + L_.db;
+
+  if (!geo.ok()) return;
+  const int c = blockIdx.x, h = blockIdx.y;
+  if (c >= geo.num_chunks_total()) return;
+  const int n = geo.seq_of_chunk(c);
+  const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * C;
+  const int L = min(C, geo.seq_end(n) - t0);
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const float* r_ = ws + rec.record_floats * ((size_t)c * H + h);
+  const float* S0 = states + ((size_t)c * H + h) * Dk * Dv;   // state entering the chunk
+  const float* dS1 = dstates + ((size_t)c * H + h) * Dk * Dv; // cotangent of the state leaving it
+
+  // ---- P0: inputs, record, cumulative decay
+  for (int idx = tid; idx < C * Dk; idx += nt) {
+    const int r = idx / Dk, a = idx - r * Dk;
+    const bool in = r < L;
+    const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
+    sK[idx] = in ? to_f32(k[gi]) : 0.f;
+    sQ[idx] = in ? to_f32(q[gi]) : 0.f;
+    sG[idx] = in ? log_alpha[gi] : 0.f;
+    X4[idx] = r_[rec.off_w + idx];
+  }
+  for (int idx = tid; idx < C * Dv; idx += nt) {
+    const int r = idx / Dv, jj = idx - r * Dv;
+    const bool in = r < L;
+    const size_t gi = ((size_t)(t0 + r) * H + h) * Dv + jj;
+    sV[idx] = in ? to_f32(v[gi]) : 0.f;
+    sdO[idx] = in ? to_f32(d_o[gi]) : 0.f;
+    sdV[idx] = in ? dvp[gi] : 0.f;
+  }
+  for (int idx = tid; idx < C * C; idx += nt) {
+    sT[idx] = r_[rec.off_t + idx];
+    sP[idx] = r_[rec.off_aqk + idx];
+    sB[idx] = r_[rec.off_b + idx];
+  }
+  for (int r = tid; r < C; r += nt) sbeta[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+  __syncthreads();
+  for (int a = tid; a < Dk; a += nt) {
+    float acc = 0.f;
+    for (int r = 0; r < C; ++r) {
+      acc += sG[r * Dk + a];
+      sG[r * Dk + a] = acc;
+    }
+  }
+
+  // ---- P1: products with the chunk-start state S (rows streamed 32 at a time)
+  constexpr int kMaxPer = (C * 128 + kBwdThreads - 1) / kBwdThreads;  // outputs of V' per thread
+  float vp[kMaxPer];
+#pragma unroll
+  for (int m = 0; m < kMaxPer; ++m) {
+    const int idx = tid + m * nt;
+    vp[m] = idx < C * Dv ? r_[rec.off_u + idx] : 0.f;
+  }
+  for (int a0 = 0; a0 < Dk; a0 += 32) {
+    const int na = min(32, Dk - a0);
+    __syncthreads();  // previous slice consumed (and, the first time, the cumsum done)
+    for (int idx = tid; idx < na * Dv; idx += nt) {
+      Y1[idx] = S0[(size_t)a0 * Dv + idx];
+      Y2[idx] = dS1[(size_t)a0 * Dv + idx];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kMaxPer; ++m) {  // V' = U - W S
+      const int idx = tid + m * nt;
+      if (idx < C * Dv) {
+        const int r = idx / Dv, jj = idx - r * Dv;
+        float acc = 0.f;
+        for (int aa = 0; aa < na; ++aa) acc += X4[r * Dk + a0 + aa] * Y1[aa * Dv + jj];
+        vp[m] -= acc;
+      }
+    }
+    for (int idx = tid; idx < C * 32; idx += nt) {  // dQt = dO S^T, dW = -dV' S^T
+      const int r = idx >> 5, aa = idx & 31;
+      if (aa < na) {
+        float s1 = 0.f, s2 = 0.f;
+        for (int jj = 0; jj < Dv; ++jj) {
+          const float sv = Y1[aa * Dv + jj];
+          s1 += sdO[r * Dv + jj] * sv;
+          s2 += sdV[r * Dv + jj] * sv;
+        }
+        X2[r * Dk + a0 + aa] = s1;
+        X3[r * Dk + a0 + aa] = -s2;
+      }
+    }
+    for (int aa = tid; aa < na; aa += nt) {  // dgamma_C = rowsum(dS' . S)
+      float s = 0.f;
+      for (int jj = 0; jj < Dv; ++jj) s += Y2[aa * Dv + jj] * Y1[aa * Dv + jj];
+      sdgam[a0 + aa] = s;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < kMaxPer; ++m) {
+    const int idx = tid + m * nt;
+    if (idx < C * Dv) X1[idx] = vp[m];
+  }
+  // ---- P2: dKt = V' dS'^T (W is dead: its buffer takes dKt)
+  for (int a0 = 0; a0 < Dk; a0 += 32) {
+    const int na = min(32, Dk - a0);
+    __syncthreads();
+    for (int idx = tid; idx < na * Dv; idx += nt) Y2[idx] = dS1[(size_t)a0 * Dv + idx];
+    __syncthreads();
+    for (int idx = tid; idx < C * 32; idx += nt) {
+      const int i = idx >> 5, aa = idx & 31;
+      if (aa < na) {
+        float s = 0.f;
+        for (int jj = 0; jj < Dv; ++jj) s += X1[i * Dv + jj] * Y2[aa * Dv + jj];
+        X4[i * Dk + a0 + aa] = s;
+      }
+    }
+  }
+  __syncthreads();
+  // ---- P3: C x C products
+  for (int idx = tid; idx < C * Dk; idx += nt) Y1[idx] = sK[idx] * expf(sG[idx]);  // Gamma.K
+  for (int idx = tid; idx < C * C; idx += nt) {  // dP = Tril(dO V'^T)
+    const int r = idx / C, i = idx - r * C;
+    float s = 0.f;
+    if (i <= r)
+      for (int jj = 0; jj < Dv; ++jj) s += sdO[r * Dv + jj] * X1[i * Dv + jj];
+    sdP[idx] = s;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += nt) {  // dM = Tril(dW (Gamma.K)^T + dV' V^T)
+    const int r = idx / C, i = idx - r * C;
+    float s = 0.f;
+    if (i <= r) {
+      for (int a = 0; a < Dk; ++a) s += X3[r * Dk + a] * Y1[i * Dk + a];
+      for (int jj = 0; jj < Dv; ++jj) s += sdV[r * Dv + jj] * sV[i * Dv + jj];
+    }
+    sdM[idx] = s;
+  }
+  __syncthreads();
+  for (int i = tid; i < C; i += nt) {  // dbeta from M = T Diag(beta)
+    float s = 0.f;
+    for (int r = i; r < C; ++r) s += sdM[r * C + i] * sT[r * C + i];
+    sdb[i] = s;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += nt) sdM[idx] *= sbeta[idx % C];  // dT
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += nt) {  // X = dT T^T
+    const int p = idx / C, i = idx - p * C;
+    float s = 0.f;
+    for (int qq = 0; qq <= i; ++qq) s += sdM[p * C + qq] * sT[i * C + qq];
+    sX[idx] = s;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * C; idx += nt) {  // dA = -StrictTril(T^T X)
+    const int r = idx / C, i = idx - r * C;
+    float s = 0.f;
+    if (i < r)
+      for (int p = r; p < C; ++p) s += sT[p * C + r] * sX[p * C + i];
+    sdM[idx] = -s;
+  }
+  __syncthreads();
+  for (int r = tid; r < C; r += nt) {  // dbeta from A = StrictTril(Diag(beta) B)
+    float s = 0.f;
+    for (int i = 0; i < r; ++i) s += sdM[r * C + i] * sB[r * C + i];
+    sdb[r] += s;
+  }
+  // ---- P4: d(Gamma.K) = M^T dW, dV = M^T dV'
+  for (int idx = tid; idx < C * Dk; idx += nt) {
+    const int i = idx / Dk, a = idx - i * Dk;
+    float s = 0.f;
+    for (int r = i; r < C; ++r) s += sT[r * C + i] * X3[r * Dk + a];
+    Y2[idx] = s * sbeta[i];
+  }
+  for (int idx = tid; idx < C * Dv; idx += nt) {
+    const int i = idx / Dv, jj = idx - i * Dv;
+    float s = 0.f;
+    for (int r = i; r < C; ++r) s += sT[r * C + i] * sdV[r * Dv + jj];
+    if (i < L) dv[((size_t)(t0 + i) * H + h) * Dv + jj] = from_f32<Tin>(s * sbeta[i]);
+  }
+  __syncthreads();
+  // ---- P5: elementwise maps of Qt, Gamma.K, Kt onto q, k, g
+  for (int idx = tid; idx < C * Dk; idx += nt) {
+    const int a = idx % Dk;
+    const float g = sG[idx], e = expf(g), et = expf(sG[(C - 1) * Dk + a] - g);
+    const float dqt = X2[idx], dkg = Y2[idx], dkt = X4[idx];
+    X1[idx] = dqt * sQ[idx] * e + dkg * Y1[idx] - dkt * sK[idx] * et;  // dg
+    X2[idx] = dqt * e;                                                 // dq
+    X3[idx] = dkg * e + dkt * et;                                      // dk
+  }
+  __syncthreads();
+  // ratio-form products through A and P, one thread per key channel; then d log_alpha
+  for (int a = tid; a < Dk; a += nt) {
+    for (int r = 0; r < C; ++r) {
+      const float kr = sK[r * Dk + a], qr = sQ[r * Dk + a], gr = sG[r * Dk + a];
+      const float br = sbeta[r];
+      float dk_r = 0.f, dq_r = 0.f, dg_r = 0.f;
+      for (int i = 0; i <= r; ++i) {
+        const float e = expf(gr - sG[i * Dk + a]);
+        const float pa = sdP[r * C + i];
+        const float aa = i < r ? sdM[r * C + i] * br : 0.f;
+        const float t1 = e * sK[i * Dk + a];
+        dk_r += aa * t1;
+        dq_r += pa * t1;
+        const float w = aa * kr + pa * qr;
+        const float s = w * t1;
+        dg_r += s;
+        X1[i * Dk + a] -= s;
+        X3[i * Dk + a] += e * w;
+      }
+      X3[r * Dk + a] += dk_r;
+      X2[r * Dk + a] += dq_r;
+      X1[r * Dk + a] += dg_r;
+    }
+    // g_C enters Kt and gamma_C
+    const float gc = sG[(C - 1) * Dk + a];
+    float dgc = sdgam[a] * expf(gc);
+    for (int i = 0; i < C; ++i)
+      dgc += X4[i * Dk + a] * sK[i * Dk + a] * expf(gc - sG[i * Dk + a]);
+    X1[(C - 1) * Dk + a] += dgc;
+    float acc = 0.f;  // d log_alpha_j = sum_{r >= j} dg_r
+    for (int r = C - 1; r >= 0; --r) {
+      acc += X1[r * Dk + a];
+      X1[r * Dk + a] = acc;
+    }
+  }
+  __syncthreads();
+  // ---- P6: outputs
+  for (int idx = tid; idx < C * Dk; idx += nt) {
+    const int r = idx / Dk, a = idx - r * Dk;
+    if (r < L) {
+      const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
+      dq[gi] = from_f32<Tin>(X2[idx]);
+      dk[gi] = from_f32<Tin>(X3[idx]);
+      dla[gi] = X1[idx];
+    }
+  }
+  for (int r = tid; r < L; r += nt) dbeta[(size_t)(t0 + r) * H + h] = sdb[r];
+}
+
+size_t bwd_state_smem_bytes(int C, int Dk) {
+  return sizeof(float) * ((size_t)Dk * kBwSlice + 3 * (size_t)C * Dk + (size_t)C * C + Dk +
+                          2 * (size_t)C * kBwSlice);
+}
+size_t bwd_local_smem_bytes(int Dk, int Dv) {
+  return sizeof(float) * (size_t)BwdSmem::make(Dk, Dv).total;
+}
+
+template <typename Tin>
+static cudaError_t launch_bwd_typed(const BackwardArgs& b, const SeqGeometry& geo, int max_chunks,
+                                    float* records, const SimtRecord& rec, float* states,
+                                    float* dstates, float* dvp, cudaStream_t stream) {
+  const PrefillArgs& a = b.fwd;
+  cudaError_t err =
+      launch_forward_for_backward(a, geo, max_chunks, records, rec, states, stream);
+  if (err != cudaSuccess) return err;
+  const size_t sm3 = bwd_state_smem_bytes(a.C, a.Dk), sm4 = bwd_local_smem_bytes(a.Dk, a.Dv);
+  err = cudaFuncSetAttribute(chunk_state_bwd_kernel<Tin>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(chunk_local_bwd_kernel<Tin>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm4);
+  if (err != cudaSuccess) return err;
+  {
+    ProfileScope prof("chunk_state_bwd", stream);
+    chunk_state_bwd_kernel<Tin><<<dim3(a.N, a.H, ceil_div(a.Dv, kBwSlice)), kBwdThreads, sm3,
+                                  stream>>>(records, rec, geo, a.H, a.Dk, a.Dv,
+                                            (const Tin*)b.d_o, b.d_final, b.d_initial, dstates,
+                                            dvp);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  if (max_chunks == 0) return cudaSuccess;
+  ProfileScope prof("chunk_local_bwd", stream);
+  chunk_local_bwd_kernel<Tin><<<dim3(max_chunks, a.H), kBwdThreads, sm4, stream>>>(
+      (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
+      a.Dv, records, rec, states, dstates, dvp, (const Tin*)b.d_o, (Tin*)b.dq, (Tin*)b.dk,
+      (Tin*)b.dv, b.dlog_alpha, b.dbeta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_bwd(const BackwardArgs& b, const SeqGeometry& geo, int max_chunks,
+                             float* records, const SimtRecord& rec, float* states,
+                             float* dstates, float* dvp, cudaStream_t stream) {
+  if (b.fwd.dtype == KDA_DTYPE_BF16)
+    return launch_bwd_typed<__nv_bfloat16>(b, geo, max_chunks, records, rec, states, dstates,
+                                           dvp, stream);
+  return launch_bwd_typed<float>(b, geo, max_chunks, records, rec, states, dstates, dvp, stream);
+}
+
+}  // namespace kda

@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     if (lane == 0) {
       sA[r * C + i] = (i < r) ? sb[r] * akk : 0.f;
       gAqk[r * C + i] = aqk;
+      if (rec.off_b != SimtRecord::kNone) out[rec.off_b + r * C + i] = (i < r) ? akk : 0.f;
     }
   }
   for (int idx = tid; idx < C * C; idx += nt) {  // upper triangles
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     if (i > r) {
       sA[idx] = 0.f;
       gAqk[idx] = 0.f;
+      if (rec.off_b != SimtRecord::kNone) out[rec.off_b + idx] = 0.f;
     }
   }
   __syncthreads();
@@ -200,8 +202,11 @@ __global__ void __launch_bounds__(kSimtThreads)
     }
     __syncthreads();
   }
-  // M = (I + A)^{-1} Diag(beta)
-  for (int idx = tid; idx < C * C; idx += nt) sT[idx] *= sb[idx % C];
+  // M = (I + A)^{-1} Diag(beta)  (the backward pass keeps (I + A)^{-1} itself)
+  for (int idx = tid; idx < C * C; idx += nt) {
+    if (rec.off_t != SimtRecord::kNone) out[rec.off_t + idx] = sT[idx];
+    sT[idx] *= sb[idx % C];
+  }
 
   // Kt = (gamma_C/gamma_i) k_i, Qt = gamma_r q_r, gamma_C; then sk <- Gamma.K
   const float* gC = sg + (C - 1) * Dk;
@@ -241,7 +246,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(kSimtThreads)
     chunk_state_simt_kernel(const float* __restrict__ ws, SimtRecord rec, SeqGeometry geo, int H,
                             int Dk, int Dv, const float* __restrict__ initial_state,
-                            float* __restrict__ final_state, Tin* __restrict__ o) {
+                            float* __restrict__ final_state, Tin* __restrict__ o,
+                            float* __restrict__ states_out) {
   extern __shared__ float smem[];
   const int C = geo.C;
   float* sS = smem;               // [Dk][32] state slice
@@ -285,6 +291,13 @@ __global__ void __launch_bounds__(kSimtThreads)
     }
     for (int idx = tid; idx < C * C; idx += nt) sAq[idx] = r_[rec.off_aqk + idx];
     for (int cc = tid; cc < Dk; cc += nt) sGam[cc] = r_[rec.off_gam + cc];
+    if (states_out) {  // the state entering this chunk, for the backward pass
+      float* so = states_out + ((size_t)c * H + h) * Dk * Dv;
+      for (int idx = tid; idx < Dk * kSlice; idx += nt) {
+        const int cc = idx / kSlice, jj = idx - cc * kSlice;
+        if (jj < NV) so[(size_t)cc * Dv + j0 + jj] = sS[idx];
+      }
+    }
     __syncthreads();
 
     // V' = U - W S  and  O_inter = Qt S
@@ -312,7 +325,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       if (r < C) {
         float acc = o1[m];
         for (int i = 0; i <= r; ++i) acc += sAq[r * C + i] * sVp[i * kSlice + j];
-        if (r < L && j < NV) o[((size_t)(t0 + r) * H + h) * Dv + j0 + j] = from_f32<Tin>(acc);
+        if (o && r < L && j < NV) o[((size_t)(t0 + r) * H + h) * Dv + j0 + j] = from_f32<Tin>(acc);
       }
     }
     // S = Diag(gamma_C) S + Kt^T V'  (Eq. 8); each thread owns its (cc, j) elements
@@ -363,11 +376,48 @@ static cudaError_t launch_simt_typed(const PrefillArgs& a, const SeqGeometry& ge
   dim3 g2(a.N, a.H, ceil_div(a.Dv, kSlice));
   ProfileScope prof("chunk_state_simt", stream);
   chunk_state_simt_kernel<Tin><<<g2, kSimtThreads, sm2, stream>>>(
-      records, rec, geo, a.H, a.Dk, a.Dv, a.initial_state, a.final_state, (Tin*)a.o);
+      records, rec, geo, a.H, a.Dk, a.Dv, a.initial_state, a.final_state, (Tin*)a.o, nullptr);
   err = cudaGetLastError();
   if (err != cudaSuccess || !a.fz.onorm) return err;
   return launch_output_norm_gate(a.o, a.dtype, a.fz, (long long)a.B * a.T * a.H, a.H, a.Dv,
                                  a.cu_seqlens ? a.cu_seqlens + a.N : nullptr, stream);
+}
+
+template <typename Tin>
+static cudaError_t launch_fwd_for_bwd_typed(const PrefillArgs& a, const SeqGeometry& geo,
+                                            int max_chunks, float* records, const SimtRecord& rec,
+                                            float* states, cudaStream_t stream) {
+  const size_t sm1 = simt_local_smem_bytes(a.C, a.Dk, a.Dv);
+  const size_t sm2 = simt_state_smem_bytes(a.C, a.Dk);
+  cudaError_t err;
+  err = cudaFuncSetAttribute(chunk_local_simt_kernel<Tin>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(chunk_state_simt_kernel<Tin>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  if (err != cudaSuccess) return err;
+  if (max_chunks > 0) {
+    ProfileScope prof("bwd_chunk_local_fwd", stream);
+    chunk_local_simt_kernel<Tin><<<dim3(max_chunks, a.H), kSimtThreads, sm1, stream>>>(
+        (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
+        a.Dv, records, rec, a.fz);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  ProfileScope prof("bwd_chunk_state_fwd", stream);
+  chunk_state_simt_kernel<Tin><<<dim3(a.N, a.H, ceil_div(a.Dv, kSlice)), kSimtThreads, sm2,
+                                 stream>>>(records, rec, geo, a.H, a.Dk, a.Dv, a.initial_state,
+                                           nullptr, (Tin*)nullptr, states);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_forward_for_backward(const PrefillArgs& a, const SeqGeometry& geo,
+                                        int max_chunks, float* records, const SimtRecord& rec,
+                                        float* states, cudaStream_t stream) {
+  if (a.dtype == KDA_DTYPE_BF16)
+    return launch_fwd_for_bwd_typed<__nv_bfloat16>(a, geo, max_chunks, records, rec, states,
+                                                   stream);
+  return launch_fwd_for_bwd_typed<float>(a, geo, max_chunks, records, rec, states, stream);
 }
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,

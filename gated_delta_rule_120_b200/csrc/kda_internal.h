@@ -56,13 +56,23 @@ struct PrefillArgs {
 
 // Per (chunk, head) record of the fp32 CUDA-core path, in floats:
 //   W [C][Dk], U [C][Dv], Kt [C][Dk], Qt [C][Dk], A_qk [C][C], gamma_C [Dk]
+//   (+ for the backward pass: T = (I + A_kk)^{-1} [C][C] and the strictly lower
+//    B[r][i] = sum_c k_r[c] k_i[c] gamma_r[c]/gamma_i[c] [C][C], i.e. A_kk without Diag(beta))
 struct SimtRecord {
+  static constexpr size_t kNone = ~(size_t)0;
   size_t record_floats;
   size_t off_w, off_u, off_kt, off_qt, off_aqk, off_gam;
+  size_t off_t = kNone, off_b = kNone;
 
-  static SimtRecord make(int C, int Dk, int Dv) {
+  static SimtRecord make(int C, int Dk, int Dv, bool for_backward = false) {
     SimtRecord r;
     size_t o = 0;
+    if (for_backward) {
+      r.off_t = o;
+      o += (size_t)C * C;
+      r.off_b = o;
+      o += (size_t)C * C;
+    }
     r.off_w = o;
     o += (size_t)C * Dk;
     r.off_u = o;
@@ -102,6 +112,28 @@ cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
                                 float* records, const SimtRecord& rec, cudaStream_t stream);
+
+// The fp32 chunk kernels run for the backward pass: records with T and B, and the state at the
+// start of every chunk (states [chunks, H, Dk, Dv]) instead of the output.
+cudaError_t launch_forward_for_backward(const PrefillArgs& a, const SeqGeometry& geo,
+                                        int max_chunks, float* records, const SimtRecord& rec,
+                                        float* states, cudaStream_t stream);
+
+// Arguments of one kda_chunk_bwd call after host validation.
+struct BackwardArgs {
+  PrefillArgs fwd;          // inputs, geometry sizes; fwd.o unused, fwd.C = backward chunk
+  const void* d_o;          // [B,T,H,Dv], input dtype
+  const float* d_final;     // [N,H,Dk,Dv] or null
+  void* dq;                 // [B,T,H,Dk], input dtype
+  void* dk;
+  void* dv;                 // [B,T,H,Dv]
+  float* dlog_alpha;        // [B,T,H,Dk]
+  float* dbeta;             // [B,T,H]
+  float* d_initial;         // [N,H,Dk,Dv] or null
+};
+cudaError_t launch_chunk_bwd(const BackwardArgs& b, const SeqGeometry& geo, int max_chunks,
+                             float* records, const SimtRecord& rec, float* states,
+                             float* dstates, float* dvp, cudaStream_t stream);
 
 size_t simt_local_smem_bytes(int C, int Dk, int Dv);
 

@@ -7,4 +7,5 @@
 #include "kda_chunk_simt.cu"
 #include "kda_chunk_tc.cu"
 #include "kda_epilogue.cu"
+#include "kda_chunk_bwd.cu"
 #include "kda_noalloc.cu"

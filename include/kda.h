@@ -237,6 +237,44 @@ KDA_API kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const
                                              kda_stream_t stream);
 
 /*
+ * kda_chunk_bwd — backward pass of the operator (reverse-mode derivative of kda_chunk_fwd).
+ *
+ * The pages motivate it through training ("Kimi Linear: An Expressive, Efficient Attention
+ * Architecture", paper-graph-ui walkthrough, §3.4 "Chunkwise Parallelization": the UT transform
+ * is what makes the chunk form trainable; "FLOPs Accounting and Inference Strategy": training
+ * FLOPs). Computes the gradients of L = <d_o, o> + <d_final_state, final_state> with respect to
+ * every input of the same call of kda_chunk_fwd (same q, k, v, log_alpha, beta, initial_state,
+ * cu_seqlens, num_seqs, B, T, H, Dk, Dv; no prologue or epilogue fusion).
+ *
+ *   d_o             device, o's layout [B,T,H,Dv] and q's dtype: the output cotangent
+ *   d_final_state   device fp32 [N,H,Dk,Dv], or NULL for zero
+ *   dq, dk          device [B,T,H,Dk], q's dtype (written for every token of a sequence)
+ *   dv              device [B,T,H,Dv], q's dtype
+ *   dlog_alpha      device fp32 [B,T,H,Dk]
+ *   dbeta           device fp32 [B,T,H]
+ *   d_initial_state device fp32 [N,H,Dk,Dv], or NULL (not computed)
+ *   workspace       device, >= kda_chunk_bwd_workspace_size(...) bytes, 256-byte aligned
+ *
+ * The pass runs the fp32 chunk kernels forward once more (chunks of 32 tokens, whatever chunk
+ * the forward call used; the result does not depend on it), keeping the state entering every
+ * chunk, then a sequential backward state pass and a parallel chunk-local pass; all arithmetic
+ * is fp32 on CUDA cores, for fp32 and bf16 inputs alike. Supported: 1 <= Dk, Dv <= 128. Tokens
+ * outside every sequence (varlen) are not written. Arguments are checked on the host (pointers
+ * aligned to their element size); a bad cu_seqlens is reported by kda_last_device_error().
+ */
+KDA_API kda_status_t kda_chunk_bwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t Dk,
+                                                  int32_t Dv, int32_t num_seqs,
+                                                  kda_dtype_t qkv_dtype, size_t* bytes);
+KDA_API kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v,
+                                   kda_dtype_t qkv_dtype, const float* log_alpha,
+                                   const float* beta, const float* initial_state,
+                                   const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                                   int32_t T, int32_t H, int32_t Dk, int32_t Dv, const void* d_o,
+                                   const float* d_final_state, void* dq, void* dk, void* dv,
+                                   float* dlog_alpha, float* dbeta, float* d_initial_state,
+                                   void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_last_device_error — read and clear the per-device status word that the kernels set
  * (KDA_ERR_INVALID_ARG for a bad cu_seqlens, KDA_ERR_TIMEOUT for a bounded wait that gave up).
  * Synchronises `stream`. Returns KDA_OK when no kernel reported a fault.

@@ -147,3 +147,23 @@ def test_fusion_struct_layout_matches_the_header(tmp_path):
                                           text=True).stdout.split()]
     want = [ctypes.sizeof(kda.Fusion)] + [getattr(kda.Fusion, f).offset for f in fields]
     assert got == want
+
+
+def test_backward_workspace_and_argument_errors_on_host(L):
+    """The backward's size query and its host-side argument checks (no device work)."""
+    import ctypes
+
+    sz = ctypes.c_size_t(0)
+    assert L.kda_chunk_bwd_workspace_size(2, 4096, 32, 128, 128, 2, 1, ctypes.byref(sz)) == 0
+    # records (T and B included) + two state arrays + dV' for 256 chunks x 32 heads
+    assert sz.value > 2 * 256 * 32 * 128 * 128 * 4
+    assert L.kda_chunk_bwd_workspace_size(2, 64, 4, 256, 128, 2, 0, ctypes.byref(sz)) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_bwd_workspace_size(2, 64, 0, 64, 64, 2, 0, ctypes.byref(sz)) == \
+        kda.KDA_ERR_INVALID_ARG
+    # null tensors with tokens present -> INVALID_ARG before any launch
+    args = [None] * 3 + [0] + [None] * 4 + [1, 1, 16, 1, 32, 32] + [None] * 9 + [0, None]
+    assert L.kda_chunk_bwd(*args) == kda.KDA_ERR_INVALID_ARG
+    # N != B without cu_seqlens
+    args = [None] * 3 + [0] + [None] * 4 + [3, 2, 0, 1, 32, 32] + [None] * 9 + [0, None]
+    assert L.kda_chunk_bwd(*args) == kda.KDA_ERR_INVALID_ARG

@@ -206,6 +206,35 @@ def prefill_kernel_bytes(name, spec, max_chunks, rec_bytes):
     return None
 
 
+def library_source_hash() -> str:
+    """sha256 over the paths and contents of the files libkda.so is built from."""
+    import hashlib
+
+    from gated_delta_rule_120_b200 import _build
+
+    h = hashlib.sha256()
+    for p in _build.sources():
+        h.update(os.path.relpath(p, _build.ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture, or None
+    when there is none or the library sources changed since it was taken."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("workload") != workload:
+        return None
+    return rec["dram_bytes_per_launch"] if rec.get("source_sha256") == library_source_hash() \
+        else None
+
+
 def profile_pass(fn, steps, dev):
     import torch
 
@@ -494,7 +523,8 @@ def main():
     achieved = top_bytes / (top_ms / 1e3) / 1e9 if top_bytes else None
     hbm_peak = peaks["hbm_gbs"]
     roof = {"kernel": top["name"], "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-            "unit": "GB/s", "frac": (achieved / hbm_peak) if achieved else None, "traffic": None,
+            "unit": "GB/s", "frac": (achieved / hbm_peak) if achieved else None,
+            "traffic": captured_traffic(top["name"], spec.name),
             "peak_source": f"{peak_src} HBM copy bandwidth",
             "launch_ms": top_ms,
             "kernels": [{"name": p["name"], "launches_per_step": p["launches"] / args.steps,

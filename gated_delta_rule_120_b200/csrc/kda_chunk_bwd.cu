@@ -123,30 +123,37 @@ __global__ void __launch_bounds__(kBwdThreads)
 // ----------------------------------------------------------------------------------------------
 constexpr int kBwdC = 32;
 
+// Shared-memory rows are padded by one float (ldk = Dk + 1, ldv = Dv + 1, ldc = C + 1) so that
+// the products below, whose lanes walk down the rows of one operand, hit 32 different banks.
 struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
+  int ldk, ldv, ldm, ldc;
   int K, Q, G, V, dO, dV, X1, X2, X3, X4, Y1, Y2, T, P, B, dP, dM, X, beta, dgam, db, total;
   __host__ __device__ static BwdSmem make(int Dk, int Dv) {
     const int C = kBwdC, Dm = Dk > Dv ? Dk : Dv;
     BwdSmem s;
+    s.ldk = Dk + 1;
+    s.ldv = Dv + 1;
+    s.ldm = Dm + 1;
+    s.ldc = C + 1;
     int o = 0;
-    s.K = o; o += C * Dk;
-    s.Q = o; o += C * Dk;
-    s.G = o; o += C * Dk;
-    s.V = o; o += C * Dv;
-    s.dO = o; o += C * Dv;
-    s.dV = o; o += C * Dv;
-    s.X1 = o; o += C * Dm;   // V', then dg
-    s.X2 = o; o += C * Dk;   // dQt, then dq
-    s.X3 = o; o += C * Dk;   // dW, then dk
-    s.X4 = o; o += C * Dk;   // W, then dKt
-    s.Y1 = o; o += C * Dm;   // chunk-start state rows, then Gamma.K
-    s.Y2 = o; o += C * Dm;   // cotangent rows, then d(Gamma.K)
-    s.T = o; o += C * C;
-    s.P = o; o += C * C;
-    s.B = o; o += C * C;
-    s.dP = o; o += C * C;
-    s.dM = o; o += C * C;    // dM, then dT, then dA
-    s.X = o; o += C * C;
+    s.K = o; o += C * s.ldk;
+    s.Q = o; o += C * s.ldk;
+    s.G = o; o += C * s.ldk;
+    s.V = o; o += C * s.ldv;
+    s.dO = o; o += C * s.ldv;
+    s.dV = o; o += C * s.ldv;
+    s.X1 = o; o += C * s.ldm;   // V' (ldv), then dg (ldk)
+    s.X2 = o; o += C * s.ldk;   // dQt, then dq
+    s.X3 = o; o += C * s.ldk;   // dW, then dk
+    s.X4 = o; o += C * s.ldk;   // W, then dKt
+    s.Y1 = o; o += C * s.ldm;   // chunk-start state rows (ldv), then Gamma.K (ldk)
+    s.Y2 = o; o += C * s.ldm;   // cotangent rows (ldv), then d(Gamma.K) (ldk)
+    s.T = o; o += C * s.ldc;
+    s.P = o; o += C * s.ldc;
+    s.B = o; o += C * s.ldc;
+    s.dP = o; o += C * s.ldc;
+    s.dM = o; o += C * s.ldc;   // dM, then dT, then dA
+    s.X = o; o += C * s.ldc;
     s.beta = o; o += C;
     s.dgam = o; o += Dk;
     s.db = o; o += C;
@@ -168,6 +175,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   extern __shared__ float smem[];
   constexpr int C = kBwdC;
   const BwdSmem L_ = BwdSmem::make(Dk, Dv);
+  const int ldk = L_.ldk, ldv = L_.ldv, ldc = L_.ldc;
   float* sK = smem + L_.K;
   float* sQ = smem + L_.Q;
   float* sG = smem + L_.G;
@@ -206,31 +214,32 @@ __global__ void __launch_bounds__(kBwdThreads)
     const int r = idx / Dk, a = idx - r * Dk;
     const bool in = r < L;
     const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
-    sK[idx] = in ? to_f32(k[gi]) : 0.f;
-    sQ[idx] = in ? to_f32(q[gi]) : 0.f;
-    sG[idx] = in ? log_alpha[gi] : 0.f;
-    X4[idx] = r_[rec.off_w + idx];
+    sK[r * ldk + a] = in ? to_f32(k[gi]) : 0.f;
+    sQ[r * ldk + a] = in ? to_f32(q[gi]) : 0.f;
+    sG[r * ldk + a] = in ? log_alpha[gi] : 0.f;
+    X4[r * ldk + a] = r_[rec.off_w + idx];
   }
   for (int idx = tid; idx < C * Dv; idx += nt) {
     const int r = idx / Dv, jj = idx - r * Dv;
     const bool in = r < L;
     const size_t gi = ((size_t)(t0 + r) * H + h) * Dv + jj;
-    sV[idx] = in ? to_f32(v[gi]) : 0.f;
-    sdO[idx] = in ? to_f32(d_o[gi]) : 0.f;
-    sdV[idx] = in ? dvp[gi] : 0.f;
+    sV[r * ldv + jj] = in ? to_f32(v[gi]) : 0.f;
+    sdO[r * ldv + jj] = in ? to_f32(d_o[gi]) : 0.f;
+    sdV[r * ldv + jj] = in ? dvp[gi] : 0.f;
   }
   for (int idx = tid; idx < C * C; idx += nt) {
-    sT[idx] = r_[rec.off_t + idx];
-    sP[idx] = r_[rec.off_aqk + idx];
-    sB[idx] = r_[rec.off_b + idx];
+    const int r = idx / C, i = idx - r * C;
+    sT[r * ldc + i] = r_[rec.off_t + idx];
+    sP[r * ldc + i] = r_[rec.off_aqk + idx];
+    sB[r * ldc + i] = r_[rec.off_b + idx];
   }
   for (int r = tid; r < C; r += nt) sbeta[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
   __syncthreads();
   for (int a = tid; a < Dk; a += nt) {
     float acc = 0.f;
     for (int r = 0; r < C; ++r) {
-      acc += sG[r * Dk + a];
-      sG[r * Dk + a] = acc;
+      acc += sG[r * ldk + a];
+      sG[r * ldk + a] = acc;
     }
   }
 
@@ -246,8 +255,9 @@ __global__ void __launch_bounds__(kBwdThreads)
     const int na = min(32, Dk - a0);
     __syncthreads();  // previous slice consumed (and, the first time, the cumsum done)
     for (int idx = tid; idx < na * Dv; idx += nt) {
-      Y1[idx] = S0[(size_t)a0 * Dv + idx];
-      Y2[idx] = dS1[(size_t)a0 * Dv + idx];
+      const int aa = idx / Dv, jj = idx - aa * Dv;
+      Y1[aa * ldv + jj] = S0[(size_t)a0 * Dv + idx];
+      Y2[aa * ldv + jj] = dS1[(size_t)a0 * Dv + idx];
     }
     __syncthreads();
 #pragma unroll
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(kBwdThreads)
       if (idx < C * Dv) {
         const int r = idx / Dv, jj = idx - r * Dv;
         float acc = 0.f;
-        for (int aa = 0; aa < na; ++aa) acc += X4[r * Dk + a0 + aa] * Y1[aa * Dv + jj];
+        for (int aa = 0; aa < na; ++aa) acc += X4[r * ldk + a0 + aa] * Y1[aa * ldv + jj];
         vp[m] -= acc;
       }
     }
@@ -265,17 +275,17 @@ __global__ void __launch_bounds__(kBwdThreads)
       if (aa < na) {
         float s1 = 0.f, s2 = 0.f;
         for (int jj = 0; jj < Dv; ++jj) {
-          const float sv = Y1[aa * Dv + jj];
-          s1 += sdO[r * Dv + jj] * sv;
-          s2 += sdV[r * Dv + jj] * sv;
+          const float sv = Y1[aa * ldv + jj];
+          s1 += sdO[r * ldv + jj] * sv;
+          s2 += sdV[r * ldv + jj] * sv;
         }
-        X2[r * Dk + a0 + aa] = s1;
-        X3[r * Dk + a0 + aa] = -s2;
+        X2[r * ldk + a0 + aa] = s1;
+        X3[r * ldk + a0 + aa] = -s2;
       }
     }
     for (int aa = tid; aa < na; aa += nt) {  // dgamma_C = rowsum(dS' . S)
       float s = 0.f;
-      for (int jj = 0; jj < Dv; ++jj) s += Y2[aa * Dv + jj] * Y1[aa * Dv + jj];
+      for (int jj = 0; jj < Dv; ++jj) s += Y2[aa * ldv + jj] * Y1[aa * ldv + jj];
       sdgam[a0 + aa] = s;
     }
   }
@@ -283,129 +293,139 @@ __global__ void __launch_bounds__(kBwdThreads)
 #pragma unroll
   for (int m = 0; m < kMaxPer; ++m) {
     const int idx = tid + m * nt;
-    if (idx < C * Dv) X1[idx] = vp[m];
+    if (idx < C * Dv) X1[(idx / Dv) * ldv + idx % Dv] = vp[m];
   }
   // ---- P2: dKt = V' dS'^T (W is dead: its buffer takes dKt)
   for (int a0 = 0; a0 < Dk; a0 += 32) {
     const int na = min(32, Dk - a0);
     __syncthreads();
-    for (int idx = tid; idx < na * Dv; idx += nt) Y2[idx] = dS1[(size_t)a0 * Dv + idx];
+    for (int idx = tid; idx < na * Dv; idx += nt) {
+      const int aa = idx / Dv, jj = idx - aa * Dv;
+      Y2[aa * ldv + jj] = dS1[(size_t)a0 * Dv + idx];
+    }
     __syncthreads();
     for (int idx = tid; idx < C * 32; idx += nt) {
       const int i = idx >> 5, aa = idx & 31;
       if (aa < na) {
         float s = 0.f;
-        for (int jj = 0; jj < Dv; ++jj) s += X1[i * Dv + jj] * Y2[aa * Dv + jj];
-        X4[i * Dk + a0 + aa] = s;
+        for (int jj = 0; jj < Dv; ++jj) s += X1[i * ldv + jj] * Y2[aa * ldv + jj];
+        X4[i * ldk + a0 + aa] = s;
       }
     }
   }
   __syncthreads();
   // ---- P3: C x C products
-  for (int idx = tid; idx < C * Dk; idx += nt) Y1[idx] = sK[idx] * expf(sG[idx]);  // Gamma.K
+  for (int idx = tid; idx < C * Dk; idx += nt) {  // Gamma.K
+    const int r = idx / Dk, a = idx - r * Dk;
+    Y1[r * ldk + a] = sK[r * ldk + a] * expf(sG[r * ldk + a]);
+  }
   for (int idx = tid; idx < C * C; idx += nt) {  // dP = Tril(dO V'^T)
     const int r = idx / C, i = idx - r * C;
     float s = 0.f;
     if (i <= r)
-      for (int jj = 0; jj < Dv; ++jj) s += sdO[r * Dv + jj] * X1[i * Dv + jj];
-    sdP[idx] = s;
+      for (int jj = 0; jj < Dv; ++jj) s += sdO[r * ldv + jj] * X1[i * ldv + jj];
+    sdP[r * ldc + i] = s;
   }
   __syncthreads();
   for (int idx = tid; idx < C * C; idx += nt) {  // dM = Tril(dW (Gamma.K)^T + dV' V^T)
     const int r = idx / C, i = idx - r * C;
     float s = 0.f;
     if (i <= r) {
-      for (int a = 0; a < Dk; ++a) s += X3[r * Dk + a] * Y1[i * Dk + a];
-      for (int jj = 0; jj < Dv; ++jj) s += sdV[r * Dv + jj] * sV[i * Dv + jj];
+      for (int a = 0; a < Dk; ++a) s += X3[r * ldk + a] * Y1[i * ldk + a];
+      for (int jj = 0; jj < Dv; ++jj) s += sdV[r * ldv + jj] * sV[i * ldv + jj];
     }
-    sdM[idx] = s;
+    sdM[r * ldc + i] = s;
   }
   __syncthreads();
   for (int i = tid; i < C; i += nt) {  // dbeta from M = T Diag(beta)
     float s = 0.f;
-    for (int r = i; r < C; ++r) s += sdM[r * C + i] * sT[r * C + i];
+    for (int r = i; r < C; ++r) s += sdM[r * ldc + i] * sT[r * ldc + i];
     sdb[i] = s;
   }
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += nt) sdM[idx] *= sbeta[idx % C];  // dT
+  for (int idx = tid; idx < C * C; idx += nt) {  // dT
+    const int r = idx / C, i = idx - r * C;
+    sdM[r * ldc + i] *= sbeta[i];
+  }
   __syncthreads();
   for (int idx = tid; idx < C * C; idx += nt) {  // X = dT T^T
     const int p = idx / C, i = idx - p * C;
     float s = 0.f;
-    for (int qq = 0; qq <= i; ++qq) s += sdM[p * C + qq] * sT[i * C + qq];
-    sX[idx] = s;
+    for (int qq = 0; qq <= i; ++qq) s += sdM[p * ldc + qq] * sT[i * ldc + qq];
+    sX[p * ldc + i] = s;
   }
   __syncthreads();
   for (int idx = tid; idx < C * C; idx += nt) {  // dA = -StrictTril(T^T X)
     const int r = idx / C, i = idx - r * C;
     float s = 0.f;
     if (i < r)
-      for (int p = r; p < C; ++p) s += sT[p * C + r] * sX[p * C + i];
-    sdM[idx] = -s;
+      for (int p = r; p < C; ++p) s += sT[p * ldc + r] * sX[p * ldc + i];
+    sdM[r * ldc + i] = -s;
   }
   __syncthreads();
   for (int r = tid; r < C; r += nt) {  // dbeta from A = StrictTril(Diag(beta) B)
     float s = 0.f;
-    for (int i = 0; i < r; ++i) s += sdM[r * C + i] * sB[r * C + i];
+    for (int i = 0; i < r; ++i) s += sdM[r * ldc + i] * sB[r * ldc + i];
     sdb[r] += s;
   }
   // ---- P4: d(Gamma.K) = M^T dW, dV = M^T dV'
   for (int idx = tid; idx < C * Dk; idx += nt) {
     const int i = idx / Dk, a = idx - i * Dk;
     float s = 0.f;
-    for (int r = i; r < C; ++r) s += sT[r * C + i] * X3[r * Dk + a];
-    Y2[idx] = s * sbeta[i];
+    for (int r = i; r < C; ++r) s += sT[r * ldc + i] * X3[r * ldk + a];
+    Y2[i * ldk + a] = s * sbeta[i];
   }
   for (int idx = tid; idx < C * Dv; idx += nt) {
     const int i = idx / Dv, jj = idx - i * Dv;
     float s = 0.f;
-    for (int r = i; r < C; ++r) s += sT[r * C + i] * sdV[r * Dv + jj];
+    for (int r = i; r < C; ++r) s += sT[r * ldc + i] * sdV[r * ldv + jj];
     if (i < L) dv[((size_t)(t0 + i) * H + h) * Dv + jj] = from_f32<Tin>(s * sbeta[i]);
   }
   __syncthreads();
   // ---- P5: elementwise maps of Qt, Gamma.K, Kt onto q, k, g
   for (int idx = tid; idx < C * Dk; idx += nt) {
-    const int a = idx % Dk;
-    const float g = sG[idx], e = expf(g), et = expf(sG[(C - 1) * Dk + a] - g);
-    const float dqt = X2[idx], dkg = Y2[idx], dkt = X4[idx];
-    X1[idx] = dqt * sQ[idx] * e + dkg * Y1[idx] - dkt * sK[idx] * et;  // dg
-    X2[idx] = dqt * e;                                                 // dq
-    X3[idx] = dkg * e + dkt * et;                                      // dk
+    const int r = idx / Dk, a = idx - r * Dk;
+    const int x = r * ldk + a;
+    const float g = sG[x], e = expf(g), et = expf(sG[(C - 1) * ldk + a] - g);
+    const float dqt = X2[x], dkg = Y2[x], dkt = X4[x];
+    X1[x] = dqt * sQ[x] * e + dkg * Y1[x] - dkt * sK[x] * et;  // dg
+    X2[x] = dqt * e;                                           // dq
+    X3[x] = dkg * e + dkt * et;                                // dk
   }
   __syncthreads();
   // ratio-form products through A and P, one thread per key channel; then d log_alpha
   for (int a = tid; a < Dk; a += nt) {
     for (int r = 0; r < C; ++r) {
-      const float kr = sK[r * Dk + a], qr = sQ[r * Dk + a], gr = sG[r * Dk + a];
+      const float kr = sK[r * ldk + a], qr = sQ[r * ldk + a], gr = sG[r * ldk + a];
       const float br = sbeta[r];
       float dk_r = 0.f, dq_r = 0.f, dg_r = 0.f;
       for (int i = 0; i <= r; ++i) {
-        const float e = expf(gr - sG[i * Dk + a]);
-        const float pa = sdP[r * C + i];
-        const float aa = i < r ? sdM[r * C + i] * br : 0.f;
-        const float t1 = e * sK[i * Dk + a];
+        const float e = __expf(gr - sG[i * ldk + a]);
+        const float pa = sdP[r * ldc + i];
+        const float aa = i < r ? sdM[r * ldc + i] * br : 0.f;
+        const float t1 = e * sK[i * ldk + a];
         dk_r += aa * t1;
         dq_r += pa * t1;
         const float w = aa * kr + pa * qr;
         const float s = w * t1;
         dg_r += s;
-        X1[i * Dk + a] -= s;
-        X3[i * Dk + a] += e * w;
+        X1[i * ldk + a] -= s;
+        X3[i * ldk + a] += e * w;
       }
-      X3[r * Dk + a] += dk_r;
-      X2[r * Dk + a] += dq_r;
-      X1[r * Dk + a] += dg_r;
+      X3[r * ldk + a] += dk_r;
+      X2[r * ldk + a] += dq_r;
+      X1[r * ldk + a] += dg_r;
     }
     // g_C enters Kt and gamma_C
-    const float gc = sG[(C - 1) * Dk + a];
+    const float gc = sG[(C - 1) * ldk + a];
     float dgc = sdgam[a] * expf(gc);
     for (int i = 0; i < C; ++i)
-      dgc += X4[i * Dk + a] * sK[i * Dk + a] * expf(gc - sG[i * Dk + a]);
-    X1[(C - 1) * Dk + a] += dgc;
+      dgc += X4[i * ldk + a] * sK[i * ldk + a] * expf(gc - sG[i * ldk + a]);
+    X1[(C - 1) * ldk + a] += dgc;
     float acc = 0.f;  // d log_alpha_j = sum_{r >= j} dg_r
     for (int r = C - 1; r >= 0; --r) {
-      acc += X1[r * Dk + a];
-      X1[r * Dk + a] = acc;
+      acc += X1[r * ldk + a];
+      X1[r * ldk + a] = acc;
     }
   }
   __syncthreads();
@@ -414,9 +434,10 @@ __global__ void __launch_bounds__(kBwdThreads)
     const int r = idx / Dk, a = idx - r * Dk;
     if (r < L) {
       const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
-      dq[gi] = from_f32<Tin>(X2[idx]);
-      dk[gi] = from_f32<Tin>(X3[idx]);
-      dla[gi] = X1[idx];
+      const int x = r * ldk + a;
+      dq[gi] = from_f32<Tin>(X2[x]);
+      dk[gi] = from_f32<Tin>(X3[x]);
+      dla[gi] = X1[x];
     }
   }
   for (int r = tid; r < L; r += nt) dbeta[(size_t)(t0 + r) * H + h] = sdb[r];

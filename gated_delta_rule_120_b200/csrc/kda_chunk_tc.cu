@@ -178,16 +178,6 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   const int L = min(kC, geo.seq_end(n) - t0);
   uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)c * H + h);
 
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, kK1Tmem);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_mbar_init();
-  }
-
   // ---- phase 1: raw k, q, v straight into their operand tiles; log decay into registers ------
   const int cg = tid & 15, rg = tid >> 4;  // thread = 8 channels (one 16-byte chunk) x 4 rows
   float g[4][8];
@@ -214,6 +204,17 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     }
   }
   if (tid < kC) sBeta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+  // the tensor memory and the barrier are first used in phase 3: set them up while the loads
+  // above are in flight
+  if (warp == 7) {
+    tmem_alloc(tmem_slot, kK1Tmem);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (tid == 224) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
   if (fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log decays
     const float neg_a = -expf(fz.A_log[h]);
     float bias[8];
@@ -747,7 +748,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 7) {  // the allocating warp frees
     tc_fence_after();
     tmem_dealloc(tmem, kK1Tmem);
   }

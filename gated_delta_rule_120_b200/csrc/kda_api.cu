@@ -76,7 +76,7 @@ kda_status_t check_backward_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, i
   } else if (N != B) {
     return KDA_ERR_INVALID_ARG;
   }
-  if (Dk > 128 || Dv > 128) return KDA_ERR_UNSUPPORTED;
+  if (Dk > 128 || Dv > 128 || Dk % 4 != 0 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
   const long long tokens = (long long)B * T;
   const long long elems = tokens * H * (long long)(Dk > Dv ? Dk : Dv);
   if (tokens > INT32_MAX || elems > (1LL << 40)) return KDA_ERR_UNSUPPORTED;

@@ -34,6 +34,19 @@ namespace kda {
 constexpr int kBwdThreads = 256;
 constexpr int kBwSlice = 32;  // value columns per CTA of the state pass
 
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+__device__ __forceinline__ void fma4(float s, float4 b, float4& acc) {
+  acc.x = fmaf(s, b.x, acc.x);
+  acc.y = fmaf(s, b.y, acc.y);
+  acc.z = fmaf(s, b.z, acc.z);
+  acc.w = fmaf(s, b.w, acc.w);
+}
+
+
 // ----------------------------------------------------------------------------------------------
 // state pass: one CTA per (sequence, head, 32-column slice of d_v), chunks in reverse order
 // ----------------------------------------------------------------------------------------------
@@ -49,15 +62,15 @@ __global__ void __launch_bounds__(kBwdThreads)
   float* sW = sdS + Dk * kBwSlice;   // [C][Dk]
   float* sKt = sW + C * Dk;          // [C][Dk]
   float* sQt = sKt + C * Dk;         // [C][Dk]
-  float* sP = sQt + C * Dk;          // [C][C]
-  float* sGam = sP + C * C;          // [Dk]
+  float* sPt = sQt + C * Dk;         // [C][C] P transposed: sPt[i][r] = P[r][i]
+  float* sGam = sPt + C * C;         // [Dk]
   float* sdO = sGam + Dk;            // [C][32]
   float* sdV = sdO + C * kBwSlice;   // [C][32]
 
   if (!geo.ok()) return;
   const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kBwSlice;
   const int NV = min(kBwSlice, Dv - j0);
-  const int tid = threadIdx.x, nt = blockDim.x, j = tid & 31, rg = tid >> 5, ng = nt >> 5;
+  const int tid = threadIdx.x, nt = blockDim.x, j = tid & 31, rg = tid >> 5;
   const size_t sbase = ((size_t)n * H + h) * Dk * Dv;
 
   for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
@@ -78,7 +91,10 @@ __global__ void __launch_bounds__(kBwdThreads)
       sKt[idx] = r_[rec.off_kt + idx];
       sQt[idx] = r_[rec.off_qt + idx];
     }
-    for (int idx = tid; idx < C * C; idx += nt) sP[idx] = r_[rec.off_aqk + idx];
+    for (int idx = tid; idx < C * C; idx += nt) {
+      const int r = idx / C, i = idx - r * C;
+      sPt[i * C + r] = r_[rec.off_aqk + idx];
+    }
     for (int a = tid; a < Dk; a += nt) sGam[a] = r_[rec.off_gam + a];
     for (int idx = tid; idx < C * kBwSlice; idx += nt) {
       const int r = idx / kBwSlice, jj = idx - r * kBwSlice;
@@ -92,21 +108,70 @@ __global__ void __launch_bounds__(kBwdThreads)
       }
     }
     __syncthreads();
-    // dV'[i][j] = sum_{r >= i} P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j]
-    for (int i = rg; i < C; i += ng) {
-      float acc = 0.f;
-      for (int r = i; r < C; ++r) acc += sP[r * C + i] * sdO[r * kBwSlice + j];
-      for (int a = 0; a < Dk; ++a) acc += sKt[i * Dk + a] * sdS[a * kBwSlice + j];
-      sdV[i * kBwSlice + j] = acc;
-      if (i < L && j < NV) dvp[((size_t)(t0 + i) * H + h) * Dv + j0 + j] = acc;
+    // dV'[i][j] = sum_r P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j] (P[r][i] = 0 for r < i);
+    // this thread: rows i = rg + 8u, column j; float4 along r and a
+    {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int r = 0; r < C; r += 4) {
+        const float o0 = sdO[r * kBwSlice + j], o1 = sdO[(r + 1) * kBwSlice + j];
+        const float o2 = sdO[(r + 2) * kBwSlice + j], o3 = sdO[(r + 3) * kBwSlice + j];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 p = ld4(sPt + (rg + 8 * u) * C + r);
+          acc[u] = fmaf(p.x, o0, fmaf(p.y, o1, fmaf(p.z, o2, fmaf(p.w, o3, acc[u]))));
+        }
+      }
+      for (int a = 0; a < Dk; a += 4) {
+        const float s0 = sdS[a * kBwSlice + j], s1 = sdS[(a + 1) * kBwSlice + j];
+        const float s2 = sdS[(a + 2) * kBwSlice + j], s3 = sdS[(a + 3) * kBwSlice + j];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 kt = ld4(sKt + (rg + 8 * u) * Dk + a);
+          acc[u] = fmaf(kt.x, s0, fmaf(kt.y, s1, fmaf(kt.z, s2, fmaf(kt.w, s3, acc[u]))));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = rg + 8 * u;
+        sdV[i * kBwSlice + j] = acc[u];
+        if (i < L && j < NV) dvp[((size_t)(t0 + i) * H + h) * Dv + j0 + j] = acc[u];
+      }
     }
     __syncthreads();
-    // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV'  (each thread owns its (a, j) elements)
-    for (int a = rg; a < Dk; a += ng) {
-      float acc = sGam[a] * sdS[a * kBwSlice + j];
-      for (int r = 0; r < C; ++r)
-        acc += sQt[r * Dk + a] * sdO[r * kBwSlice + j] - sW[r * Dk + a] * sdV[r * kBwSlice + j];
-      sdS[a * kBwSlice + j] = acc;
+    // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV'; this thread: rows a in the groups of four
+    // {4 (rg + 8 u) .. + 3}, column j (each thread rewrites only its own elements)
+    for (int g0 = 4 * rg; g0 < Dk; g0 += 4 * 8 * 4) {
+      float4 acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int a = g0 + 32 * u;
+        acc[u] = a < Dk ? make_float4(sGam[a] * sdS[a * kBwSlice + j],
+                                      sGam[a + 1] * sdS[(a + 1) * kBwSlice + j],
+                                      sGam[a + 2] * sdS[(a + 2) * kBwSlice + j],
+                                      sGam[a + 3] * sdS[(a + 3) * kBwSlice + j])
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int r = 0; r < C; ++r) {
+        const float o = sdO[r * kBwSlice + j], dvv = -sdV[r * kBwSlice + j];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int a = g0 + 32 * u;
+          if (a < Dk) {
+            fma4(o, ld4(sQt + r * Dk + a), acc[u]);
+            fma4(dvv, ld4(sW + r * Dk + a), acc[u]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int a = g0 + 32 * u;
+        if (a < Dk) {
+          sdS[a * kBwSlice + j] = acc[u].x;
+          sdS[(a + 1) * kBwSlice + j] = acc[u].y;
+          sdS[(a + 2) * kBwSlice + j] = acc[u].z;
+          sdS[(a + 3) * kBwSlice + j] = acc[u].w;
+        }
+      }
     }
   }
   __syncthreads();
@@ -123,18 +188,22 @@ __global__ void __launch_bounds__(kBwdThreads)
 // ----------------------------------------------------------------------------------------------
 constexpr int kBwdC = 32;
 
-// Shared-memory rows are padded by one float (ldk = Dk + 1, ldv = Dv + 1, ldc = C + 1) so that
-// the products below, whose lanes walk down the rows of one operand, hit 32 different banks.
+// Shared-memory rows are padded by four floats (ld = D + 4): rows stay 16-byte aligned for
+// float4 accesses, and consecutive rows start 4 banks apart. The products are register-tiled:
+// a thread owns output rows {tm, tm + 16} and, along the other dimension, either columns
+// {tn, tn + 16} (contractions over d_k / d_v of two row-major operands, float4 along the
+// contraction) or two float4 column groups {4 tn .. 4 tn + 3, 64 + 4 tn .. 64 + 4 tn + 3}
+// (contractions over the chunk rows). Requires Dk, Dv multiples of 4.
 struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
   int ldk, ldv, ldm, ldc;
-  int K, Q, G, V, dO, dV, X1, X2, X3, X4, Y1, Y2, T, P, B, dP, dM, X, beta, dgam, db, total;
+  int K, Q, G, V, dO, dV, X1, X2, X3, X4, Y1, Y2, T, B, dP, dM, X, beta, dgam, db, total;
   __host__ __device__ static BwdSmem make(int Dk, int Dv) {
     const int C = kBwdC, Dm = Dk > Dv ? Dk : Dv;
     BwdSmem s;
-    s.ldk = Dk + 1;
-    s.ldv = Dv + 1;
-    s.ldm = Dm + 1;
-    s.ldc = C + 1;
+    s.ldk = Dk + 4;
+    s.ldv = Dv + 4;
+    s.ldm = Dm + 4;
+    s.ldc = C + 4;
     int o = 0;
     s.K = o; o += C * s.ldk;
     s.Q = o; o += C * s.ldk;
@@ -149,7 +218,6 @@ struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
     s.Y1 = o; o += C * s.ldm;   // chunk-start state rows (ldv), then Gamma.K (ldk)
     s.Y2 = o; o += C * s.ldm;   // cotangent rows (ldv), then d(Gamma.K) (ldk)
     s.T = o; o += C * s.ldc;
-    s.P = o; o += C * s.ldc;
     s.B = o; o += C * s.ldc;
     s.dP = o; o += C * s.ldc;
     s.dM = o; o += C * s.ldc;   // dM, then dT, then dA
@@ -162,6 +230,22 @@ struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
   }
 };
 
+// acc[u][w] += sum_{k < K} X[(tm + 16u) * ldx + k] * Y[(tn + 16w) * ldy + k]  (K multiple of 4)
+__device__ __forceinline__ void abt_2x2(const float* X, int ldx, const float* Y, int ldy, int K,
+                                        int tm, int tn, float (&acc)[2][2]) {
+  const float* x0 = X + tm * ldx;
+  const float* x1 = X + (tm + 16) * ldx;
+  const float* y0 = Y + tn * ldy;
+  const float* y1 = Y + (tn + 16) * ldy;
+  for (int k = 0; k < K; k += 4) {
+    const float4 a0 = ld4(x0 + k), a1 = ld4(x1 + k), b0 = ld4(y0 + k), b1 = ld4(y1 + k);
+    acc[0][0] = dot4(a0, b0, acc[0][0]);
+    acc[0][1] = dot4(a0, b1, acc[0][1]);
+    acc[1][0] = dot4(a1, b0, acc[1][0]);
+    acc[1][1] = dot4(a1, b1, acc[1][1]);
+  }
+}
+
 template <typename Tin>
 __global__ void __launch_bounds__(kBwdThreads)
     chunk_local_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
@@ -172,7 +256,7 @@ __global__ void __launch_bounds__(kBwdThreads)
                            const float* __restrict__ dvp, const Tin* __restrict__ d_o,
                            Tin* __restrict__ dq, Tin* __restrict__ dk, Tin* __restrict__ dv,
                            float* __restrict__ dla, float* __restrict__ dbeta) {
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   constexpr int C = kBwdC;
   const BwdSmem L_ = BwdSmem::make(Dk, Dv);
   const int ldk = L_.ldk, ldv = L_.ldv, ldc = L_.ldc;
@@ -189,7 +273,6 @@ __global__ void __launch_bounds__(kBwdThreads)
   float* Y1 = smem + L_.Y1;
   float* Y2 = smem + L_.Y2;
   float* sT = smem + L_.T;
-  float* sP = smem + L_.P;
   float* sB = smem + L_.B;
   float* sdP = smem + L_.dP;
   float* sdM = smem + L_.dM;
@@ -205,9 +288,11 @@ __global__ void __launch_bounds__(kBwdThreads)
   const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * C;
   const int L = min(C, geo.seq_end(n) - t0);
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int tm = tid >> 4, tn = tid & 15;  // register-tile coordinates
   const float* r_ = ws + rec.record_floats * ((size_t)c * H + h);
   const float* S0 = states + ((size_t)c * H + h) * Dk * Dv;   // state entering the chunk
   const float* dS1 = dstates + ((size_t)c * H + h) * Dk * Dv; // cotangent of the state leaving it
+  const int Dv4 = Dv >> 2;
 
   // ---- P0: inputs, record, cumulative decay
   for (int idx = tid; idx < C * Dk; idx += nt) {
@@ -230,7 +315,6 @@ __global__ void __launch_bounds__(kBwdThreads)
   for (int idx = tid; idx < C * C; idx += nt) {
     const int r = idx / C, i = idx - r * C;
     sT[r * ldc + i] = r_[rec.off_t + idx];
-    sP[r * ldc + i] = r_[rec.off_aqk + idx];
     sB[r * ldc + i] = r_[rec.off_b + idx];
   }
   for (int r = tid; r < C; r += nt) sbeta[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
@@ -244,73 +328,85 @@ __global__ void __launch_bounds__(kBwdThreads)
   }
 
   // ---- P1: products with the chunk-start state S (rows streamed 32 at a time)
-  constexpr int kMaxPer = (C * 128 + kBwdThreads - 1) / kBwdThreads;  // outputs of V' per thread
-  float vp[kMaxPer];
+  // V' = U - W S: this thread's rows {tm, tm + 16}, column groups {4 tn, 64 + 4 tn}
+  float4 vp[2][2];
 #pragma unroll
-  for (int m = 0; m < kMaxPer; ++m) {
-    const int idx = tid + m * nt;
-    vp[m] = idx < C * Dv ? r_[rec.off_u + idx] : 0.f;
-  }
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int j = 4 * tn + 64 * w;
+      vp[u][w] = j < Dv ? ld4(r_ + rec.off_u + (tm + 16 * u) * Dv + j)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   for (int a0 = 0; a0 < Dk; a0 += 32) {
     const int na = min(32, Dk - a0);
     __syncthreads();  // previous slice consumed (and, the first time, the cumsum done)
-    for (int idx = tid; idx < na * Dv; idx += nt) {
-      const int aa = idx / Dv, jj = idx - aa * Dv;
-      Y1[aa * ldv + jj] = S0[(size_t)a0 * Dv + idx];
-      Y2[aa * ldv + jj] = dS1[(size_t)a0 * Dv + idx];
+    for (int idx = tid; idx < na * Dv4; idx += nt) {
+      const int aa = idx / Dv4, j4 = idx - aa * Dv4;
+      st4(Y1 + aa * ldv + 4 * j4, ld4(S0 + (size_t)(a0 + aa) * Dv + 4 * j4));
+      st4(Y2 + aa * ldv + 4 * j4, ld4(dS1 + (size_t)(a0 + aa) * Dv + 4 * j4));
     }
     __syncthreads();
+    for (int aa = 0; aa < na; ++aa) {
+      const float w0 = X4[tm * ldk + a0 + aa], w1 = X4[(tm + 16) * ldk + a0 + aa];
 #pragma unroll
-    for (int m = 0; m < kMaxPer; ++m) {  // V' = U - W S
-      const int idx = tid + m * nt;
-      if (idx < C * Dv) {
-        const int r = idx / Dv, jj = idx - r * Dv;
-        float acc = 0.f;
-        for (int aa = 0; aa < na; ++aa) acc += X4[r * ldk + a0 + aa] * Y1[aa * ldv + jj];
-        vp[m] -= acc;
+      for (int w = 0; w < 2; ++w) {
+        const int j = 4 * tn + 64 * w;
+        if (j < Dv) {
+          const float4 sv = ld4(Y1 + aa * ldv + j);
+          fma4(-w0, sv, vp[0][w]);
+          fma4(-w1, sv, vp[1][w]);
+        }
       }
     }
-    for (int idx = tid; idx < C * 32; idx += nt) {  // dQt = dO S^T, dW = -dV' S^T
-      const int r = idx >> 5, aa = idx & 31;
-      if (aa < na) {
-        float s1 = 0.f, s2 = 0.f;
-        for (int jj = 0; jj < Dv; ++jj) {
-          const float sv = Y1[aa * ldv + jj];
-          s1 += sdO[r * ldv + jj] * sv;
-          s2 += sdV[r * ldv + jj] * sv;
+    if (tn < na || tn + 16 < na) {  // dQt = dO S^T, dW = -dV' S^T over this slice's columns
+      float a1[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, a2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      abt_2x2(sdO, ldv, Y1, ldv, Dv, tm, tn, a1);
+      abt_2x2(sdV, ldv, Y1, ldv, Dv, tm, tn, a2);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int aa = tn + 16 * w;
+          if (aa < na) {
+            X2[(tm + 16 * u) * ldk + a0 + aa] = a1[u][w];
+            X3[(tm + 16 * u) * ldk + a0 + aa] = -a2[u][w];
+          }
         }
-        X2[r * ldk + a0 + aa] = s1;
-        X3[r * ldk + a0 + aa] = -s2;
-      }
     }
     for (int aa = tid; aa < na; aa += nt) {  // dgamma_C = rowsum(dS' . S)
       float s = 0.f;
-      for (int jj = 0; jj < Dv; ++jj) s += Y2[aa * ldv + jj] * Y1[aa * ldv + jj];
+      for (int j = 0; j < Dv; j += 4) s = dot4(ld4(Y2 + aa * ldv + j), ld4(Y1 + aa * ldv + j), s);
       sdgam[a0 + aa] = s;
     }
   }
   __syncthreads();
 #pragma unroll
-  for (int m = 0; m < kMaxPer; ++m) {
-    const int idx = tid + m * nt;
-    if (idx < C * Dv) X1[(idx / Dv) * ldv + idx % Dv] = vp[m];
-  }
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int j = 4 * tn + 64 * w;
+      if (j < Dv) st4(X1 + (tm + 16 * u) * ldv + j, vp[u][w]);
+    }
   // ---- P2: dKt = V' dS'^T (W is dead: its buffer takes dKt)
   for (int a0 = 0; a0 < Dk; a0 += 32) {
     const int na = min(32, Dk - a0);
     __syncthreads();
-    for (int idx = tid; idx < na * Dv; idx += nt) {
-      const int aa = idx / Dv, jj = idx - aa * Dv;
-      Y2[aa * ldv + jj] = dS1[(size_t)a0 * Dv + idx];
+    for (int idx = tid; idx < na * Dv4; idx += nt) {
+      const int aa = idx / Dv4, j4 = idx - aa * Dv4;
+      st4(Y2 + aa * ldv + 4 * j4, ld4(dS1 + (size_t)(a0 + aa) * Dv + 4 * j4));
     }
     __syncthreads();
-    for (int idx = tid; idx < C * 32; idx += nt) {
-      const int i = idx >> 5, aa = idx & 31;
-      if (aa < na) {
-        float s = 0.f;
-        for (int jj = 0; jj < Dv; ++jj) s += X1[i * ldv + jj] * Y2[aa * ldv + jj];
-        X4[i * ldk + a0 + aa] = s;
-      }
+    if (tn < na || tn + 16 < na) {
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      abt_2x2(X1, ldv, Y2, ldv, Dv, tm, tn, acc);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int aa = tn + 16 * w;
+          if (aa < na) X4[(tm + 16 * u) * ldk + a0 + aa] = acc[u][w];
+        }
     }
   }
   __syncthreads();
@@ -319,22 +415,29 @@ __global__ void __launch_bounds__(kBwdThreads)
     const int r = idx / Dk, a = idx - r * Dk;
     Y1[r * ldk + a] = sK[r * ldk + a] * expf(sG[r * ldk + a]);
   }
-  for (int idx = tid; idx < C * C; idx += nt) {  // dP = Tril(dO V'^T)
-    const int r = idx / C, i = idx - r * C;
-    float s = 0.f;
-    if (i <= r)
-      for (int jj = 0; jj < Dv; ++jj) s += sdO[r * ldv + jj] * X1[i * ldv + jj];
-    sdP[r * ldc + i] = s;
+  {  // dP = Tril(dO V'^T)
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    abt_2x2(sdO, ldv, X1, ldv, Dv, tm, tn, acc);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int r = tm + 16 * u, i = tn + 16 * w;
+        sdP[r * ldc + i] = i <= r ? acc[u][w] : 0.f;
+      }
   }
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += nt) {  // dM = Tril(dW (Gamma.K)^T + dV' V^T)
-    const int r = idx / C, i = idx - r * C;
-    float s = 0.f;
-    if (i <= r) {
-      for (int a = 0; a < Dk; ++a) s += X3[r * ldk + a] * Y1[i * ldk + a];
-      for (int jj = 0; jj < Dv; ++jj) s += sdV[r * ldv + jj] * sV[i * ldv + jj];
-    }
-    sdM[r * ldc + i] = s;
+  {  // dM = Tril(dW (Gamma.K)^T + dV' V^T)
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    abt_2x2(X3, ldk, Y1, ldk, Dk, tm, tn, acc);
+    abt_2x2(sdV, ldv, sV, ldv, Dv, tm, tn, acc);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int r = tm + 16 * u, i = tn + 16 * w;
+        sdM[r * ldc + i] = i <= r ? acc[u][w] : 0.f;
+      }
   }
   __syncthreads();
   for (int i = tid; i < C; i += nt) {  // dbeta from M = T Diag(beta)
@@ -348,11 +451,13 @@ __global__ void __launch_bounds__(kBwdThreads)
     sdM[r * ldc + i] *= sbeta[i];
   }
   __syncthreads();
-  for (int idx = tid; idx < C * C; idx += nt) {  // X = dT T^T
-    const int p = idx / C, i = idx - p * C;
-    float s = 0.f;
-    for (int qq = 0; qq <= i; ++qq) s += sdM[p * ldc + qq] * sT[i * ldc + qq];
-    sX[p * ldc + i] = s;
+  {  // X = dT T^T
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    abt_2x2(sdM, ldc, sT, ldc, C, tm, tn, acc);
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 2; ++w) sX[(tm + 16 * u) * ldc + tn + 16 * w] = acc[u][w];
   }
   __syncthreads();
   for (int idx = tid; idx < C * C; idx += nt) {  // dA = -StrictTril(T^T X)
@@ -368,18 +473,51 @@ __global__ void __launch_bounds__(kBwdThreads)
     for (int i = 0; i < r; ++i) s += sdM[r * ldc + i] * sB[r * ldc + i];
     sdb[r] += s;
   }
-  // ---- P4: d(Gamma.K) = M^T dW, dV = M^T dV'
-  for (int idx = tid; idx < C * Dk; idx += nt) {
-    const int i = idx / Dk, a = idx - i * Dk;
-    float s = 0.f;
-    for (int r = i; r < C; ++r) s += sT[r * ldc + i] * X3[r * ldk + a];
-    Y2[i * ldk + a] = s * sbeta[i];
-  }
-  for (int idx = tid; idx < C * Dv; idx += nt) {
-    const int i = idx / Dv, jj = idx - i * Dv;
-    float s = 0.f;
-    for (int r = i; r < C; ++r) s += sT[r * ldc + i] * sdV[r * ldv + jj];
-    if (i < L) dv[((size_t)(t0 + i) * H + h) * Dv + jj] = from_f32<Tin>(s * sbeta[i]);
+  // ---- P4: d(Gamma.K) = M^T dW, dV = M^T dV' (rows {tm, tm + 16}, column groups)
+  {
+    float4 gk[2][2], gv[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 2; ++w)
+        gk[u][w] = gv[u][w] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = tm; r < C; ++r) {  // M[r][i] = 0 for r < i: rows below tm only
+      const float m0 = sT[r * ldc + tm];
+      const float m1 = r >= tm + 16 ? sT[r * ldc + tm + 16] : 0.f;
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int a = 4 * tn + 64 * w;
+        if (a < Dk) {
+          const float4 x = ld4(X3 + r * ldk + a);
+          fma4(m0, x, gk[0][w]);
+          fma4(m1, x, gk[1][w]);
+        }
+        if (a < Dv) {
+          const float4 x = ld4(sdV + r * ldv + a);
+          fma4(m0, x, gv[0][w]);
+          fma4(m1, x, gv[1][w]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = tm + 16 * u;
+      const float b = sbeta[i];
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int a = 4 * tn + 64 * w;
+        if (a < Dk)
+          st4(Y2 + i * ldk + a, make_float4(gk[u][w].x * b, gk[u][w].y * b, gk[u][w].z * b,
+                                            gk[u][w].w * b));
+        if (a < Dv && i < L) {
+          Tin* dst = dv + ((size_t)(t0 + i) * H + h) * Dv + a;
+          dst[0] = from_f32<Tin>(gv[u][w].x * b);
+          dst[1] = from_f32<Tin>(gv[u][w].y * b);
+          dst[2] = from_f32<Tin>(gv[u][w].z * b);
+          dst[3] = from_f32<Tin>(gv[u][w].w * b);
+        }
+      }
+    }
   }
   __syncthreads();
   // ---- P5: elementwise maps of Qt, Gamma.K, Kt onto q, k, g
@@ -393,8 +531,11 @@ __global__ void __launch_bounds__(kBwdThreads)
     X3[x] = dkg * e + dkt * et;                                // dk
   }
   __syncthreads();
-  // ratio-form products through A and P, one thread per key channel; then d log_alpha
-  for (int a = tid; a < Dk; a += nt) {
+  // ratio-form products through A and P: threads [0, Dk) accumulate along rows (row r over
+  // i <= r) into the dk / dq / dg buffers, threads [128, 128 + Dk) along columns (column i over
+  // r >= i) into the dead Gamma.K / d(Gamma.K) buffers; each thread owns one key channel
+  if (tid < Dk) {
+    const int a = tid;
     for (int r = 0; r < C; ++r) {
       const float kr = sK[r * ldk + a], qr = sQ[r * ldk + a], gr = sG[r * ldk + a];
       const float br = sbeta[r];
@@ -404,18 +545,39 @@ __global__ void __launch_bounds__(kBwdThreads)
         const float pa = sdP[r * ldc + i];
         const float aa = i < r ? sdM[r * ldc + i] * br : 0.f;
         const float t1 = e * sK[i * ldk + a];
-        dk_r += aa * t1;
-        dq_r += pa * t1;
-        const float w = aa * kr + pa * qr;
-        const float s = w * t1;
-        dg_r += s;
-        X1[i * ldk + a] -= s;
-        X3[i * ldk + a] += e * w;
+        dk_r = fmaf(aa, t1, dk_r);
+        dq_r = fmaf(pa, t1, dq_r);
+        dg_r = fmaf(fmaf(aa, kr, pa * qr), t1, dg_r);
       }
       X3[r * ldk + a] += dk_r;
       X2[r * ldk + a] += dq_r;
       X1[r * ldk + a] += dg_r;
     }
+  } else if (tid >= 128 && tid - 128 < Dk) {
+    const int a = tid - 128;
+    for (int i = 0; i < C; ++i) {
+      const float ki = sK[i * ldk + a], gi = sG[i * ldk + a];
+      float dk_i = 0.f, dg_i = 0.f;
+      for (int r = i; r < C; ++r) {
+        const float e = __expf(sG[r * ldk + a] - gi);
+        const float pa = sdP[r * ldc + i];
+        const float aa = i < r ? sdM[r * ldc + i] * sbeta[r] : 0.f;
+        const float w = fmaf(aa, sK[r * ldk + a], pa * sQ[r * ldk + a]) * e;
+        dk_i += w;
+        dg_i = fmaf(-w, ki, dg_i);
+      }
+      Y1[i * ldk + a] = dk_i;
+      Y2[i * ldk + a] = dg_i;
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < C * Dk; idx += nt) {
+    const int r = idx / Dk, a = idx - r * Dk;
+    X3[r * ldk + a] += Y1[r * ldk + a];
+    X1[r * ldk + a] += Y2[r * ldk + a];
+  }
+  __syncthreads();
+  for (int a = tid; a < Dk; a += nt) {
     // g_C enters Kt and gamma_C
     const float gc = sG[(C - 1) * ldk + a];
     float dgc = sdgam[a] * expf(gc);

@@ -307,10 +307,14 @@ __global__ void __launch_bounds__(kSimtThreads)
       const int r = rg + m * ng;
       float aw = 0.f, aq = 0.f;
       if (r < C) {
-        for (int cc = 0; cc < Dk; ++cc) {
-          const float s = sS[cc * kSlice + j];
-          aw += sW[r * Dk + cc] * s;
-          aq += sQt[r * Dk + cc] * s;
+        if (o) {
+          for (int cc = 0; cc < Dk; ++cc) {
+            const float s = sS[cc * kSlice + j];
+            aw += sW[r * Dk + cc] * s;
+            aq += sQt[r * Dk + cc] * s;
+          }
+        } else {  // only the states are wanted
+          for (int cc = 0; cc < Dk; ++cc) aw += sW[r * Dk + cc] * sS[cc * kSlice + j];
         }
         sVp[r * kSlice + j] = sU[r * kSlice + j] - aw;
       }
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const int r = rg + m * ng;
-      if (r < C) {
+      if (o && r < C) {
         float acc = o1[m];
         for (int i = 0; i <= r; ++i) acc += sAq[r * C + i] * sVp[i * kSlice + j];
         if (o && r < L && j < NV) o[((size_t)(t0 + r) * H + h) * Dv + j0 + j] = from_f32<Tin>(acc);

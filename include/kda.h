@@ -258,7 +258,8 @@ KDA_API kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const
  * The pass runs the fp32 chunk kernels forward once more (chunks of 32 tokens, whatever chunk
  * the forward call used; the result does not depend on it), keeping the state entering every
  * chunk, then a sequential backward state pass and a parallel chunk-local pass; all arithmetic
- * is fp32 on CUDA cores, for fp32 and bf16 inputs alike. Supported: 1 <= Dk, Dv <= 128. Tokens
+ * is fp32 on CUDA cores, for fp32 and bf16 inputs alike. Supported: Dk, Dv multiples of 4 in
+ * [4, 128] (anything else: KDA_ERR_UNSUPPORTED). Tokens
  * outside every sequence (varlen) are not written. Arguments are checked on the host (pointers
  * aligned to their element size); a bad cu_seqlens is reported by kda_last_device_error().
  */

@@ -220,10 +220,12 @@ def library_source_hash() -> str:
     return h.hexdigest()
 
 
-def captured_traffic(kernel: str, workload: str):
+def captured_traffic(kernel: str, workload: str, path: str | None = None):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture, or None
     when there is none or the library sources changed since it was taken."""
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "traffic.json")
+    if path is None:
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel)

@@ -46,3 +46,25 @@ def test_two_ranks_agree_on_max_time_and_rate():
 def test_single_rank_is_identity():
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
     assert bench.whole_job_rate(100.0, 1, 1000.0) == pytest.approx(100.0)
+
+
+def test_captured_traffic_follows_the_library_sources(tmp_path):
+    """The roofline's DRAM traffic comes from the committed ncu capture only while the library
+    sources hash to the value recorded with it; any other hash (or workload) gives None."""
+    import json
+
+    import bench
+
+    real = bench.library_source_hash()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"chunk_local_tc": {"workload": "w", "dram_bytes_per_launch": 123,
+                              "source_sha256": real}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    path = str(prof / "traffic.json")
+    assert bench.captured_traffic("chunk_local_tc", "w", path) == 123
+    assert bench.captured_traffic("chunk_local_tc", "other", path) is None
+    assert bench.captured_traffic("chunk_state_tc", "w", path) is None
+    rec["chunk_local_tc"]["source_sha256"] = "0" * 64
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.captured_traffic("chunk_local_tc", "w", path) is None

@@ -314,7 +314,9 @@ def run_prefill_e2e(spec, x, o, fs, ws, dev, steps, warmup, world):
     return ms, h2d, d2h
 
 
-def run_decode(spec, n_steps, dev, warmup, world, rank):
+def run_decode(spec, n_steps, dev, warmup, world, rank, fused=False):
+    """Decode steps over the pre-staged inputs of every step; with ``fused`` each step also runs
+    the layer's prologue (q/k L2 norm, decay gate from the raw gate) and output epilogue."""
     import torch
 
     import gated_delta_rule_120_b200 as kda
@@ -323,11 +325,20 @@ def run_decode(spec, n_steps, dev, warmup, world, rank):
     state = kda_synth.decode_state(spec, 2004 + 10 * rank, dev)
     x = kda_synth.decode_step_inputs(spec, 2004 + 10 * rank, n_steps, dev)
     o = torch.empty((spec.N, spec.H, spec.Dv), dtype=x["q"].dtype, device=dev)
+    fusion = None
+    if fused:
+        g = torch.Generator(device=dev).manual_seed(2104 + 10 * rank)
+        fusion = dict(qk_l2norm=True, eps=1e-6,
+                      A_log=torch.log(torch.rand((spec.H,), generator=g, device=dev) * 15 + 1) - 2,
+                      dt_bias=torch.randn((spec.H, spec.Dk), generator=g, device=dev) * 0.5,
+                      out_norm=True, out_norm_eps=1e-5,
+                      out_norm_weight=torch.rand((spec.Dv,), generator=g, device=dev) + 0.5,
+                      out_gate=torch.randn(o.shape, generator=g, device=dev).to(o.dtype))
 
     def step(i):
         s = i % n_steps
         kda.kda_recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["log_alpha"][s], x["beta"][s],
-                               state, o=o)
+                               state, o=o, fusion=fusion)
 
     ms = timed(step, n_steps, warmup, world, dev)
     prof = profile_pass(step, min(n_steps, 64), dev)
@@ -619,6 +630,14 @@ def main():
         tbytes = roofline.decode_total_bytes(dspec.N, dspec.H, dspec.Dk, dspec.Dv, 2)
         per = dms / args.decode_steps
         kms = dprof[0]["total_ms"] / dprof[0]["launches"]
+        # the same decode steps with the layer's prologue and output epilogue fused in
+        fsteps = min(256, args.decode_steps)
+        fdms, _ = run_decode(dspec, fsteps, dev, 3, world, rank, fused=True)
+        fper = fdms / fsteps
+        fused_decode = {"workload": dspec.name + "_fused_prologue_epilogue", "steps": fsteps,
+                        "ms_per_step": fper,
+                        "state_gbs": world * sbytes / (fper / 1e3) / 1e9,
+                        "frac_hbm_state": sbytes / (fper / 1e3) / 1e9 / hbm_peak}
         extra["decode"] = {
             "workload": dspec.name, "steps": args.decode_steps, "ms_per_step": per,
             "state_gbs": world * sbytes / (per / 1e3) / 1e9,
@@ -626,7 +645,8 @@ def main():
             "total_gbs": world * tbytes / (per / 1e3) / 1e9,
             "kernel": {"name": dprof[0]["name"], "ms_per_launch": kms,
                        "achieved_gbs": tbytes / (kms / 1e3) / 1e9,
-                       "frac": tbytes / (kms / 1e3) / 1e9 / hbm_peak}}
+                       "frac": tbytes / (kms / 1e3) / 1e9 / hbm_peak},
+            "fused": fused_decode}
         torch.cuda.empty_cache()
 
     cpu = None

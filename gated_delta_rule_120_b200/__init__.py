@@ -33,7 +33,7 @@ ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
                "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
                "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused",
-               "kda_chunk_bwd_workspace_size", "kda_chunk_bwd")
+               "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_recurrent_step_fused")
 
 
 class Fusion(ctypes.Structure):
@@ -94,6 +94,9 @@ def lib() -> ctypes.CDLL:
                                                   i32, i32, i32, i32, i32, i32,
                                                   ctypes.POINTER(Fusion), vp]
             L.kda_recurrent_fwd_fused.restype = ctypes.c_int
+            L.kda_recurrent_step_fused.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i32,
+                                                   i32, i32, i32, ctypes.POINTER(Fusion), vp]
+            L.kda_recurrent_step_fused.restype = ctypes.c_int
             L.kda_chunk_bwd_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int,
                                                                    ctypes.POINTER(sz)]
             L.kda_chunk_bwd_workspace_size.restype = ctypes.c_int
@@ -296,9 +299,10 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_sta
     return dq, dk, dv, dla, db, ds0
 
 
-def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
+def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None, fusion=None):
     """One decode token per sequence: q, k [N,H,Dk], v [N,H,Dv], log_alpha [N,H,Dk] fp32,
-    beta [N,H] fp32; ``state`` [N,H,Dk,Dv] fp32 is updated in place. Returns o [N,H,Dv]."""
+    beta [N,H] fp32; ``state`` [N,H,Dk,Dv] fp32 is updated in place. Returns o [N,H,Dv].
+    ``fusion``: as for :func:`kda_chunk_fwd` (out_gate then has o's shape [N,H,Dv])."""
     dev = q.device
     N, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -311,9 +315,13 @@ def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None):
         raise ValueError("state must be [N,H,Dk,Dv]")
     if o is None:
         o = torch.empty((N, H, Dv), dtype=q.dtype, device=dev)
-    code = lib().kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
-                                    _ptr(beta), _ptr(state), _ptr(o), N, H, Dk, Dv,
-                                    _stream_handle(dev))
+    fz = _fusion(fusion, dev, H, Dk, v)
+    args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), _ptr(state),
+            _ptr(o), N, H, Dk, Dv)
+    if fz is None:
+        code = lib().kda_recurrent_step(*args, _stream_handle(dev))
+    else:
+        code = lib().kda_recurrent_step_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_recurrent_step")
     return o
 

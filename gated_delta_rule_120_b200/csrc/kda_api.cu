@@ -331,6 +331,26 @@ kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, kda_dty
                                        (float*)(ws + lay.rec_base), rec, stream));
 }
 
+kda_status_t recurrent_step_impl(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                 const float* log_alpha, const float* beta, float* state, void* o,
+                                 int32_t N, int32_t H, int32_t Dk, int32_t Dv, const Fusion* fz,
+                                 kda_stream_t stream) {
+  if (N < 0 || H < 0 || Dk <= 0 || Dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H == 0) return KDA_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;  // q, k, v, o need element alignment only
+  if (!aligned(state, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
+      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+    return KDA_ERR_INVALID_ARG;
+  if (fz && fz->onorm && ((fz->og && !aligned(fz->og, es)) || (fz->ow && !aligned(fz->ow, 16))))
+    return KDA_ERR_INVALID_ARG;
+  return from_cuda(launch_decode_step(q, k, v, dt, log_alpha, beta, state, o, N, H, Dk, Dv, fz,
+                                      (cudaStream_t)stream));
+}
+
 kda_status_t recurrent_fwd_impl(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                 const float* log_alpha, const float* beta, float* pool,
                                 const int32_t* state_indices, void* o, int32_t N, int32_t T,
@@ -386,18 +406,20 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda
                                 const float* log_alpha, const float* beta, float* state, void* o,
                                 int32_t N, int32_t H, int32_t Dk, int32_t Dv,
                                 kda_stream_t stream) {
-  if (N < 0 || H < 0 || Dk <= 0 || Dv <= 0) return KDA_ERR_INVALID_ARG;
-  if (dt != KDA_DTYPE_F32 && dt != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
-  if (Dk > 128 || Dv > 128 || Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
-  if ((long long)N * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
-  if ((long long)N * H == 0) return KDA_OK;
-  if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
-  const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;  // q, k, v, o need element alignment only
-  if (!aligned(state, 16) || !aligned(q, es) || !aligned(k, es) || !aligned(v, es) ||
-      !aligned(o, es) || !aligned(log_alpha, 4) || !aligned(beta, 4))
-    return KDA_ERR_INVALID_ARG;
-  return from_cuda(launch_decode_step(q, k, v, dt, log_alpha, beta, state, o, N, H, Dk, Dv,
-                                      (cudaStream_t)stream));
+  return recurrent_step_impl(q, k, v, dt, log_alpha, beta, state, o, N, H, Dk, Dv, nullptr,
+                             stream);
+}
+
+kda_status_t kda_recurrent_step_fused(const void* q, const void* k, const void* v,
+                                      kda_dtype_t dt, const float* log_alpha_or_gate,
+                                      const float* beta, float* state, void* o, int32_t N,
+                                      int32_t H, int32_t Dk, int32_t Dv,
+                                      const kda_fusion_t* fusion, kda_stream_t stream) {
+  Fusion fz;
+  const kda_status_t st = to_fusion(fusion, &fz);
+  if (st != KDA_OK) return st;
+  return recurrent_step_impl(q, k, v, dt, log_alpha_or_gate, beta, state, o, N, H, Dk, Dv,
+                             fusion ? &fz : nullptr, stream);
 }
 
 kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void* v, kda_dtype_t dt,

@@ -333,19 +333,26 @@ constexpr int kDsThreads = kDsCompute + 32;    // + producer warp
 
 struct DsLayout {
   uint32_t state_bytes, la_off, q_off, k_off, v_off, stage_bytes, vec_tx;
+  uint32_t og_off, bias_off;  // fused step: output gate row and the head's dt_bias row
+  uint32_t og_bytes, bias_bytes;  // 0 when the fused step has no such input
 };
 
 __host__ __device__ inline uint32_t align16u(uint32_t x) { return (x + 15u) & ~15u; }
 
-static DsLayout make_ds_layout(int Dk, int Dv, int es) {
+static DsLayout make_ds_layout(int Dk, int Dv, int es, bool gate_row = false,
+                               bool bias_row = false) {
   DsLayout L;
   L.state_bytes = (uint32_t)Dk * Dv * 4;
   L.la_off = L.state_bytes;
   L.q_off = L.la_off + align16u((uint32_t)Dk * 4);
   L.k_off = L.q_off + align16u((uint32_t)Dk * es);
   L.v_off = L.k_off + align16u((uint32_t)Dk * es);
-  L.stage_bytes = (L.v_off + align16u((uint32_t)Dv * es) + 127u) & ~127u;
-  L.vec_tx = (uint32_t)Dk * 4 + 2u * Dk * es + (uint32_t)Dv * es;
+  L.og_off = L.v_off + align16u((uint32_t)Dv * es);
+  L.og_bytes = gate_row ? (uint32_t)Dv * es : 0u;
+  L.bias_off = L.og_off + align16u(L.og_bytes);
+  L.bias_bytes = bias_row ? (uint32_t)Dk * 4 : 0u;
+  L.stage_bytes = (L.bias_off + align16u(L.bias_bytes) + 127u) & ~127u;
+  L.vec_tx = (uint32_t)Dk * 4 + 2u * Dk * es + (uint32_t)Dv * es + L.og_bytes + L.bias_bytes;
   return L;
 }
 
@@ -362,19 +369,23 @@ __device__ __forceinline__ bool block_all(bool pred, uint32_t bar_id, uint32_t n
   return r != 0;
 }
 
-template <typename Tin>
+// kFused: the prologue and epilogue of kda_fusion_t (log_alpha holds the raw gate when A_log is
+// given; q and k normalised through the reductions; output RMSNorm x sigmoid gate in warp 0).
+template <typename Tin, bool kFused>
 __global__ void __launch_bounds__(kDsThreads, 1)
     decode_stream_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                          const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                          const float* __restrict__ beta, float* __restrict__ state,
-                         Tin* __restrict__ o, int NH, int Dk, int Dv, DsLayout lay) {
+                         Tin* __restrict__ o, int NH, int Dk, int Dv, DsLayout lay, int H,
+                         Fusion fz) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((128 - (sm100::smem_u32(smem_raw) & 127)) & 127);
   uint8_t* stages = sm;
   float4* s_e = reinterpret_cast<float4*>(sm + kDsStages * lay.stage_bytes);  // [8][32]
   float4* s_p = s_e + 8 * 32;                                                 // [8][32]
   float* s_kq = reinterpret_cast<float*>(s_p + 8 * 32);                        // [8]
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_kq + 8);                      // [kDsStages]
+  float* s_ss = s_kq + 8;                                                      // [2][8] (fused)
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_kq + 24);                     // [kDsStages]
   uint64_t* computed = full + kDsStages;                                       // [kDsStages]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -404,6 +415,12 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         sm100::bulk_g2s(st + lay.q_off, q + head * Dk, Dk * es, full + s);
         sm100::bulk_g2s(st + lay.k_off, k + head * Dk, Dk * es, full + s);
         sm100::bulk_g2s(st + lay.v_off, v + head * Dv, Dv * es, full + s);
+        if (kFused && lay.og_bytes)
+          sm100::bulk_g2s(st + lay.og_off, reinterpret_cast<const Tin*>(fz.og) + head * Dv,
+                          lay.og_bytes, full + s);
+        if (kFused && lay.bias_bytes)
+          sm100::bulk_g2s(st + lay.bias_off, fz.dt_bias + (head % (size_t)H) * Dk,
+                          lay.bias_bytes, full + s);
       };
       for (int it = 0; it < count && it < kDsStages; ++it) issue_load(it);
       for (int it = 0; it < count; ++it) {
@@ -431,11 +448,16 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     const bool col_ok = col < Dv;
     const int row0 = warp * kDecRowsPerWarp;
     float b_next = count > 0 ? beta[first] : 0.f;
+    // fused gate: -exp(A_log[h]) of the next head, fetched a head ahead like beta
+    float na_next = (kFused && fz.A_log && count > 0) ? -expf(fz.A_log[first % H]) : 0.f;
     for (int it = 0; it < count; ++it) {
       const int s = it % kDsStages;
       const size_t head = (size_t)first + (size_t)it * stride;
       const float b = b_next;
       if (it + 1 < count) b_next = beta[head + stride];
+      const float neg_a = na_next;
+      if (kFused && fz.A_log && it + 1 < count)
+        na_next = -expf(fz.A_log[(head + stride) % (size_t)H]);
       const bool ok = sm100::mbar_wait(full + s, (it / kDsStages) & 1);
       if (!block_all(ok, 1, kDsCompute)) break;
       uint8_t* st = stages + (size_t)s * lay.stage_bytes;
@@ -445,7 +467,13 @@ __global__ void __launch_bounds__(kDsThreads, 1)
       const Tin* vv = reinterpret_cast<const Tin*>(st + lay.v_off);
       // decay of this warp's 16 rows: lanes 0..15 evaluate one each, shuffled to the warp
       const int rl = row0 + (lane & 15);
-      const float a_mine = (rl < Dk) ? expf(la[rl]) : 1.f;
+      float la_mine = (rl < Dk) ? la[rl] : 0.f;
+      if (kFused && fz.A_log && rl < Dk) {  // fused gate: raw gate -> log decay
+        const float bias = lay.bias_bytes ? reinterpret_cast<const float*>(st + lay.bias_off)[rl]
+                                          : 0.f;
+        la_mine = neg_a * softplus_f(la_mine + bias);
+      }
+      const float a_mine = (rl < Dk) ? expf(la_mine) : 1.f;
       float4* Srow = reinterpret_cast<float4*>(st) + (col >> 2);
       const int vstride = Dv >> 2;
       float4 sreg[kDecRowsPerWarp];
@@ -455,7 +483,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         sreg[i] = (col_ok && r < Dk) ? Srow[r * vstride] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
-      float kq = 0.f;
+      float kq = 0.f, ssk = 0.f, ssq = 0.f;
       float kr_[kDecRowsPerWarp];
 #pragma unroll
       for (int i = 0; i < kDecRowsPerWarp; ++i) {
@@ -465,13 +493,23 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         const float qr = (r < Dk) ? to_f32(qv[r]) : 0.f;
         kr_[i] = kr;
         kq += kr * qr;
+        if (kFused) {
+          ssk += kr * kr;
+          ssq += qr * qr;
+        }
         sreg[i].x *= a; sreg[i].y *= a; sreg[i].z *= a; sreg[i].w *= a;
         e.x += sreg[i].x * kr; e.y += sreg[i].y * kr; e.z += sreg[i].z * kr; e.w += sreg[i].w * kr;
         p.x += sreg[i].x * qr; p.y += sreg[i].y * qr; p.z += sreg[i].z * qr; p.w += sreg[i].w * qr;
       }
       s_e[warp * 32 + lane] = e;
       s_p[warp * 32 + lane] = p;
-      if (lane == 0) s_kq[warp] = kq;
+      if (lane == 0) {
+        s_kq[warp] = kq;
+        if (kFused) {
+          s_ss[warp] = ssk;
+          s_ss[8 + warp] = ssq;
+        }
+      }
       sm100::named_barrier_sync(1, kDsCompute);
       e = make_float4(0.f, 0.f, 0.f, 0.f);
       p = e;
@@ -482,6 +520,20 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         e.x += ew.x; e.y += ew.y; e.z += ew.z; e.w += ew.w;
         p.x += pw.x; p.y += pw.y; p.z += pw.z; p.w += pw.w;
         kq += s_kq[w];
+      }
+      float ik = 1.f;
+      if (kFused && fz.l2) {  // fused L2 norm, applied to the reductions and to the update
+        float sk = 0.f, sq = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          sk += s_ss[w];
+          sq += s_ss[8 + w];
+        }
+        ik = rsqrtf(sk + fz.eps);
+        const float iq = rsqrtf(sq + fz.eps);
+        e.x *= ik; e.y *= ik; e.z *= ik; e.w *= ik;
+        p.x *= iq; p.y *= iq; p.z *= iq; p.w *= iq;
+        kq *= ik * iq;
       }
       float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
       if (col_ok) {
@@ -494,17 +546,40 @@ __global__ void __launch_bounds__(kDsThreads, 1)
       for (int i = 0; i < kDecRowsPerWarp; ++i) {
         const int r = row0 + i;
         if (col_ok && r < Dk) {
+          const float kn = kr_[i] * ik;
           float4 t = sreg[i];
-          t.x += kr_[i] * u.x; t.y += kr_[i] * u.y; t.z += kr_[i] * u.z; t.w += kr_[i] * u.w;
+          t.x += kn * u.x; t.y += kn * u.y; t.z += kn * u.z; t.w += kn * u.w;
           Srow[r * vstride] = t;
         }
       }
-      if (warp == 0 && col_ok) {
-        Tin* op = o + head * Dv + col;
-        op[0] = from_f32<Tin>(p.x + kq * u.x);
-        op[1] = from_f32<Tin>(p.y + kq * u.y);
-        op[2] = from_f32<Tin>(p.z + kq * u.z);
-        op[3] = from_f32<Tin>(p.w + kq * u.w);
+      if (warp == 0) {
+        float4 y = make_float4(p.x + kq * u.x, p.y + kq * u.y, p.z + kq * u.z, p.w + kq * u.w);
+        if (kFused && fz.onorm) {  // output epilogue: head-wise RMSNorm x sigmoid gate
+          float ss = col_ok ? y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w : 0.f;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
+          if (col_ok) {
+            float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+                              : make_float4(1.f, 1.f, 1.f, 1.f);
+            if (lay.og_bytes) {  // the output gate row staged with the head's vectors
+              const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off) + col;
+              wv.x *= sigmoid_f(to_f32(gp[0]));
+              wv.y *= sigmoid_f(to_f32(gp[1]));
+              wv.z *= sigmoid_f(to_f32(gp[2]));
+              wv.w *= sigmoid_f(to_f32(gp[3]));
+            }
+            y = make_float4(y.x * inv * wv.x, y.y * inv * wv.y, y.z * inv * wv.z,
+                            y.w * inv * wv.w);
+          }
+        }
+        if (col_ok) {
+          Tin* op = o + head * Dv + col;
+          op[0] = from_f32<Tin>(y.x);
+          op[1] = from_f32<Tin>(y.y);
+          op[2] = from_f32<Tin>(y.z);
+          op[3] = from_f32<Tin>(y.w);
+        }
       }
       sm100::fence_proxy_async_smem();
       sm100::named_barrier_sync(1, kDsCompute);
@@ -516,15 +591,36 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 
 static int g_num_sms[64] = {0};
 
+template <typename Tin, bool kFused>
+static cudaError_t launch_stream_typed(const void* q, const void* k, const void* v,
+                                       const float* log_alpha, const float* beta, float* state,
+                                       void* o, int heads, int Dk, int Dv, const DsLayout& lay,
+                                       int grid, size_t smem, int H, const Fusion& fz,
+                                       cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(decode_stream_kernel<Tin, kFused>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  decode_stream_kernel<Tin, kFused><<<grid, kDsThreads, smem, stream>>>(
+      (const Tin*)q, (const Tin*)k, (const Tin*)v, log_alpha, beta, state, (Tin*)o, heads, Dk,
+      Dv, lay, H, fz);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                const float* log_alpha, const float* beta, float* state, void* o,
-                               int N, int H, int Dk, int Dv, cudaStream_t stream) {
+                               int N, int H, int Dk, int Dv, const Fusion* fz,
+                               cudaStream_t stream) {
   const long long heads = (long long)N * H;
   if (heads == 0) return cudaSuccess;
   const int es = dt == KDA_DTYPE_BF16 ? 2 : 4;
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
   const bool streamable = (Dk * es) % 16 == 0 && (Dv * es) % 16 == 0 && (Dk * 4) % 16 == 0 &&
-                          al16(q) && al16(k) && al16(v) && al16(log_alpha) && al16(state);
+                          al16(q) && al16(k) && al16(v) && al16(log_alpha) && al16(state) &&
+                          (!fz || ((!fz->onorm || !fz->og || al16(fz->og)) &&
+                                   (!fz->A_log || !fz->dt_bias || al16(fz->dt_bias))));
+  if (fz && !streamable)  // the fused step on other shapes: the token-by-token kernel with T = 1
+    return launch_recurrent_multi(q, k, v, dt, log_alpha, beta, state, nullptr, o, N, 1, H, Dk,
+                                  Dv, N, *fz, stream);
   if (streamable) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -535,27 +631,25 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_
       if (err != cudaSuccess) return err;
       if (dev >= 0 && dev < 64) g_num_sms[dev] = nsm;
     }
-    const DsLayout lay = make_ds_layout(Dk, Dv, es);
+    const DsLayout lay = make_ds_layout(Dk, Dv, es, fz && fz->onorm && fz->og,
+                                        fz && fz->A_log && fz->dt_bias);
     const size_t smem = (size_t)kDsStages * lay.stage_bytes + 2 * 8 * 32 * sizeof(float4) +
-                        8 * sizeof(float) + 2 * kDsStages * sizeof(uint64_t) + 128;
+                        24 * sizeof(float) + 2 * kDsStages * sizeof(uint64_t) + 128;
     const int grid = (int)(heads < nsm ? heads : nsm);
-    ProfileScope prof("decode_stream", stream);
-    if (dt == KDA_DTYPE_BF16) {
-      err = cudaFuncSetAttribute(decode_stream_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err != cudaSuccess) return err;
-      decode_stream_kernel<__nv_bfloat16><<<grid, kDsThreads, smem, stream>>>(
-          (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha,
-          beta, state, (__nv_bfloat16*)o, (int)heads, Dk, Dv, lay);
-    } else {
-      err = cudaFuncSetAttribute(decode_stream_kernel<float>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err != cudaSuccess) return err;
-      decode_stream_kernel<float><<<grid, kDsThreads, smem, stream>>>(
-          (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, state, (float*)o,
-          (int)heads, Dk, Dv, lay);
-    }
-    return cudaGetLastError();
+    const Fusion none;
+    ProfileScope prof(fz ? "decode_stream_fused" : "decode_stream", stream);
+    if (dt == KDA_DTYPE_BF16)
+      return fz ? launch_stream_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, state, o,
+                                                           (int)heads, Dk, Dv, lay, grid, smem,
+                                                           H, *fz, stream)
+                : launch_stream_typed<__nv_bfloat16, false>(q, k, v, log_alpha, beta, state, o,
+                                                            (int)heads, Dk, Dv, lay, grid, smem,
+                                                            H, none, stream);
+    return fz ? launch_stream_typed<float, true>(q, k, v, log_alpha, beta, state, o, (int)heads,
+                                                 Dk, Dv, lay, grid, smem, H, *fz, stream)
+              : launch_stream_typed<float, false>(q, k, v, log_alpha, beta, state, o,
+                                                  (int)heads, Dk, Dv, lay, grid, smem, H, none,
+                                                  stream);
   }
   dim3 grid((unsigned)heads), block(kDecThreads);
   ProfileScope prof("decode_step", stream);

@@ -100,7 +100,8 @@ size_t tc_state_smem_bytes();
 
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                const float* log_alpha, const float* beta, float* state, void* o,
-                               int N, int H, int Dk, int Dv, cudaStream_t stream);
+                               int N, int H, int Dk, int Dv, const Fusion* fz,
+                               cudaStream_t stream);
 
 cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
                                    const float* log_alpha, const float* beta, float* pool,

@@ -227,6 +227,15 @@ KDA_API kda_status_t kda_chunk_fwd_fused(const void* q, const void* k, const voi
                                          void* workspace, size_t workspace_bytes,
                                          const kda_fusion_t* fusion, kda_stream_t stream);
 
+/* kda_recurrent_step with the fusion above (the serving decode step with the layer's prologue
+ * and epilogue); fusion == NULL is exactly kda_recurrent_step. The streaming kernel runs it when
+ * the shapes and pointers allow 16-byte bulk copies, the token-by-token kernel otherwise. */
+KDA_API kda_status_t kda_recurrent_step_fused(const void* q, const void* k, const void* v,
+                                              kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,
+                                              const float* beta, float* state, void* o, int32_t N,
+                                              int32_t H, int32_t Dk, int32_t Dv,
+                                              const kda_fusion_t* fusion, kda_stream_t stream);
+
 /* kda_recurrent_fwd with the fusion above; fusion == NULL is exactly kda_recurrent_fwd. */
 KDA_API kda_status_t kda_recurrent_fwd_fused(const void* q, const void* k, const void* v,
                                              kda_dtype_t qkv_dtype, const float* log_alpha_or_gate,

@@ -166,9 +166,10 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return world * units_per_rank / (max_ms / 1e3)
 
 
-def timed(fn, steps, warmup, world, dev):
+def timed(fn, steps, warmup, world, dev, join=None):
     """W untimed warm-up steps, then K steps between a barrier + synchronize on both sides;
-    device time from CUDA events on the launching stream, max over ranks."""
+    device time from CUDA events on the launching stream, max over ranks. `join` (optional) makes
+    the launching stream wait for work that `fn` queued on other streams before the end event."""
     import torch
 
     for i in range(warmup):
@@ -180,7 +181,9 @@ def timed(fn, steps, warmup, world, dev):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s)
     for i in range(steps):
-        fn(i)
+        fn(warmup + i)
+    if join is not None:
+        join()
     e1.record(s)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -286,8 +289,10 @@ def run_prefill(spec, seeds, dev, steps, warmup, world):
 
 
 def run_prefill_e2e(spec, x, o, fs, ws, dev, steps, warmup, world):
-    """Public-API end to end: pinned host inputs -> device, kda_chunk_fwd, o and final state back
-    to pinned host memory, every step."""
+    """Public-API end to end: every step copies its inputs from pinned host memory to the device,
+    runs kda_chunk_fwd and copies o and the final state back to pinned host memory. Steps are
+    pipelined as a serving loop would: host->device copies on one stream, the operator on the
+    launching stream, device->host copies on a third, two buffer sets, events between them."""
     import torch
 
     import gated_delta_rule_120_b200 as kda
@@ -295,22 +300,48 @@ def run_prefill_e2e(spec, x, o, fs, ws, dev, steps, warmup, world):
     names = ["q", "k", "v", "log_alpha", "beta"] + \
         (["initial_state"] if x["initial_state"] is not None else [])
     host = {n: x[n].cpu().pin_memory() for n in names}
-    dbuf = {n: torch.empty_like(x[n]) for n in names}
+    dbuf = [{n: torch.empty_like(x[n]) for n in names} for _ in range(2)]
+    obuf = [(o, fs), (torch.empty_like(o), torch.empty_like(fs))]
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    computed, out_free = [ev(), ev()], [ev(), ev()]
+    last_out = [None]
 
     def step(i):
-        for n in names:
-            dbuf[n].copy_(host[n], non_blocking=True)
-        kda.kda_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
-                          initial_state=dbuf.get("initial_state"), chunk=spec.chunk, o=o,
-                          final_state=fs, workspace=ws)
-        ho.copy_(o, non_blocking=True)
-        hs.copy_(fs, non_blocking=True)
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(in_free[b])
+            for n in names:
+                dbuf[b][n].copy_(host[n], non_blocking=True)
+            in_ready[b].record(s_in)
+        comp.wait_event(in_ready[b])
+        if i >= 2:
+            comp.wait_event(out_free[b])
+        d, (ob, fb) = dbuf[b], obuf[b]
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                          initial_state=d.get("initial_state"), chunk=spec.chunk, o=ob,
+                          final_state=fb, workspace=ws)
+        in_free[b].record(comp)
+        computed[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[b])
+            ho.copy_(ob, non_blocking=True)
+            hs.copy_(fb, non_blocking=True)
+            out_free[b].record(s_out)
+        last_out[0] = out_free[b]
 
-    ms = timed(step, steps, warmup, world, dev)
+    def join():
+        comp.wait_event(last_out[0])
+
+    ms = timed(step, steps, warmup, world, dev, join=join)
+    torch.cuda.synchronize(dev)
     return ms, h2d, d2h
 
 

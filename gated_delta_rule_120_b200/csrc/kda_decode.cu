@@ -302,10 +302,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
 }
 
-cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
-                                   const float* log_alpha, const float* beta, float* pool,
-                                   const int32_t* idx, void* o, int N, int T, int H, int Dk,
-                                   int Dv, int P, const Fusion& fz, cudaStream_t stream) {
+static cudaError_t launch_recurrent_blockwise(const void* q, const void* k, const void* v,
+                                              kda_dtype_t dt, const float* log_alpha,
+                                              const float* beta, float* pool, const int32_t* idx,
+                                              void* o, int N, int T, int H, int Dk, int Dv, int P,
+                                              const Fusion& fz, cudaStream_t stream) {
   const long long heads = (long long)N * H;
   if (heads == 0 || T == 0) return cudaSuccess;
   ProfileScope prof("recurrent_multi", stream);
@@ -589,7 +590,368 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   __syncthreads();
 }
 
+// ---------------------------------------------------------------------------------------------
+// Streaming multi-token variant of the recurrent mode (T <= kRsMaxT tokens per sequence): one
+// persistent CTA per SM walks its (sequence, head) items through a two-stage ring. The producer
+// warp bulk-loads the item's state (from the pool row given by the state index) and all T
+// tokens' vectors at once, and bulk-stores the state back after the last token; the eight compute
+// warps keep the state in registers across the T tokens (two block reductions per token), so
+// no token waits on global memory and the state crosses HBM once per call.
+// ---------------------------------------------------------------------------------------------
+constexpr int kRsStages = 2;
+constexpr int kRsMaxT = 32;
+
+struct RsLayout {
+  uint32_t state_bytes, la_off, q_off, k_off, v_off, og_off, bias_off, stage_bytes;
+  uint32_t la_row, qk_row, v_row, og_row;  // bytes of one token's row in the stage
+  uint32_t bias_bytes, vec_tx;
+};
+
+static RsLayout make_rs_layout(int T, int Dk, int Dv, int es, bool gate_rows, bool bias_row) {
+  RsLayout L;
+  L.state_bytes = (uint32_t)Dk * Dv * 4;
+  L.la_row = align16u((uint32_t)Dk * 4);
+  L.qk_row = align16u((uint32_t)Dk * es);
+  L.v_row = align16u((uint32_t)Dv * es);
+  L.og_row = gate_rows ? L.v_row : 0u;
+  L.la_off = L.state_bytes;
+  L.q_off = L.la_off + (uint32_t)T * L.la_row;
+  L.k_off = L.q_off + (uint32_t)T * L.qk_row;
+  L.v_off = L.k_off + (uint32_t)T * L.qk_row;
+  L.og_off = L.v_off + (uint32_t)T * L.v_row;
+  L.bias_off = L.og_off + (uint32_t)T * L.og_row;
+  L.bias_bytes = bias_row ? (uint32_t)Dk * 4 : 0u;
+  L.stage_bytes = (L.bias_off + L.bias_bytes + 127u) & ~127u;
+  L.vec_tx = (uint32_t)T * ((uint32_t)Dk * 4 + 2u * Dk * es + (uint32_t)Dv * es +
+                            (gate_rows ? (uint32_t)Dv * es : 0u)) +
+             L.bias_bytes;
+  return L;
+}
+
+template <typename Tin, bool kFused>
+__global__ void __launch_bounds__(kDsThreads, 1)
+    recurrent_stream_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                            const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                            const float* __restrict__ beta, float* __restrict__ pool,
+                            const int32_t* __restrict__ state_indices, Tin* __restrict__ o,
+                            int NH, int T, int H, int Dk, int Dv, int P, RsLayout lay, Fusion fz) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((128 - (sm100::smem_u32(smem_raw) & 127)) & 127);
+  uint8_t* stages = sm;
+  float4* s_e = reinterpret_cast<float4*>(sm + kRsStages * lay.stage_bytes);  // [8][32]
+  float4* s_p = s_e + 8 * 32;                                                 // [8][32]
+  float* s_kq = reinterpret_cast<float*>(s_p + 8 * 32);                        // [8]
+  float* s_ss = s_kq + 8;                                                      // [2][8]
+  float* s_beta = s_ss + 16;                                   // [2][kRsMaxT + 1] (+ -exp(A_log))
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_beta + 2 * (kRsMaxT + 2));    // [kRsStages]
+  uint64_t* computed = full + kRsStages;                                       // [kRsStages]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int first = blockIdx.x, stride = gridDim.x;
+  const int count = first < NH ? (NH - first + stride - 1) / stride : 0;
+  const uint32_t es = sizeof(Tin);
+  // pool row of an item, -1 to skip it (padding entry or an index past the pool)
+  auto slot_of = [&](int it) -> int {
+    const int item = first + it * stride, n = item / H;
+    const int sl = state_indices ? state_indices[n] : n;
+    return (sl >= 0 && sl < P) ? sl : -1;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kRsStages; ++i) {
+      sm100::mbar_init(full + i, 1);
+      sm100::mbar_init(computed + i, 1);
+    }
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kDsCompute / 32) {
+    // ---------------------------------------------------------------- producer warp
+    auto issue_load = [&](int it, int slot) {
+      const int s = it % kRsStages;
+      if (slot < 0) {  // nothing to load: complete the phase so the compute warps move on
+        if (lane == 0) sm100::mbar_arrive(full + s);
+        return;
+      }
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+      if (lane == 0) {
+        sm100::mbar_arrive_expect_tx(full + s, lay.state_bytes + lay.vec_tx);
+        sm100::bulk_g2s(st, pool + ((size_t)slot * H + h) * Dk * Dv, lay.state_bytes, full + s);
+        if (kFused && lay.bias_bytes)
+          sm100::bulk_g2s(st + lay.bias_off, fz.dt_bias + (size_t)h * Dk, lay.bias_bytes,
+                          full + s);
+      }
+      for (int t = lane; t < T; t += 32) {  // one token's rows per lane
+        const size_t base = ((size_t)n * T + t) * H + h;
+        sm100::bulk_g2s(st + lay.la_off + t * lay.la_row, log_alpha + base * Dk, Dk * 4,
+                        full + s);
+        sm100::bulk_g2s(st + lay.q_off + t * lay.qk_row, q + base * Dk, Dk * es, full + s);
+        sm100::bulk_g2s(st + lay.k_off + t * lay.qk_row, k + base * Dk, Dk * es, full + s);
+        sm100::bulk_g2s(st + lay.v_off + t * lay.v_row, v + base * Dv, Dv * es, full + s);
+        if (kFused && lay.og_row)
+          sm100::bulk_g2s(st + lay.og_off + t * lay.og_row,
+                          reinterpret_cast<const Tin*>(fz.og) + base * Dv, Dv * es, full + s);
+      }
+    };
+    int slot_cur[kRsStages];
+    for (int it = 0; it < count && it < kRsStages; ++it) {
+      slot_cur[it] = slot_of(it);
+      issue_load(it, slot_cur[it]);
+    }
+    for (int it = 0; it < count; ++it) {
+      const int s = it % kRsStages;
+      bool ok = sm100::mbar_wait(computed + s, (it / kRsStages) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0 && slot_cur[s] >= 0) {
+        const int item = first + it * stride, h = item % H;
+        sm100::bulk_s2g(pool + ((size_t)slot_cur[s] * H + h) * Dk * Dv,
+                        stages + (size_t)s * lay.stage_bytes, lay.state_bytes);
+        sm100::bulk_commit();
+      }
+      if (it + kRsStages < count) {
+        if (lane == 0) sm100::bulk_wait_read_all();  // the stage is free once its store read it
+        __syncwarp();
+        slot_cur[s] = slot_of(it + kRsStages);
+        issue_load(it + kRsStages, slot_cur[s]);
+      }
+    }
+    if (lane == 0) {
+      sm100::bulk_wait_all();
+      // loads that were issued but never consumed (only after a timeout) must land first
+      for (int it = 0; it < count && it < kRsStages; ++it) {
+        const int last = count - 1 - it;
+        if (last >= 0)
+          sm100::mbar_wait(full + last % kRsStages, (last / kRsStages) & 1, 100000000ull);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    const int col = lane * 4;
+    const bool col_ok = col < Dv;
+    const int row0 = warp * kDecRowsPerWarp;
+    // per-token beta (and -exp(A_log[h]) for the fused gate) of an item, one item ahead
+    auto stage_scalars = [&](int it) {
+      float* dst = s_beta + (it & 1) * (kRsMaxT + 2);
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      if (tid < T) dst[tid] = beta[((size_t)n * T + tid) * H + h];
+      if (kFused && tid == 32 && fz.A_log) dst[kRsMaxT] = -expf(fz.A_log[h]);
+    };
+    if (count > 0) stage_scalars(0);
+    sm100::named_barrier_sync(1, kDsCompute);
+    for (int it = 0; it < count; ++it) {
+      const int s = it % kRsStages;
+      const int item = first + it * stride, n = item / H;
+      const int slot_raw = state_indices ? state_indices[n] : n;
+      const bool ok = sm100::mbar_wait(full + s, (it / kRsStages) & 1);
+      if (!block_all(ok, 1, kDsCompute)) break;
+      if (it + 1 < count) stage_scalars(it + 1);  // read after this item's barriers
+      if (slot_raw < 0 || slot_raw >= P) {
+        if (slot_raw >= P && tid == 0) raise_status(kStatusBadSeqlens);
+        sm100::named_barrier_sync(1, kDsCompute);
+        if (tid == 0) sm100::mbar_arrive(computed + s);
+        continue;
+      }
+      uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+      const float* sb = s_beta + (it & 1) * (kRsMaxT + 2);
+      float4* Srow = reinterpret_cast<float4*>(st) + (col >> 2);
+      const int vstride = Dv >> 2;
+      float4 sreg[kDecRowsPerWarp];
+#pragma unroll
+      for (int i = 0; i < kDecRowsPerWarp; ++i) {
+        const int r = row0 + i;
+        sreg[i] = (col_ok && r < Dk) ? Srow[r * vstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const int rl = row0 + (lane & 15);
+      const float bias_r = (kFused && fz.A_log && lay.bias_bytes && rl < Dk)
+                               ? reinterpret_cast<const float*>(st + lay.bias_off)[rl]
+                               : 0.f;
+      for (int t = 0; t < T; ++t) {
+        const float* la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row);
+        const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row);
+        const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row);
+        const Tin* vv = reinterpret_cast<const Tin*>(st + lay.v_off + t * lay.v_row);
+        float la_mine = (rl < Dk) ? la[rl] : 0.f;
+        if (kFused && fz.A_log && rl < Dk) la_mine = sb[kRsMaxT] * softplus_f(la_mine + bias_r);
+        const float a_mine = (rl < Dk) ? expf(la_mine) : 1.f;
+        float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
+        float kq = 0.f, ssk = 0.f, ssq = 0.f;
+        float kr_[kDecRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kDecRowsPerWarp; ++i) {
+          const int r = row0 + i;
+          const float a = __shfl_sync(0xffffffffu, a_mine, i);
+          const float kr = (r < Dk) ? to_f32(kv[r]) : 0.f;
+          const float qr = (r < Dk) ? to_f32(qv[r]) : 0.f;
+          kr_[i] = kr;
+          kq += kr * qr;
+          if (kFused) {
+            ssk += kr * kr;
+            ssq += qr * qr;
+          }
+          sreg[i].x *= a; sreg[i].y *= a; sreg[i].z *= a; sreg[i].w *= a;
+          e.x += sreg[i].x * kr; e.y += sreg[i].y * kr; e.z += sreg[i].z * kr; e.w += sreg[i].w * kr;
+          p.x += sreg[i].x * qr; p.y += sreg[i].y * qr; p.z += sreg[i].z * qr; p.w += sreg[i].w * qr;
+        }
+        s_e[warp * 32 + lane] = e;
+        s_p[warp * 32 + lane] = p;
+        if (lane == 0) {
+          s_kq[warp] = kq;
+          if (kFused) {
+            s_ss[warp] = ssk;
+            s_ss[8 + warp] = ssq;
+          }
+        }
+        sm100::named_barrier_sync(1, kDsCompute);
+        e = make_float4(0.f, 0.f, 0.f, 0.f);
+        p = e;
+        kq = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const float4 ew = s_e[w * 32 + lane], pw = s_p[w * 32 + lane];
+          e.x += ew.x; e.y += ew.y; e.z += ew.z; e.w += ew.w;
+          p.x += pw.x; p.y += pw.y; p.z += pw.z; p.w += pw.w;
+          kq += s_kq[w];
+        }
+        float ik = 1.f;
+        if (kFused && fz.l2) {
+          float sk = 0.f, sq = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            sk += s_ss[w];
+            sq += s_ss[8 + w];
+          }
+          ik = rsqrtf(sk + fz.eps);
+          const float iq = rsqrtf(sq + fz.eps);
+          e.x *= ik; e.y *= ik; e.z *= ik; e.w *= ik;
+          p.x *= iq; p.y *= iq; p.z *= iq; p.w *= iq;
+          kq *= ik * iq;
+        }
+        const float b = sb[t];
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (col_ok) {
+          u.x = b * (to_f32(vv[col]) - e.x);
+          u.y = b * (to_f32(vv[col + 1]) - e.y);
+          u.z = b * (to_f32(vv[col + 2]) - e.z);
+          u.w = b * (to_f32(vv[col + 3]) - e.w);
+        }
+#pragma unroll
+        for (int i = 0; i < kDecRowsPerWarp; ++i) {
+          const float kn = kr_[i] * ik;
+          sreg[i].x += kn * u.x; sreg[i].y += kn * u.y; sreg[i].z += kn * u.z; sreg[i].w += kn * u.w;
+        }
+        if (warp == 0) {
+          float4 y = make_float4(p.x + kq * u.x, p.y + kq * u.y, p.z + kq * u.z, p.w + kq * u.w);
+          if (kFused && fz.onorm) {
+            float ss = col_ok ? y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w : 0.f;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
+            if (col_ok) {
+              float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+                                : make_float4(1.f, 1.f, 1.f, 1.f);
+              if (lay.og_row) {
+                const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off + t * lay.og_row) + col;
+                wv.x *= sigmoid_f(to_f32(gp[0]));
+                wv.y *= sigmoid_f(to_f32(gp[1]));
+                wv.z *= sigmoid_f(to_f32(gp[2]));
+                wv.w *= sigmoid_f(to_f32(gp[3]));
+              }
+              y = make_float4(y.x * inv * wv.x, y.y * inv * wv.y, y.z * inv * wv.z,
+                              y.w * inv * wv.w);
+            }
+          }
+          if (col_ok) {
+            Tin* op = o + (((size_t)n * T + t) * H + (item - n * H)) * Dv + col;
+            op[0] = from_f32<Tin>(y.x);
+            op[1] = from_f32<Tin>(y.y);
+            op[2] = from_f32<Tin>(y.z);
+            op[3] = from_f32<Tin>(y.w);
+          }
+        }
+        sm100::named_barrier_sync(1, kDsCompute);  // s_e / s_p are rewritten by the next token
+      }
+#pragma unroll
+      for (int i = 0; i < kDecRowsPerWarp; ++i) {
+        const int r = row0 + i;
+        if (col_ok && r < Dk) Srow[r * vstride] = sreg[i];
+      }
+      sm100::fence_proxy_async_smem();
+      sm100::named_barrier_sync(1, kDsCompute);
+      if (tid == 0) sm100::mbar_arrive(computed + s);
+    }
+  }
+  __syncthreads();
+}
+
+template <typename Tin, bool kFused>
+static cudaError_t launch_rs_typed(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, float* pool,
+                                   const int32_t* idx, void* o, int heads, int T, int H, int Dk,
+                                   int Dv, int P, const RsLayout& lay, int grid, size_t smem,
+                                   const Fusion& fz, cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(recurrent_stream_kernel<Tin, kFused>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  recurrent_stream_kernel<Tin, kFused><<<grid, kDsThreads, smem, stream>>>(
+      (const Tin*)q, (const Tin*)k, (const Tin*)v, log_alpha, beta, pool, idx, (Tin*)o, heads, T,
+      H, Dk, Dv, P, lay, fz);
+  return cudaGetLastError();
+}
+
 static int g_num_sms[64] = {0};
+
+static int num_sms_cached() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int nsm = (dev >= 0 && dev < 64) ? g_num_sms[dev] : 0;
+  if (nsm == 0) {
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) g_num_sms[dev] = nsm;
+  }
+  return nsm;
+}
+
+cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, kda_dtype_t dt,
+                                   const float* log_alpha, const float* beta, float* pool,
+                                   const int32_t* idx, void* o, int N, int T, int H, int Dk,
+                                   int Dv, int P, const Fusion& fz, cudaStream_t stream) {
+  const long long heads = (long long)N * H;
+  if (heads == 0 || T == 0) return cudaSuccess;
+  const int es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  const bool fused = fz.l2 || fz.A_log || fz.onorm;
+  const bool gate_rows = fz.onorm && fz.og, bias_row = fz.A_log && fz.dt_bias;
+  const RsLayout lay = make_rs_layout(T, Dk, Dv, es, gate_rows, bias_row);
+  const size_t smem = (size_t)kRsStages * lay.stage_bytes + 2 * 8 * 32 * sizeof(float4) +
+                      (24 + 2 * (kRsMaxT + 2)) * sizeof(float) +
+                      2 * kRsStages * sizeof(uint64_t) + 128;
+  const bool streamable = T <= kRsMaxT && (Dk * es) % 16 == 0 && (Dv * es) % 16 == 0 &&
+                          (Dk * 4) % 16 == 0 && al16(q) && al16(k) && al16(v) &&
+                          al16(log_alpha) && al16(pool) && (!gate_rows || al16(fz.og)) &&
+                          (!bias_row || al16(fz.dt_bias)) && smem <= 227u * 1024u &&
+                          heads <= INT32_MAX;
+  if (!streamable)
+    return launch_recurrent_blockwise(q, k, v, dt, log_alpha, beta, pool, idx, o, N, T, H, Dk,
+                                      Dv, P, fz, stream);
+  const int nsm = num_sms_cached();
+  if (nsm <= 0) return cudaErrorUnknown;
+  const int grid = (int)(heads < nsm ? heads : nsm);
+  ProfileScope prof(fused ? "recurrent_stream_fused" : "recurrent_stream", stream);
+  if (dt == KDA_DTYPE_BF16)
+    return fused ? launch_rs_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, pool, idx, o,
+                                                        (int)heads, T, H, Dk, Dv, P, lay, grid,
+                                                        smem, fz, stream)
+                 : launch_rs_typed<__nv_bfloat16, false>(q, k, v, log_alpha, beta, pool, idx, o,
+                                                         (int)heads, T, H, Dk, Dv, P, lay, grid,
+                                                         smem, fz, stream);
+  return fused ? launch_rs_typed<float, true>(q, k, v, log_alpha, beta, pool, idx, o, (int)heads,
+                                              T, H, Dk, Dv, P, lay, grid, smem, fz, stream)
+               : launch_rs_typed<float, false>(q, k, v, log_alpha, beta, pool, idx, o,
+                                               (int)heads, T, H, Dk, Dv, P, lay, grid, smem, fz,
+                                               stream);
+}
 
 template <typename Tin, bool kFused>
 static cudaError_t launch_stream_typed(const void* q, const void* k, const void* v,

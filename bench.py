@@ -557,11 +557,10 @@ def main():
     # roofline of the dominant kernel
     prof = pre["prof"]
     launches_per_step = sum(p["launches"] for p in prof) / args.steps
-    rec_bytes = pre["ws_bytes"]  # placeholder, replaced below by the per-record size
     n_chunks = chunk_count(spec)
     top = prof[0]
-    ws_records = pre["ws_bytes"] - 256
-    rec_bytes = ws_records // max(1, n_chunks * spec.H)
+    # bytes of one (chunk, head) record: the workspace past its 256-byte header, per record
+    rec_bytes = (pre["ws_bytes"] - 256) // max(1, n_chunks * spec.H)
     top_bytes = prefill_kernel_bytes(top["name"], spec, n_chunks, rec_bytes)
     top_ms = top["total_ms"] / top["launches"]
     achieved = top_bytes / (top_ms / 1e3) / 1e9 if top_bytes else None

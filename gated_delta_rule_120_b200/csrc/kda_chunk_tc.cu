@@ -722,6 +722,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   tc_fence_after();
 
   // ---- phase 5: W = M Kg, then U = M V, through TMEM [0, 128) -------------------------------
+  // the state kernel launched after this one may start its set-up now; it waits for this grid's
+  // completion before it reads any record
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   uint32_t phase = nwait & 1;
 #pragma unroll 1
   for (int which = 0; which < 2 && alive; ++which) {
@@ -852,6 +855,9 @@ __global__ void __launch_bounds__(kK2Threads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
+    // launched as a programmatic dependent of the chunk-local kernel: the records are complete
+    // and visible only after this wait (the set-up above overlapped that kernel's tail)
+    if (lane == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     // lane 0 copies the record; with the gated output epilogue the whole warp also copies the
     // chunk's gate rows (128 bytes of this CTA's columns per row)
     const bool gate_rows = kNorm && fz.og != nullptr;
@@ -1144,25 +1150,29 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  if (!norm) {
-    ProfileScope prof("chunk_state_tc", stream);
-    tc::chunk_state_tc_kernel<false><<<dim3(a.N, a.H, 2), tc::kK2Threads, sm2, stream>>>(
-        records, geo, a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o, a.fz);
-    return cudaGetLastError();
-  }
-  // the two column halves of a (sequence, head) form one cluster
+  // programmatic dependent launch: the state kernel's set-up (tensor memory, barriers, initial
+  // state) overlaps the chunk-local kernel's last wave; its producer waits for the records
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.N, a.H, 2);
   cfg.blockDim = dim3(tc::kK2Threads);
   cfg.dynamicSmemBytes = (size_t)sm2;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 2;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (!norm) {
+    ProfileScope prof("chunk_state_tc", stream);
+    return cudaLaunchKernelEx(&cfg, tc::chunk_state_tc_kernel<false>, (const uint8_t*)records, geo,
+                              (int)a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o, a.fz);
+  }
+  // the two column halves of a (sequence, head) form one cluster
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 2;
+  cfg.numAttrs = 2;
   ProfileScope prof("chunk_state_tc_norm", stream);
   return cudaLaunchKernelEx(&cfg, tc::chunk_state_tc_kernel<true>, (const uint8_t*)records, geo,
                             (int)a.H, a.initial_state, a.final_state, (__nv_bfloat16*)a.o, a.fz);

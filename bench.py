@@ -613,6 +613,24 @@ def main():
                         for p in lp["prof"]]}
         del lp
         torch.cuda.empty_cache()
+        # packed variable-length batch: 16 sequences, lengths log-uniform in [256, 32768]
+        vspec = kda_synth.varlen_spec(1003)
+        vsteps = max(2, args.steps // 5)
+        vp = run_prefill(vspec, [2003 + 10 * rank], dev, vsteps, 2, world)
+        vms = vp["ms"] / vsteps
+        vmin = roofline.prefill_min_bytes(vspec.token_heads(), vspec.num_seqs, vspec.H, vspec.Dk,
+                                          vspec.Dv, 2, False, True)
+        veq13 = sum(roofline.eq13_flops(n_tok, 64, 128) for n_tok in vspec.seqlens) * vspec.H
+        extra["varlen_prefill"] = {
+            "workload": vspec.name, "sequences": vspec.num_seqs,
+            "tokens": vspec.total_tokens, "longest": max(vspec.seqlens),
+            "tokens_per_s": world * vspec.total_tokens / (vms / 1e3),
+            "ms_per_call": vms, "frac_hbm_min_bytes": vmin / (vms / 1e3) / 1e9 / hbm_peak,
+            "eq13_tflops": veq13 / (vms / 1e3) / 1e12,
+            "kernels": [{"name": p["name"], "ms_per_launch": p["total_ms"] / p["launches"]}
+                        for p in vp["prof"]]}
+        del vp
+        torch.cuda.empty_cache()
     # the fused prologue on the standard workload
     fms = run_fused_prefill(spec, 2001 + 10 * rank, dev, args.steps, args.warmup, world)
     extra["fused_prologue_prefill"] = {

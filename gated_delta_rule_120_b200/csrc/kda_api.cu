@@ -14,7 +14,8 @@ inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 // Workspace layout of one prefill call:
 //   [0, 256)                 header: int32 `valid` flag written by the chunk-map kernel
-//   [256, 256 + off_bytes)   int32 chunk_off[N+1] (packed varlen batches only)
+//   [256, 256 + off_bytes)   int32 chunk_off[N+1], then int32 order[N] (the sequences longest
+//                            first), for packed varlen batches only
 //   [rec_base, ...)          per (chunk, head) records of the kernel path
 struct WsLayout {
   size_t chunk_off_base;
@@ -54,7 +55,7 @@ WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
   const long long tokens = (long long)B * T;
   w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
   w.chunk_off_base = 256;
-  const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * ((size_t)N + 1), 256) : 0;
+  const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * (2 * (size_t)N + 1), 256) : 0;
   w.rec_base = w.chunk_off_base + off_bytes;
   w.rec_bytes = is_tc_path(dt) ? TcRecordBytes
                                : SimtRecord::make(C, Dk, Dv).record_floats * sizeof(float);
@@ -189,7 +190,8 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtyp
   int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
   if (varlen) {
     st = from_cuda(
-        launch_chunk_map(cu_seqlens, N, (int)tokens, kBwdChunk, chunk_off, valid, stream));
+        launch_chunk_map(cu_seqlens, N, (int)tokens, kBwdChunk, chunk_off, valid, nullptr,
+                         stream));
     if (st != KDA_OK) return st;
   }
   SeqGeometry geo;
@@ -292,10 +294,12 @@ kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, kda_dty
   int32_t* valid = (int32_t*)ws;
   int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
   if (varlen) {
-    st = from_cuda(launch_chunk_map(cu_seqlens, N, (int)tokens, C, chunk_off, valid, stream));
+    st = from_cuda(launch_chunk_map(cu_seqlens, N, (int)tokens, C, chunk_off, valid,
+                                    chunk_off + N + 1, stream));
     if (st != KDA_OK) return st;
   }
   SeqGeometry geo;
+  if (varlen) geo.order = chunk_off + N + 1;
   geo.cu_seqlens = cu_seqlens;
   geo.chunk_off = chunk_off;
   geo.valid = valid;

@@ -31,10 +31,14 @@ constexpr int kSimtThreads = 256;
 // chunk map for packed variable-length batches: chunk_off[n] = sum_{m<n} ceil(len_m / C).
 // Validates cu_seqlens (cu[0] == 0, non-decreasing, cu[N] <= total) and records the verdict in
 // `valid`; the other kernels do nothing when it is 0 and the per-device status word is raised.
+// With `order` it also writes the sequences by decreasing chunk count (ties by index) for up to
+// blockDim.x sequences, the identity beyond that.
 // ----------------------------------------------------------------------------------------------
 __global__ void chunk_map_kernel(const int32_t* __restrict__ cu, int N, int total, int C,
-                                 int32_t* __restrict__ chunk_off, int32_t* __restrict__ valid) {
+                                 int32_t* __restrict__ chunk_off, int32_t* __restrict__ valid,
+                                 int32_t* __restrict__ order) {
   __shared__ int s_sum[1024];
+  __shared__ int s_cnt[1024];
   __shared__ int s_bad;
   const int tid = threadIdx.x, nt = blockDim.x;
   if (tid == 0) s_bad = (cu[0] != 0 || cu[N] > total) ? 1 : 0;
@@ -63,6 +67,24 @@ __global__ void chunk_map_kernel(const int32_t* __restrict__ cu, int N, int tota
     run += len > 0 ? (len + C - 1) / C : 0;
   }
   if (tid == nt - 1) chunk_off[N] = s_sum[nt - 1];
+  if (order) {
+    if (N <= nt) {  // rank = number of sequences ahead of this one
+      const int len = tid < N ? cu[tid + 1] - cu[tid] : 0;
+      const int cnt = len > 0 ? (len + C - 1) / C : 0;
+      s_cnt[tid] = cnt;
+      __syncthreads();
+      if (tid < N) {
+        int rank = 0;
+        for (int m = 0; m < N; ++m) {
+          const int cm = s_cnt[m];
+          rank += (cm > cnt || (cm == cnt && m < tid)) ? 1 : 0;
+        }
+        order[rank] = tid;
+      }
+    } else {
+      for (int n = tid; n < N; n += nt) order[n] = n;
+    }
+  }
   __syncthreads();
   if (tid == 0) {
     *valid = s_bad ? 0 : 1;
@@ -71,9 +93,9 @@ __global__ void chunk_map_kernel(const int32_t* __restrict__ cu, int N, int tota
 }
 
 cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
-                             int32_t* valid, cudaStream_t stream) {
+                             int32_t* valid, int32_t* order, cudaStream_t stream) {
   ProfileScope prof("chunk_map", stream);
-  chunk_map_kernel<<<1, 1024, 0, stream>>>(cu, N, total, C, chunk_off, valid);
+  chunk_map_kernel<<<1, 1024, 0, stream>>>(cu, N, total, C, chunk_off, valid, order);
   return cudaGetLastError();
 }
 

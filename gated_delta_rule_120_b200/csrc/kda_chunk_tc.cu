@@ -257,24 +257,22 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     gcp[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
   }
   cp_async_wait_all();
-  __syncthreads();
+  // the threads of the chunk's last rows hold g_C: fast mode iff every channel's is above -60
+  float gmin = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) gmin = fminf(gmin, g[3][j]);
+  const bool fast = __syncthreads_and(rg != 15 || gmin >= -kFastDecayLimit) != 0;
   float egc[8];
-  bool ok = true;
-  float gcv[8];
   {
     const float4* gcp = reinterpret_cast<const float4*>(sGC + cg * 8);
     const float4 a = gcp[0], b = gcp[1];
-    gcv[0] = a.x; gcv[1] = a.y; gcv[2] = a.z; gcv[3] = a.w;
-    gcv[4] = b.x; gcv[5] = b.y; gcv[6] = b.z; gcv[7] = b.w;
-  }
+    const float gcv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float gcj = gcv[j];
-    ok = ok && (gcj >= -kFastDecayLimit);
-    egc[j] = __expf(gcj);  // only scales a bf16 operand; the carried gamma_C uses expf
+    for (int j = 0; j < 8; ++j)
+      egc[j] = __expf(gcv[j]);  // only scales a bf16 operand; the carried gamma_C uses expf
   }
   int mode = kModeFast;
-  if (!__syncthreads_and(ok)) {
+  if (!fast) {
     bool blocks_ok = true;  // every channel's decay within every 16-row block
     if (tid < kD) {
       float prev = 0.f;
@@ -400,16 +398,13 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       tmem_ld32(tmem_at(tmem, sp * 32, half * 64 + part * 32), va);
       tmem_ld_wait();
       if (lane < 16) {
-        if (half == 0) {
+        if (half == 0) {  // the inverse reads only the strictly lower triangle: no mask
           const float br = sBeta[r];
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const int i = part * 32 + j4 * 4;
-            sts4(sA, r, i >> 2,
-                 make_float4(i < r ? br * va[4 * j4] : 0.f, i + 1 < r ? br * va[4 * j4 + 1] : 0.f,
-                             i + 2 < r ? br * va[4 * j4 + 2] : 0.f,
-                             i + 3 < r ? br * va[4 * j4 + 3] : 0.f));
-          }
+          for (int j4 = 0; j4 < 8; ++j4)
+            sts4(sA, r, part * 8 + j4,
+                 make_float4(br * va[4 * j4], br * va[4 * j4 + 1], br * va[4 * j4 + 2],
+                             br * va[4 * j4 + 3]));
         } else {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
@@ -500,16 +495,12 @@ __global__ void __launch_bounds__(kK1Threads, 3)
               for (int j = 0; j < 16; ++j) va[j] = 0.f;
             }
             if (lane < 16) {
-              if (half == 0) {
+              if (half == 0) {  // only the strictly lower triangle is read: no mask
 #pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
-                  const int i = 16 * u + 4 * j4;
-                  sts4(sA, r, i >> 2,
-                       make_float4(i < r ? br * va[4 * j4] : 0.f,
-                                   i + 1 < r ? br * va[4 * j4 + 1] : 0.f,
-                                   i + 2 < r ? br * va[4 * j4 + 2] : 0.f,
-                                   i + 3 < r ? br * va[4 * j4 + 3] : 0.f));
-                }
+                for (int j4 = 0; j4 < 4; ++j4)
+                  sts4(sA, r, 4 * u + j4,
+                       make_float4(br * va[4 * j4], br * va[4 * j4 + 1], br * va[4 * j4 + 2],
+                                   br * va[4 * j4 + 3]));
               } else {
 #pragma unroll
                 for (int c8 = 0; c8 < 2; ++c8) {
@@ -818,7 +809,10 @@ __global__ void __launch_bounds__(kK2Threads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM::Tmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM::Flags);
 
-  const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * 64;
+  // one CTA per (sequence, head, 64-column half), linear in that order with the sequence slowest:
+  // the longest sequences' chains are dispatched first
+  const int n = geo.seq_at_rank((int)(blockIdx.x / (2u * (unsigned)H)));
+  const int h = (int)((blockIdx.x >> 1) % (unsigned)H), j0 = (int)(blockIdx.x & 1u) * 64;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tb = geo.seq_begin(n), te = geo.seq_end(n);
   const int nchunks = te > tb ? ceil_div(te - tb, kC) : 0;
@@ -1150,10 +1144,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
+  if (2LL * a.N * a.H > INT32_MAX) return cudaErrorInvalidConfiguration;
   // programmatic dependent launch: the state kernel's set-up (tensor memory, barriers, initial
   // state) overlaps the chunk-local kernel's last wave; its producer waits for the records
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.N, a.H, 2);
+  cfg.gridDim = dim3(2u * (unsigned)a.N * (unsigned)a.H);
   cfg.blockDim = dim3(tc::kK2Threads);
   cfg.dynamicSmemBytes = (size_t)sm2;
   cfg.stream = stream;
@@ -1169,9 +1164,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
   }
   // the two column halves of a (sequence, head) form one cluster
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.x = 2;
   attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 2;
+  attr[1].val.clusterDim.z = 1;
   cfg.numAttrs = 2;
   ProfileScope prof("chunk_state_tc_norm", stream);
   return cudaLaunchKernelEx(&cfg, tc::chunk_state_tc_kernel<true>, (const uint8_t*)records, geo,

@@ -73,6 +73,9 @@ struct SeqGeometry {
   int32_t N;
   int32_t T;  // tokens per sequence when cu_seqlens == nullptr
   int32_t C;
+  // device [N], or nullptr: sequence indices by decreasing chunk count (packed varlen batches),
+  // so that kernels whose work per sequence is a serial chain start the longest chains first
+  const int32_t* order = nullptr;
 
   __device__ __forceinline__ bool ok() const { return cu_seqlens == nullptr || *valid != 0; }
 
@@ -88,6 +91,8 @@ struct SeqGeometry {
   __device__ __forceinline__ int first_chunk(int n) const {
     return cu_seqlens ? chunk_off[n] : n * ceil_div(T, C);
   }
+  // Sequence at position `i` of the longest-first order (the identity without one).
+  __device__ __forceinline__ int seq_at_rank(int i) const { return order ? order[i] : i; }
   // Sequence that owns global chunk `c` (c < num_chunks_total()).
   __device__ __forceinline__ int seq_of_chunk(int c) const {
     if (!cu_seqlens) return c / ceil_div(T, C);

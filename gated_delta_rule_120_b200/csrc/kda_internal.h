@@ -109,7 +109,7 @@ cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, 
                                    int Dv, int P, const Fusion& fz, cudaStream_t stream);
 
 cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
-                             int32_t* valid, cudaStream_t stream);
+                             int32_t* valid, int32_t* order, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
                                 float* records, const SimtRecord& rec, cudaStream_t stream);

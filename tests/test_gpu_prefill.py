@@ -139,6 +139,28 @@ def test_bf16_varlen_small(cuda_device):
     _check(spec, 51, cuda_device, TOL_BF16_O, TOL_BF16_S)
 
 
+@pytest.mark.parametrize("lens", [
+    (3, 300, 0, 130, 64, 1, 257, 64),  # the state kernel runs the sequences longest first
+    tuple([0, 300] + [(7 * i) % 41 for i in range(1098)]),  # past the ranked count: index order
+], ids=["ranked", "1100_sequences"])
+def test_bf16_varlen_initial_states_follow_their_sequences(cuda_device, lens):
+    """Every sequence starts from its own initial state and returns its own final state, whatever
+    order the state kernel visits the sequences in."""
+    H = 2 if len(lens) < 100 else 1
+    spec = PrefillSpec("t", B=1, T=sum(lens), H=H, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                       decay="fast", init_std=0.0, seqlens=lens)
+    inp = kda_synth.prefill_inputs(spec, 57, cuda_device)
+    g = torch.Generator(device=cuda_device).manual_seed(58)
+    inp["initial_state"] = torch.randn((len(lens), H, 128, 128), generator=g,
+                                       device=cuda_device) * 0.02
+    o, s = _run(inp, 64)
+    o_ref, s_ref = _oracle(inp, 1, spec.T)
+    assert rel_err(o, o_ref) <= TOL_BF16_O
+    assert rel_err(s, s_ref) <= TOL_BF16_S
+    empty = [n for n, L in enumerate(lens) if L == 0]
+    assert torch.equal(s[empty], inp["initial_state"][empty])
+
+
 def _sampled_heads_check(spec, seed, dev, heads, seqs=None):
     """Full-size run on the GPU; the oracle recomputes selected (sequence, head) pairs."""
     inp = kda_synth.prefill_inputs(spec, seed, dev)

@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kBwdThreads)
                            int Dk, int Dv, const Tin* __restrict__ d_o,
                            const float* __restrict__ d_final, float* __restrict__ d_initial,
                            float* __restrict__ dstates, float* __restrict__ dvp) {
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   const int C = geo.C;
   float* sdS = smem;                 // [Dk][32] cotangent of the state leaving the chunk
   float* sW = sdS + Dk * kBwSlice;   // [C][Dk]
@@ -86,10 +86,15 @@ __global__ void __launch_bounds__(kBwdThreads)
     const int L = min(C, te - t0);
     const float* r_ = ws + rec.record_floats * ((size_t)c * H + h);
     __syncthreads();  // the previous chunk is done with the staging buffers
-    for (int idx = tid; idx < C * Dk; idx += nt) {
-      sW[idx] = r_[rec.off_w + idx];
-      sKt[idx] = r_[rec.off_kt + idx];
-      sQt[idx] = r_[rec.off_qt + idx];
+    {  // record sections are 16-byte aligned (d_k multiple of 4, C multiple of 16)
+      const float4* w4 = reinterpret_cast<const float4*>(r_ + rec.off_w);
+      const float4* k4 = reinterpret_cast<const float4*>(r_ + rec.off_kt);
+      const float4* q4 = reinterpret_cast<const float4*>(r_ + rec.off_qt);
+      for (int idx = tid; idx < C * Dk / 4; idx += nt) {
+        reinterpret_cast<float4*>(sW)[idx] = w4[idx];
+        reinterpret_cast<float4*>(sKt)[idx] = k4[idx];
+        reinterpret_cast<float4*>(sQt)[idx] = q4[idx];
+      }
     }
     for (int idx = tid; idx < C * C; idx += nt) {
       const int r = idx / C, i = idx - r * C;
@@ -102,9 +107,11 @@ __global__ void __launch_bounds__(kBwdThreads)
     }
     {  // the cotangent entering from the right of this chunk, for the chunk-local pass
       float* dst = dstates + ((size_t)c * H + h) * Dk * Dv;
-      for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
-        const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
-        if (jj < NV) dst[(size_t)a * Dv + j0 + jj] = sdS[idx];
+      for (int idx = tid; idx < Dk * kBwSlice / 4; idx += nt) {
+        const int a = idx / (kBwSlice / 4), q = idx - a * (kBwSlice / 4);
+        if (4 * q < NV)
+          *reinterpret_cast<float4*>(dst + (size_t)a * Dv + j0 + 4 * q) =
+              reinterpret_cast<const float4*>(sdS)[idx];
       }
     }
     __syncthreads();

@@ -51,7 +51,7 @@ __device__ __forceinline__ void fma4(float s, float4 b, float4& acc) {
 // state pass: one CTA per (sequence, head, 32-column slice of d_v), chunks in reverse order
 // ----------------------------------------------------------------------------------------------
 template <typename Tin>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 2)
     chunk_state_bwd_kernel(const float* __restrict__ ws, SimtRecord rec, SeqGeometry geo, int H,
                            int Dk, int Dv, const Tin* __restrict__ d_o,
                            const float* __restrict__ d_final, float* __restrict__ d_initial,
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   if (!geo.ok()) return;
   const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kBwSlice;
   const int NV = min(kBwSlice, Dv - j0);
-  const int tid = threadIdx.x, nt = blockDim.x, j = tid & 31, rg = tid >> 5;
+  const int tid = threadIdx.x, nt = blockDim.x;
   const size_t sbase = ((size_t)n * H + h) * Dk * Dv;
 
   for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
@@ -115,69 +115,89 @@ __global__ void __launch_bounds__(kBwdThreads)
       }
     }
     __syncthreads();
-    // dV'[i][j] = sum_r P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j] (P[r][i] = 0 for r < i);
-    // this thread: rows i = rg + 8u, column j; float4 along r and a
+    // dV'[i][j] = sum_r P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j] (P[r][i] = 0 for r < i):
+    // 2 x 4 tiles (rows i0, i0 + 1; columns 4 jq .. 4 jq + 3), the d_k part split 64 / C ways
     {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int r = 0; r < C; r += 4) {
-        const float o0 = sdO[r * kBwSlice + j], o1 = sdO[(r + 1) * kBwSlice + j];
-        const float o2 = sdO[(r + 2) * kBwSlice + j], o3 = sdO[(r + 3) * kBwSlice + j];
+      const float4* Kt4 = reinterpret_cast<const float4*>(sKt);
+      const float4* S4 = reinterpret_cast<const float4*>(sdS);  // [Dk][8]
+      const float4* O4 = reinterpret_cast<const float4*>(sdO);  // [C][8]
+      const int dq = Dk >> 2, split = 64 / C;
+      const int ip = (tid >> 3) % (C >> 1), jq = tid & 7, sp = tid / (4 * C);
+      const int i0 = 2 * ip, i1 = i0 + 1;
+      const int kq = (dq + split - 1) / split, q0 = sp * kq, q1 = min(dq, q0 + kq);
+      float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+      for (int q = q0; q < q1; ++q) {
+        const float4 x0 = Kt4[i0 * dq + q], x1 = Kt4[i1 * dq + q];
+        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 p = ld4(sPt + (rg + 8 * u) * C + r);
-          acc[u] = fmaf(p.x, o0, fmaf(p.y, o1, fmaf(p.z, o2, fmaf(p.w, o3, acc[u]))));
+        for (int k = 0; k < 4; ++k) {
+          const float4 sv = S4[(4 * q + k) * 8 + jq];
+          fma4(xa[k], sv, acc[0]);
+          fma4(xb[k], sv, acc[1]);
         }
       }
-      for (int a = 0; a < Dk; a += 4) {
-        const float s0 = sdS[a * kBwSlice + j], s1 = sdS[(a + 1) * kBwSlice + j];
-        const float s2 = sdS[(a + 2) * kBwSlice + j], s3 = sdS[(a + 3) * kBwSlice + j];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 kt = ld4(sKt + (rg + 8 * u) * Dk + a);
-          acc[u] = fmaf(kt.x, s0, fmaf(kt.y, s1, fmaf(kt.z, s2, fmaf(kt.w, s3, acc[u]))));
+      if (sp == 0) {  // the A_qk part (contraction over the chunk rows r >= i)
+        for (int r = i0; r < C; ++r) {
+          const float4 ov = O4[r * 8 + jq];
+          fma4(sPt[i0 * C + r], ov, acc[0]);
+          if (r >= i1) fma4(sPt[i1 * C + r], ov, acc[1]);
         }
       }
+      float4* sRed = reinterpret_cast<float4*>(sdV + C * kBwSlice);  // [split][C][8]
+      if (split > 1) {
+        sRed[(sp * C + i0) * 8 + jq] = acc[0];
+        sRed[(sp * C + i1) * 8 + jq] = acc[1];
+        __syncthreads();
+        if (sp == 0)
+          for (int s2 = 1; s2 < split; ++s2)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = rg + 8 * u;
-        sdV[i * kBwSlice + j] = acc[u];
-        if (i < L && j < NV) dvp[((size_t)(t0 + i) * H + h) * Dv + j0 + j] = acc[u];
+            for (int u = 0; u < 2; ++u) {
+              const float4 p = sRed[(s2 * C + i0 + u) * 8 + jq];
+              acc[u].x += p.x; acc[u].y += p.y; acc[u].z += p.z; acc[u].w += p.w;
+            }
+      }
+      if (sp == 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = i0 + u;
+          const float4 val = acc[u];
+          reinterpret_cast<float4*>(sdV)[i * 8 + jq] = val;
+          if (i < L && 4 * jq < NV)
+            *reinterpret_cast<float4*>(dvp + ((size_t)(t0 + i) * H + h) * Dv + j0 + 4 * jq) = val;
+        }
       }
     }
     __syncthreads();
-    // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV'; this thread: rows a in the groups of four
-    // {4 (rg + 8 u) .. + 3}, column j (each thread rewrites only its own elements)
-    for (int g0 = 4 * rg; g0 < Dk; g0 += 4 * 8 * 4) {
-      float4 acc[4];
+    // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV': 4 x 4 tiles (rows 4 aq .. 4 aq + 3), each
+    // thread rewrites only its own tile
+    {
+      const float4* Q4 = reinterpret_cast<const float4*>(sQt);
+      const float4* W4 = reinterpret_cast<const float4*>(sW);
+      const float4* O4 = reinterpret_cast<const float4*>(sdO);
+      const float4* V4 = reinterpret_cast<const float4*>(sdV);
+      float4* S4 = reinterpret_cast<float4*>(sdS);
+      const int dq = Dk >> 2;
+      for (int t = tid; t < dq * 8; t += nt) {
+        const int aq = t >> 3, jq = t & 7;
+        float4 acc[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int a = g0 + 32 * u;
-        acc[u] = a < Dk ? make_float4(sGam[a] * sdS[a * kBwSlice + j],
-                                      sGam[a + 1] * sdS[(a + 1) * kBwSlice + j],
-                                      sGam[a + 2] * sdS[(a + 2) * kBwSlice + j],
-                                      sGam[a + 3] * sdS[(a + 3) * kBwSlice + j])
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      for (int r = 0; r < C; ++r) {
-        const float o = sdO[r * kBwSlice + j], dvv = -sdV[r * kBwSlice + j];
+        for (int e = 0; e < 4; ++e) {
+          const float g = sGam[4 * aq + e];
+          const float4 sv = S4[(4 * aq + e) * 8 + jq];
+          acc[e] = make_float4(g * sv.x, g * sv.y, g * sv.z, g * sv.w);
+        }
+        for (int r = 0; r < C; ++r) {
+          const float4 qv = Q4[r * dq + aq], wv = W4[r * dq + aq];
+          const float4 ov = O4[r * 8 + jq], dv = V4[r * 8 + jq];
+          const float qx[4] = {qv.x, qv.y, qv.z, qv.w}, wx[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int a = g0 + 32 * u;
-          if (a < Dk) {
-            fma4(o, ld4(sQt + r * Dk + a), acc[u]);
-            fma4(dvv, ld4(sW + r * Dk + a), acc[u]);
+          for (int e = 0; e < 4; ++e) {
+            fma4(qx[e], ov, acc[e]);
+            fma4(-wx[e], dv, acc[e]);
           }
         }
-      }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int a = g0 + 32 * u;
-        if (a < Dk) {
-          sdS[a * kBwSlice + j] = acc[u].x;
-          sdS[(a + 1) * kBwSlice + j] = acc[u].y;
-          sdS[(a + 2) * kBwSlice + j] = acc[u].z;
-          sdS[(a + 3) * kBwSlice + j] = acc[u].w;
-        }
+        for (int e = 0; e < 4; ++e) S4[(4 * aq + e) * 8 + jq] = acc[e];
       }
     }
   }
@@ -613,8 +633,9 @@ __global__ void __launch_bounds__(kBwdThreads)
 }
 
 size_t bwd_state_smem_bytes(int C, int Dk) {
+  // + the split-contraction partial sums of dV' ([64 / C][C][32])
   return sizeof(float) * ((size_t)Dk * kBwSlice + 3 * (size_t)C * Dk + (size_t)C * C + Dk +
-                          2 * (size_t)C * kBwSlice);
+                          2 * (size_t)C * kBwSlice + 64 * (size_t)kBwSlice);
 }
 size_t bwd_local_smem_bytes(int Dk, int Dv) {
   return sizeof(float) * (size_t)BwdSmem::make(Dk, Dv).total;

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kSimtThreads)
                             const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                             const float* __restrict__ beta, SeqGeometry geo, int H, int Dk, int Dv,
                             float* __restrict__ ws, SimtRecord rec, Fusion fz) {
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   const int C = geo.C;
   float* sk = smem;            // [C][Dk]  k, later Gamma.K
   float* sq = sk + C * Dk;     // [C][Dk]
@@ -186,7 +186,9 @@ __global__ void __launch_bounds__(kSimtThreads)
     const int i = p - r * (r + 1) / 2;
     float akk = 0.f, aqk = 0.f;
     for (int cc = lane; cc < Dk; cc += 32) {
-      const float f = expf(sg[r * Dk + cc] - sg[i * Dk + cc]);  // gamma_r / gamma_i <= 1
+      // gamma_r / gamma_i <= 1; the fast exponential's relative error (a few 1e-7 plus the
+      // argument's rounding, < 1e-5 for any argument above -87) is far below fp32 parity needs
+      const float f = __expf(sg[r * Dk + cc] - sg[i * Dk + cc]);
       const float ki = sk[i * Dk + cc] * f;
       akk += sk[r * Dk + cc] * ki;
       aqk += sq[r * Dk + cc] * ki;
@@ -212,18 +214,23 @@ __global__ void __launch_bounds__(kSimtThreads)
   }
   __syncthreads();
 
-  // (I + A)^{-1} by forward substitution: row r = e_r - sum_{j<r} A[r][j] row j
-  for (int r = 0; r < C; ++r) {
-    for (int cc = tid; cc < C; cc += nt) {
-      float val = 0.f;
-      if (cc <= r) {
-        val = (cc == r) ? 1.f : 0.f;
-        for (int j = cc; j < r; ++j) val -= sA[r * C + j] * sT[j * C + cc];
+  // (I + A)^{-1} by forward substitution, one lane per column of the inverse (warps 0 and 1
+  // for C = 64), the column held in registers: T[r][cc] = [r == cc] - sum_{cc<=j<r} A[r][j] T[j][cc]
+  if (tid < C) {
+    const int cc = tid;
+    float col[64];
+#pragma unroll
+    for (int r = 0; r < 64; ++r) {
+      if (r < C) {
+        float val = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < r; ++jj) val -= sA[r * C + jj] * col[jj];  // col[j] = 0 for j < cc
+        col[r] = r >= cc ? val : 0.f;
+        sT[r * C + cc] = col[r];
       }
-      sT[r * C + cc] = val;
     }
-    __syncthreads();
   }
+  __syncthreads();
   // M = (I + A)^{-1} Diag(beta)  (the backward pass keeps (I + A)^{-1} itself)
   for (int idx = tid; idx < C * C; idx += nt) {
     if (rec.off_t != SimtRecord::kNone) out[rec.off_t + idx] = sT[idx];
@@ -236,14 +243,38 @@ __global__ void __launch_bounds__(kSimtThreads)
     const int cc = idx % Dk;
     const float g = sg[idx];
     const float kk = sk[idx];
-    out[rec.off_kt + idx] = kk * expf(gC[cc] - g);
-    out[rec.off_qt + idx] = sq[idx] * expf(g);
-    sk[idx] = kk * expf(g);
+    const float eg = __expf(g);  // operand scales (arguments <= 0); the carried gamma_C uses expf
+    out[rec.off_kt + idx] = kk * __expf(gC[cc] - g);
+    out[rec.off_qt + idx] = sq[idx] * eg;
+    sk[idx] = kk * eg;
   }
   for (int cc = tid; cc < Dk; cc += nt) out[rec.off_gam + cc] = expf(gC[cc]);
   __syncthreads();
 
   // W = M (Gamma.K), U = M V
+  if ((Dk & 3) == 0 && (Dv & 3) == 0) {  // 2 x 4 register tiles, float4 rows and record stores
+    const int dq = Dk >> 2, vq = Dv >> 2;
+    const float4* k4 = reinterpret_cast<const float4*>(sk);
+    const float4* v4 = reinterpret_cast<const float4*>(sv);
+    for (int t = tid; t < (C >> 1) * (dq + vq); t += nt) {
+      const int rp = t / (dq + vq), cq = t - rp * (dq + vq);
+      const int r0 = 2 * rp, r1 = r0 + 1;
+      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+      for (int i = 0; i <= r1; ++i) {  // M is lower triangular: M[r0][r1] = 0
+        const float m0 = sT[r0 * C + i], m1 = sT[r1 * C + i];
+        const float4 x = cq < dq ? k4[i * dq + cq] : v4[i * vq + (cq - dq)];
+        a0.x = fmaf(m0, x.x, a0.x); a0.y = fmaf(m0, x.y, a0.y);
+        a0.z = fmaf(m0, x.z, a0.z); a0.w = fmaf(m0, x.w, a0.w);
+        a1.x = fmaf(m1, x.x, a1.x); a1.y = fmaf(m1, x.y, a1.y);
+        a1.z = fmaf(m1, x.z, a1.z); a1.w = fmaf(m1, x.w, a1.w);
+      }
+      float* dst = cq < dq ? out + rec.off_w + 4 * cq : out + rec.off_u + 4 * (cq - dq);
+      const int ld = cq < dq ? Dk : Dv;
+      *reinterpret_cast<float4*>(dst + r0 * ld) = a0;
+      *reinterpret_cast<float4*>(dst + r1 * ld) = a1;
+    }
+    return;
+  }
   const int wu = Dk + Dv;
   for (int idx = tid; idx < C * wu; idx += nt) {
     const int r = idx / wu, cc = idx - r * wu;

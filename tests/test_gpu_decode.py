@@ -70,6 +70,35 @@ def test_decode_full_size_sampled(cuda_device):
     assert torch.isfinite(state).all()
 
 
+def test_decode_all_steps_sampled(cuda_device):
+    """The decode workload end to end: 256 sequences x 32 heads, all of its 1024 steps on the
+    same in-place states. Inputs are drawn 64 steps at a time (step s from its own seed, as in
+    one 1024-step draw); 16 sampled sequences (all heads) follow in the oracle, o compared at
+    every step and the states after the last one."""
+    spec = kda_synth.DECODE
+    block = 64
+    state = kda_synth.decode_state(spec, 2005, cuda_device)
+    pick = np.sort(np.random.default_rng(1).choice(spec.N, 16, replace=False))
+    S_ref = to_np(state[pick])
+    worst_o = 0.0
+    for b in range(spec.steps // block):
+        steps = kda_synth.decode_step_inputs(spec, 2005 + block * b, block, cuda_device)
+        outs = []
+        for s in range(block):
+            o = kda.kda_recurrent_step(steps["q"][s], steps["k"][s], steps["v"][s],
+                                       steps["log_alpha"][s], steps["beta"][s], state)
+            outs.append(o[pick].cpu())
+        torch.cuda.synchronize()
+        host = {k: v[:, pick].cpu() for k, v in steps.items()}
+        o_ref, S_ref = _oracle_steps(S_ref, host, block)
+        worst_o = max(worst_o, rel_err(torch.stack(outs), o_ref))
+        del steps
+    assert kda.kda_last_device_error() == kda.KDA_OK
+    assert worst_o <= TOL_DECODE_O, worst_o
+    assert rel_err(state[pick], S_ref) <= TOL_DECODE_S
+    assert torch.isfinite(state).all()
+
+
 def test_decode_is_deterministic(cuda_device):
     spec = kda_synth.DecodeSpec("t", N=64, H=8, Dk=128, Dv=128, steps=1, dtype="bf16",
                                 decay="slow", init_std=0.02)

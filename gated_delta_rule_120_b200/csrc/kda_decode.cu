@@ -885,6 +885,311 @@ __global__ void __launch_bounds__(kDsThreads, 1)
   __syncthreads();
 }
 
+// ---------------------------------------------------------------------------------------------
+// Column-layout variant of the streaming recurrent mode (d_k = d_v = 128, T tokens that fit the
+// shared-memory budget): the same producer warp and two-stage ring, eight compute warps, each
+// owning 16 columns of the state over all 128 rows: lane = (row group rg of 16 rows, column quad
+// cq), so a thread holds a 16 x 4 tile in registers. A token's reductions
+// e_j = sum_i S'[i][j] k_i and p_j = sum_i S'[i][j] q_i then end in three lane exchanges inside
+// the warp instead of a block-wide reduction, so the token loop has no barrier. The per-token decays exp(log alpha),
+// k.q, the norms and beta are computed for all T tokens of an item in one pass before it, and
+// the outputs (with the head-wise norm and gate when fused) are written by one pass after it.
+// ---------------------------------------------------------------------------------------------
+constexpr int kRcCompute = 256;                // 8 compute warps
+constexpr int kRcThreads = kRcCompute + 32;    // + producer warp
+constexpr int kRcD = 128;
+
+__device__ __forceinline__ void load8_f32(const float* p, float (&x)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void load8_in(const float* p, float (&x)[8]) { load8_f32(p, x); }
+__device__ __forceinline__ void load8_in(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+template <typename Tin, bool kFused>
+__global__ void __launch_bounds__(kRcThreads, 1)
+    recurrent_cols_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                          const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                          const float* __restrict__ beta, float* __restrict__ pool,
+                          const int32_t* __restrict__ state_indices, Tin* __restrict__ o, int NH,
+                          int T, int H, int P, RsLayout lay, Fusion fz) {
+  constexpr int D = kRcD;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((128 - (sm100::smem_u32(smem_raw) & 127)) & 127);
+  uint8_t* stages = sm;
+  float* s_alpha = reinterpret_cast<float*>(sm + kRsStages * lay.stage_bytes);  // [kRsMaxT][D]
+  float* s_y = s_alpha + kRsMaxT * D;                                           // [kRsMaxT][D]
+  float4* s_tok = reinterpret_cast<float4*>(s_y + kRsMaxT * D);  // [kRsMaxT]: kq, 1/|k|, 1/|q|, beta
+  float* s_beta = reinterpret_cast<float*>(s_tok + kRsMaxT);     // [2][kRsMaxT + 2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_beta + 2 * (kRsMaxT + 2));  // [kRsStages]
+  uint64_t* computed = full + kRsStages;                                     // [kRsStages]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int first = blockIdx.x, stride = gridDim.x;
+  const int count = first < NH ? (NH - first + stride - 1) / stride : 0;
+  const uint32_t es = sizeof(Tin);
+  auto slot_of = [&](int it) -> int {
+    const int item = first + it * stride, n = item / H;
+    const int sl = state_indices ? state_indices[n] : n;
+    return (sl >= 0 && sl < P) ? sl : -1;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kRsStages; ++i) {
+      sm100::mbar_init(full + i, 1);
+      sm100::mbar_init(computed + i, 1);
+    }
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kRcCompute / 32) {
+    // ---------------------------------------------------------------- producer warp
+    auto issue_load = [&](int it, int slot) {
+      const int s = it % kRsStages;
+      if (slot < 0) {
+        if (lane == 0) sm100::mbar_arrive(full + s);
+        return;
+      }
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+      if (lane == 0) {
+        sm100::mbar_arrive_expect_tx(full + s, lay.state_bytes + lay.vec_tx);
+        sm100::bulk_g2s(st, pool + ((size_t)slot * H + h) * D * D, lay.state_bytes, full + s);
+        if (kFused && lay.bias_bytes)
+          sm100::bulk_g2s(st + lay.bias_off, fz.dt_bias + (size_t)h * D, lay.bias_bytes, full + s);
+      }
+      for (int t = lane; t < T; t += 32) {
+        const size_t base = ((size_t)n * T + t) * H + h;
+        sm100::bulk_g2s(st + lay.la_off + t * lay.la_row, log_alpha + base * D, D * 4, full + s);
+        sm100::bulk_g2s(st + lay.q_off + t * lay.qk_row, q + base * D, D * es, full + s);
+        sm100::bulk_g2s(st + lay.k_off + t * lay.qk_row, k + base * D, D * es, full + s);
+        sm100::bulk_g2s(st + lay.v_off + t * lay.v_row, v + base * D, D * es, full + s);
+        if (kFused && lay.og_row)
+          sm100::bulk_g2s(st + lay.og_off + t * lay.og_row,
+                          reinterpret_cast<const Tin*>(fz.og) + base * D, D * es, full + s);
+      }
+    };
+    int slot_cur[kRsStages];
+    for (int it = 0; it < count && it < kRsStages; ++it) {
+      slot_cur[it] = slot_of(it);
+      issue_load(it, slot_cur[it]);
+    }
+    for (int it = 0; it < count; ++it) {
+      const int s = it % kRsStages;
+      bool ok = sm100::mbar_wait(computed + s, (it / kRsStages) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (lane == 0 && slot_cur[s] >= 0) {
+        const int item = first + it * stride, h = item % H;
+        sm100::bulk_s2g(pool + ((size_t)slot_cur[s] * H + h) * D * D,
+                        stages + (size_t)s * lay.stage_bytes, lay.state_bytes);
+        sm100::bulk_commit();
+      }
+      if (it + kRsStages < count) {
+        if (lane == 0) sm100::bulk_wait_read_all();  // the stage is free once its store read it
+        __syncwarp();
+        slot_cur[s] = slot_of(it + kRsStages);
+        issue_load(it + kRsStages, slot_cur[s]);
+      }
+    }
+    if (lane == 0) {
+      sm100::bulk_wait_all();
+      for (int it = 0; it < count && it < kRsStages; ++it) {
+        const int last = count - 1 - it;
+        if (last >= 0)
+          sm100::mbar_wait(full + last % kRsStages, (last / kRsStages) & 1, 100000000ull);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    const int rg = lane >> 2, cq = lane & 3;
+    const int r0 = 16 * rg, c0 = 16 * warp + 4 * cq;  // rows r0 .. r0 + 15, columns c0 .. c0 + 3
+    auto stage_scalars = [&](int it) {  // beta (and -exp(A_log[h])) of an item, one item ahead
+      float* dst = s_beta + (it & 1) * (kRsMaxT + 2);
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      if (tid < T) dst[tid] = beta[((size_t)n * T + tid) * H + h];
+      if (kFused && tid == 32 && fz.A_log) dst[kRsMaxT] = -expf(fz.A_log[h]);
+    };
+    if (count > 0) stage_scalars(0);
+    sm100::named_barrier_sync(1, kRcCompute);
+    for (int it = 0; it < count; ++it) {
+      const int s = it % kRsStages;
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      const int slot_raw = state_indices ? state_indices[n] : n;
+      const bool ok = sm100::mbar_wait(full + s, (it / kRsStages) & 1);
+      if (!block_all(ok, 1, kRcCompute)) break;
+      const float* sb = s_beta + (it & 1) * (kRsMaxT + 2);
+      if (slot_raw < 0 || slot_raw >= P) {
+        if (slot_raw >= P && tid == 0) raise_status(kStatusBadSeqlens);
+        if (it + 1 < count) stage_scalars(it + 1);
+        sm100::named_barrier_sync(1, kRcCompute);
+        if (tid == 0) sm100::mbar_arrive(computed + s);
+        continue;
+      }
+      uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+      // pre-pass: every token's decays; k.q, inverse norms and beta per token (one warp each)
+      for (int e = tid; e < T * D; e += kRcCompute) {
+        const int t = e >> 7, i = e & (D - 1);
+        float la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row)[i];
+        if (kFused && fz.A_log) {
+          const float bias = lay.bias_bytes ? reinterpret_cast<const float*>(st + lay.bias_off)[i]
+                                            : 0.f;
+          la = sb[kRsMaxT] * softplus_f(la + bias);
+        }
+        s_alpha[e] = expf(la);
+      }
+      for (int t = warp; t < T; t += kRcCompute / 32) {
+        float kx[4], qx[4];
+        const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + 4 * lane;
+        const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + 4 * lane;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          kx[c] = to_f32(kv[c]);
+          qx[c] = to_f32(qv[c]);
+        }
+        float kq = 0.f, ssk = 0.f, ssq = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          kq = fmaf(kx[c], qx[c], kq);
+          ssk = fmaf(kx[c], kx[c], ssk);
+          ssq = fmaf(qx[c], qx[c], ssq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          kq += __shfl_xor_sync(0xffffffffu, kq, off);
+          ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+          ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+        }
+        if (lane == 0) {
+          float ik = 1.f, iq = 1.f;
+          if (kFused && fz.l2) {
+            ik = rsqrtf(ssk + fz.eps);
+            iq = rsqrtf(ssq + fz.eps);
+          }
+          s_tok[t] = make_float4(kq * ik * iq, ik, iq, sb[t]);
+        }
+      }
+      if (it + 1 < count) stage_scalars(it + 1);  // the other buffer; read after this barrier
+      sm100::named_barrier_sync(1, kRcCompute);
+
+      float4 S[16];
+      float* Sst = reinterpret_cast<float*>(st);
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) S[ii] = *reinterpret_cast<const float4*>(Sst + (r0 + ii) * D + c0);
+      for (int t = 0; t < T; ++t) {
+        const float* al = s_alpha + t * D + r0;
+        const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + r0;
+        const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + r0;
+        float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
+#pragma unroll
+        for (int i8 = 0; i8 < 2; ++i8) {  // S' = Diag(alpha) S; e, p over this thread's rows
+          float a[8], kk[8], qv8[8];
+          load8_f32(al + 8 * i8, a);
+          load8_in(kv + 8 * i8, kk);
+          load8_in(qv + 8 * i8, qv8);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4& sv = S[8 * i8 + u];
+            sv.x *= a[u]; sv.y *= a[u]; sv.z *= a[u]; sv.w *= a[u];
+            e.x = fmaf(sv.x, kk[u], e.x); e.y = fmaf(sv.y, kk[u], e.y);
+            e.z = fmaf(sv.z, kk[u], e.z); e.w = fmaf(sv.w, kk[u], e.w);
+            p.x = fmaf(sv.x, qv8[u], p.x); p.y = fmaf(sv.y, qv8[u], p.y);
+            p.z = fmaf(sv.z, qv8[u], p.z); p.w = fmaf(sv.w, qv8[u], p.w);
+          }
+        }
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {  // over the eight row groups of the warp
+          e.x += __shfl_xor_sync(0xffffffffu, e.x, off);
+          e.y += __shfl_xor_sync(0xffffffffu, e.y, off);
+          e.z += __shfl_xor_sync(0xffffffffu, e.z, off);
+          e.w += __shfl_xor_sync(0xffffffffu, e.w, off);
+          p.x += __shfl_xor_sync(0xffffffffu, p.x, off);
+          p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+          p.z += __shfl_xor_sync(0xffffffffu, p.z, off);
+          p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+        }
+        const float4 tk = s_tok[t];  // k.q (normalised), 1/|k|, 1/|q|, beta
+        const Tin* vv = reinterpret_cast<const Tin*>(st + lay.v_off + t * lay.v_row) + c0;
+        const float4 u = make_float4(tk.w * (to_f32(vv[0]) - e.x * tk.y),
+                                     tk.w * (to_f32(vv[1]) - e.y * tk.y),
+                                     tk.w * (to_f32(vv[2]) - e.z * tk.y),
+                                     tk.w * (to_f32(vv[3]) - e.w * tk.y));
+        if (rg == 0)  // o_t = S'^T q + (k.q) beta (v - e)
+          *reinterpret_cast<float4*>(s_y + t * D + c0) =
+              make_float4(p.x * tk.z + tk.x * u.x, p.y * tk.z + tk.x * u.y,
+                          p.z * tk.z + tk.x * u.z, p.w * tk.z + tk.x * u.w);
+        const float4 ku = make_float4(tk.y * u.x, tk.y * u.y, tk.y * u.z, tk.y * u.w);
+#pragma unroll
+        for (int i8 = 0; i8 < 2; ++i8) {  // S = S' + k (beta (v - e))^T
+          float kk[8];
+          load8_in(kv + 8 * i8, kk);
+#pragma unroll
+          for (int u8 = 0; u8 < 8; ++u8) {
+            float4& sv = S[8 * i8 + u8];
+            sv.x = fmaf(kk[u8], ku.x, sv.x); sv.y = fmaf(kk[u8], ku.y, sv.y);
+            sv.z = fmaf(kk[u8], ku.z, sv.z); sv.w = fmaf(kk[u8], ku.w, sv.w);
+          }
+        }
+      }
+#pragma unroll
+      for (int ii = 0; ii < 16; ++ii) *reinterpret_cast<float4*>(Sst + (r0 + ii) * D + c0) = S[ii];
+      sm100::named_barrier_sync(1, kRcCompute);  // s_y complete
+      // outputs: one warp per token row, four columns per lane (head-wise norm x gate if fused)
+      for (int t = warp; t < T; t += kRcCompute / 32) {
+        float4 y = reinterpret_cast<const float4*>(s_y + t * D)[lane];
+        if (kFused && fz.onorm) {
+          float ss = y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float inv = rsqrtf(ss * (1.f / D) + fz.oeps);
+          float4 wv = fz.ow ? reinterpret_cast<const float4*>(fz.ow)[lane]
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+          if (lay.og_row) {
+            const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off + t * lay.og_row) + 4 * lane;
+            wv.x *= sigmoid_f(to_f32(gp[0]));
+            wv.y *= sigmoid_f(to_f32(gp[1]));
+            wv.z *= sigmoid_f(to_f32(gp[2]));
+            wv.w *= sigmoid_f(to_f32(gp[3]));
+          }
+          y = make_float4(y.x * inv * wv.x, y.y * inv * wv.y, y.z * inv * wv.z, y.w * inv * wv.w);
+        }
+        Tin* op = o + (((size_t)n * T + t) * H + h) * D + 4 * lane;
+        op[0] = from_f32<Tin>(y.x);
+        op[1] = from_f32<Tin>(y.y);
+        op[2] = from_f32<Tin>(y.z);
+        op[3] = from_f32<Tin>(y.w);
+      }
+      sm100::fence_proxy_async_smem();
+      sm100::named_barrier_sync(1, kRcCompute);
+      if (tid == 0) sm100::mbar_arrive(computed + s);
+    }
+  }
+  __syncthreads();
+}
+
+template <typename Tin, bool kFused>
+static cudaError_t launch_rc_typed(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, float* pool,
+                                   const int32_t* idx, void* o, int heads, int T, int H, int P,
+                                   const RsLayout& lay, int grid, size_t smem, const Fusion& fz,
+                                   cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(recurrent_cols_kernel<Tin, kFused>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  recurrent_cols_kernel<Tin, kFused><<<grid, kRcThreads, smem, stream>>>(
+      (const Tin*)q, (const Tin*)k, (const Tin*)v, log_alpha, beta, pool, idx, (Tin*)o, heads, T,
+      H, P, lay, fz);
+  return cudaGetLastError();
+}
+
 template <typename Tin, bool kFused>
 static cudaError_t launch_rs_typed(const void* q, const void* k, const void* v,
                                    const float* log_alpha, const float* beta, float* pool,
@@ -938,6 +1243,27 @@ cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, 
   const int nsm = num_sms_cached();
   if (nsm <= 0) return cudaErrorUnknown;
   const int grid = (int)(heads < nsm ? heads : nsm);
+  // d = 128: the column layout, when its per-item buffers fit beside the two stages
+  const size_t smem_cols = (size_t)kRsStages * lay.stage_bytes +
+                           2 * (size_t)kRsMaxT * kRcD * sizeof(float) + kRsMaxT * sizeof(float4) +
+                           2 * (kRsMaxT + 2) * sizeof(float) + 2 * kRsStages * sizeof(uint64_t) +
+                           128;
+  if (Dk == kRcD && Dv == kRcD && (!fz.ow || al16(fz.ow)) && smem_cols <= 227u * 1024u) {
+    ProfileScope prof(fused ? "recurrent_cols_fused" : "recurrent_cols", stream);
+    if (dt == KDA_DTYPE_BF16)
+      return fused ? launch_rc_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, pool, idx, o,
+                                                          (int)heads, T, H, P, lay, grid,
+                                                          smem_cols, fz, stream)
+                   : launch_rc_typed<__nv_bfloat16, false>(q, k, v, log_alpha, beta, pool, idx,
+                                                           o, (int)heads, T, H, P, lay, grid,
+                                                           smem_cols, fz, stream);
+    return fused ? launch_rc_typed<float, true>(q, k, v, log_alpha, beta, pool, idx, o,
+                                                (int)heads, T, H, P, lay, grid, smem_cols, fz,
+                                                stream)
+                 : launch_rc_typed<float, false>(q, k, v, log_alpha, beta, pool, idx, o,
+                                                 (int)heads, T, H, P, lay, grid, smem_cols, fz,
+                                                 stream);
+  }
   ProfileScope prof(fused ? "recurrent_stream_fused" : "recurrent_stream", stream);
   if (dt == KDA_DTYPE_BF16)
     return fused ? launch_rs_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, pool, idx, o,

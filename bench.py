@@ -209,14 +209,27 @@ def prefill_kernel_bytes(name, spec, max_chunks, rec_bytes):
     return None
 
 
-def library_source_hash() -> str:
-    """sha256 over the paths and contents of the files libkda.so is built from."""
+# The files each captured kernel is compiled from: its own source and the headers that source
+# includes (the library is one translation unit, but a kernel's code depends only on these).
+KERNEL_SOURCES = {
+    "chunk_local_tc": ["csrc/kda_chunk_tc.cu", "csrc/kda_common.cuh", "csrc/kda_sm100.cuh",
+                       "csrc/kda_internal.h", "../include/kda.h"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str | None:
+    """sha256 over the paths and contents of the files `kernel` is compiled from, or None for a
+    kernel without a source list."""
     import hashlib
 
     from gated_delta_rule_120_b200 import _build
 
+    files = KERNEL_SOURCES.get(kernel)
+    if files is None:
+        return None
     h = hashlib.sha256()
-    for p in _build.sources():
+    for rel in files:
+        p = os.path.normpath(os.path.join(_build.PKG, rel))
         h.update(os.path.relpath(p, _build.ROOT).encode())
         with open(p, "rb") as f:
             h.update(f.read())
@@ -225,7 +238,7 @@ def library_source_hash() -> str:
 
 def captured_traffic(kernel: str, workload: str, path: str | None = None):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture, or None
-    when there is none or the library sources changed since it was taken."""
+    when there is none or the kernel's sources changed since it was taken."""
     if path is None:
         path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
                             "traffic.json")
@@ -236,8 +249,8 @@ def captured_traffic(kernel: str, workload: str, path: str | None = None):
         return None
     if not rec or rec.get("workload") != workload:
         return None
-    return rec["dram_bytes_per_launch"] if rec.get("source_sha256") == library_source_hash() \
-        else None
+    digest = kernel_source_hash(kernel)
+    return rec["dram_bytes_per_launch"] if digest and rec.get("source_sha256") == digest else None
 
 
 def profile_pass(fn, steps, dev):

@@ -48,14 +48,15 @@ def test_single_rank_is_identity():
     assert bench.whole_job_rate(100.0, 1, 1000.0) == pytest.approx(100.0)
 
 
-def test_captured_traffic_follows_the_library_sources(tmp_path):
-    """The roofline's DRAM traffic comes from the committed ncu capture only while the library
+def test_captured_traffic_follows_the_kernel_sources(tmp_path):
+    """The roofline's DRAM traffic comes from the committed ncu capture only while the kernel's
     sources hash to the value recorded with it; any other hash (or workload) gives None."""
     import json
 
     import bench
 
-    real = bench.library_source_hash()
+    real = bench.kernel_source_hash("chunk_local_tc")
+    assert real and bench.kernel_source_hash("no_such_kernel") is None
     prof = tmp_path / "profiles"
     prof.mkdir()
     rec = {"chunk_local_tc": {"workload": "w", "dram_bytes_per_launch": 123,

@@ -20,12 +20,12 @@
 //
 // The ratio exp(g_r - g_i) inside A_kk and A_qk is split into two bf16 factors around a reference
 // log decay, and each factor must stay inside bf16 range. Three cases per (chunk, head):
-//   fast   every channel decays by less than exp(-60) over the chunk: one reference (the chunk
+//   fast   every channel decays by less than exp(-L) over the chunk: one reference (the chunk
 //          start), K/Gamma = k * exp(-g), one pair of MMAs;
-//   blocks some channel decays harder, but none by more than exp(-60) within any 16-row block:
+//   blocks some channel decays harder, but none by more than exp(-L) within any 16-row block:
 //          row block R takes the reference g at the end of block R-1, so the row factor
 //          k_r exp(g_r - ref_R) is <= 1 and the column factor k_i exp(ref_R - g_i) is <= 1 for
-//          earlier blocks and <= exp(60) inside block R; three rounds of MMAs cover the four row
+//          earlier blocks and <= exp(L) inside block R; three rounds of MMAs cover the four row
 //          blocks (the column tile is rebuilt per reference);
 //   exact  otherwise: a CUDA-core evaluation of every product with ratios exp(g_r - g_i) <= 1.
 #include "kda_common.cuh"
@@ -39,7 +39,12 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr float kFastDecayLimit = 60.f;  // log-decay range bound for one bf16 factorisation
+// Log-decay range bound L of one bf16 factorisation: the factors k exp(+-g) stay below
+// |k| exp(L) inside bf16's range. L = 80 when the keys are L2-normalised in the kernel
+// (|k| <= 1; the discarded upper triangle of A_kk may overflow in its fp32 accumulator without
+// being read), L = 60 for caller-provided keys (any |k| below ~1e12).
+constexpr float kDecayLimitNormalisedKeys = 80.f;
+constexpr float kDecayLimitRawKeys = 60.f;
 constexpr int kModeFast = 0, kModeBlocks = 1, kModeExact = 2;
 
 // record layout (bytes) of one (chunk, head). QW is a [128 x 128] tile (64-column blocks
@@ -257,11 +262,12 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     gcp[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
   }
   cp_async_wait_all();
-  // the threads of the chunk's last rows hold g_C: fast mode iff every channel's is above -60
+  // the threads of the chunk's last rows hold g_C: fast mode iff every channel's is above -L
+  const float decay_limit = fz.l2 ? kDecayLimitNormalisedKeys : kDecayLimitRawKeys;
   float gmin = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) gmin = fminf(gmin, g[3][j]);
-  const bool fast = __syncthreads_and(rg != 15 || gmin >= -kFastDecayLimit) != 0;
+  const bool fast = __syncthreads_and(rg != 15 || gmin >= -decay_limit) != 0;
   float egc[8];
   {
     const float4* gcp = reinterpret_cast<const float4*>(sGC + cg * 8);
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 #pragma unroll
       for (int R = 0; R < 4; ++R) {
         const float next = sRef[R * kD + tid];
-        blocks_ok = blocks_ok && (prev - next <= kFastDecayLimit);
+        blocks_ok = blocks_ok && (prev - next <= decay_limit);
         prev = next;
       }
     }

@@ -61,6 +61,29 @@ def test_chunk_fused_bf16(cuda_device, mode):
     assert rel_err(s, s_ref) <= TOL_BF16_S
 
 
+def test_chunk_decays_between_the_two_bounds(cuda_device):
+    """Chunks whose strongest channels decay by exp(-70) over 64 tokens: with the in-kernel L2
+    norm (|k| <= 1) they take the single-reference evaluation (bound exp(-80)), with caller-
+    normalised keys the block-reference one (bound exp(-60)); both match the oracle."""
+    B, T, H = 1, 250, 2
+    x = _raw_inputs(B, T, H, 128, 128, "bf16", 710, cuda_device)
+    la = -torch.nn.functional.softplus(x["gate"]) * 0.5
+    la[..., :16] = -70.0 / 64.0
+    x["gate"] = la
+    s0 = torch.randn((B, H, 128, 128), device=cuda_device) * 0.02
+    qn = (x["q"].float() / x["q"].float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    kn = (x["k"].float() / x["k"].float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+    for fusion, q, k in (({"eps": 1e-6, "qk_l2norm": True}, x["q"], x["k"]), ({}, qn, kn)):
+        o, s = kda.kda_chunk_fwd(q, k, x["v"], la, x["beta"], initial_state=s0, chunk=64,
+                                 fusion=fusion or None)
+        torch.cuda.synchronize()
+        assert kda.kda_last_device_error() == kda.KDA_OK
+        y = dict(x, q=q, k=k)
+        o_ref, s_ref = _oracle_fused(y, fusion, s0.cpu(), np.array([0, T]))
+        assert rel_err(o.reshape(-1, H, 128), o_ref) <= TOL_BF16_O
+        assert rel_err(s, s_ref) <= TOL_BF16_S
+
+
 def test_chunk_fused_f32_varlen(cuda_device):
     lens = [5, 70, 0, 33]
     T, H, Dk, Dv = sum(lens), 2, 48, 20

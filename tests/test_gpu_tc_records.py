@@ -58,17 +58,18 @@ def chunk_reference(k, q, v, la, beta, L):
                 gam=np.exp(g[-1]))
 
 
-def chunk_mode(la_chunk: np.ndarray) -> str:
+def chunk_mode(la_chunk: np.ndarray, limit: float = 60.0) -> str:
     """Which evaluation of A_kk / A_qk the kernel picks for one chunk of one head: "fast" when
-    every channel decays by at most exp(-60) over the chunk, "blocks" when it does so within
-    every 16-row block, "exact" otherwise."""
+    every channel decays by at most exp(-limit) over the chunk, "blocks" when it does so within
+    every 16-row block, "exact" otherwise. The limit is 60 for caller-provided keys and 80 when
+    the kernel L2-normalises them."""
     g = np.concatenate([np.zeros((1, la_chunk.shape[1])), np.cumsum(la_chunk, axis=0)])
-    if g[-1].min() >= -60:
+    if g[-1].min() >= -limit:
         return "fast"
     ends = [min(16 * (R + 1), la_chunk.shape[0]) for R in range(4)]
     starts = [min(16 * R, la_chunk.shape[0]) for R in range(4)]
     drops = [(g[s] - g[e]).max() for s, e in zip(starts, ends)]
-    return "blocks" if max(drops) <= 60 else "exact"
+    return "blocks" if max(drops) <= limit else "exact"
 
 
 # per-chunk decay scalings: (channels scaled, factor); 1 = the plain recipe

@@ -241,16 +241,20 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     sc[1] = make_float4(g[3][4], g[3][5], g[3][6], g[3][7]);
   }
   __syncthreads();
-  {
-    float pre[8];
+  if (tid < kD) {  // exclusive prefix over the 16 row groups in place, one channel per thread
+    float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) pre[j] = 0.f;
-    for (int r2 = 0; r2 < rg; ++r2) {
-      const float4* sc = reinterpret_cast<const float4*>(sScan + r2 * kD + cg * 8);
-      const float4 a = sc[0], b = sc[1];
-      pre[0] += a.x; pre[1] += a.y; pre[2] += a.z; pre[3] += a.w;
-      pre[4] += b.x; pre[5] += b.y; pre[6] += b.z; pre[7] += b.w;
+    for (int r2 = 0; r2 < 16; ++r2) {
+      const float x = sScan[r2 * kD + tid];
+      sScan[r2 * kD + tid] = acc;
+      acc += x;
     }
+  }
+  __syncthreads();
+  {
+    const float4* sc = reinterpret_cast<const float4*>(sScan + rg * kD + cg * 8);
+    const float4 a = sc[0], b = sc[1];
+    const float pre[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll

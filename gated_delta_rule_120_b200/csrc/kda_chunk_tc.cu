@@ -1091,7 +1091,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
               float f[8];
               unpack8(graw[q8], f);
 #pragma unroll
-              for (int j = 0; j < 8; ++j) gt[q8 * 8 + j] = __fdividef(1.f, 1.f + __expf(-f[j]));
+              for (int j = 0; j < 8; ++j)  // sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU op
+                gt[q8 * 8 + j] = fmaf(0.5f, tanh_approx(0.5f * f[j]), 0.5f);
             }
           } else {
 #pragma unroll

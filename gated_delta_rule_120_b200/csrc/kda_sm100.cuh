@@ -264,6 +264,13 @@ __device__ __forceinline__ uint32_t tmem_at(uint32_t base, uint32_t lane, uint32
   return base + (lane << 16) + col;
 }
 
+// Hardware tanh approximation (one MUFU operation; relative error ~2^-10.7).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------------------- bf16 packing
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

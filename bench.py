@@ -692,7 +692,7 @@ def main():
         per = dms / args.decode_steps
         kms = dprof[0]["total_ms"] / dprof[0]["launches"]
         # the same decode steps with the layer's prologue and output epilogue fused in
-        fsteps = min(256, args.decode_steps)
+        fsteps = args.decode_steps  # as many steps as the plain run, so the two compare
         fdms, _ = run_decode(dspec, fsteps, dev, 3, world, rank, fused=True)
         fper = fdms / fsteps
         fused_decode = {"workload": dspec.name + "_fused_prologue_epilogue", "steps": fsteps,

@@ -309,7 +309,8 @@ __global__ void __launch_bounds__(kBwdThreads)
   float* sdb = smem + L_.db;
 
   if (!geo.ok()) return;
-  const int c = blockIdx.x, h = blockIdx.y;
+  const ChunkItem item = chunk_item();
+  const int c = item.c, h = item.h;
   if (c >= geo.num_chunks_total()) return;
   const int n = geo.seq_of_chunk(c);
   const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * C;
@@ -667,7 +668,7 @@ static cudaError_t launch_bwd_typed(const BackwardArgs& b, const SeqGeometry& ge
   }
   if (max_chunks == 0) return cudaSuccess;
   ProfileScope prof("chunk_local_bwd", stream);
-  chunk_local_bwd_kernel<Tin><<<dim3(max_chunks, a.H), kBwdThreads, sm4, stream>>>(
+  chunk_local_bwd_kernel<Tin><<<item_grid(max_chunks, a.H), kBwdThreads, sm4, stream>>>(
       (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
       a.Dv, records, rec, states, dstates, dvp, (const Tin*)b.d_o, (Tin*)b.dq, (Tin*)b.dk,
       (Tin*)b.dv, b.dlog_alpha, b.dbeta);

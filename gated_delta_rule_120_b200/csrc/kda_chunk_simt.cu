@@ -119,7 +119,8 @@ __global__ void __launch_bounds__(kSimtThreads)
   float* sb = sT + C * C;      // [C]
 
   if (!geo.ok()) return;
-  const int c = blockIdx.x, h = blockIdx.y;
+  const ChunkItem item = chunk_item();
+  const int c = item.c, h = item.h;
   if (c >= geo.num_chunks_total()) return;
   const int n = geo.seq_of_chunk(c);
   const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * C;
@@ -582,7 +583,7 @@ static cudaError_t launch_simt_typed(const PrefillArgs& a, const SeqGeometry& ge
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
   if (err != cudaSuccess) return err;
   if (max_chunks > 0) {
-    dim3 g1(max_chunks, a.H);
+    const dim3 g1 = item_grid(max_chunks, a.H);
     ProfileScope prof("chunk_local_simt", stream);
     chunk_local_simt_kernel<Tin><<<g1, kSimtThreads, sm1, stream>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
@@ -615,7 +616,7 @@ static cudaError_t launch_fwd_for_bwd_typed(const PrefillArgs& a, const SeqGeome
   if (err != cudaSuccess) return err;
   if (max_chunks > 0) {
     ProfileScope prof("bwd_chunk_local_fwd", stream);
-    chunk_local_simt_kernel<Tin><<<dim3(max_chunks, a.H), kSimtThreads, sm1, stream>>>(
+    chunk_local_simt_kernel<Tin><<<item_grid(max_chunks, a.H), kSimtThreads, sm1, stream>>>(
         (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, a.log_alpha, a.beta, geo, a.H, a.Dk,
         a.Dv, records, rec, a.fz);
     err = cudaGetLastError();

@@ -28,6 +28,7 @@
 // forward pass used (the result does not depend on the chunk size).
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_items.cuh"
 
 namespace kda {
 

@@ -22,6 +22,7 @@
 // = 0): they add nothing and their outputs are not written.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_items.cuh"
 
 namespace kda {
 

@@ -161,8 +161,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
                           uint8_t* __restrict__ ws_records, Fusion fz) {
   extern __shared__ uint8_t smem_raw[];
   if (!geo.ok()) return;
-  const ChunkItem item = chunk_item();
-  const int c = item.c, h = item.h;
+  const int c = blockIdx.x, h = blockIdx.y;
   if (c >= geo.num_chunks_total()) return;
 
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -1150,7 +1149,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
   if (err != cudaSuccess) return err;
   if (max_chunks > 0) {
     ProfileScope prof("chunk_local_tc", stream);
-    tc::chunk_local_tc_kernel<<<item_grid(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
+    tc::chunk_local_tc_kernel<<<dim3(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
         a.log_alpha, a.beta, geo, a.H, records, a.fz);
     err = cudaGetLastError();

@@ -108,21 +108,4 @@ struct SeqGeometry {
   }
 };
 
-// ---------------------------------------------------------------------------------------------
-// Chunk-local work items (chunk c, head h) are dispatched with the head index fastest (grid x =
-// head, y and z = chunk): the blocks resident at one time then cover whole token rows ([H, d],
-// contiguous in the [tokens, H, d] layout) of a few consecutive chunks instead of one 256-byte
-// piece per 8 KB row. Chunks beyond 65535 continue in z.
-// ---------------------------------------------------------------------------------------------
-struct ChunkItem {
-  int c, h;
-};
-__device__ __forceinline__ ChunkItem chunk_item() {
-  return ChunkItem{(int)(blockIdx.z * gridDim.y + blockIdx.y), (int)blockIdx.x};
-}
-inline dim3 item_grid(int max_chunks, int H) {  // max_chunks > 0
-  const int cy = max_chunks < 65535 ? max_chunks : 65535;
-  return dim3((unsigned)H, (unsigned)cy, (unsigned)ceil_div(max_chunks, cy));
-}
-
 }  // namespace kda

@@ -27,6 +27,20 @@ struct WsLayout {
 
 bool is_tc_path(kda_dtype_t dt) { return dt == KDA_DTYPE_BF16; }
 
+// Upper bound on the chunks of one call: every sequence may end in a partial chunk.
+long long max_chunks_of(int32_t B, int32_t T, int32_t C, int32_t N, bool varlen) {
+  const long long tokens = (long long)B * T;
+  return varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
+}
+
+// Launch-grid limits of the chunk kernels: the head index is a grid y extent (<= 65535) in the
+// chunk-state kernels, and chunk x head items and 2 x sequence x head chains are counted in int.
+// Bounding the items also keeps every workspace size far inside size_t.
+bool grid_limits_ok(int32_t B, int32_t T, int32_t H, int32_t C, int32_t N, bool varlen) {
+  if (H > 65535) return false;
+  return max_chunks_of(B, T, C, N, varlen) * H <= INT32_MAX && 2LL * N * H <= INT32_MAX;
+}
+
 kda_status_t check_prefill_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
                                  int32_t C, int32_t N, kda_dtype_t dt, bool varlen) {
   if (B < 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || N < 0 || C <= 0)
@@ -46,14 +60,14 @@ kda_status_t check_prefill_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, in
   const long long tokens = (long long)B * T;
   const long long elems = tokens * H * (long long)(Dk > Dv ? Dk : Dv);
   if (tokens > INT32_MAX || elems > (1LL << 40)) return KDA_ERR_UNSUPPORTED;
+  if (!grid_limits_ok(B, T, H, C, N, varlen)) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
 
 WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv, int32_t C,
                         int32_t N, bool varlen, kda_dtype_t dt) {
   WsLayout w;
-  const long long tokens = (long long)B * T;
-  w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
+  w.max_chunks = max_chunks_of(B, T, C, N, varlen);
   w.chunk_off_base = 256;
   const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * (2 * (size_t)N + 1), 256) : 0;
   w.rec_base = w.chunk_off_base + off_bytes;
@@ -81,6 +95,7 @@ kda_status_t check_backward_shape(int32_t B, int32_t T, int32_t H, int32_t Dk, i
   const long long tokens = (long long)B * T;
   const long long elems = tokens * H * (long long)(Dk > Dv ? Dk : Dv);
   if (tokens > INT32_MAX || elems > (1LL << 40)) return KDA_ERR_UNSUPPORTED;
+  if (!grid_limits_ok(B, T, H, kBwdChunk, N, varlen)) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
 
@@ -95,13 +110,12 @@ struct BwdLayout {
 BwdLayout backward_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv, int32_t N,
                           bool varlen) {
   BwdLayout w;
-  const int32_t C = kBwdChunk;
   const long long tokens = (long long)B * T;
-  w.max_chunks = varlen ? (tokens + C - 1) / C + N : (long long)B * ((T + C - 1) / C);
+  w.max_chunks = max_chunks_of(B, T, kBwdChunk, N, varlen);
   w.chunk_off_base = 256;
   const size_t off_bytes = varlen ? align_up(sizeof(int32_t) * ((size_t)N + 1), 256) : 0;
   w.rec_base = w.chunk_off_base + off_bytes;
-  const size_t rec_bytes = SimtRecord::make(C, Dk, Dv, true).record_floats * sizeof(float);
+  const size_t rec_bytes = SimtRecord::make(kBwdChunk, Dk, Dv, true).record_floats * sizeof(float);
   const size_t state_bytes = (size_t)Dk * Dv * sizeof(float);
   w.states_base = w.rec_base + (size_t)w.max_chunks * H * rec_bytes;
   w.dstates_base = align_up(w.states_base + (size_t)w.max_chunks * H * state_bytes, 256);

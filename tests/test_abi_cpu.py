@@ -63,6 +63,25 @@ def test_workspace_size_queries(L):
     del out
 
 
+def test_grid_limits_are_refused_on_host(L):
+    """Shapes beyond the kernels' launch grids are UNSUPPORTED before any size is computed: more
+    than 65535 heads, or more chunk x head items (here 2^30 empty sequences x 4 heads) or sequence
+    x head chains than an int counts; the largest fitting head count still sizes."""
+    F32, BF16 = kda.KDA_DTYPE_F32, kda.KDA_DTYPE_BF16
+    assert _ws(1, 64, 65536, 32, 32, 64, 1, F32)[0] == kda.KDA_ERR_UNSUPPORTED
+    assert _ws(1, 0, 4, 32, 32, 64, 1 << 30, F32)[0] == kda.KDA_ERR_UNSUPPORTED
+    assert _ws(1, 0, 2, 32, 32, 64, 1 << 29, F32)[0] == kda.KDA_ERR_UNSUPPORTED  # 2 N H = 2^31
+    rc, n = _ws(1, 64, 65535, 32, 32, 64, 1, F32)
+    assert rc == kda.KDA_OK and n > 65535 * 64 * 32 * 4
+    assert _fwd(H=65536) == kda.KDA_ERR_UNSUPPORTED
+    assert _fwd(dt=F32, Dk=32, Dv=32, cu=FAKE, B=1, T=0, N=1 << 30, H=4) == kda.KDA_ERR_UNSUPPORTED
+    sz = ctypes.c_size_t(0)
+    assert L.kda_chunk_bwd_workspace_size(1, 64, 65536, 32, 32, 1, F32, ctypes.byref(sz)) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert L.kda_chunk_bwd_workspace_size(1, 0, 4, 32, 32, 1 << 30, BF16, ctypes.byref(sz)) == \
+        kda.KDA_ERR_UNSUPPORTED
+
+
 FAKE = 1 << 20  # a 256-aligned non-null address: never dereferenced, the host rejects first
 
 

@@ -97,6 +97,10 @@ KDA_API kda_status_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t 
  *                   256-byte aligned; its contents on entry are ignored.
  * Supported: qkv_dtype BF16 with Dk = Dv = 128, chunk = 64 (tensor-core path); qkv_dtype F32
  * with 1 <= Dk, Dv <= 128 and Dv a multiple of 4 (CUDA-core fp32 path).
+ * Size limits (else KDA_ERR_UNSUPPORTED, before any launch): B*T <= INT32_MAX tokens,
+ * B*T*H*max(Dk, Dv) <= 2^40 elements, H <= 65535, (chunks + N) * H <= INT32_MAX and
+ * 2 * N * H <= INT32_MAX (chunks = ceil(B*T / chunk); the same limits hold for kda_chunk_bwd
+ * with chunk = 32).
  * Tokens past cu_seqlens[N] are neither read nor written.
  */
 KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,

@@ -6,10 +6,19 @@ the current stream. There is no CPU fallback: without the built library every ca
 
 Entry points (same names as the C ABI):
   kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk=64, ...)
-      chunkwise prefill -> (o, final_state)
-  kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None)
+      chunkwise prefill -> (o, final_state); ``fusion=`` adds the q/k L2 norm, the decay gate and
+      the output epilogue (kda_chunk_fwd_fused)
+  kda_chunk_fwd_noalloc(...)  the same prefill on the library's own scratch array
+  kda_chunk_bwd(q, k, v, log_alpha, beta, d_o, ...)  gradients of the prefill
+  kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None, fusion=None)
       one decode token per sequence, ``state`` updated in place -> o
-  kda_chunk_fwd_workspace_size(...), kda_last_device_error(), kda_status_string(code)
+  kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, ...)
+      a few tokens per sequence against pooled states -> o
+  kda_chunk_fwd_workspace_size(...), kda_chunk_bwd_workspace_size(...), kda_last_device_error(),
+  kda_status_string(code), kda_profile_enable(), kda_profile_read()
+
+Every tensor must be contiguous and on the device of q; caller-provided outputs and workspaces are
+checked for device, dtype and shape (size) before anything is launched.
 """
 from __future__ import annotations
 
@@ -146,18 +155,65 @@ def _stream_handle(device: torch.device):
 
 
 def _need(t: torch.Tensor, name: str, device, dtype=None):
-    if not t.is_cuda or t.device != device:
-        raise ValueError(f"{name} must be on {device}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor, got one on {t.device}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _need_inputs(q, k, v, log_alpha, beta):
+    """q, k [*lead, Dk] and v [*lead, Dv] in one dtype (bf16 or fp32), log_alpha [*lead, Dk] and
+    beta [*lead] fp32, all contiguous on q's device."""
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dev, q.dtype)
+    _dtype_code(q)
+    _need(log_alpha, "log_alpha", dev, torch.float32)
+    _need(beta, "beta", dev, torch.float32)
+    lead, Dk = tuple(q.shape[:-1]), q.shape[-1]
+    if tuple(k.shape) != lead + (Dk,) or tuple(log_alpha.shape) != lead + (Dk,) or \
+            tuple(v.shape[:-1]) != lead or tuple(beta.shape) != lead:
+        raise ValueError("inconsistent q/k/v/log_alpha/beta shapes")
+
+
+def _out(t, name: str, device, dtype, shape):
+    """A caller-provided output (or None -> a new tensor): the call writes `shape` elements of
+    `dtype` through it."""
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _need(t, name, device, dtype)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _workspace(ws, device, nbytes: int):
+    """The caller's workspace when it is a contiguous device buffer of at least `nbytes` bytes,
+    else a new one. Returns (tensor, its size in bytes)."""
+    if ws is not None:
+        _need(ws, "workspace", device)
+        if ws.numel() * ws.element_size() >= nbytes:
+            return ws, ws.numel() * ws.element_size()
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    return ws, ws.numel()
+
+
+def _size_dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"dtype {dtype} not supported (bf16 or fp32)")
+
+
 def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, chunk: int,
                                  num_seqs: int, dtype: torch.dtype) -> int:
     out = ctypes.c_size_t(0)
-    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    code = _size_dtype_code(dtype)
     _check(lib().kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, num_seqs, code,
                                               ctypes.byref(out)), "kda_chunk_fwd_workspace_size")
     return int(out.value)
@@ -196,6 +252,26 @@ def _fusion(fusion, dev, H, Dk, o_like=None):
                   None if w is None else w.data_ptr(), None if og is None else og.data_ptr())
 
 
+def _prefill_checks(q, k, v, log_alpha, beta, initial_state, cu_seqlens) -> int:
+    """Checks of the prefill inputs ([B,T,H,D] layout); returns the number of sequences N."""
+    dev = q.device
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,Dk]")
+    _need_inputs(q, k, v, log_alpha, beta)
+    B, _, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if initial_state is not None:
+        _need(initial_state, "initial_state", dev, torch.float32)
+        if tuple(initial_state.shape) != (N, H, Dk, Dv):
+            raise ValueError("initial_state must be [N,H,Dk,Dv]")
+    return N
+
+
 def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
                   output_final_state: bool = True, o=None, final_state=None, workspace=None,
                   fusion=None):
@@ -212,45 +288,28 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     dev = q.device
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, dev, q.dtype)
-    _need(log_alpha, "log_alpha", dev, torch.float32)
-    _need(beta, "beta", dev, torch.float32)
-    if tuple(k.shape) != (B, T, H, Dk) or tuple(log_alpha.shape) != (B, T, H, Dk) or \
-            tuple(v.shape[:3]) != (B, T, H) or tuple(beta.shape) != (B, T, H):
-        raise ValueError("inconsistent q/k/v/log_alpha/beta shapes")
-    if cu_seqlens is not None:
-        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
-        N = cu_seqlens.numel() - 1
-    else:
-        N = B
-    if initial_state is not None:
-        _need(initial_state, "initial_state", dev, torch.float32)
-        if tuple(initial_state.shape) != (N, H, Dk, Dv):
-            raise ValueError("initial_state must be [N,H,Dk,Dv]")
-    if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
-    if output_final_state and final_state is None:
-        final_state = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
+    N = _prefill_checks(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    o = _out(o, "o", dev, q.dtype, (B, T, H, Dv))
+    final_state = _out(final_state, "final_state", dev, torch.float32, (N, H, Dk, Dv)) \
+        if output_final_state else None
     ws_bytes = kda_chunk_fwd_workspace_size(B, T, H, Dk, Dv, chunk, N, q.dtype)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    workspace, ws_len = _workspace(workspace, dev, ws_bytes)
     fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
-            _ptr(final_state if output_final_state else None), _ptr(workspace), workspace.numel())
+            _ptr(final_state), _ptr(workspace), ws_len)
     if fz is None:
         code = lib().kda_chunk_fwd(*args, _stream_handle(dev))
     else:
         code = lib().kda_chunk_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_chunk_fwd")
-    return o, (final_state if output_final_state else None)
+    return o, final_state
 
 
 def kda_chunk_bwd_workspace_size(B: int, T: int, H: int, Dk: int, Dv: int, num_seqs: int,
                                  dtype: torch.dtype) -> int:
     out = ctypes.c_size_t(0)
-    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    code = _size_dtype_code(dtype)
     _check(lib().kda_chunk_bwd_workspace_size(B, T, H, Dk, Dv, num_seqs, code, ctypes.byref(out)),
            "kda_chunk_bwd_workspace_size")
     return int(out.value)
@@ -264,36 +323,25 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_sta
     dev = q.device
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
-        _need(t, n, dev, q.dtype)
-    _need(log_alpha, "log_alpha", dev, torch.float32)
-    _need(beta, "beta", dev, torch.float32)
-    if tuple(k.shape) != (B, T, H, Dk) or tuple(log_alpha.shape) != (B, T, H, Dk) or \
-            tuple(v.shape[:3]) != (B, T, H) or tuple(beta.shape) != (B, T, H) or \
-            tuple(d_o.shape) != tuple(v.shape):
-        raise ValueError("inconsistent q/k/v/log_alpha/beta/d_o shapes")
-    if cu_seqlens is not None:
-        _need(cu_seqlens, "cu_seqlens", dev, torch.int32)
-        N = cu_seqlens.numel() - 1
-    else:
-        N = B
-    for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
-        if t is not None:
-            _need(t, n, dev, torch.float32)
-            if tuple(t.shape) != (N, H, Dk, Dv):
-                raise ValueError(f"{n} must be [N,H,Dk,Dv]")
+    N = _prefill_checks(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    _need(d_o, "d_o", dev, q.dtype)
+    if tuple(d_o.shape) != tuple(v.shape):
+        raise ValueError("d_o must have v's shape")
+    if d_final_state is not None:
+        _need(d_final_state, "d_final_state", dev, torch.float32)
+        if tuple(d_final_state.shape) != (N, H, Dk, Dv):
+            raise ValueError("d_final_state must be [N,H,Dk,Dv]")
     dq, dk = torch.zeros_like(q), torch.zeros_like(k)
     dv = torch.zeros_like(v)
     dla = torch.zeros_like(log_alpha)
     db = torch.zeros_like(beta)
     ds0 = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev) if need_d_initial else None
     ws_bytes = kda_chunk_bwd_workspace_size(B, T, H, Dk, Dv, N, q.dtype)
-    if workspace is None or workspace.numel() < ws_bytes:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    workspace, ws_len = _workspace(workspace, dev, ws_bytes)
     code = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
                                _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk,
                                Dv, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv),
-                               _ptr(dla), _ptr(db), _ptr(ds0), _ptr(workspace), workspace.numel(),
+                               _ptr(dla), _ptr(db), _ptr(ds0), _ptr(workspace), ws_len,
                                _stream_handle(dev))
     _check(code, "kda_chunk_bwd")
     return dq, dk, dv, dla, db, ds0
@@ -304,17 +352,15 @@ def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None, fusion=None):
     beta [N,H] fp32; ``state`` [N,H,Dk,Dv] fp32 is updated in place. Returns o [N,H,Dv].
     ``fusion``: as for :func:`kda_chunk_fwd` (out_gate then has o's shape [N,H,Dv])."""
     dev = q.device
+    if q.dim() != 3:
+        raise ValueError("q must be [N,H,Dk]")
+    _need_inputs(q, k, v, log_alpha, beta)
     N, H, Dk = q.shape
     Dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, dev, q.dtype)
-    _need(log_alpha, "log_alpha", dev, torch.float32)
-    _need(beta, "beta", dev, torch.float32)
     _need(state, "state", dev, torch.float32)
     if tuple(state.shape) != (N, H, Dk, Dv):
         raise ValueError("state must be [N,H,Dk,Dv]")
-    if o is None:
-        o = torch.empty((N, H, Dv), dtype=q.dtype, device=dev)
+    o = _out(o, "o", dev, q.dtype, (N, H, Dv))
     fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), _ptr(state),
             _ptr(o), N, H, Dk, Dv)
@@ -334,12 +380,11 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, 
     state_pool [P,H,Dk,Dv] fp32 updated in place; state_indices int32 [N] on the device (negative
     entries skip their sequence) or None for pool rows 0..N-1. Returns o [N,T,H,Dv]."""
     dev = q.device
+    if q.dim() != 4:
+        raise ValueError("q must be [N,T,H,Dk]")
+    _need_inputs(q, k, v, log_alpha, beta)
     N, T, H, Dk = q.shape
     Dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, dev, q.dtype)
-    _need(log_alpha, "log_alpha", dev, torch.float32)
-    _need(beta, "beta", dev, torch.float32)
     _need(state_pool, "state_pool", dev, torch.float32)
     P = state_pool.shape[0]
     if tuple(state_pool.shape[1:]) != (H, Dk, Dv):
@@ -348,8 +393,7 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, 
         _need(state_indices, "state_indices", dev, torch.int32)
         if state_indices.numel() != N:
             raise ValueError("state_indices must have N entries")
-    if o is None:
-        o = torch.empty((N, T, H, Dv), dtype=q.dtype, device=dev)
+    o = _out(o, "o", dev, q.dtype, (N, T, H, Dv))
     fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(state_pool), _ptr(state_indices), _ptr(o), N, T, H, Dk, Dv, P)
@@ -395,11 +439,9 @@ def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None, cu_seqle
     dev = q.device
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
-    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
-    if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=q.dtype, device=dev)
-    if final_state is None:
-        final_state = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev)
+    N = _prefill_checks(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    o = _out(o, "o", dev, q.dtype, (B, T, H, Dv))
+    final_state = _out(final_state, "final_state", dev, torch.float32, (N, H, Dk, Dv))
     code = lib().kda_chunk_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
         _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),

@@ -186,3 +186,26 @@ def test_backward_workspace_and_argument_errors_on_host(L):
     # N != B without cu_seqlens
     args = [None] * 3 + [0] + [None] * 4 + [3, 2, 0, 1, 32, 32] + [None] * 9 + [0, None]
     assert L.kda_chunk_bwd(*args) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU fallback: host tensors are refused by every entry point before anything reaches the
+    library, and the size queries refuse dtypes the library has no kernel for."""
+    import torch
+
+    q = torch.zeros((1, 64, 2, 32))
+    beta = torch.zeros((1, 64, 2))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.kda_chunk_fwd(q, q, q, q, beta, chunk=32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.kda_chunk_fwd_noalloc(q, q, q, q, beta, chunk=32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.kda_chunk_bwd(q, q, q, q, beta, q)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.kda_recurrent_fwd(q, q, q, q, beta, torch.zeros((1, 2, 32, 32)))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kda.kda_recurrent_step(q[0], q[0], q[0], q[0], beta[0], torch.zeros((64, 2, 32, 32)))
+    with pytest.raises(TypeError):
+        kda.kda_chunk_fwd_workspace_size(1, 64, 2, 128, 128, 64, 1, torch.float16)
+    with pytest.raises(TypeError):
+        kda.kda_chunk_bwd_workspace_size(1, 64, 2, 128, 128, 1, torch.float16)

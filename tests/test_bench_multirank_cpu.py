@@ -33,7 +33,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_agree_on_max_time_and_rate():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:  # no fork of this multi-threaded process
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

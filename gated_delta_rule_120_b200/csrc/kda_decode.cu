@@ -15,6 +15,8 @@
 // thread), reduced, updated and stored once: 2 x 64 KiB of HBM traffic per head, nothing else
 // of note. Loads and stores use the streaming cache hint: the state of a decode batch is larger
 // than L2 and is not reused within the step.
+#include <atomic>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -1205,15 +1207,17 @@ static cudaError_t launch_rs_typed(const void* q, const void* k, const void* v,
   return cudaGetLastError();
 }
 
-static int g_num_sms[64] = {0};
+// SM count of each device (0 until first asked); calls from several host threads may fill an
+// entry concurrently, all with the same value.
+static std::atomic<int> g_num_sms[64];
 
 static int num_sms_cached() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  int nsm = (dev >= 0 && dev < 64) ? g_num_sms[dev] : 0;
+  int nsm = (dev >= 0 && dev < 64) ? g_num_sms[dev].load(std::memory_order_relaxed) : 0;
   if (nsm == 0) {
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev >= 0 && dev < 64) g_num_sms[dev] = nsm;
+    if (dev >= 0 && dev < 64) g_num_sms[dev].store(nsm, std::memory_order_relaxed);
   }
   return nsm;
 }
@@ -1310,15 +1314,8 @@ cudaError_t launch_decode_step(const void* q, const void* k, const void* v, kda_
     return launch_recurrent_multi(q, k, v, dt, log_alpha, beta, state, nullptr, o, N, 1, H, Dk,
                                   Dv, N, *fz, stream);
   if (streamable) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    int nsm = (dev >= 0 && dev < 64) ? g_num_sms[dev] : 0;
-    if (nsm == 0) {
-      err = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-      if (err != cudaSuccess) return err;
-      if (dev >= 0 && dev < 64) g_num_sms[dev] = nsm;
-    }
+    const int nsm = num_sms_cached();
+    if (nsm <= 0) return cudaErrorUnknown;
     const DsLayout lay = make_ds_layout(Dk, Dv, es, fz && fz->onorm && fz->og,
                                         fz && fz->A_log && fz->dt_bias);
     const size_t smem = (size_t)kDsStages * lay.stage_bytes + 2 * 8 * 32 * sizeof(float4) +

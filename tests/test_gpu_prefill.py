@@ -7,7 +7,7 @@ import gated_delta_rule_120_b200 as kda
 import kda_synth
 import oracle
 from kda_synth import PrefillSpec
-from tests._parity import TOL_BF16_O, TOL_BF16_S, TOL_F32, cu_list, rel_err, to_np
+from tests._parity import TOL_BF16_O, TOL_BF16_S, TOL_F32, cu_list, rel_err
 
 pytestmark = pytest.mark.gpu
 

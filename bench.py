@@ -496,6 +496,15 @@ def cpu_baseline(spec, dev, budget_s):
                        f"token-by-token recurrence, OpenMP over heads), {el:.1f} s")
 
 
+def workload_config(spec, world: int) -> dict:
+    """The `config` object of the headline line, the same for both arms."""
+    return {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
+            "d_k": spec.Dk, "d_v": spec.Dv, "chunk": spec.chunk,
+            "state": "fp32", "gates": "fp32",
+            "l2": "4 rotating input sets (>370 MB) larger than the 126 MB L2",
+            "parallelism": f"dp{world} (independent batches per GPU)"}
+
+
 def reference_arm(args, world, rank):
     """--impl reference: the fp64 CPU oracle on a bounded sample of the same workload per step."""
     if rank != 0:
@@ -525,8 +534,7 @@ def reference_arm(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H, "d": spec.Dk,
-                   "chunk": spec.chunk},
+        "config": workload_config(spec, args.gpus),
         "cpu_baseline": {"value": tokens_per_s, "unit": "tokens/s", "cores": oracle.max_threads(),
                          "kind": "oracle",
                          "sample": f"per step: 1 sequence x {heads} of {spec.H} heads x "
@@ -720,11 +728,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
-                       "d_k": spec.Dk, "d_v": spec.Dv, "chunk": spec.chunk,
-                       "state": "fp32", "gates": "fp32",
-                       "l2": "4 rotating input sets (>370 MB) larger than the 126 MB L2",
-                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "config": workload_config(spec, world),
             "roofline": roof, "prefill_path": path, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "clocks": clocks, **extra,

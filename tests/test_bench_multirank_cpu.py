@@ -69,3 +69,30 @@ def test_captured_traffic_follows_the_kernel_sources(tmp_path):
     rec["chunk_local_tc"]["source_sha256"] = "0" * 64
     (prof / "traffic.json").write_text(json.dumps(rec))
     assert bench.captured_traffic("chunk_local_tc", "w", path) is None
+
+
+def test_reference_arm_line_follows_the_contract():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON line with
+    the headline keys, our arm's config object, a cpu_baseline describing the run and an e2e
+    equal to its own value with no host-device bytes."""
+    import json
+    import subprocess
+    import sys
+
+    import kda_synth
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    run = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert run.returncode == 0, run.stderr[-2000:]
+    line = json.loads(run.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 1 and line["value"] > 0
+    assert line["config"] == bench.workload_config(kda_synth.STANDARD, 1)
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1

@@ -37,12 +37,13 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED = 0, 1, 2
 KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_WORKSPACE = 3, 4, 5
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 
-# every symbol include/kda.h declares
+# every symbol the headers under include/ declare
 ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
                "kda_chunk_fwd", "kda_recurrent_step", "kda_last_device_error",
                "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
                "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused",
-               "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_recurrent_step_fused")
+               "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_recurrent_step_fused",
+               "kda_selftest_wait_timeout")
 
 
 class Fusion(ctypes.Structure):
@@ -122,6 +123,8 @@ def lib() -> ctypes.CDLL:
             L.kda_profile_read.argtypes = [ctypes.POINTER(ProfileEntry), ctypes.c_int32,
                                            ctypes.POINTER(ctypes.c_int32)]
             L.kda_profile_read.restype = ctypes.c_int
+            L.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+            L.kda_selftest_wait_timeout.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -410,6 +413,16 @@ def kda_last_device_error(device=None) -> int:
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
     return int(lib().kda_last_device_error(_stream_handle(dev)))
+
+
+def kda_selftest_wait_timeout(limit_ns: int = 10_000_000, device=None) -> None:
+    """Run the bounded-wait give-up path on purpose (include/kda_selftest.h): one block waits on
+    an mbarrier phase that nothing completes and gives up after ``limit_ns``; the timeout is then
+    reported by :func:`kda_last_device_error` on the same device."""
+    dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                        torch.cuda.current_device())
+    _check(lib().kda_selftest_wait_timeout(int(limit_ns), _stream_handle(dev)),
+           "kda_selftest_wait_timeout")
 
 
 def kda_profile_enable(enable: bool = True) -> None:

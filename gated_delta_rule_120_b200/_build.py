@@ -23,7 +23,8 @@ NVCC_FLAGS = [
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(ROOT, "include", "kda.h")])
+                  glob.glob(os.path.join(CSRC, "*.h")) +
+                  glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def up_to_date() -> bool:

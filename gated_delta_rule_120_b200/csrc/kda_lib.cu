@@ -1,5 +1,5 @@
 // kda_lib.cu — single translation unit of libkda.so. The kernel files share one per-device
-// status word (defined in kda_api.cu), so they are compiled together rather than linked with
+// status word (defined in kda_common.cuh), so they are compiled together rather than linked with
 // relocatable device code.
 #include "kda_api.cu"
 #include "kda_profile.cu"
@@ -9,3 +9,4 @@
 #include "kda_epilogue.cu"
 #include "kda_chunk_bwd.cu"
 #include "kda_noalloc.cu"
+#include "kda_selftest.cu"

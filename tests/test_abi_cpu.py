@@ -19,8 +19,11 @@ def L():
 
 
 def declared_symbols():
-    with open(os.path.join(ROOT, "include", "kda.h")) as f:
-        src = f.read()
+    src = ""
+    for name in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if name.endswith(".h"):
+            with open(os.path.join(ROOT, "include", name)) as f:
+                src += f.read()
     return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", src)))
 
 
@@ -209,3 +212,9 @@ def test_binding_refuses_host_tensors():
         kda.kda_chunk_fwd_workspace_size(1, 64, 2, 128, 128, 64, 1, torch.float16)
     with pytest.raises(TypeError):
         kda.kda_chunk_bwd_workspace_size(1, 64, 2, 128, 128, 1, torch.float16)
+
+
+def test_selftest_limit_is_checked_on_host(L):
+    """The failure-detection self-test refuses limits outside [1 ns, 1 s] before launching."""
+    assert L.kda_selftest_wait_timeout(0, None) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_selftest_wait_timeout(1_000_000_001, None) == kda.KDA_ERR_INVALID_ARG

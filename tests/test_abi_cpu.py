@@ -218,3 +218,23 @@ def test_selftest_limit_is_checked_on_host(L):
     """The failure-detection self-test refuses limits outside [1 ns, 1 s] before launching."""
     assert L.kda_selftest_wait_timeout(0, None) == kda.KDA_ERR_INVALID_ARG
     assert L.kda_selftest_wait_timeout(1_000_000_001, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_headers_compile_as_c_and_the_library_links(L, tmp_path):
+    """A C99 program (tests/c_abi/kda_abi_check.c) includes the headers with no CUDA or C++ header,
+    links libkda.so and gets the host-side answers of the ABI."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    exe = tmp_path / "kda_abi_check"
+    pkg = os.path.dirname(_build.LIB)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi", "kda_abi_check.c"),
+                    "-L", pkg, "-lkda", f"-Wl,-rpath,{pkg}", "-o", str(exe)], check=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert run.stdout.startswith("ok ")

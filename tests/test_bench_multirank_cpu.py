@@ -96,3 +96,27 @@ def test_reference_arm_line_follows_the_contract():
                            "d2h_bytes_per_step": 0}
     cpu = line["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1
+
+
+def test_roofline_byte_accounting_matches_the_layouts():
+    """The bench's algorithmic bytes, counted by hand from the tensor layouts of the standard
+    prefill (B=2, T=4096, H=32, d=128, bf16, C=64: 4096 (chunk, head) items) and the decode."""
+    import kda_synth
+    from gated_delta_rule_120_b200 import roofline
+
+    spec = kda_synth.STANDARD
+    items = 2 * 4096 // 64 * 32
+    per_item_inputs = 3 * 64 * 128 * 2 + 64 * 128 * 4 + 64 * 4  # q, k, v bf16; log alpha; beta
+    assert per_item_inputs == 82_176
+    rec = 74_240
+    assert bench.prefill_kernel_bytes("chunk_local_tc", spec, 128, rec) == \
+        items * (per_item_inputs + rec)
+    o_bytes = 2 * 4096 * 32 * 128 * 2
+    state = 2 * 32 * 128 * 128 * 4
+    assert bench.prefill_kernel_bytes("chunk_state_tc", spec, 128, rec) == \
+        items * rec + o_bytes + 2 * state  # initial state read, final state written
+    # the path's minimum: 1540 B per token-head plus the two states
+    assert roofline.prefill_min_bytes(2 * 4096 * 32, 2, 32, 128, 128, 2, True, True) == \
+        2 * 4096 * 32 * 1540 + 2 * state
+    # decode: every state read once and written once
+    assert roofline.decode_state_bytes(256, 32, 128, 128) == 2 * 256 * 32 * 128 * 128 * 4

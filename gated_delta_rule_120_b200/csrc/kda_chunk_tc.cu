@@ -16,7 +16,7 @@
 //        D1 = W S, D2 = Qt S  ->  V' = U - D1  ->  D3 = Kt^T V', D2 += A_qk V'
 //        S = Diag(gamma_C) S + D3 (Eq. 8, fp32 in registers),  O = D2 (Eq. 9)
 //      Warp roles: a bulk-copy producer (double-buffered records), a single MMA-issuing thread,
-//      and four epilogue warps that hold the fp32 state slice (one row of S per thread).
+//      8 epilogue warps, 32 columns of S each (one row of S per thread, in fp32 registers).
 //
 // The ratio exp(g_r - g_i) inside A_kk and A_qk is split into two bf16 factors around a reference
 // log decay, and each factor must stay inside bf16 range. Three cases per (chunk, head):

@@ -238,3 +238,27 @@ def test_headers_compile_as_c_and_the_library_links(L, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, run.stdout + run.stderr
     assert run.stdout.startswith("ok ")
+
+
+def test_product_path_never_reaches_the_oracle(L):
+    """The oracle is test infrastructure: the package's Python files, the CUDA sources and the
+    headers never name it, and libkda.so links no library besides the C/C++ runtime (the CUDA
+    runtime is linked statically)."""
+    import shutil
+    import subprocess
+
+    pkg = os.path.dirname(_build.LIB)
+    roots = [pkg, os.path.join(pkg, "csrc"), os.path.join(ROOT, "include")]
+    for d in roots:
+        for name in os.listdir(d):
+            if name.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(d, name)) as f:
+                    assert "oracle" not in f.read().lower(), os.path.join(d, name)
+    readelf = shutil.which("readelf")
+    if readelf is None:
+        pytest.skip("no readelf")
+    dyn = subprocess.run([readelf, "-d", _build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    needed = re.findall(r"\(NEEDED\)\s+Shared library: \[([^\]]+)\]", dyn)
+    assert needed and all(re.match(r"(libstdc\+\+|libgcc_s|libc|libm|ld-linux|libdl|librt|"
+                                   r"libpthread)", n) for n in needed), needed

@@ -262,3 +262,16 @@ def test_product_path_never_reaches_the_oracle(L):
     needed = re.findall(r"\(NEEDED\)\s+Shared library: \[([^\]]+)\]", dyn)
     assert needed and all(re.match(r"(libstdc\+\+|libgcc_s|libc|libm|ld-linux|libdl|librt|"
                                    r"libpthread)", n) for n in needed), needed
+
+
+def test_oracle_shares_nothing_with_the_library():
+    """The other direction: the oracle's C source includes only system headers and its Python
+    module imports nothing from the package, the CUDA sources or the synthetic-input module."""
+    odir = os.path.join(ROOT, "oracle")
+    with open(os.path.join(odir, "kda_oracle.c")) as f:
+        src = f.read()
+    assert re.findall(r'#include\s+"', src) == []  # no local header at all
+    with open(os.path.join(odir, "__init__.py")) as f:
+        py = f.read()
+    for name in ("gated_delta_rule_120_b200", "kda_synth", "csrc", "libkda.so"):
+        assert name not in py, name

@@ -496,6 +496,36 @@ def cpu_baseline(spec, dev, budget_s):
                        f"token-by-token recurrence, OpenMP over heads), {el:.1f} s")
 
 
+DATASHEET_BF16_TFLOPS = 2250.0  # nominal dense bf16 tensor-core peak of one B200
+
+
+def prefill_path_figures(spec, ms_step: float, hbm_peak: float, tc_peak: float) -> dict:
+    """Path-level figures of one prefill step of `spec` taking `ms_step` ms: minimum HBM bytes and
+    their rate, the three FLOP counts (Eq. 13, triangular halves excluded, full issued tiles) as
+    rates, Eq. 13 as a fraction of the measured and of the datasheet tensor-core peak, and the
+    fraction of the min(TC, HBM) roofline floor. Peaks in GB/s and TFLOP/s."""
+    from gated_delta_rule_120_b200 import roofline
+
+    sec = ms_step / 1e3
+    heads = spec.B * spec.H
+    min_bytes = roofline.prefill_min_bytes(spec.token_heads(), spec.num_seqs, spec.H, spec.Dk,
+                                           spec.Dv, 2, spec.init_std > 0, True)
+    eq13 = roofline.eq13_flops(spec.T, spec.chunk, spec.Dk) * heads
+    path = {"min_bytes": min_bytes, "achieved_gbs": min_bytes / sec / 1e9,
+            "frac_hbm": min_bytes / sec / 1e9 / hbm_peak,
+            "eq13_flops": eq13, "eq13_tflops": eq13 / sec / 1e12,
+            "frac_tc_peak_eq13": eq13 / sec / 1e12 / tc_peak,
+            "frac_tc_datasheet_eq13": eq13 / sec / 1e12 / DATASHEET_BF16_TFLOPS,
+            "triangular_tflops": roofline.triangular_flops(spec.T, spec.chunk, spec.Dk) *
+            heads / sec / 1e12,
+            "issued_tile_tflops": roofline.issued_tile_flops(spec.T, spec.chunk, spec.Dk) *
+            heads / sec / 1e12,
+            "roofline_floor_ms": 1e3 * max(min_bytes / (hbm_peak * 1e9),
+                                           eq13 / (tc_peak * 1e12))}
+    path["frac_min_roofline"] = path["roofline_floor_ms"] / ms_step
+    return path
+
+
 def workload_config(spec, world: int) -> dict:
     """The `config` object of the headline line, the same for both arms."""
     return {"workload": spec.name, "B": spec.B, "T": spec.T, "H": spec.H,
@@ -596,19 +626,7 @@ def main():
                          "share": p["total_ms"] / sum(q["total_ms"] for q in prof)}
                         for p in prof]}
     # path-level figures for the prefill step
-    min_bytes = roofline.prefill_min_bytes(spec.token_heads(), spec.num_seqs, spec.H, spec.Dk,
-                                           spec.Dv, 2, spec.init_std > 0, True)
-    eq13 = roofline.eq13_flops(spec.T, spec.chunk, spec.Dk) * spec.B * spec.H
-    tc_peak = peaks["bf16_tflops"]
-    path = {"min_bytes": min_bytes, "achieved_gbs": min_bytes / (ms_step / 1e3) / 1e9,
-            "frac_hbm": min_bytes / (ms_step / 1e3) / 1e9 / hbm_peak,
-            "eq13_flops": eq13, "eq13_tflops": eq13 / (ms_step / 1e3) / 1e12,
-            "frac_tc_peak_eq13": eq13 / (ms_step / 1e3) / 1e12 / tc_peak,
-            "issued_tile_tflops": roofline.issued_tile_flops(spec.T, spec.chunk, spec.Dk) *
-            spec.B * spec.H / (ms_step / 1e3) / 1e12,
-            "roofline_floor_ms": 1e3 * max(min_bytes / (hbm_peak * 1e9),
-                                           eq13 / (tc_peak * 1e12))}
-    path["frac_min_roofline"] = path["roofline_floor_ms"] / ms_step
+    path = prefill_path_figures(spec, ms_step, hbm_peak, peaks["bf16_tflops"])
 
     # public-API end to end
     e2e_ms, h2d, d2h = run_prefill_e2e(spec, pre["sets"][0], pre["o"], pre["fs"], pre["ws"], dev,

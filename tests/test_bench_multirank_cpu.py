@@ -120,3 +120,22 @@ def test_roofline_byte_accounting_matches_the_layouts():
         2 * 4096 * 32 * 1540 + 2 * state
     # decode: every state read once and written once
     assert roofline.decode_state_bytes(256, 32, 128, 128) == 2 * 256 * 32 * 128 * 128 * 4
+
+
+def test_prefill_path_figures():
+    """The path-level figures of the standard prefill at a given step time: minimum bytes, the
+    three FLOP-count rates (Eq. 13 < triangular < issued tiles), both tensor-core fractions and
+    the roofline-floor fraction; the values of a recorded bench line are reproduced."""
+    import kda_synth
+
+    spec = kda_synth.STANDARD
+    p = bench.prefill_path_figures(spec, 0.2712591886520386, 6543.4, 1623.7)
+    assert p["min_bytes"] == 412_090_368
+    assert p["eq13_flops"] == 520_093_696 * 2 * 32
+    assert p["eq13_tflops"] == pytest.approx(122.70919451395272, rel=1e-12)
+    assert p["frac_tc_peak_eq13"] == pytest.approx(0.07557380951773894, rel=1e-12)
+    assert p["frac_tc_datasheet_eq13"] == pytest.approx(p["eq13_tflops"] / 2250.0)
+    assert p["eq13_tflops"] < p["triangular_tflops"] < p["issued_tile_tflops"]
+    floor_ms = 1e3 * max(412_090_368 / 6543.4e9, p["eq13_flops"] / 1623.7e12)
+    assert p["roofline_floor_ms"] == pytest.approx(floor_ms)
+    assert p["frac_min_roofline"] == pytest.approx(floor_ms / 0.2712591886520386)

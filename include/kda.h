@@ -154,8 +154,8 @@ KDA_API kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const v
  *   state           device fp32 [N,H,Dk,Dv], read and overwritten; 16-byte aligned.
  *   o               device [N,H,Dv], dtype qkv_dtype: o = S_new^T q.
  * q, k, v and o need the alignment of their element type; log_alpha and beta 4 bytes.
- * Supported: 1 <= Dk <= 128, 4 <= Dv <= 128 with Dv a multiple of 4, either dtype.
- * The state is streamed once from HBM and written once.
+ * Supported: 1 <= Dk <= 128, 4 <= Dv <= 128 (Dv % 4 == 0), either dtype, N * H <= INT32_MAX
+ * (else KDA_ERR_UNSUPPORTED). The state is streamed once from HBM and written once.
  */
 KDA_API kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
                                 const float* log_alpha, const float* beta, float* state, void* o,
@@ -176,7 +176,7 @@ KDA_API kda_status_t kda_recurrent_step(const void* q, const void* k, const void
  *                   (no state update, its o is left untouched). Entries must be distinct; an
  *                   entry >= P is skipped too and reported as KDA_ERR_INVALID_ARG through
  *                   kda_last_device_error(). NULL means pool row n (then P >= N is required).
- * Supported: as kda_recurrent_step (1 <= Dk <= 128, 4 <= Dv <= 128, Dv % 4 == 0), T >= 0.
+ * Supported: as kda_recurrent_step, T >= 0 and N * T * H * max(Dk, Dv) <= 2^40.
  * For longer sequences kda_chunk_fwd is the faster path.
  */
 KDA_API kda_status_t kda_recurrent_fwd(const void* q, const void* k, const void* v,

@@ -11,6 +11,15 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running case")
+    config.addinivalue_line("markers", "late: run after the other tests (the newest checks)")
+
+
+def pytest_collection_modifyitems(config, items):
+    """Tests marked `late` run after all others, in their collected order, so that when a run
+    stops at its first failure a failure among the newest checks cannot hide the results of the
+    established ones."""
+    items[:] = [i for i in items if i.get_closest_marker("late") is None] + \
+        [i for i in items if i.get_closest_marker("late") is not None]
 
 
 @pytest.fixture(scope="session")

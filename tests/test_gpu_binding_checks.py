@@ -7,7 +7,7 @@ import torch
 import gated_delta_rule_120_b200 as kda
 import kda_synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
 
 
 def _prefill_args(dev):

@@ -12,7 +12,7 @@ import torch
 import gated_delta_rule_120_b200 as kda
 import kda_synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
 
 GUARD = 4096  # guard elements after each buffer
 

@@ -10,7 +10,7 @@ import kda_synth
 import oracle
 from tests._parity import TOL_F32, rel_err
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
 
 
 def test_bounded_wait_gives_up_and_the_context_survives(cuda_device):

@@ -9,7 +9,7 @@ import torch
 import gated_delta_rule_120_b200 as kda
 import kda_synth
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late]
 
 
 def test_recurrent_mode_replays_bit_exactly(cuda_device):

@@ -190,31 +190,11 @@ def timed(fn, steps, warmup, world, dev, join=None):
     return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
 
-# Algorithmic bytes one launch of each kernel must move (inputs read once, outputs written once);
-# the workspace records are the split design's intermediates, written by one kernel and read by
-# the next, and count for both.
-def prefill_kernel_bytes(name, spec, max_chunks, rec_bytes):
-    th = spec.token_heads()
-    qkv = 2 if spec.dtype == "bf16" else 4
-    inputs = th * ((2 * spec.Dk + spec.Dv) * qkv + 4 * spec.Dk + 4)
-    out_o = th * spec.Dv * qkv
-    states = spec.num_seqs * spec.H * spec.Dk * spec.Dv * 4
-    recs = max_chunks * spec.H * rec_bytes
-    if name.startswith("chunk_local"):
-        return inputs + recs
-    if name.startswith("chunk_state"):
-        return recs + out_o + states * (2 if spec.init_std > 0 else 1)
-    if name.startswith("chunk_map"):
-        return 8 * (spec.num_seqs + 1)
-    return None
-
-
 # The files each captured kernel is compiled from: its own source and the headers that source
 # includes (the library is one translation unit, but a kernel's code depends only on these).
-KERNEL_SOURCES = {
-    "chunk_local_tc": ["csrc/kda_chunk_tc.cu", "csrc/kda_common.cuh", "csrc/kda_sm100.cuh",
-                       "csrc/kda_internal.h", "../include/kda.h"],
-}
+_TC_SOURCES = ["csrc/kda_chunk_tc.cu", "csrc/kda_common.cuh", "csrc/kda_sm100.cuh",
+               "csrc/kda_internal.h", "../include/kda.h"]
+KERNEL_SOURCES = {"chunk_local_tc": _TC_SOURCES, "chunk_state_tc": _TC_SOURCES}
 
 
 def kernel_source_hash(kernel: str) -> str | None:
@@ -237,17 +217,18 @@ def kernel_source_hash(kernel: str) -> str | None:
 
 
 def captured_traffic(kernel: str, workload: str, path: str | None = None):
-    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture, or None
-    when there is none or the kernel's sources changed since it was taken."""
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu captures
+    (profiles/traffic.json, records keyed "kernel@workload"), or None when there is none or the
+    kernel's sources changed since it was taken."""
     if path is None:
         path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
                             "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
+            rec = json.load(f).get("records", {}).get(f"{kernel}@{workload}")
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("workload") != workload:
+    if not rec:
         return None
     digest = kernel_source_hash(kernel)
     return rec["dram_bytes_per_launch"] if digest and rec.get("source_sha256") == digest else None
@@ -496,6 +477,49 @@ def cpu_baseline(spec, dev, budget_s):
                        f"token-by-token recurrence, OpenMP over heads), {el:.1f} s")
 
 
+def prefill_roofline(spec, ms_step: float, prof, steps: int, hbm_peak: float,
+                     peak_src: str) -> dict:
+    """Roofline of one prefill call (the path: every kernel of kda_chunk_fwd) against the method's
+    algorithmic bytes (per token-head q, k, v, o in the input dtype, log_alpha fp32, beta fp32;
+    the fp32 states in and out), with each kernel's share of those bytes beside its own CUDA-event
+    time. `traffic` is the DRAM bytes the path's kernels really moved, from the committed ncu
+    captures (None while any is missing or stale); its ratio to the algorithmic bytes shows the
+    cost of the records the chunk-local kernel writes and the state kernel reads."""
+    from gated_delta_rule_120_b200 import roofline
+
+    qkv = 2 if spec.dtype == "bf16" else 4
+    th = spec.token_heads()
+    dims = (th, spec.num_seqs, spec.H, spec.Dk, spec.Dv, qkv, spec.init_std > 0, True)
+    alg = roofline.prefill_min_bytes(*dims)
+    total = sum(p["total_ms"] for p in prof) or 1.0
+    kernels, traffic, complete = [], 0.0, True
+    for p in sorted(prof, key=lambda p: -p["total_ms"]):
+        ms = p["total_ms"] / p["launches"]
+        share = roofline.prefill_kernel_share_bytes(p["name"], *dims)
+        tr = captured_traffic(p["name"], spec.name)
+        per_step = p["launches"] / steps
+        kernels.append({
+            "name": p["name"], "launches_per_step": per_step, "ms_per_launch": ms,
+            "share": p["total_ms"] / total, "algorithmic_bytes": share,
+            "achieved_gbs": share / (ms / 1e3) / 1e9 if share else None,
+            "frac": share / (ms / 1e3) / 1e9 / hbm_peak if share else None,
+            "traffic": tr, "traffic_over_algorithmic": tr / share if tr and share else None})
+        if tr is None:
+            complete = False
+        else:
+            traffic += tr * per_step
+    achieved = alg / (ms_step / 1e3) / 1e9
+    return {"kernel": "kda_chunk_fwd (" + " + ".join(k["name"] for k in kernels) + ")",
+            "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": traffic if complete else None,
+            "traffic_over_algorithmic": traffic / alg if complete else None,
+            "algorithmic_bytes": alg,
+            "algorithmic_basis": "per token-head q, k, v, o in the input dtype + log_alpha fp32 + "
+                                 "beta fp32 (1540 B at d = 128, bf16) + fp32 states in and out",
+            "peak_source": f"{peak_src} HBM copy bandwidth", "launch_ms": ms_step,
+            "dominant_kernel": kernels[0]["name"] if kernels else None, "kernels": kernels}
+
+
 DATASHEET_BF16_TFLOPS = 2250.0  # nominal dense bf16 tensor-core peak of one B200
 
 
@@ -605,26 +629,11 @@ def main():
     tokens = spec.total_tokens
     value = whole_job_rate(tokens * args.steps, world, pre["ms"])
 
-    # roofline of the dominant kernel
+    # roofline of the prefill path, with each kernel's share of the algorithmic bytes
     prof = pre["prof"]
     launches_per_step = sum(p["launches"] for p in prof) / args.steps
-    n_chunks = chunk_count(spec)
-    top = prof[0]
-    # bytes of one (chunk, head) record: the workspace past its 256-byte header, per record
-    rec_bytes = (pre["ws_bytes"] - 256) // max(1, n_chunks * spec.H)
-    top_bytes = prefill_kernel_bytes(top["name"], spec, n_chunks, rec_bytes)
-    top_ms = top["total_ms"] / top["launches"]
-    achieved = top_bytes / (top_ms / 1e3) / 1e9 if top_bytes else None
     hbm_peak = peaks["hbm_gbs"]
-    roof = {"kernel": top["name"], "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-            "unit": "GB/s", "frac": (achieved / hbm_peak) if achieved else None,
-            "traffic": captured_traffic(top["name"], spec.name),
-            "peak_source": f"{peak_src} HBM copy bandwidth",
-            "launch_ms": top_ms,
-            "kernels": [{"name": p["name"], "launches_per_step": p["launches"] / args.steps,
-                         "ms_per_launch": p["total_ms"] / p["launches"],
-                         "share": p["total_ms"] / sum(q["total_ms"] for q in prof)}
-                        for p in prof]}
+    roof = prefill_roofline(spec, ms_step, prof, args.steps, hbm_peak, peak_src)
     # path-level figures for the prefill step
     path = prefill_path_figures(spec, ms_step, hbm_peak, peaks["bf16_tflops"])
 
@@ -640,16 +649,16 @@ def main():
     extra = {}
     if not args.no_long:
         lspec = kda_synth.LONG
-        lp = run_prefill(lspec, [2002 + 10 * rank], dev, max(2, args.steps // 5), 1, world)
-        lms = lp["ms"] / max(2, args.steps // 5)
-        lmin = roofline.prefill_min_bytes(lspec.token_heads(), 1, lspec.H, lspec.Dk, lspec.Dv, 2,
-                                          False, True)
+        lsteps = max(2, args.steps // 5)
+        lp = run_prefill(lspec, [2002 + 10 * rank], dev, lsteps, 1, world)
+        lms = lp["ms"] / lsteps
+        lpath = prefill_path_figures(lspec, lms, hbm_peak, peaks["bf16_tflops"])
         extra["long_prefill"] = {
             "workload": lspec.name, "tokens_per_s": world * lspec.total_tokens / (lms / 1e3),
-            "ms_per_call": lms, "frac_hbm_min_bytes": lmin / (lms / 1e3) / 1e9 / hbm_peak,
-            "eq13_tflops": roofline.eq13_flops(lspec.T, 64, 128) * lspec.H / (lms / 1e3) / 1e12,
-            "kernels": [{"name": p["name"], "ms_per_launch": p["total_ms"] / p["launches"]}
-                        for p in lp["prof"]]}
+            "ms_per_call": lms, "frac_hbm_min_bytes": lpath["frac_hbm"],
+            "eq13_tflops": lpath["eq13_tflops"],
+            "roofline": prefill_roofline(lspec, lms, lp["prof"], lsteps, hbm_peak, peak_src),
+            "prefill_path": lpath}
         del lp
         torch.cuda.empty_cache()
         # packed variable-length batch: 16 sequences, lengths log-uniform in [256, 32768]

@@ -157,6 +157,12 @@ def _stream_handle(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _on(device: torch.device):
+    """Make `device` current around an ABI call: the library launches on (and looks up per-device
+    state of) the current device, which must own the tensors and the stream passed to it."""
+    return torch.cuda.device(device)
+
+
 def _need(t: torch.Tensor, name: str, device, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor, got one on {t.device}")
@@ -301,10 +307,11 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
             _ptr(final_state), _ptr(workspace), ws_len)
-    if fz is None:
-        code = lib().kda_chunk_fwd(*args, _stream_handle(dev))
-    else:
-        code = lib().kda_chunk_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
+    with _on(dev):
+        if fz is None:
+            code = lib().kda_chunk_fwd(*args, _stream_handle(dev))
+        else:
+            code = lib().kda_chunk_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_chunk_fwd")
     return o, final_state
 
@@ -341,11 +348,12 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_sta
     ds0 = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=dev) if need_d_initial else None
     ws_bytes = kda_chunk_bwd_workspace_size(B, T, H, Dk, Dv, N, q.dtype)
     workspace, ws_len = _workspace(workspace, dev, ws_bytes)
-    code = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
-                               _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk,
-                               Dv, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk), _ptr(dv),
-                               _ptr(dla), _ptr(db), _ptr(ds0), _ptr(workspace), ws_len,
-                               _stream_handle(dev))
+    with _on(dev):
+        code = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha),
+                                   _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H,
+                                   Dk, Dv, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(dla), _ptr(db), _ptr(ds0), _ptr(workspace),
+                                   ws_len, _stream_handle(dev))
     _check(code, "kda_chunk_bwd")
     return dq, dk, dv, dla, db, ds0
 
@@ -367,10 +375,11 @@ def kda_recurrent_step(q, k, v, log_alpha, beta, state, o=None, fusion=None):
     fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta), _ptr(state),
             _ptr(o), N, H, Dk, Dv)
-    if fz is None:
-        code = lib().kda_recurrent_step(*args, _stream_handle(dev))
-    else:
-        code = lib().kda_recurrent_step_fused(*args, ctypes.byref(fz), _stream_handle(dev))
+    with _on(dev):
+        if fz is None:
+            code = lib().kda_recurrent_step(*args, _stream_handle(dev))
+        else:
+            code = lib().kda_recurrent_step_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_recurrent_step")
     return o
 
@@ -400,10 +409,11 @@ def kda_recurrent_fwd(q, k, v, log_alpha, beta, state_pool, state_indices=None, 
     fz = _fusion(fusion, dev, H, Dk, v)
     args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
             _ptr(state_pool), _ptr(state_indices), _ptr(o), N, T, H, Dk, Dv, P)
-    if fz is None:
-        code = lib().kda_recurrent_fwd(*args, _stream_handle(dev))
-    else:
-        code = lib().kda_recurrent_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
+    with _on(dev):
+        if fz is None:
+            code = lib().kda_recurrent_fwd(*args, _stream_handle(dev))
+        else:
+            code = lib().kda_recurrent_fwd_fused(*args, ctypes.byref(fz), _stream_handle(dev))
     _check(code, "kda_recurrent_fwd")
     return o
 
@@ -412,7 +422,8 @@ def kda_last_device_error(device=None) -> int:
     """Read and clear the device status word (synchronises the current stream)."""
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
-    return int(lib().kda_last_device_error(_stream_handle(dev)))
+    with _on(dev):
+        return int(lib().kda_last_device_error(_stream_handle(dev)))
 
 
 def kda_selftest_wait_timeout(limit_ns: int = 10_000_000, device=None) -> None:
@@ -421,8 +432,9 @@ def kda_selftest_wait_timeout(limit_ns: int = 10_000_000, device=None) -> None:
     reported by :func:`kda_last_device_error` on the same device."""
     dev = torch.device(device) if device is not None else torch.device("cuda",
                                                                         torch.cuda.current_device())
-    _check(lib().kda_selftest_wait_timeout(int(limit_ns), _stream_handle(dev)),
-           "kda_selftest_wait_timeout")
+    with _on(dev):
+        code = lib().kda_selftest_wait_timeout(int(limit_ns), _stream_handle(dev))
+    _check(code, "kda_selftest_wait_timeout")
 
 
 def kda_profile_enable(enable: bool = True) -> None:
@@ -455,9 +467,10 @@ def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None, cu_seqle
     N = _prefill_checks(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
     o = _out(o, "o", dev, q.dtype, (B, T, H, Dv))
     final_state = _out(final_state, "final_state", dev, torch.float32, (N, H, Dk, Dv))
-    code = lib().kda_chunk_fwd_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
-        _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
-        _ptr(final_state), _stream_handle(dev))
+    with _on(dev):  # the scratch array used is the current device's
+        code = lib().kda_chunk_fwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(log_alpha), _ptr(beta),
+            _ptr(initial_state), _ptr(cu_seqlens), N, B, T, H, Dk, Dv, chunk, _ptr(o),
+            _ptr(final_state), _stream_handle(dev))
     _check(code, "kda_chunk_fwd_noalloc")
     return o, final_state

@@ -50,3 +50,22 @@ def decode_total_bytes(N: int, H: int, Dk: int, Dv: int, qkv_bytes: int) -> int:
     """All bytes of one decode step: state in/out, q, k, v, log_alpha, beta in, o out."""
     per_head = (2 * Dk + Dv) * qkv_bytes + 4 * Dk + 4 + Dv * qkv_bytes
     return decode_state_bytes(N, H, Dk, Dv) + N * H * per_head
+
+
+def prefill_kernel_share_bytes(name: str, token_heads: int, num_seqs: int, H: int, Dk: int,
+                               Dv: int, qkv_bytes: int, with_initial_state: bool,
+                               with_final_state: bool) -> int | None:
+    """The part of prefill_min_bytes that falls to one kernel of the two-kernel prefill: the
+    chunk-local kernel reads every input once (q, k, v, log_alpha, beta); the state kernel writes
+    o and reads / writes the fp32 states; the varlen chunk map reads cu_seqlens and writes the
+    chunk offsets. The per-(chunk, head) records one kernel writes and the next reads are the split
+    design's intermediates, not the method's work: they show up in measured traffic only."""
+    states = num_seqs * H * Dk * Dv * 4
+    if name.startswith("chunk_local"):
+        return token_heads * ((2 * Dk + Dv) * qkv_bytes + 4 * Dk + 4)
+    if name.startswith("chunk_state"):
+        return token_heads * Dv * qkv_bytes + \
+            states * (int(with_initial_state) + int(with_final_state))
+    if name.startswith("chunk_map"):
+        return 8 * (num_seqs + 1)
+    return None

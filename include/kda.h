@@ -126,7 +126,10 @@ KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, 
  *     KDA_NOALLOC_SCRATCH_BYTES is rejected with KDA_ERR_WORKSPACE before anything is launched.
  *   - Set-up: the first call on a device looks up the device address of the scratch array (with
  *     that device current), so make that first call before any stream capture; the current
- *     device must be the one that owns the pointers.
+ *     device must be the one that owns the pointers. The address is kept for the life of the
+ *     process: resetting the device (cudaDeviceReset, or anything else that destroys and
+ *     re-creates its primary context) leaves it stale, so do not call this entry point on a
+ *     device after resetting it in the same process.
  *   - Sharing: all calls on a device share the one array and it keeps the last call's contents.
  *     Nothing in it needs clearing (every byte a call reads was written earlier in that call),
  *     but calls that overlap on the GPU (different streams, or different host threads) race on

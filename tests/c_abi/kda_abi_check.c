@@ -10,6 +10,14 @@
 #include "kda.h"
 #include "kda_selftest.h"
 
+/* the no-allocation entry point's declaration and its scratch limit are part of the C ABI */
+typedef char kda_noalloc_limit_is_64_mib[(KDA_NOALLOC_SCRATCH_BYTES == ((size_t)64 << 20)) ? 1 : -1];
+static kda_status_t (*const kda_noalloc_entry)(const void*, const void*, const void*, kda_dtype_t,
+                                               const float*, const float*, const float*,
+                                               const int32_t*, int32_t, int32_t, int32_t, int32_t,
+                                               int32_t, int32_t, int32_t, void*, float*,
+                                               kda_stream_t) = kda_chunk_fwd_noalloc;
+
 static int fails = 0;
 #define CHECK(cond)                                          \
   do {                                                       \
@@ -43,6 +51,7 @@ int main(void) {
   CHECK(kda_chunk_fwd(NULL, NULL, NULL, KDA_DTYPE_F32, NULL, NULL, NULL, NULL, 0, 0, 0, 1, 32, 32,
                       32, NULL, NULL, NULL, 0, NULL) == KDA_OK);
   CHECK(kda_selftest_wait_timeout(0, NULL) == KDA_ERR_INVALID_ARG);
+  CHECK(kda_noalloc_entry != NULL);
   if (fails == 0) printf("ok %s\n", kda_version());
   return fails != 0;
 }

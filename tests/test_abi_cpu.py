@@ -275,3 +275,12 @@ def test_oracle_shares_nothing_with_the_library():
         py = f.read()
     for name in ("gated_delta_rule_120_b200", "kda_synth", "csrc", "libkda.so"):
         assert name not in py, name
+
+
+def test_noalloc_limit_matches_the_header():
+    """The binding's copy of the no-allocation scratch limit is the value include/kda.h declares."""
+    with open(os.path.join(ROOT, "include", "kda.h")) as f:
+        m = re.search(r"#define\s+KDA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)",
+                      f.read())
+    assert m, "KDA_NOALLOC_SCRATCH_BYTES not found"
+    assert kda.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

@@ -57,16 +57,17 @@ def test_captured_traffic_follows_the_kernel_sources(tmp_path):
 
     real = bench.kernel_source_hash("chunk_local_tc")
     assert real and bench.kernel_source_hash("no_such_kernel") is None
+    assert bench.kernel_source_hash("chunk_state_tc") == real  # one source list for both kernels
     prof = tmp_path / "profiles"
     prof.mkdir()
-    rec = {"chunk_local_tc": {"workload": "w", "dram_bytes_per_launch": 123,
-                              "source_sha256": real}}
+    rec = {"records": {"chunk_local_tc@w": {"dram_bytes_per_launch": 123,
+                                            "source_sha256": real}}}
     (prof / "traffic.json").write_text(json.dumps(rec))
     path = str(prof / "traffic.json")
     assert bench.captured_traffic("chunk_local_tc", "w", path) == 123
     assert bench.captured_traffic("chunk_local_tc", "other", path) is None
     assert bench.captured_traffic("chunk_state_tc", "w", path) is None
-    rec["chunk_local_tc"]["source_sha256"] = "0" * 64
+    rec["records"]["chunk_local_tc@w"]["source_sha256"] = "0" * 64
     (prof / "traffic.json").write_text(json.dumps(rec))
     assert bench.captured_traffic("chunk_local_tc", "w", path) is None
 
@@ -100,24 +101,39 @@ def test_reference_arm_line_follows_the_contract():
 
 def test_roofline_byte_accounting_matches_the_layouts():
     """The bench's algorithmic bytes, counted by hand from the tensor layouts of the standard
-    prefill (B=2, T=4096, H=32, d=128, bf16, C=64: 4096 (chunk, head) items) and the decode."""
+    prefill (B=2, T=4096, H=32, d=128, bf16, C=64: 4096 (chunk, head) items) and the decode. Each
+    kernel's share is its part of the method's minimum (inputs to the chunk-local kernel, o and
+    the states to the state kernel); the shares add up to the path's minimum, and the records
+    between the kernels count for neither."""
     import kda_synth
     from gated_delta_rule_120_b200 import roofline
 
     spec = kda_synth.STANDARD
+    th = 2 * 4096 * 32
     items = 2 * 4096 // 64 * 32
     per_item_inputs = 3 * 64 * 128 * 2 + 64 * 128 * 4 + 64 * 4  # q, k, v bf16; log alpha; beta
     assert per_item_inputs == 82_176
-    rec = 74_240
-    assert bench.prefill_kernel_bytes("chunk_local_tc", spec, 128, rec) == \
-        items * (per_item_inputs + rec)
+    dims = (th, 2, 32, 128, 128, 2, True, True)
+    k1 = roofline.prefill_kernel_share_bytes("chunk_local_tc", *dims)
+    assert k1 == items * per_item_inputs
     o_bytes = 2 * 4096 * 32 * 128 * 2
     state = 2 * 32 * 128 * 128 * 4
-    assert bench.prefill_kernel_bytes("chunk_state_tc", spec, 128, rec) == \
-        items * rec + o_bytes + 2 * state  # initial state read, final state written
-    # the path's minimum: 1540 B per token-head plus the two states
-    assert roofline.prefill_min_bytes(2 * 4096 * 32, 2, 32, 128, 128, 2, True, True) == \
-        2 * 4096 * 32 * 1540 + 2 * state
+    k2 = roofline.prefill_kernel_share_bytes("chunk_state_tc", *dims)
+    assert k2 == o_bytes + 2 * state  # o written, initial state read, final state written
+    # the path's minimum: 1540 B per token-head plus the two states = the two shares
+    assert roofline.prefill_min_bytes(*dims) == th * 1540 + 2 * state == k1 + k2
+    assert roofline.prefill_kernel_share_bytes("something_else", *dims) is None
+    # the roofline block of a step: path frac from the path bytes, kernel fracs from the shares
+    prof = [{"name": "chunk_local_tc", "launches": 4, "total_ms": 0.8},
+            {"name": "chunk_state_tc", "launches": 4, "total_ms": 0.4}]
+    roof = bench.prefill_roofline(spec, 0.3, prof, 4, 6543.4, "measured")
+    assert roof["algorithmic_bytes"] == k1 + k2
+    assert roof["achieved"] == pytest.approx((k1 + k2) / 0.3e-3 / 1e9)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / 6543.4)
+    assert roof["dominant_kernel"] == "chunk_local_tc"
+    kk = {k["name"]: k for k in roof["kernels"]}
+    assert kk["chunk_local_tc"]["achieved_gbs"] == pytest.approx(k1 / 0.2e-3 / 1e9)
+    assert kk["chunk_state_tc"]["share"] == pytest.approx(1 / 3)
     # decode: every state read once and written once
     assert roofline.decode_state_bytes(256, 32, 128, 128) == 2 * 256 * 32 * 128 * 128 * 4
 

@@ -1,4 +1,6 @@
 """GPU parity of kda_chunk_fwd (chunkwise prefill) against the fp64 oracle, through the C ABI."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -184,21 +186,39 @@ def _sampled_heads_check(spec, seed, dev, heads, seqs=None):
         worst_s = max(worst_s, rel_err(s[n:n + 1][:, heads], s_ref))
     assert worst_o <= TOL_BF16_O, worst_o
     assert worst_s <= TOL_BF16_S, worst_s
-    return inp, o, s
+    return worst_o, worst_s
 
 
-def test_bf16_long_prefill_sampled(cuda_device):
-    """B=1, T=131072, H=32: two heads recomputed by the oracle end to end (o and final state)."""
-    _sampled_heads_check(kda_synth.LONG, 1002, cuda_device, heads=[0, 17])
+# eight of the 32 heads, spread over the head index range
+SAMPLED_HEADS = [0, 5, 9, 14, 17, 22, 26, 31]
+
+# Final-state error (max-abs / max |S| over the sampled heads) of the bf16 tensor-core path
+# against the fp64 oracle as the sequence grows, slow-decay distributions of the long prefill.
+# The bound is the bf16 tolerance; the ceilings are the values measured on a B200 with headroom,
+# so that a precision regression (an operand rounded once more, a carry leaving fp32) shows up
+# long before the tolerance is reached.
+STATE_ERR_CEILING = {4096: 2e-2, 32768: 2e-2, 131072: 2e-2}
+
+
+@pytest.mark.parametrize("T", [4096, 32768, 131072])
+def test_bf16_state_error_vs_sequence_length(cuda_device, T):
+    """B=1, H=32, slow decay: the state carried over T / 64 chunk steps (fp32 carry, bf16
+    operands in the correction terms) stays within its ceiling; T = 131072 is the long prefill
+    workload itself (same seed)."""
+    spec = kda_synth.LONG if T == kda_synth.LONG.T else \
+        dataclasses.replace(kda_synth.LONG, name=f"prefill_B1_T{T}_H32_d128", T=T)
+    eo, es = _sampled_heads_check(spec, 1002, cuda_device, heads=SAMPLED_HEADS)
+    print(f"STATE_ERR T={T} o={eo:.3e} state={es:.3e}")
+    assert es <= STATE_ERR_CEILING[T], es
 
 
 def test_bf16_varlen_workload_sampled(cuda_device):
     """16 packed sequences with log-uniform lengths in [256, 32768]: the shortest and the longest
-    sequence, two heads each, recomputed by the oracle."""
+    sequence, eight heads each, recomputed by the oracle."""
     spec = kda_synth.varlen_spec(1003)
     lens = np.asarray(spec.seqlens)
     pick = [int(np.argmin(lens)), int(np.argmax(lens))]
-    _sampled_heads_check(spec, 1003, cuda_device, heads=[3, 30], seqs=pick)
+    _sampled_heads_check(spec, 1003, cuda_device, heads=SAMPLED_HEADS, seqs=pick)
 
 
 # ------------------------------------------------------------------ invariants and edge cases

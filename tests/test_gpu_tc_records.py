@@ -45,11 +45,13 @@ def chunk_reference(k, q, v, la, beta, L):
     G = np.zeros((C, 128)); b = np.zeros(C)
     K[:L], Q[:L], V[:L], G[:L], b[:L] = k, q, v, la, beta
     g = np.cumsum(G, axis=0)
-    ratio = np.exp(g[:, None, :] - g[None, :, :])  # [r, i, c] = gamma_r / gamma_i
-    akk = np.einsum("rc,ic,ric->ri", K, K, np.where(np.arange(C)[:, None, None] >=
-                                                    np.arange(C)[None, :, None], ratio, 0.0))
-    aqk = np.einsum("rc,ic,ric->ri", Q, K, np.where(np.arange(C)[:, None, None] >=
-                                                    np.arange(C)[None, :, None], ratio, 0.0))
+    # [r, i, c] = gamma_r / gamma_i on the causal pairs i <= r (exponent <= 0), 0 elsewhere: the
+    # mask is applied before the exponential, so no masked pair overflows and a NaN would show
+    causal = np.arange(C)[:, None, None] >= np.arange(C)[None, :, None]
+    ratio = np.zeros((C, C, 128))
+    np.exp(g[:, None, :] - g[None, :, :], out=ratio, where=np.broadcast_to(causal, ratio.shape))
+    akk = np.einsum("rc,ic,ric->ri", K, K, ratio)
+    aqk = np.einsum("rc,ic,ric->ri", Q, K, ratio)
     A = np.tril(b[:, None] * akk, -1)
     M = np.linalg.inv(np.eye(C) + A) * b[None, :]
     W = M @ (np.exp(g) * K)

@@ -97,6 +97,9 @@ __device__ __forceinline__ float4 lds4(const float* base, int r, int c4) {  // c
 __device__ __forceinline__ void sts4(float* base, int r, int c4, float4 v) {
   *reinterpret_cast<float4*>(base + sidx(r, 4 * c4)) = v;
 }
+// the level product Y (fp32 32 x 32) of the inverse: column groups of four XOR-ed by (row % 8),
+// so that eight consecutive rows of one group, or eight groups of one row, hit distinct banks
+__device__ __forceinline__ int yidx(int r, int c4) { return r * 32 + 4 * (c4 ^ (r & 7)); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
@@ -668,24 +671,26 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       sts4(sT, 16 * (bb + 1) + rr, 4 * bb + cq, make_float4(-t.x, -t.y, -t.z, -t.w));
     }
     __syncthreads();
-    // stage 3: Y = A21 T11 (32 x 32, K over k >= c), one strip per thread
-    const int r3 = tid >> 3, c3 = tid & 7;  // row 0..31, column group 0..7
+    // stage 3: Y = A21 T11 (32 x 32, K over k >= c); warp = column group (so the triangular
+    // extent of the sum is the same across the warp), lane = row
     {
+      const int c3w = warp, r3w = lane;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int k4 = 0; k4 < 8; ++k4) {
-        if (k4 < c3) continue;
-        const float4 a = lds4(sA, 32 + r3, k4);
-        const float4 t0 = lds4(sT, 4 * k4 + 0, c3), t1 = lds4(sT, 4 * k4 + 1, c3);
-        const float4 t2 = lds4(sT, 4 * k4 + 2, c3), t3 = lds4(sT, 4 * k4 + 3, c3);
+        if (k4 < c3w) continue;
+        const float4 a = lds4(sA, 32 + r3w, k4);
+        const float4 t0 = lds4(sT, 4 * k4 + 0, c3w), t1 = lds4(sT, 4 * k4 + 1, c3w);
+        const float4 t2 = lds4(sT, 4 * k4 + 2, c3w), t3 = lds4(sT, 4 * k4 + 3, c3w);
         acc.x += a.x * t0.x + a.y * t1.x + a.z * t2.x + a.w * t3.x;
         acc.y += a.x * t0.y + a.y * t1.y + a.z * t2.y + a.w * t3.y;
         acc.z += a.x * t0.z + a.y * t1.z + a.z * t2.z + a.w * t3.z;
         acc.w += a.x * t0.w + a.y * t1.w + a.z * t2.w + a.w * t3.w;
       }
-      *reinterpret_cast<float4*>(sX + r3 * 32 + 4 * c3) = acc;
+      *reinterpret_cast<float4*>(sX + yidx(r3w, c3w)) = acc;
     }
     __syncthreads();
+    const int r3 = tid >> 3, c3 = tid & 7;
     // T21 = -T22 Y (K over k <= r)
     {
       float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -693,8 +698,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       for (int k4 = 0; k4 < 8; ++k4) {
         if (4 * k4 > r3) continue;
         const float4 a = lds4(sT, 32 + r3, 8 + k4);
-        const float4* yr = reinterpret_cast<const float4*>(sX + (4 * k4) * 32 + 4 * c3);
-        const float4 y0 = yr[0], y1 = yr[8], y2 = yr[16], y3 = yr[24];
+        const float4 y0 = *reinterpret_cast<const float4*>(sX + yidx(4 * k4 + 0, c3));
+        const float4 y1 = *reinterpret_cast<const float4*>(sX + yidx(4 * k4 + 1, c3));
+        const float4 y2 = *reinterpret_cast<const float4*>(sX + yidx(4 * k4 + 2, c3));
+        const float4 y3 = *reinterpret_cast<const float4*>(sX + yidx(4 * k4 + 3, c3));
         t.x += a.x * y0.x + a.y * y1.x + a.z * y2.x + a.w * y3.x;
         t.y += a.x * y0.y + a.y * y1.y + a.z * y2.y + a.w * y3.y;
         t.z += a.x * y0.z + a.y * y1.z + a.z * y2.z + a.w * y3.z;

@@ -194,10 +194,10 @@ SAMPLED_HEADS = [0, 5, 9, 14, 17, 22, 26, 31]
 
 # Final-state error (max-abs / max |S| over the sampled heads) of the bf16 tensor-core path
 # against the fp64 oracle as the sequence grows, slow-decay distributions of the long prefill.
-# The bound is the bf16 tolerance; the ceilings are the values measured on a B200 with headroom,
-# so that a precision regression (an operand rounded once more, a carry leaving fp32) shows up
-# long before the tolerance is reached.
-STATE_ERR_CEILING = {4096: 2e-2, 32768: 2e-2, 131072: 2e-2}
+# The bound is the bf16 tolerance (2e-2); the ceilings are the values measured on a B200 (3.85e-3,
+# 3.51e-3, 3.95e-3) with 50 % headroom, so that a precision regression (an operand rounded once
+# more, a carry leaving fp32) shows up long before the tolerance is reached.
+STATE_ERR_CEILING = {4096: 6e-3, 32768: 6e-3, 131072: 6e-3}
 
 
 @pytest.mark.parametrize("T", [4096, 32768, 131072])

@@ -891,7 +891,9 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 // Column-layout variant of the streaming recurrent mode (d_k = d_v = 128, T tokens that fit the
 // shared-memory budget): the same producer warp and two-stage ring, eight compute warps, each
 // owning 16 columns of the state over all 128 rows: lane = (row group rg of 16 rows, column quad
-// cq), so a thread holds a 16 x 4 tile in registers. A token's reductions
+// cq), so a thread holds a 16 x 4 tile in registers, as packed fp32 pairs of adjacent rows: the
+// decay, the two reductions and the update each take one fma/mul .f32x2 per row pair and column,
+// with the rows' decays, keys and queries read from shared memory as pairs. A token's reductions
 // e_j = sum_i S'[i][j] k_i and p_j = sum_i S'[i][j] q_i then end in three lane exchanges inside
 // the warp instead of a block-wide reduction, so the token loop has no barrier. The per-token decays exp(log alpha),
 // k.q, the norms and beta are computed for all T tokens of an item in one pass before it, and
@@ -1082,15 +1084,28 @@ __global__ void __launch_bounds__(kRcThreads, 1)
       if (it + 1 < count) stage_scalars(it + 1);  // the other buffer; read after this barrier
       sm100::named_barrier_sync(1, kRcCompute);
 
-      float4 S[16];
+      // the thread's 16 x 4 state tile as 8 row pairs x 4 columns: SP[4 jr + c] holds
+      // (S[r0 + 2 jr][c0 + c], S[r0 + 2 jr + 1][c0 + c]), so the per-row decays, keys and queries
+      // enter the packed products as adjacent pairs straight from shared memory
+      f32x2 SP[32];
       float* Sst = reinterpret_cast<float*>(st);
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) S[ii] = *reinterpret_cast<const float4*>(Sst + (r0 + ii) * D + c0);
+      for (int jr = 0; jr < 8; ++jr) {
+        const float4 lo = *reinterpret_cast<const float4*>(Sst + (r0 + 2 * jr) * D + c0);
+        const float4 hi = *reinterpret_cast<const float4*>(Sst + (r0 + 2 * jr + 1) * D + c0);
+        SP[4 * jr + 0] = f2_pack(lo.x, hi.x);
+        SP[4 * jr + 1] = f2_pack(lo.y, hi.y);
+        SP[4 * jr + 2] = f2_pack(lo.z, hi.z);
+        SP[4 * jr + 3] = f2_pack(lo.w, hi.w);
+      }
       for (int t = 0; t < T; ++t) {
         const float* al = s_alpha + t * D + r0;
         const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + r0;
         const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + r0;
-        float4 e = make_float4(0.f, 0.f, 0.f, 0.f), p = e;
+        f32x2 ep[4], pp[4];  // per column: partial sums over the even and the odd rows
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ep[c] = pp[c] = 0ull;
+        f32x2 kp[8];  // (k_r, k_r+1) pairs, kept for the update
 #pragma unroll
         for (int i8 = 0; i8 < 2; ++i8) {  // S' = Diag(alpha) S; e, p over this thread's rows
           float a[8], kk[8], qv8[8];
@@ -1098,14 +1113,27 @@ __global__ void __launch_bounds__(kRcThreads, 1)
           load8_in(kv + 8 * i8, kk);
           load8_in(qv + 8 * i8, qv8);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float4& sv = S[8 * i8 + u];
-            sv.x *= a[u]; sv.y *= a[u]; sv.z *= a[u]; sv.w *= a[u];
-            e.x = fmaf(sv.x, kk[u], e.x); e.y = fmaf(sv.y, kk[u], e.y);
-            e.z = fmaf(sv.z, kk[u], e.z); e.w = fmaf(sv.w, kk[u], e.w);
-            p.x = fmaf(sv.x, qv8[u], p.x); p.y = fmaf(sv.y, qv8[u], p.y);
-            p.z = fmaf(sv.z, qv8[u], p.z); p.w = fmaf(sv.w, qv8[u], p.w);
+          for (int u = 0; u < 4; ++u) {
+            const int jr = 4 * i8 + u;
+            const f32x2 ap = f2_pack(a[2 * u], a[2 * u + 1]);
+            kp[jr] = f2_pack(kk[2 * u], kk[2 * u + 1]);
+            const f32x2 qp = f2_pack(qv8[2 * u], qv8[2 * u + 1]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              SP[4 * jr + c] = f2_mul(SP[4 * jr + c], ap);
+              ep[c] = f2_fma(SP[4 * jr + c], kp[jr], ep[c]);
+              pp[c] = f2_fma(SP[4 * jr + c], qp, pp[c]);
+            }
           }
+        }
+        float4 e, p;
+        {
+          const float2 e0 = f2_unpack(ep[0]), e1 = f2_unpack(ep[1]), e2 = f2_unpack(ep[2]),
+                       e3 = f2_unpack(ep[3]);
+          const float2 p0 = f2_unpack(pp[0]), p1 = f2_unpack(pp[1]), p2 = f2_unpack(pp[2]),
+                       p3 = f2_unpack(pp[3]);
+          e = make_float4(e0.x + e0.y, e1.x + e1.y, e2.x + e2.y, e3.x + e3.y);
+          p = make_float4(p0.x + p0.y, p1.x + p1.y, p2.x + p2.y, p3.x + p3.y);
         }
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {  // over the eight row groups of the warp
@@ -1128,21 +1156,20 @@ __global__ void __launch_bounds__(kRcThreads, 1)
           *reinterpret_cast<float4*>(s_y + t * D + c0) =
               make_float4(p.x * tk.z + tk.x * u.x, p.y * tk.z + tk.x * u.y,
                           p.z * tk.z + tk.x * u.z, p.w * tk.z + tk.x * u.w);
-        const float4 ku = make_float4(tk.y * u.x, tk.y * u.y, tk.y * u.z, tk.y * u.w);
+        const f32x2 ku[4] = {f2_pack(tk.y * u.x, tk.y * u.x), f2_pack(tk.y * u.y, tk.y * u.y),
+                             f2_pack(tk.y * u.z, tk.y * u.z), f2_pack(tk.y * u.w, tk.y * u.w)};
 #pragma unroll
-        for (int i8 = 0; i8 < 2; ++i8) {  // S = S' + k (beta (v - e))^T
-          float kk[8];
-          load8_in(kv + 8 * i8, kk);
+        for (int jr = 0; jr < 8; ++jr)  // S = S' + k (beta (v - e))^T
 #pragma unroll
-          for (int u8 = 0; u8 < 8; ++u8) {
-            float4& sv = S[8 * i8 + u8];
-            sv.x = fmaf(kk[u8], ku.x, sv.x); sv.y = fmaf(kk[u8], ku.y, sv.y);
-            sv.z = fmaf(kk[u8], ku.z, sv.z); sv.w = fmaf(kk[u8], ku.w, sv.w);
-          }
-        }
+          for (int c = 0; c < 4; ++c) SP[4 * jr + c] = f2_fma(kp[jr], ku[c], SP[4 * jr + c]);
       }
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) *reinterpret_cast<float4*>(Sst + (r0 + ii) * D + c0) = S[ii];
+      for (int jr = 0; jr < 8; ++jr) {
+        const float2 s0 = f2_unpack(SP[4 * jr + 0]), s1 = f2_unpack(SP[4 * jr + 1]);
+        const float2 s2 = f2_unpack(SP[4 * jr + 2]), s3 = f2_unpack(SP[4 * jr + 3]);
+        *reinterpret_cast<float4*>(Sst + (r0 + 2 * jr) * D + c0) = make_float4(s0.x, s1.x, s2.x, s3.x);
+        *reinterpret_cast<float4*>(Sst + (r0 + 2 * jr + 1) * D + c0) = make_float4(s0.y, s1.y, s2.y, s3.y);
+      }
       sm100::named_barrier_sync(1, kRcCompute);  // s_y complete
       // outputs: one warp per token row, four columns per lane (head-wise norm x gate if fused)
       for (int t = warp; t < T; t += kRcCompute / 32) {

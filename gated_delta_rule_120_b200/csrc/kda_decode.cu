@@ -893,13 +893,21 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 // owning 16 columns of the state over all 128 rows: lane = (row group rg of 16 rows, column quad
 // cq), so a thread holds a 16 x 4 tile in registers, as packed fp32 pairs of adjacent rows: the
 // decay, the two reductions and the update each take one fma/mul .f32x2 per row pair and column,
-// with the rows' decays, keys and queries read from shared memory as pairs. A token's reductions
+// with the rows' decays, keys and queries read from shared memory as pairs. For T <= 16, an item
+// whose rows decay by less than e^-60 over the call runs in the running-decay form: with D_t the
+// product of the row's decays from the item start, S_t = Diag(D_t) Shat_t, so
+// e = Shat^T (D_t k), p = Shat^T (D_t q) and Shat += (k / D_t) (beta (v - e))^T need no per-token
+// decay of the state; D_t k, D_t q and k / D_t are formed once per token before the loop and the
+// state is scaled by D_T after it (fp32 throughout: every term keeps its relative precision).
+// A token's reductions
 // e_j = sum_i S'[i][j] k_i and p_j = sum_i S'[i][j] q_i then end in three lane exchanges inside
 // the warp instead of a block-wide reduction, so the token loop has no barrier. The per-token decays exp(log alpha),
 // k.q, the norms and beta are computed for all T tokens of an item in one pass before it, and
 // the outputs (with the head-wise norm and gate when fused) are written by one pass after it.
 // ---------------------------------------------------------------------------------------------
 constexpr int kRcCompute = 256;                // 8 compute warps
+// the running-decay form keeps 1 / D_t below e^60: its terms stay far inside fp32's range
+constexpr float kRcLazyLimit = 60.f;
 constexpr int kRcThreads = kRcCompute + 32;    // + producer warp
 constexpr int kRcD = 128;
 
@@ -935,6 +943,10 @@ __global__ void __launch_bounds__(kRcThreads, 1)
   float* s_beta = reinterpret_cast<float*>(s_tok + kRsMaxT);     // [2][kRsMaxT + 2]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_beta + 2 * (kRsMaxT + 2));  // [kRsStages]
   uint64_t* computed = full + kRsStages;                                     // [kRsStages]
+  // running-decay form (T <= kRsMaxT / 2): D_t k, D_t q in the decay area, k / D_t beside the
+  // outputs; D_T per row and the item's form flag after the barriers
+  float* s_dT = reinterpret_cast<float*>(computed + kRsStages);  // [D]
+  int* s_lazy = reinterpret_cast<int*>(s_dT + D);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int first = blockIdx.x, stride = gridDim.x;
@@ -1039,16 +1051,63 @@ __global__ void __launch_bounds__(kRcThreads, 1)
         continue;
       }
       uint8_t* st = stages + (size_t)s * lay.stage_bytes;
-      // pre-pass: every token's decays; k.q, inverse norms and beta per token (one warp each)
-      for (int e = tid; e < T * D; e += kRcCompute) {
-        const int t = e >> 7, i = e & (D - 1);
-        float la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row)[i];
-        if (kFused && fz.A_log) {
-          const float bias = lay.bias_bytes ? reinterpret_cast<const float*>(st + lay.bias_off)[i]
-                                            : 0.f;
-          la = sb[kRsMaxT] * softplus_f(la + bias);
+      // pre-pass: the running log decay of every row over the item decides the form; then either
+      // every token's decays (token form) or the scaled keys and queries (running-decay form);
+      // k.q, inverse norms and beta per token (one warp each)
+      float* s_khat = s_alpha;
+      float* s_qhat = s_alpha + T * D;
+      float* s_ktil = s_y + (kRsMaxT / 2) * D;
+      if (tid == 0) *s_lazy = T <= kRsMaxT / 2;
+      sm100::named_barrier_sync(1, kRcCompute);
+      if (tid < D) {
+        float G = 0.f;
+        for (int t = 0; t < T; ++t) {
+          float la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row)[tid];
+          if (kFused && fz.A_log) {
+            const float bias = lay.bias_bytes
+                                   ? reinterpret_cast<const float*>(st + lay.bias_off)[tid]
+                                   : 0.f;
+            la = sb[kRsMaxT] * softplus_f(la + bias);
+          }
+          G += la;
         }
-        s_alpha[e] = expf(la);
+        s_dT[tid] = expf(G);
+        if (!(G >= -kRcLazyLimit)) *s_lazy = 0;
+      }
+      sm100::named_barrier_sync(1, kRcCompute);
+      const bool lazy = *s_lazy != 0;
+      if (lazy) {
+        if (tid < D) {  // row tid: D_t = exp(sum of the decays up to t)
+          float G = 0.f;
+          for (int t = 0; t < T; ++t) {
+            float la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row)[tid];
+            if (kFused && fz.A_log) {
+              const float bias = lay.bias_bytes
+                                     ? reinterpret_cast<const float*>(st + lay.bias_off)[tid]
+                                     : 0.f;
+              la = sb[kRsMaxT] * softplus_f(la + bias);
+            }
+            G += la;
+            const float Dt = expf(G), Di = expf(-G);
+            const float kx = to_f32(reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row)[tid]);
+            const float qx = to_f32(reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row)[tid]);
+            s_khat[t * D + tid] = Dt * kx;
+            s_qhat[t * D + tid] = Dt * qx;
+            s_ktil[t * D + tid] = Di * kx;
+          }
+        }
+      } else {
+        for (int e = tid; e < T * D; e += kRcCompute) {
+          const int t = e >> 7, i = e & (D - 1);
+          float la = reinterpret_cast<const float*>(st + lay.la_off + t * lay.la_row)[i];
+          if (kFused && fz.A_log) {
+            const float bias = lay.bias_bytes
+                                   ? reinterpret_cast<const float*>(st + lay.bias_off)[i]
+                                   : 0.f;
+            la = sb[kRsMaxT] * softplus_f(la + bias);
+          }
+          s_alpha[e] = expf(la);
+        }
       }
       for (int t = warp; t < T; t += kRcCompute / 32) {
         float kx[4], qx[4];
@@ -1099,13 +1158,34 @@ __global__ void __launch_bounds__(kRcThreads, 1)
         SP[4 * jr + 3] = f2_pack(lo.w, hi.w);
       }
       for (int t = 0; t < T; ++t) {
-        const float* al = s_alpha + t * D + r0;
-        const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + r0;
-        const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + r0;
+        f32x2 kp[8];  // (k_r, k_r+1) pairs for the update: k / D_t (running form) or k
         f32x2 ep[4], pp[4];  // per column: partial sums over the even and the odd rows
 #pragma unroll
         for (int c = 0; c < 4; ++c) ep[c] = pp[c] = 0ull;
-        f32x2 kp[8];  // (k_r, k_r+1) pairs, kept for the update
+        if (lazy) {
+          const float4* kh = reinterpret_cast<const float4*>(s_khat + t * D + r0);
+          const float4* qh = reinterpret_cast<const float4*>(s_qhat + t * D + r0);
+          const float4* kt4 = reinterpret_cast<const float4*>(s_ktil + t * D + r0);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float4 a = kh[m], b = qh[m], c4 = kt4[m];
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              const int jr = 2 * m + hlf;
+              const f32x2 khp = hlf ? f2_pack(a.z, a.w) : f2_pack(a.x, a.y);
+              const f32x2 qhp = hlf ? f2_pack(b.z, b.w) : f2_pack(b.x, b.y);
+              kp[jr] = hlf ? f2_pack(c4.z, c4.w) : f2_pack(c4.x, c4.y);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                ep[c] = f2_fma(SP[4 * jr + c], khp, ep[c]);
+                pp[c] = f2_fma(SP[4 * jr + c], qhp, pp[c]);
+              }
+            }
+          }
+        } else {
+        const float* al = s_alpha + t * D + r0;
+        const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + r0;
+        const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + r0;
 #pragma unroll
         for (int i8 = 0; i8 < 2; ++i8) {  // S' = Diag(alpha) S; e, p over this thread's rows
           float a[8], kk[8], qv8[8];
@@ -1125,6 +1205,7 @@ __global__ void __launch_bounds__(kRcThreads, 1)
               pp[c] = f2_fma(SP[4 * jr + c], qp, pp[c]);
             }
           }
+        }
         }
         float4 e, p;
         {
@@ -1162,6 +1243,14 @@ __global__ void __launch_bounds__(kRcThreads, 1)
         for (int jr = 0; jr < 8; ++jr)  // S = S' + k (beta (v - e))^T
 #pragma unroll
           for (int c = 0; c < 4; ++c) SP[4 * jr + c] = f2_fma(kp[jr], ku[c], SP[4 * jr + c]);
+      }
+      if (lazy) {  // S = Diag(D_T) Shat
+#pragma unroll
+        for (int jr = 0; jr < 8; ++jr) {
+          const f32x2 dp = f2_pack(s_dT[r0 + 2 * jr], s_dT[r0 + 2 * jr + 1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) SP[4 * jr + c] = f2_mul(SP[4 * jr + c], dp);
+        }
       }
 #pragma unroll
       for (int jr = 0; jr < 8; ++jr) {
@@ -1278,7 +1367,7 @@ cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, 
   const size_t smem_cols = (size_t)kRsStages * lay.stage_bytes +
                            2 * (size_t)kRsMaxT * kRcD * sizeof(float) + kRsMaxT * sizeof(float4) +
                            2 * (kRsMaxT + 2) * sizeof(float) + 2 * kRsStages * sizeof(uint64_t) +
-                           128;
+                           (kRcD + 4) * sizeof(float) + 128;
   if (Dk == kRcD && Dv == kRcD && (!fz.ow || al16(fz.ow)) && smem_cols <= 227u * 1024u) {
     ProfileScope prof(fused ? "recurrent_cols_fused" : "recurrent_cols", stream);
     if (dt == KDA_DTYPE_BF16)

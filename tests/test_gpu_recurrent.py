@@ -73,3 +73,29 @@ def test_recurrent_fwd_index_beyond_pool_is_reported(cuda_device):
     assert kda.kda_last_device_error() == kda.KDA_ERR_INVALID_ARG
     assert torch.isfinite(pool).all()
     assert kda.kda_last_device_error() == kda.KDA_OK
+
+
+def test_recurrent_fwd_strong_and_mild_decays_in_one_launch(cuda_device):
+    """Items whose decay over the call stays mild and items whose rows decay below e^-60 within
+    the call (the kernel keeps the second kind on its token-by-token form) in one launch, against
+    the oracle at the recurrent mode's tolerances."""
+    N, T, H = 8, 12, 3
+    x = _inputs(N, T, H, 128, 128, "bf16", 670, cuda_device)
+    la = x["log_alpha"].clone()
+    la[1::2] *= 25.0  # odd sequences: about -40 per token on average over 12 tokens
+    x["log_alpha"] = la
+    g = torch.Generator(device=cuda_device).manual_seed(71)
+    pool = torch.randn((N, H, 128, 128), generator=g, device=cuda_device) * 0.05
+    pool0 = pool.clone()
+    o = kda.kda_recurrent_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool)
+    torch.cuda.synchronize()
+    assert kda.kda_last_device_error() == kda.KDA_OK
+    cu = np.arange(N + 1, dtype=np.int64) * T
+    o_ref, s_ref = oracle.recurrent(*(x[n_].cpu().reshape(N * T, H, -1) if n_ != "beta"
+                                      else x[n_].cpu().reshape(N * T, H)
+                                      for n_ in ("q", "k", "v", "log_alpha", "beta")),
+                                    initial_state=pool0.cpu(), cu_seqlens=cu)
+    assert torch.isfinite(pool).all()
+    assert rel_err(o.reshape(-1, H, 128), o_ref) <= TOL_DECODE_O
+    assert rel_err(pool, s_ref) <= TOL_DECODE_S
+

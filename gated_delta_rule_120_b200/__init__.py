@@ -31,7 +31,8 @@ import torch
 from . import roofline  # noqa: F401  (work counts used by the benchmark)
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libkda.so")
+# KDA_LIBRARY selects another build of the library (e.g. the bounds-checked libkda_checked.so)
+LIB_PATH = os.environ.get("KDA_LIBRARY") or os.path.join(_PKG, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED = 0, 1, 2
 KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_WORKSPACE = 3, 4, 5
@@ -43,7 +44,7 @@ ABI_SYMBOLS = ("kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size
                "kda_profile_enable", "kda_profile_read", "kda_chunk_fwd_noalloc",
                "kda_recurrent_fwd", "kda_chunk_fwd_fused", "kda_recurrent_fwd_fused",
                "kda_chunk_bwd_workspace_size", "kda_chunk_bwd", "kda_recurrent_step_fused",
-               "kda_selftest_wait_timeout")
+               "kda_selftest_wait_timeout", "kda_selftest_bounds")
 
 
 class Fusion(ctypes.Structure):
@@ -125,6 +126,8 @@ def lib() -> ctypes.CDLL:
             L.kda_profile_read.restype = ctypes.c_int
             L.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
             L.kda_selftest_wait_timeout.restype = ctypes.c_int
+            L.kda_selftest_bounds.argtypes = [vp, sz, vp]
+            L.kda_selftest_bounds.restype = ctypes.c_int
             _lib = L
     return _lib
 

@@ -10,6 +10,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkda.so")
+# the bounds-checked build (-DKDA_BOUNDS_CHECK): every global access of the prefill, decode and
+# recurrent-mode kernels is tested against the extent of its buffer (a debugging substitute for a
+# memory checker); load it with KDA_LIBRARY=<path> before importing the package
+LIB_CHECKED = os.path.join(PKG, "libkda_checked.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -27,28 +31,31 @@ def sources() -> list[str]:
                   glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/kda_lib.cu into gated_delta_rule_120_b200/libkda.so (no-op when current)."""
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-I", CSRC,
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile csrc/kda_lib.cu into gated_delta_rule_120_b200/libkda.so (no-op when current);
+    with ``checked`` the bounds-checked build libkda_checked.so instead."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [NVCC, *NVCC_FLAGS, *(["-DKDA_BOUNDS_CHECK"] if checked else []),
+           "-I", os.path.join(ROOT, "include"), "-I", CSRC,
            "-o", tmp, os.path.join(CSRC, "kda_lib.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                checked="--checked" in sys.argv))

@@ -79,6 +79,21 @@ WsLayout prefill_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
 
 kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// one entry of a call's bounds table (bytes = 0 leaves the role empty: any access is reported)
+inline void set_extent(BoundsTable& t, BufRole role, const void* base, size_t bytes) {
+  t.base[role] = bytes ? base : nullptr;
+  t.bytes[role] = bytes;
+}
+
+// the extents of the fusion descriptor's buffers
+void fusion_extents(BoundsTable& t, const Fusion& fz, size_t gate_bytes, int32_t H, int32_t Dk,
+                    int32_t Dv) {
+  set_extent(t, kBufALog, fz.A_log, fz.A_log ? (size_t)H * 4 : 0);
+  set_extent(t, kBufDtBias, fz.dt_bias, fz.dt_bias ? (size_t)H * Dk * 4 : 0);
+  set_extent(t, kBufGate, fz.og, fz.og ? gate_bytes : 0);
+  set_extent(t, kBufNormW, fz.ow, fz.ow ? (size_t)Dv * 4 : 0);
+}
+
 // Backward pass: chunk of 32 tokens, fp32 arithmetic for both input dtypes.
 constexpr int32_t kBwdChunk = 32;
 
@@ -125,6 +140,17 @@ BwdLayout backward_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t D
 }
 
 }  // namespace
+
+cudaError_t register_bounds(const BoundsTable& t, cudaStream_t stream) {
+#ifdef KDA_BOUNDS_CHECK
+  return cudaMemcpyToSymbolAsync(g_bounds, &t, sizeof(t), 0, cudaMemcpyHostToDevice, stream);
+#else
+  (void)t;
+  (void)stream;
+  return cudaSuccess;
+#endif
+}
+
 }  // namespace kda
 
 using namespace kda;
@@ -199,6 +225,13 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtyp
     return KDA_ERR_WORKSPACE;
 
   cudaStream_t stream = (cudaStream_t)stream_;
+  if (kBoundsChecked) {  // the varlen chunk map is the instrumented kernel of this call
+    BoundsTable t = {};
+    set_extent(t, kBufWork, workspace, workspace_bytes);
+    set_extent(t, kBufCuSeqlens, cu_seqlens, varlen ? ((size_t)N + 1) * 4 : 0);
+    st = from_cuda(register_bounds(t, stream));
+    if (st != KDA_OK) return st;
+  }
   char* ws = (char*)workspace;
   int32_t* valid = (int32_t*)ws;
   int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
@@ -304,6 +337,24 @@ kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v, kda_dty
     return KDA_ERR_WORKSPACE;
 
   cudaStream_t stream = (cudaStream_t)stream_;
+  if (kBoundsChecked) {
+    BoundsTable t = {};
+    const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4, th = (size_t)tokens * H;
+    const size_t states = (size_t)N * H * Dk * Dv * 4;
+    set_extent(t, kBufQ, q, th * Dk * es);
+    set_extent(t, kBufK, k, th * Dk * es);
+    set_extent(t, kBufV, v, th * Dv * es);
+    set_extent(t, kBufO, o, th * Dv * es);
+    set_extent(t, kBufLogAlpha, log_alpha, th * Dk * 4);
+    set_extent(t, kBufBeta, beta, th * 4);
+    set_extent(t, kBufInitial, initial_state, initial_state ? states : 0);
+    set_extent(t, kBufFinal, final_state, final_state ? states : 0);
+    set_extent(t, kBufWork, workspace, workspace_bytes);
+    set_extent(t, kBufCuSeqlens, cu_seqlens, varlen ? ((size_t)N + 1) * 4 : 0);
+    fusion_extents(t, fz, th * Dv * es, H, Dk, Dv);
+    st = from_cuda(register_bounds(t, stream));
+    if (st != KDA_OK) return st;
+  }
   char* ws = (char*)workspace;
   int32_t* valid = (int32_t*)ws;
   int32_t* chunk_off = (int32_t*)(ws + lay.chunk_off_base);
@@ -365,6 +416,20 @@ kda_status_t recurrent_step_impl(const void* q, const void* k, const void* v, kd
     return KDA_ERR_INVALID_ARG;
   if (fz && fz->onorm && ((fz->og && !aligned(fz->og, es)) || (fz->ow && !aligned(fz->ow, 16))))
     return KDA_ERR_INVALID_ARG;
+  if (kBoundsChecked) {
+    BoundsTable t = {};
+    const size_t nh = (size_t)N * H;
+    set_extent(t, kBufQ, q, nh * Dk * es);
+    set_extent(t, kBufK, k, nh * Dk * es);
+    set_extent(t, kBufV, v, nh * Dv * es);
+    set_extent(t, kBufO, o, nh * Dv * es);
+    set_extent(t, kBufLogAlpha, log_alpha, nh * Dk * 4);
+    set_extent(t, kBufBeta, beta, nh * 4);
+    set_extent(t, kBufState, state, nh * Dk * Dv * 4);
+    if (fz) fusion_extents(t, *fz, nh * Dv * es, H, Dk, Dv);
+    const kda_status_t st = from_cuda(register_bounds(t, (cudaStream_t)stream));
+    if (st != KDA_OK) return st;
+  }
   return from_cuda(launch_decode_step(q, k, v, dt, log_alpha, beta, state, o, N, H, Dk, Dv, fz,
                                       (cudaStream_t)stream));
 }
@@ -388,6 +453,21 @@ kda_status_t recurrent_fwd_impl(const void* q, const void* k, const void* v, kda
       (state_indices && !aligned(state_indices, 4)) || (fz.onorm && fz.og && !aligned(fz.og, es)) ||
       (fz.onorm && fz.ow && !aligned(fz.ow, 16)))
     return KDA_ERR_INVALID_ARG;
+  if (kBoundsChecked) {
+    BoundsTable t = {};
+    const size_t nth = (size_t)N * T * H;
+    set_extent(t, kBufQ, q, nth * Dk * es);
+    set_extent(t, kBufK, k, nth * Dk * es);
+    set_extent(t, kBufV, v, nth * Dv * es);
+    set_extent(t, kBufO, o, nth * Dv * es);
+    set_extent(t, kBufLogAlpha, log_alpha, nth * Dk * 4);
+    set_extent(t, kBufBeta, beta, nth * 4);
+    set_extent(t, kBufState, pool, (size_t)P * H * Dk * Dv * 4);
+    set_extent(t, kBufIndices, state_indices, state_indices ? (size_t)N * 4 : 0);
+    fusion_extents(t, fz, nth * Dv * es, H, Dk, Dv);
+    const kda_status_t st = from_cuda(register_bounds(t, (cudaStream_t)stream));
+    if (st != KDA_OK) return st;
+  }
   return from_cuda(launch_recurrent_multi(q, k, v, dt, log_alpha, beta, pool, state_indices, o, N,
                                           T, H, Dk, Dv, P, fz, (cudaStream_t)stream));
 }
@@ -473,7 +553,7 @@ kda_status_t kda_last_device_error(kda_stream_t stream) {
     if (e != cudaSuccess) return KDA_ERR_CUDA;
   }
   if (bits & kStatusTimeout) return KDA_ERR_TIMEOUT;
-  if (bits & kStatusBadSeqlens) return KDA_ERR_INVALID_ARG;
+  if (bits & (kStatusBadSeqlens | kStatusBounds)) return KDA_ERR_INVALID_ARG;
   return KDA_OK;
 }
 

@@ -42,6 +42,10 @@ __global__ void chunk_map_kernel(const int32_t* __restrict__ cu, int N, int tota
   __shared__ int s_cnt[1024];
   __shared__ int s_bad;
   const int tid = threadIdx.x, nt = blockDim.x;
+  if (!KDA_IN_BOUNDS(kBufCuSeqlens, cu, (N + 1) * 4ull) || !KDA_IN_BOUNDS(kBufWork, valid, 4) ||
+      !KDA_IN_BOUNDS(kBufWork, chunk_off, (N + 1) * 4ull) ||
+      (order && !KDA_IN_BOUNDS(kBufWork, order, N * 4ull)))
+    return;  // (uniform: the whole block leaves)
   if (tid == 0) s_bad = (cu[0] != 0 || cu[N] > total) ? 1 : 0;
   const int per = (N + nt - 1) / nt;
   const int lo = min(N, tid * per), hi = min(N, lo + per);
@@ -95,6 +99,10 @@ __global__ void chunk_map_kernel(const int32_t* __restrict__ cu, int N, int tota
 
 cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t* chunk_off,
                              int32_t* valid, int32_t* order, cudaStream_t stream) {
+  if (kBoundsChecked) {  // a map that skips its accesses leaves the call's kernels disabled
+    const cudaError_t err = cudaMemsetAsync(valid, 0, sizeof(int32_t), stream);
+    if (err != cudaSuccess) return err;
+  }
   ProfileScope prof("chunk_map", stream);
   chunk_map_kernel<<<1, 1024, 0, stream>>>(cu, N, total, C, chunk_off, valid, order);
   return cudaGetLastError();

@@ -185,6 +185,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * kC;
   const int L = min(kC, geo.seq_end(n) - t0);
   uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)c * H + h);
+  if (!KDA_IN_BOUNDS(kBufWork, rec, kRecBytes)) return;  // (uniform: the whole CTA leaves)
 
   // ---- phase 1: raw k, q, v straight into their operand tiles; log decay into registers ------
   const int cg = tid & 15, rg = tid >> 4;  // thread = 8 channels (one 16-byte chunk) x 4 rows
@@ -193,8 +194,11 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   for (int i = 0; i < 4; ++i) {
     const int r = rg * 4 + i;
     const uint32_t off = tile_chunk_off(r, cg, 8192);
-    if (r < L) {
-      const size_t row = (size_t)(t0 + r) * H + h;
+    const size_t row = (size_t)(t0 + r) * H + h;
+    if (r < L && KDA_IN_BOUNDS(kBufK, k + row * kD + cg * 8, 16) &&
+        KDA_IN_BOUNDS(kBufQ, q + row * kD + cg * 8, 16) &&
+        KDA_IN_BOUNDS(kBufV, v + row * kD + cg * 8, 16) &&
+        KDA_IN_BOUNDS(kBufLogAlpha, log_alpha + row * kD + cg * 8, 32)) {
       cp_async16(sb + kS1Kg + off, reinterpret_cast<const uint4*>(k + row * kD) + cg);
       cp_async16(sb + kS1Qg + off, reinterpret_cast<const uint4*>(q + row * kD) + cg);
       cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
@@ -211,7 +215,10 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       for (int j = 0; j < 8; ++j) g[i][j] = 0.f;
     }
   }
-  if (tid < kC) sBeta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+  if (tid < kC)
+    sBeta[tid] = (tid < L && KDA_IN_BOUNDS(kBufBeta, beta + (size_t)(t0 + tid) * H + h, 4))
+                     ? beta[(size_t)(t0 + tid) * H + h]
+                     : 0.f;
   // the tensor memory and the barrier are first used in phase 3: set them up while the loads
   // above are in flight
   if (warp == 7) {
@@ -224,10 +231,12 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     fence_mbar_init();
   }
   if (fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log decays
-    const float neg_a = -expf(fz.A_log[h]);
+    const float neg_a = KDA_IN_BOUNDS(kBufALog, fz.A_log + h, 4) ? -expf(fz.A_log[h]) : 0.f;
     float bias[8];
+    const bool bias_ok =
+        fz.dt_bias && KDA_IN_BOUNDS(kBufDtBias, fz.dt_bias + h * kD + cg * 8, 32);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) bias[j] = fz.dt_bias ? fz.dt_bias[h * kD + cg * 8 + j] : 0.f;
+    for (int j = 0; j < 8; ++j) bias[j] = bias_ok ? fz.dt_bias[h * kD + cg * 8 + j] : 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (rg * 4 + i < L)
@@ -449,8 +458,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
         const int i = second ? t - 48 : t;
         if (i >= 16 * R + 16) continue;
         float kc[8];
-        if (i < L) {
-          unpack8(*(reinterpret_cast<const uint4*>(k + ((size_t)(t0 + i) * H + h) * kD) + cg), kc);
+        const uint4* kci = reinterpret_cast<const uint4*>(k + ((size_t)(t0 + i) * H + h) * kD) + cg;
+        if (i < L && KDA_IN_BOUNDS(kBufK, kci, 16)) {
+          unpack8(*kci, kc);
           const float sc = fz.l2 ? sInv[i] : 1.f;
           const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i)) + cg * 8;
           const float4 ga = *reinterpret_cast<const float4*>(gi);
@@ -539,8 +549,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     for (int ii = 0; ii < 4; ++ii) {
       const int r = rg * 4 + ii;
       const uint32_t off = tile_chunk_off(r, cg, 8192);
-      if (r < L) {
-        const size_t row = (size_t)(t0 + r) * H + h;
+      const size_t row = (size_t)(t0 + r) * H + h;
+      if (r < L && KDA_IN_BOUNDS(kBufV, v + row * kD + cg * 8, 16) &&
+          KDA_IN_BOUNDS(kBufK, k + row * kD + cg * 8, 16)) {
         cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
         float kf[8];
         unpack8(*(reinterpret_cast<const uint4*>(k + row * kD) + cg), kf);
@@ -566,7 +577,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       while (r * (r + 1) / 2 > p) --r;
       const int i = p - r * (r + 1) / 2;
       float akk = 0.f, aqk = 0.f;
-      if (r < L) {
+      const size_t rowr0 = (size_t)(t0 + r) * H + h, rowi0 = (size_t)(t0 + i) * H + h;
+      if (r < L && KDA_IN_BOUNDS(kBufK, k + rowr0 * kD, 256) &&
+          KDA_IN_BOUNDS(kBufK, k + rowi0 * kD, 256) && KDA_IN_BOUNDS(kBufQ, q + rowr0 * kD, 256)) {
         const float* gr = reinterpret_cast<const float*>(rec + g_scratch_off(r));
         const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i));
         const size_t rowr = (size_t)(t0 + r) * H + h, rowi = (size_t)(t0 + i) * H + h;
@@ -857,7 +870,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     fence_mbar_init();
   }
   if (kNorm && tid < 64)
-    reinterpret_cast<float*>(sm + SM::W)[tid] = fz.ow ? fz.ow[j0 + tid] : 1.f;
+    reinterpret_cast<float*>(sm + SM::W)[tid] =
+        (fz.ow && KDA_IN_BOUNDS(kBufNormW, fz.ow + j0 + tid, 4)) ? fz.ow[j0 + tid] : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -885,17 +899,26 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         uint8_t* stage = sm + kS2Stage0 + st * kStageBytes;
         const int t0 = tb + ci * kC;
         const int L = min(kC, te - t0);
-        if (lane == 0) {
-          const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
-          mbar_arrive_expect_tx(full + st, kStageTx + (gate_rows ? (uint32_t)L * 128u : 0u));
+        const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
+        const __nv_bfloat16* g0 = reinterpret_cast<const __nv_bfloat16*>(fz.og);
+        // the gate rows of this chunk lie between its first and last row's 128 bytes
+        const bool gates_in =
+            !gate_rows ||
+            (KDA_IN_BOUNDS(kBufGate, g0 + ((size_t)t0 * H + h) * kD + j0, 128) &&
+             KDA_IN_BOUNDS(kBufGate, g0 + ((size_t)(t0 + L - 1) * H + h) * kD + j0, 128));
+        if (lane == 0 && !KDA_IN_BOUNDS(kBufWork, rec, kRecBytes)) {
+          mbar_arrive(full + st);  // nothing copied: the phase completes on the stale stage
+        } else if (lane == 0) {
+          mbar_arrive_expect_tx(full + st,
+                                kStageTx + (gate_rows && gates_in ? (uint32_t)L * 128u : 0u));
           bulk_g2s(stage + kStQW, rec + kRecQW, 32768, full + st);
           bulk_g2s(stage + kStAZ, rec + kRecAqk, 8192, full + st);
           bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
           bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
           bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
         }
-        if (gate_rows) {
-          const __nv_bfloat16* g0 = reinterpret_cast<const __nv_bfloat16*>(fz.og);
+        if (gate_rows && gates_in && (!kBoundsChecked || __shfl_sync(0xffffffffu,
+                                                                      (int)KDA_IN_BOUNDS(kBufWork, rec, kRecBytes), 0))) {
           for (int rr = lane; rr < L; rr += 32)
             bulk_g2s(stage + kStGate + rr * 128, g0 + ((size_t)(t0 + rr) * H + h) * kD + j0, 128,
                      full + st);
@@ -968,7 +991,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
                      make_uint4(0, 0, 0, 0));
     float S[32];
     const size_t sbase = (((size_t)n * H + h) * kD + row) * kD + j0 + 32 * chalf;
-    if (initial_state) {
+    if (initial_state && KDA_IN_BOUNDS(kBufInitial, initial_state + sbase, 128)) {
       const float4* src = reinterpret_cast<const float4*>(initial_state + sbase);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -1108,7 +1131,8 @@ __global__ void __launch_bounds__(kK2Threads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) va[j] = va[j] * inv * sW[j] * gt[j];
         }
-        if (r < L) {
+        if (r < L && KDA_IN_BOUNDS(kBufO, o + ((size_t)(t0 + r) * H + h) * kD + j0 + 32 * chalf,
+                                   64)) {
           uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + h) * kD + j0 +
                                                 32 * chalf);
 #pragma unroll
@@ -1121,7 +1145,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         }
       }
     }
-    if (final_state && !*abort_flag) {
+    if (final_state && !*abort_flag && KDA_IN_BOUNDS(kBufFinal, final_state + sbase, 128)) {
       float4* dst = reinterpret_cast<float4*>(final_state + sbase);
 #pragma unroll
       for (int j = 0; j < 8; ++j)

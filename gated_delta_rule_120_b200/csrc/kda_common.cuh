@@ -20,9 +20,46 @@ __device__ unsigned int g_status = 0;  // one definition: the library is a singl
 enum : unsigned int {
   kStatusBadSeqlens = 1u << 0,  // also: a state index beyond the pool
   kStatusTimeout = 1u << 1,
+  kStatusBounds = 1u << 2,      // bounds-checked build: an access outside its buffer, skipped
 };
 
 __device__ __forceinline__ void raise_status(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// ---------------------------------------------------------------------------------------------
+// Bounds-checked build (compiled with KDA_BOUNDS_CHECK, `_build.build(checked=True)`): every entry
+// point registers the byte extent of each buffer of its call in a device table (on the call's
+// stream, before its launches), and the prefill, decode and recurrent-mode kernels test each
+// global access against the extent of the buffer it belongs to. An access outside is skipped — a
+// load yields zeros, a bulk copy is left out of its barrier's byte count — and the status word
+// gets kStatusBounds, which kda_last_device_error reports as KDA_ERR_INVALID_ARG: a substitute
+// for a memory checker that never faults the GPU. The table is one per device, so calls that
+// overlap on the GPU would see each other's extents: the checked build runs one call at a time.
+// In the normal build the checks compile away.
+// ---------------------------------------------------------------------------------------------
+enum BufRole : int {
+  kBufQ = 0, kBufK, kBufV, kBufLogAlpha, kBufBeta, kBufInitial, kBufFinal, kBufO, kBufWork,
+  kBufCuSeqlens, kBufState, kBufIndices, kBufGate, kBufDtBias, kBufALog, kBufNormW, kBufRoles
+};
+struct BoundsTable {
+  const void* base[kBufRoles];
+  unsigned long long bytes[kBufRoles];
+};
+#ifdef KDA_BOUNDS_CHECK
+__device__ BoundsTable g_bounds;
+__device__ __forceinline__ bool in_bounds(int role, const void* p, unsigned long long n) {
+  const char* b = static_cast<const char*>(g_bounds.base[role]);
+  const char* c = static_cast<const char*>(p);
+  if (b != nullptr && c >= b && (unsigned long long)(c - b) + n <= g_bounds.bytes[role])
+    return true;
+  raise_status(kStatusBounds);
+  return false;
+}
+#define KDA_IN_BOUNDS(role, p, n) (::kda::in_bounds((role), (p), (n)))
+constexpr bool kBoundsChecked = true;
+#else
+#define KDA_IN_BOUNDS(role, p, n) ((void)(p), true)
+constexpr bool kBoundsChecked = false;
+#endif
 
 // ---------------------------------------------------------------------------------------------
 // Element access for the two input dtypes.

@@ -275,7 +275,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
         if (col_ok) {
-          float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+          float4 wv = (fz.ow && KDA_IN_BOUNDS(kBufNormW, fz.ow + col, 16))
+                          ? *reinterpret_cast<const float4*>(fz.ow + col)
                             : make_float4(1.f, 1.f, 1.f, 1.f);
           if (fz.og) {
             const Tin* gp = reinterpret_cast<const Tin*>(fz.og) + vec_base(t) * Dv + col;
@@ -412,6 +413,21 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         const int s = it % kDsStages;
         const size_t head = (size_t)first + (size_t)it * stride;
         uint8_t* st = stages + (size_t)s * lay.stage_bytes;
+        if (kBoundsChecked &&
+            !(KDA_IN_BOUNDS(kBufState, state + head * Dk * Dv, lay.state_bytes) &&
+              KDA_IN_BOUNDS(kBufLogAlpha, log_alpha + head * Dk, Dk * 4ull) &&
+              KDA_IN_BOUNDS(kBufQ, q + head * Dk, (size_t)Dk * es) &&
+              KDA_IN_BOUNDS(kBufK, k + head * Dk, (size_t)Dk * es) &&
+              KDA_IN_BOUNDS(kBufV, v + head * Dv, (size_t)Dv * es) &&
+              (!(kFused && lay.og_bytes) ||
+               KDA_IN_BOUNDS(kBufGate, reinterpret_cast<const Tin*>(fz.og) + head * Dv,
+                             lay.og_bytes)) &&
+              (!(kFused && lay.bias_bytes) ||
+               KDA_IN_BOUNDS(kBufDtBias, fz.dt_bias + (head % (size_t)H) * Dk,
+                             lay.bias_bytes)))) {
+          sm100::mbar_arrive(full + s);  // nothing copied: the phase completes on a stale stage
+          return;
+        }
         sm100::mbar_arrive_expect_tx(full + s, lay.state_bytes + lay.vec_tx);
         sm100::bulk_g2s(st, state + head * Dk * Dv, lay.state_bytes, full + s);
         sm100::bulk_g2s(st + lay.la_off, log_alpha + head * Dk, Dk * 4, full + s);
@@ -430,9 +446,11 @@ __global__ void __launch_bounds__(kDsThreads, 1)
         const int s = it % kDsStages;
         if (!sm100::mbar_wait(computed + s, (it / kDsStages) & 1)) break;
         const size_t head = (size_t)first + (size_t)it * stride;
-        sm100::bulk_s2g(state + head * Dk * Dv, stages + (size_t)s * lay.stage_bytes,
-                        lay.state_bytes);
-        sm100::bulk_commit();
+        if (KDA_IN_BOUNDS(kBufState, state + head * Dk * Dv, lay.state_bytes)) {
+          sm100::bulk_s2g(state + head * Dk * Dv, stages + (size_t)s * lay.stage_bytes,
+                          lay.state_bytes);
+          sm100::bulk_commit();
+        }
         if (it + kDsStages < count) {
           sm100::bulk_wait_read_all();  // the stage is free once its store has read it
           issue_load(it + kDsStages);
@@ -450,14 +468,15 @@ __global__ void __launch_bounds__(kDsThreads, 1)
     const int col = lane * 4;
     const bool col_ok = col < Dv;
     const int row0 = warp * kDecRowsPerWarp;
-    float b_next = count > 0 ? beta[first] : 0.f;
+    float b_next = (count > 0 && KDA_IN_BOUNDS(kBufBeta, beta + first, 4)) ? beta[first] : 0.f;
     // fused gate: -exp(A_log[h]) of the next head, fetched a head ahead like beta
     float na_next = (kFused && fz.A_log && count > 0) ? -expf(fz.A_log[first % H]) : 0.f;
     for (int it = 0; it < count; ++it) {
       const int s = it % kDsStages;
       const size_t head = (size_t)first + (size_t)it * stride;
       const float b = b_next;
-      if (it + 1 < count) b_next = beta[head + stride];
+      if (it + 1 < count)
+        b_next = KDA_IN_BOUNDS(kBufBeta, beta + head + stride, 4) ? beta[head + stride] : 0.f;
       const float neg_a = na_next;
       if (kFused && fz.A_log && it + 1 < count)
         na_next = -expf(fz.A_log[(head + stride) % (size_t)H]);
@@ -563,7 +582,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
           for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
           const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
           if (col_ok) {
-            float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+            float4 wv = (fz.ow && KDA_IN_BOUNDS(kBufNormW, fz.ow + col, 16))
+                          ? *reinterpret_cast<const float4*>(fz.ow + col)
                               : make_float4(1.f, 1.f, 1.f, 1.f);
             if (lay.og_bytes) {  // the output gate row staged with the head's vectors
               const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off) + col;
@@ -576,7 +596,7 @@ __global__ void __launch_bounds__(kDsThreads, 1)
                             y.w * inv * wv.w);
           }
         }
-        if (col_ok) {
+        if (col_ok && KDA_IN_BOUNDS(kBufO, o + head * Dv + col, 4ull * sizeof(Tin))) {
           Tin* op = o + head * Dv + col;
           op[0] = from_f32<Tin>(y.x);
           op[1] = from_f32<Tin>(y.y);
@@ -851,7 +871,8 @@ __global__ void __launch_bounds__(kDsThreads, 1)
             for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
             const float inv = rsqrtf(ss / (float)Dv + fz.oeps);
             if (col_ok) {
-              float4 wv = fz.ow ? *reinterpret_cast<const float4*>(fz.ow + col)
+              float4 wv = (fz.ow && KDA_IN_BOUNDS(kBufNormW, fz.ow + col, 16))
+                          ? *reinterpret_cast<const float4*>(fz.ow + col)
                                 : make_float4(1.f, 1.f, 1.f, 1.f);
               if (lay.og_row) {
                 const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off + t * lay.og_row) + col;
@@ -908,6 +929,13 @@ __global__ void __launch_bounds__(kDsThreads, 1)
 constexpr int kRcCompute = 256;                // 8 compute warps
 // the running-decay form keeps 1 / D_t below e^60: its terms stay far inside fp32's range
 constexpr float kRcLazyLimit = 60.f;
+
+// Position of row r inside a token's per-row vector in shared memory (the decays, or the scaled
+// keys and queries): the 4-row chunks of each 16-row group are permuted by ((r >> 5) & 3), so the
+// eight row groups of a warp, which read one chunk each at a time, hit eight distinct bank groups.
+__device__ __forceinline__ int rc_row(int r) {
+  return (r & ~15) | ((((r >> 2) & 3) ^ ((r >> 5) & 3)) << 2) | (r & 3);
+}
 constexpr int kRcThreads = kRcCompute + 32;    // + producer warp
 constexpr int kRcD = 128;
 
@@ -954,7 +982,9 @@ __global__ void __launch_bounds__(kRcThreads, 1)
   const uint32_t es = sizeof(Tin);
   auto slot_of = [&](int it) -> int {
     const int item = first + it * stride, n = item / H;
-    const int sl = state_indices ? state_indices[n] : n;
+    const int sl = state_indices ? (KDA_IN_BOUNDS(kBufIndices, state_indices + n, 4)
+                                        ? state_indices[n] : -1)
+                                 : n;
     return (sl >= 0 && sl < P) ? sl : -1;
   };
 
@@ -969,13 +999,31 @@ __global__ void __launch_bounds__(kRcThreads, 1)
 
   if (warp == kRcCompute / 32) {
     // ---------------------------------------------------------------- producer warp
-    auto issue_load = [&](int it, int slot) {
+    // issues the item's loads and returns the pool row its state came from (-1: none loaded)
+    auto issue_load = [&](int it, int slot) -> int {
       const int s = it % kRsStages;
+      const int item = first + it * stride, n = item / H, h = item - n * H;
+      if (slot >= 0 && kBoundsChecked) {  // every copy of the item inside its buffer, or none
+        bool ok =
+            KDA_IN_BOUNDS(kBufState, pool + ((size_t)slot * H + h) * D * D, lay.state_bytes) &&
+            (!(kFused && lay.bias_bytes) ||
+             KDA_IN_BOUNDS(kBufDtBias, fz.dt_bias + (size_t)h * D, lay.bias_bytes));
+        for (int t = lane; t < T; t += 32) {
+          const size_t base = ((size_t)n * T + t) * H + h;
+          ok = ok && KDA_IN_BOUNDS(kBufLogAlpha, log_alpha + base * D, D * 4ull) &&
+               KDA_IN_BOUNDS(kBufQ, q + base * D, (size_t)D * es) &&
+               KDA_IN_BOUNDS(kBufK, k + base * D, (size_t)D * es) &&
+               KDA_IN_BOUNDS(kBufV, v + base * D, (size_t)D * es) &&
+               (!(kFused && lay.og_row) ||
+                KDA_IN_BOUNDS(kBufGate, reinterpret_cast<const Tin*>(fz.og) + base * D,
+                              (size_t)D * es));
+        }
+        if (!__all_sync(0xffffffffu, ok)) slot = -1;
+      }
       if (slot < 0) {
         if (lane == 0) sm100::mbar_arrive(full + s);
-        return;
+        return -1;
       }
-      const int item = first + it * stride, n = item / H, h = item - n * H;
       uint8_t* st = stages + (size_t)s * lay.stage_bytes;
       if (lane == 0) {
         sm100::mbar_arrive_expect_tx(full + s, lay.state_bytes + lay.vec_tx);
@@ -993,17 +1041,15 @@ __global__ void __launch_bounds__(kRcThreads, 1)
           sm100::bulk_g2s(st + lay.og_off + t * lay.og_row,
                           reinterpret_cast<const Tin*>(fz.og) + base * D, D * es, full + s);
       }
+      return slot;
     };
     int slot_cur[kRsStages];
-    for (int it = 0; it < count && it < kRsStages; ++it) {
-      slot_cur[it] = slot_of(it);
-      issue_load(it, slot_cur[it]);
-    }
+    for (int it = 0; it < count && it < kRsStages; ++it) slot_cur[it] = issue_load(it, slot_of(it));
     for (int it = 0; it < count; ++it) {
       const int s = it % kRsStages;
       bool ok = sm100::mbar_wait(computed + s, (it / kRsStages) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
-      if (lane == 0 && slot_cur[s] >= 0) {
+      if (lane == 0 && slot_cur[s] >= 0) {  // (a row inside the pool: issue_load checked it)
         const int item = first + it * stride, h = item % H;
         sm100::bulk_s2g(pool + ((size_t)slot_cur[s] * H + h) * D * D,
                         stages + (size_t)s * lay.stage_bytes, lay.state_bytes);
@@ -1012,8 +1058,7 @@ __global__ void __launch_bounds__(kRcThreads, 1)
       if (it + kRsStages < count) {
         if (lane == 0) sm100::bulk_wait_read_all();  // the stage is free once its store read it
         __syncwarp();
-        slot_cur[s] = slot_of(it + kRsStages);
-        issue_load(it + kRsStages, slot_cur[s]);
+        slot_cur[s] = issue_load(it + kRsStages, slot_of(it + kRsStages));
       }
     }
     if (lane == 0) {
@@ -1031,15 +1076,21 @@ __global__ void __launch_bounds__(kRcThreads, 1)
     auto stage_scalars = [&](int it) {  // beta (and -exp(A_log[h])) of an item, one item ahead
       float* dst = s_beta + (it & 1) * (kRsMaxT + 2);
       const int item = first + it * stride, n = item / H, h = item - n * H;
-      if (tid < T) dst[tid] = beta[((size_t)n * T + tid) * H + h];
-      if (kFused && tid == 32 && fz.A_log) dst[kRsMaxT] = -expf(fz.A_log[h]);
+      if (tid < T)
+        dst[tid] = KDA_IN_BOUNDS(kBufBeta, beta + ((size_t)n * T + tid) * H + h, 4)
+                       ? beta[((size_t)n * T + tid) * H + h]
+                       : 0.f;
+      if (kFused && tid == 32 && fz.A_log)
+        dst[kRsMaxT] = KDA_IN_BOUNDS(kBufALog, fz.A_log + h, 4) ? -expf(fz.A_log[h]) : 0.f;
     };
     if (count > 0) stage_scalars(0);
     sm100::named_barrier_sync(1, kRcCompute);
     for (int it = 0; it < count; ++it) {
       const int s = it % kRsStages;
       const int item = first + it * stride, n = item / H, h = item - n * H;
-      const int slot_raw = state_indices ? state_indices[n] : n;
+      const int slot_raw =
+          state_indices ? (KDA_IN_BOUNDS(kBufIndices, state_indices + n, 4) ? state_indices[n] : -1)
+                        : n;
       const bool ok = sm100::mbar_wait(full + s, (it / kRsStages) & 1);
       if (!block_all(ok, 1, kRcCompute)) break;
       const float* sb = s_beta + (it & 1) * (kRsMaxT + 2);
@@ -1091,9 +1142,9 @@ __global__ void __launch_bounds__(kRcThreads, 1)
             const float Dt = expf(G), Di = expf(-G);
             const float kx = to_f32(reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row)[tid]);
             const float qx = to_f32(reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row)[tid]);
-            s_khat[t * D + tid] = Dt * kx;
-            s_qhat[t * D + tid] = Dt * qx;
-            s_ktil[t * D + tid] = Di * kx;
+            s_khat[t * D + rc_row(tid)] = Dt * kx;
+            s_qhat[t * D + rc_row(tid)] = Dt * qx;
+            s_ktil[t * D + rc_row(tid)] = Di * kx;
           }
         }
       } else {
@@ -1106,7 +1157,7 @@ __global__ void __launch_bounds__(kRcThreads, 1)
                                    : 0.f;
             la = sb[kRsMaxT] * softplus_f(la + bias);
           }
-          s_alpha[e] = expf(la);
+          s_alpha[t * D + rc_row(i)] = expf(la);
         }
       }
       for (int t = warp; t < T; t += kRcCompute / 32) {
@@ -1163,12 +1214,13 @@ __global__ void __launch_bounds__(kRcThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) ep[c] = pp[c] = 0ull;
         if (lazy) {
-          const float4* kh = reinterpret_cast<const float4*>(s_khat + t * D + r0);
-          const float4* qh = reinterpret_cast<const float4*>(s_qhat + t * D + r0);
-          const float4* kt4 = reinterpret_cast<const float4*>(s_ktil + t * D + r0);
+          const int sw = (rg >> 1) & 3;  // this row group's chunk permutation (rc_row)
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            const float4 a = kh[m], b = qh[m], c4 = kt4[m];
+            const int o4 = t * D + r0 + 4 * (m ^ sw);
+            const float4 a = *reinterpret_cast<const float4*>(s_khat + o4);
+            const float4 b = *reinterpret_cast<const float4*>(s_qhat + o4);
+            const float4 c4 = *reinterpret_cast<const float4*>(s_ktil + o4);
 #pragma unroll
             for (int hlf = 0; hlf < 2; ++hlf) {
               const int jr = 2 * m + hlf;
@@ -1186,10 +1238,16 @@ __global__ void __launch_bounds__(kRcThreads, 1)
         const float* al = s_alpha + t * D + r0;
         const Tin* kv = reinterpret_cast<const Tin*>(st + lay.k_off + t * lay.qk_row) + r0;
         const Tin* qv = reinterpret_cast<const Tin*>(st + lay.q_off + t * lay.qk_row) + r0;
+        const int sw = (rg >> 1) & 3;  // this row group's chunk permutation (rc_row)
 #pragma unroll
         for (int i8 = 0; i8 < 2; ++i8) {  // S' = Diag(alpha) S; e, p over this thread's rows
           float a[8], kk[8], qv8[8];
-          load8_f32(al + 8 * i8, a);
+          {
+            const float4 a0 = *reinterpret_cast<const float4*>(al + 4 * ((2 * i8) ^ sw));
+            const float4 a1 = *reinterpret_cast<const float4*>(al + 4 * ((2 * i8 + 1) ^ sw));
+            a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+            a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+          }
           load8_in(kv + 8 * i8, kk);
           load8_in(qv + 8 * i8, qv8);
 #pragma unroll
@@ -1268,8 +1326,9 @@ __global__ void __launch_bounds__(kRcThreads, 1)
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
           const float inv = rsqrtf(ss * (1.f / D) + fz.oeps);
-          float4 wv = fz.ow ? reinterpret_cast<const float4*>(fz.ow)[lane]
-                            : make_float4(1.f, 1.f, 1.f, 1.f);
+          float4 wv = (fz.ow && KDA_IN_BOUNDS(kBufNormW, fz.ow + 4 * lane, 16))
+                          ? reinterpret_cast<const float4*>(fz.ow)[lane]
+                          : make_float4(1.f, 1.f, 1.f, 1.f);
           if (lay.og_row) {
             const Tin* gp = reinterpret_cast<const Tin*>(st + lay.og_off + t * lay.og_row) + 4 * lane;
             wv.x *= sigmoid_f(to_f32(gp[0]));
@@ -1280,10 +1339,12 @@ __global__ void __launch_bounds__(kRcThreads, 1)
           y = make_float4(y.x * inv * wv.x, y.y * inv * wv.y, y.z * inv * wv.z, y.w * inv * wv.w);
         }
         Tin* op = o + (((size_t)n * T + t) * H + h) * D + 4 * lane;
-        op[0] = from_f32<Tin>(y.x);
-        op[1] = from_f32<Tin>(y.y);
-        op[2] = from_f32<Tin>(y.z);
-        op[3] = from_f32<Tin>(y.w);
+        if (KDA_IN_BOUNDS(kBufO, op, 4ull * sizeof(Tin))) {
+          op[0] = from_f32<Tin>(y.x);
+          op[1] = from_f32<Tin>(y.y);
+          op[2] = from_f32<Tin>(y.z);
+          op[3] = from_f32<Tin>(y.w);
+        }
       }
       sm100::fence_proxy_async_smem();
       sm100::named_barrier_sync(1, kRcCompute);

@@ -93,6 +93,11 @@ struct SimtRecord {
 // bytes of one (chunk, head) record of the bf16 tensor-core path (d = 128, C = 64)
 constexpr size_t TcRecordBytes = 74240;
 
+// Bounds-checked build: the call's buffer extents into the device table, on `stream` (a no-op
+// returning cudaSuccess in the normal build).
+struct BoundsTable;
+cudaError_t register_bounds(const BoundsTable& t, cudaStream_t stream);
+
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int max_chunks,
                               uint8_t* records, cudaStream_t stream);
 size_t tc_local_smem_bytes();

@@ -28,6 +28,18 @@ extern "C" {
  */
 KDA_API kda_status_t kda_selftest_wait_timeout(uint64_t limit_ns, kda_stream_t stream);
 
+/*
+ * kda_selftest_bounds — in the bounds-checked build of the library (compiled with
+ * KDA_BOUNDS_CHECK; see _build.build(checked=True)), registers `buffer` (device, `bytes` long) as
+ * the only extent of the call and launches one thread that tests, with the kernels' own check and
+ * without performing it, a 4-byte access starting just past the buffer's end. The check refuses
+ * it and sets the bounds bit of the status word, which kda_last_device_error(stream) then reports
+ * as KDA_ERR_INVALID_ARG. Nothing is read or written outside the buffer.
+ * Returns KDA_ERR_UNSUPPORTED in the normal build (no checks compiled in), KDA_ERR_INVALID_ARG for
+ * a null buffer or zero bytes, KDA_ERR_CUDA when a CUDA call fails, else KDA_OK.
+ */
+KDA_API kda_status_t kda_selftest_bounds(const void* buffer, size_t bytes, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -51,6 +51,15 @@ __device__ __forceinline__ void fma4(float s, float4 b, float4& acc) {
 // ----------------------------------------------------------------------------------------------
 // state pass: one CTA per (sequence, head, 32-column slice of d_v), chunks in reverse order
 // ----------------------------------------------------------------------------------------------
+constexpr int kBwdC = 32;  // chunk of the backward pass (both passes)
+constexpr int kDoPerThread = kBwdC * kBwSlice / kBwdThreads;
+
+// Each chunk step has two phases, dV' (reads Kt, P, dO, dS') and dS (reads Qt, W, gamma, dO, dV').
+// The record sections are fetched with cp.async in two groups, each a phase ahead of its use:
+// group A (W, Qt, gamma of chunk c) is issued when step c starts and lands during its dV' phase;
+// group B (Kt, P of chunk c - 1) is issued when the dV' phase of step c ends and lands during its
+// dS phase. The dO slice of chunk c - 1 is loaded into registers in the same place and stored to
+// shared memory when step c - 1 starts. The chain then waits on global memory only at its start.
 template <typename Tin>
 __global__ void __launch_bounds__(kBwdThreads, 2)
     chunk_state_bwd_kernel(const float* __restrict__ ws, SimtRecord rec, SeqGeometry geo, int H,
@@ -58,13 +67,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                            const float* __restrict__ d_final, float* __restrict__ d_initial,
                            float* __restrict__ dstates, float* __restrict__ dvp) {
   extern __shared__ __align__(16) float smem[];
-  const int C = geo.C;
+  constexpr int C = kBwdC;
   float* sdS = smem;                 // [Dk][32] cotangent of the state leaving the chunk
   float* sW = sdS + Dk * kBwSlice;   // [C][Dk]
   float* sKt = sW + C * Dk;          // [C][Dk]
   float* sQt = sKt + C * Dk;         // [C][Dk]
-  float* sPt = sQt + C * Dk;         // [C][C] P transposed: sPt[i][r] = P[r][i]
-  float* sGam = sPt + C * C;         // [Dk]
+  float* sP = sQt + C * Dk;          // [C][C] P[r][i] (read for r >= i only)
+  float* sGam = sP + C * C;          // [Dk]
   float* sdO = sGam + Dk;            // [C][32]
   float* sdV = sdO + C * kBwSlice;   // [C][32]
 
@@ -73,39 +82,56 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
   const int NV = min(kBwSlice, Dv - j0);
   const int tid = threadIdx.x, nt = blockDim.x;
   const size_t sbase = ((size_t)n * H + h) * Dk * Dv;
+  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
+  const int c_first = geo.first_chunk(n);
+  const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
+
+  // record sections are 16-byte aligned (d_k multiple of 4, C multiple of 16)
+  auto record = [&](int c) { return ws + rec.record_floats * ((size_t)c * H + h); };
+  auto issue_a = [&](int c) {
+    const float* r_ = record(c);
+    for (int idx = tid; idx < C * Dk / 4; idx += nt) {
+      cp_async_16B(sW + 4 * idx, r_ + rec.off_w + 4 * idx);
+      cp_async_16B(sQt + 4 * idx, r_ + rec.off_qt + 4 * idx);
+    }
+    for (int idx = tid; idx < Dk / 4; idx += nt) cp_async_16B(sGam + 4 * idx, r_ + rec.off_gam + 4 * idx);
+    cp_async_commit();
+  };
+  auto issue_b = [&](int c) {
+    const float* r_ = record(c);
+    for (int idx = tid; idx < C * Dk / 4; idx += nt)
+      cp_async_16B(sKt + 4 * idx, r_ + rec.off_kt + 4 * idx);
+    for (int idx = tid; idx < C * C / 4; idx += nt) cp_async_16B(sP + 4 * idx, r_ + rec.off_aqk + 4 * idx);
+    cp_async_commit();
+  };
+  float dnext[kDoPerThread];  // the dO slice of the next chunk (element tid + m * nt)
+  auto load_do = [&](int ci) {
+    const int t0 = tb + ci * C, L = min(C, te - t0);
+#pragma unroll
+    for (int m = 0; m < kDoPerThread; ++m) {
+      const int idx = tid + m * kBwdThreads, r = idx / kBwSlice, jj = idx - r * kBwSlice;
+      dnext[m] = (r < L && jj < NV)
+                     ? to_f32(d_o[((size_t)(t0 + r) * H + h) * Dv + j0 + jj])
+                     : 0.f;
+    }
+  };
 
   for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
     const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
     sdS[idx] = (d_final && jj < NV) ? d_final[sbase + (size_t)a * Dv + j0 + jj] : 0.f;
   }
-  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
-  const int c_first = geo.first_chunk(n);
-  const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
+  if (nchunks > 0) {
+    issue_b(c_first + nchunks - 1);
+    load_do(nchunks - 1);
+  }
+  __syncthreads();
   for (int ci = nchunks - 1; ci >= 0; --ci) {
     const int c = c_first + ci;
     const int t0 = tb + ci * C;
     const int L = min(C, te - t0);
-    const float* r_ = ws + rec.record_floats * ((size_t)c * H + h);
-    __syncthreads();  // the previous chunk is done with the staging buffers
-    {  // record sections are 16-byte aligned (d_k multiple of 4, C multiple of 16)
-      const float4* w4 = reinterpret_cast<const float4*>(r_ + rec.off_w);
-      const float4* k4 = reinterpret_cast<const float4*>(r_ + rec.off_kt);
-      const float4* q4 = reinterpret_cast<const float4*>(r_ + rec.off_qt);
-      for (int idx = tid; idx < C * Dk / 4; idx += nt) {
-        reinterpret_cast<float4*>(sW)[idx] = w4[idx];
-        reinterpret_cast<float4*>(sKt)[idx] = k4[idx];
-        reinterpret_cast<float4*>(sQt)[idx] = q4[idx];
-      }
-    }
-    for (int idx = tid; idx < C * C; idx += nt) {
-      const int r = idx / C, i = idx - r * C;
-      sPt[i * C + r] = r_[rec.off_aqk + idx];
-    }
-    for (int a = tid; a < Dk; a += nt) sGam[a] = r_[rec.off_gam + a];
-    for (int idx = tid; idx < C * kBwSlice; idx += nt) {
-      const int r = idx / kBwSlice, jj = idx - r * kBwSlice;
-      sdO[idx] = (r < L && jj < NV) ? to_f32(d_o[((size_t)(t0 + r) * H + h) * Dv + j0 + jj]) : 0.f;
-    }
+#pragma unroll
+    for (int m = 0; m < kDoPerThread; ++m) sdO[tid + m * kBwdThreads] = dnext[m];
+    issue_a(c);
     {  // the cotangent entering from the right of this chunk, for the chunk-local pass
       float* dst = dstates + ((size_t)c * H + h) * Dk * Dv;
       for (int idx = tid; idx < Dk * kBwSlice / 4; idx += nt) {
@@ -115,6 +141,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
               reinterpret_cast<const float4*>(sdS)[idx];
       }
     }
+    cp_async_wait<1>();  // group B of this chunk has landed (group A may be in flight)
     __syncthreads();
     // dV'[i][j] = sum_r P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j] (P[r][i] = 0 for r < i):
     // 2 x 4 tiles (rows i0, i0 + 1; columns 4 jq .. 4 jq + 3), the d_k part split 64 / C ways
@@ -122,7 +149,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
       const float4* Kt4 = reinterpret_cast<const float4*>(sKt);
       const float4* S4 = reinterpret_cast<const float4*>(sdS);  // [Dk][8]
       const float4* O4 = reinterpret_cast<const float4*>(sdO);  // [C][8]
-      const int dq = Dk >> 2, split = 64 / C;
+      constexpr int split = 64 / C;
+      const int dq = Dk >> 2;
       const int ip = (tid >> 3) % (C >> 1), jq = tid & 7, sp = tid / (4 * C);
       const int i0 = 2 * ip, i1 = i0 + 1;
       const int kq = (dq + split - 1) / split, q0 = sp * kq, q1 = min(dq, q0 + kq);
@@ -140,8 +168,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
       if (sp == 0) {  // the A_qk part (contraction over the chunk rows r >= i)
         for (int r = i0; r < C; ++r) {
           const float4 ov = O4[r * 8 + jq];
-          fma4(sPt[i0 * C + r], ov, acc[0]);
-          if (r >= i1) fma4(sPt[i1 * C + r], ov, acc[1]);
+          fma4(sP[r * C + i0], ov, acc[0]);
+          if (r >= i1) fma4(sP[r * C + i1], ov, acc[1]);
         }
       }
       float4* sRed = reinterpret_cast<float4*>(sdV + C * kBwSlice);  // [split][C][8]
@@ -167,6 +195,14 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
             *reinterpret_cast<float4*>(dvp + ((size_t)(t0 + i) * H + h) * Dv + j0 + 4 * jq) = val;
         }
       }
+    }
+    __syncthreads();  // dV' complete; Kt and P are free for the next chunk
+    if (ci > 0) {
+      issue_b(c - 1);
+      load_do(ci - 1);
+      cp_async_wait<1>();  // group A of this chunk has landed
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
     // dS = Qt^T dO + Diag(gamma_C) dS' - W^T dV': 4 x 4 tiles (rows 4 aq .. 4 aq + 3), each
@@ -201,8 +237,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
         for (int e = 0; e < 4; ++e) S4[(4 * aq + e) * 8 + jq] = acc[e];
       }
     }
+    __syncthreads();  // dS complete; W, Qt, gamma and dO are free
   }
-  __syncthreads();
   if (d_initial) {
     for (int idx = tid; idx < Dk * kBwSlice; idx += nt) {
       const int a = idx / kBwSlice, jj = idx - a * kBwSlice;
@@ -214,7 +250,6 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
 // ----------------------------------------------------------------------------------------------
 // chunk-local pass: one CTA per (chunk, head); chunk = 32 tokens
 // ----------------------------------------------------------------------------------------------
-constexpr int kBwdC = 32;
 
 // Shared-memory rows are padded by four floats (ld = D + 4): rows stay 16-byte aligned for
 // float4 accesses, and consecutive rows start 4 banks apart. The products are register-tiled:
@@ -258,6 +293,45 @@ struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
   }
 };
 
+// A 16-byte vector of Tin into fp32 shared memory (4 floats, or 8 from bf16).
+__device__ __forceinline__ void store_vec(float* p, uint4 u, float) {
+  st4(p, make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                     __uint_as_float(u.w)));
+}
+__device__ __forceinline__ void store_vec(float* p, uint4 u, __nv_bfloat16) {
+  st4(p, make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u)));
+  st4(p + 4, make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                         __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u)));
+}
+
+// A [kBwdC][D] tile of Tin rows (row r at src + r * stride; rows >= L read as zeros; D <= 128 a
+// multiple of kPer; 16-byte aligned rows) moved into fp32 shared-memory rows as 16-byte vectors:
+// load() issues every load of the thread, store() converts them once they have been issued.
+template <typename Tin>
+struct RowVec {
+  static constexpr int kPer = 16 / sizeof(Tin);                    // elements per vector
+  static constexpr int kMax = kBwdC * 128 / kPer / kBwdThreads;  // vectors per thread
+  uint4 x[kMax];
+  __device__ __forceinline__ void load(const Tin* src, size_t stride, int L, int D) {
+    const int vpr = D / kPer;
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+      const int idx = threadIdx.x + m * kBwdThreads, r = idx / vpr, c = idx - r * vpr;
+      x[m] = r < L ? __ldg(reinterpret_cast<const uint4*>(src + r * stride + c * kPer))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  __device__ __forceinline__ void store(float* dst, int ld, int D) const {
+    const int vpr = D / kPer;
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+      const int idx = threadIdx.x + m * kBwdThreads, r = idx / vpr, c = idx - r * vpr;
+      if (r < kBwdC) store_vec(dst + r * ld + c * kPer, x[m], Tin());
+    }
+  }
+};
+
 // acc[u][w] += sum_{k < K} X[(tm + 16u) * ldx + k] * Y[(tn + 16w) * ldy + k]  (K multiple of 4)
 __device__ __forceinline__ void abt_2x2(const float* X, int ldx, const float* Y, int ldy, int K,
                                         int tm, int tn, float (&acc)[2][2]) {
@@ -275,7 +349,7 @@ __device__ __forceinline__ void abt_2x2(const float* X, int ldx, const float* Y,
 }
 
 template <typename Tin>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     chunk_local_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                            const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                            const float* __restrict__ beta, SeqGeometry geo, int H, int Dk, int Dv,
@@ -323,28 +397,71 @@ __global__ void __launch_bounds__(kBwdThreads)
   const float* dS1 = dstates + ((size_t)c * H + h) * Dk * Dv; // cotangent of the state leaving it
   const int Dv4 = Dv >> 2;
 
-  // ---- P0: inputs, record, cumulative decay
-  for (int idx = tid; idx < C * Dk; idx += nt) {
-    const int r = idx / Dk, a = idx - r * Dk;
-    const bool in = r < L;
-    const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
-    sK[r * ldk + a] = in ? to_f32(k[gi]) : 0.f;
-    sQ[r * ldk + a] = in ? to_f32(q[gi]) : 0.f;
-    sG[r * ldk + a] = in ? log_alpha[gi] : 0.f;
-    X4[r * ldk + a] = r_[rec.off_w + idx];
-  }
-  for (int idx = tid; idx < C * Dv; idx += nt) {
-    const int r = idx / Dv, jj = idx - r * Dv;
-    const bool in = r < L;
-    const size_t gi = ((size_t)(t0 + r) * H + h) * Dv + jj;
-    sV[r * ldv + jj] = in ? to_f32(v[gi]) : 0.f;
-    sdO[r * ldv + jj] = in ? to_f32(d_o[gi]) : 0.f;
-    sdV[r * ldv + jj] = in ? dvp[gi] : 0.f;
-  }
-  for (int idx = tid; idx < C * C; idx += nt) {
-    const int r = idx / C, i = idx - r * C;
-    sT[r * ldc + i] = r_[rec.off_t + idx];
-    sB[r * ldc + i] = r_[rec.off_b + idx];
+  // ---- P0: inputs, record, cumulative decay. With 16-byte aligned input rows every copy is
+  // issued before any is used: the record, dV' and log_alpha by cp.async, the Tin inputs as
+  // 16-byte vectors converted once all are in flight (the record and dV' rows are always aligned).
+  const bool vec = ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                     reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(d_o) |
+                     reinterpret_cast<uintptr_t>(log_alpha)) & 15) == 0 &&
+                   Dk % RowVec<Tin>::kPer == 0 && Dv % RowVec<Tin>::kPer == 0;
+  if (vec) {
+    const size_t rowk = (size_t)H * Dk, rowv = (size_t)H * Dv;  // token strides
+    const size_t bk = ((size_t)t0 * H + h) * Dk, bv = ((size_t)t0 * H + h) * Dv;
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    RowVec<Tin> xk, xq, xv, xo;
+    xk.load(k + bk, rowk, L, Dk);
+    xq.load(q + bk, rowk, L, Dk);
+    xv.load(v + bv, rowv, L, Dv);
+    xo.load(d_o + bv, rowv, L, Dv);
+    for (int idx = tid; idx < C * (Dk / 4); idx += nt) {
+      const int r = idx / (Dk / 4), a = 4 * (idx - r * (Dk / 4));
+      cp_async_16B(X4 + r * ldk + a, r_ + rec.off_w + r * Dk + a);
+      if (r < L)
+        cp_async_16B(sG + r * ldk + a, log_alpha + bk + r * rowk + a);
+      else
+        st4(sG + r * ldk + a, zero4);
+    }
+    for (int idx = tid; idx < C * (Dv / 4); idx += nt) {
+      const int r = idx / (Dv / 4), jj = 4 * (idx - r * (Dv / 4));
+      if (r < L)
+        cp_async_16B(sdV + r * ldv + jj, dvp + bv + r * rowv + jj);
+      else
+        st4(sdV + r * ldv + jj, zero4);
+    }
+    for (int idx = tid; idx < C * (C / 4); idx += nt) {
+      const int r = idx / (C / 4), i = 4 * (idx - r * (C / 4));
+      cp_async_16B(sT + r * ldc + i, r_ + rec.off_t + r * C + i);
+      cp_async_16B(sB + r * ldc + i, r_ + rec.off_b + r * C + i);
+    }
+    cp_async_commit();
+    xk.store(sK, ldk, Dk);
+    xq.store(sQ, ldk, Dk);
+    xv.store(sV, ldv, Dv);
+    xo.store(sdO, ldv, Dv);
+    cp_async_wait<0>();
+  } else {
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, a = idx - r * Dk;
+      const bool in = r < L;
+      const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + a;
+      sK[r * ldk + a] = in ? to_f32(k[gi]) : 0.f;
+      sQ[r * ldk + a] = in ? to_f32(q[gi]) : 0.f;
+      sG[r * ldk + a] = in ? log_alpha[gi] : 0.f;
+      X4[r * ldk + a] = r_[rec.off_w + idx];
+    }
+    for (int idx = tid; idx < C * Dv; idx += nt) {
+      const int r = idx / Dv, jj = idx - r * Dv;
+      const bool in = r < L;
+      const size_t gi = ((size_t)(t0 + r) * H + h) * Dv + jj;
+      sV[r * ldv + jj] = in ? to_f32(v[gi]) : 0.f;
+      sdO[r * ldv + jj] = in ? to_f32(d_o[gi]) : 0.f;
+      sdV[r * ldv + jj] = in ? dvp[gi] : 0.f;
+    }
+    for (int idx = tid; idx < C * C; idx += nt) {
+      const int r = idx / C, i = idx - r * C;
+      sT[r * ldc + i] = r_[rec.off_t + idx];
+      sB[r * ldc + i] = r_[rec.off_b + idx];
+    }
   }
   for (int r = tid; r < C; r += nt) sbeta[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
   __syncthreads();
@@ -370,11 +487,13 @@ __global__ void __launch_bounds__(kBwdThreads)
   for (int a0 = 0; a0 < Dk; a0 += 32) {
     const int na = min(32, Dk - a0);
     __syncthreads();  // previous slice consumed (and, the first time, the cumsum done)
-    for (int idx = tid; idx < na * Dv4; idx += nt) {
+    for (int idx = tid; idx < na * Dv4; idx += nt) {  // (state rows: 16-byte aligned)
       const int aa = idx / Dv4, j4 = idx - aa * Dv4;
-      st4(Y1 + aa * ldv + 4 * j4, ld4(S0 + (size_t)(a0 + aa) * Dv + 4 * j4));
-      st4(Y2 + aa * ldv + 4 * j4, ld4(dS1 + (size_t)(a0 + aa) * Dv + 4 * j4));
+      cp_async_16B(Y1 + aa * ldv + 4 * j4, S0 + (size_t)(a0 + aa) * Dv + 4 * j4);
+      cp_async_16B(Y2 + aa * ldv + 4 * j4, dS1 + (size_t)(a0 + aa) * Dv + 4 * j4);
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
     for (int aa = 0; aa < na; ++aa) {
       const float w0 = X4[tm * ldk + a0 + aa], w1 = X4[(tm + 16) * ldk + a0 + aa];
@@ -403,10 +522,16 @@ __global__ void __launch_bounds__(kBwdThreads)
           }
         }
     }
-    for (int aa = tid; aa < na; aa += nt) {  // dgamma_C = rowsum(dS' . S)
+    {  // dgamma_C = rowsum(dS' . S): eight lanes per row, each over every eighth float4
+      const int aa = tid >> 3, part = tid & 7;
       float s = 0.f;
-      for (int j = 0; j < Dv; j += 4) s = dot4(ld4(Y2 + aa * ldv + j), ld4(Y1 + aa * ldv + j), s);
-      sdgam[a0 + aa] = s;
+      if (aa < na)
+        for (int j = 4 * part; j < Dv; j += 32)
+          s = dot4(ld4(Y2 + aa * ldv + j), ld4(Y1 + aa * ldv + j), s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (aa < na && part == 0) sdgam[a0 + aa] = s;
     }
   }
   __syncthreads();
@@ -423,8 +548,10 @@ __global__ void __launch_bounds__(kBwdThreads)
     __syncthreads();
     for (int idx = tid; idx < na * Dv4; idx += nt) {
       const int aa = idx / Dv4, j4 = idx - aa * Dv4;
-      st4(Y2 + aa * ldv + 4 * j4, ld4(dS1 + (size_t)(a0 + aa) * Dv + 4 * j4));
+      cp_async_16B(Y2 + aa * ldv + 4 * j4, dS1 + (size_t)(a0 + aa) * Dv + 4 * j4);
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     __syncthreads();
     if (tn < na || tn + 16 < na) {
       float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
@@ -648,6 +775,7 @@ static cudaError_t launch_bwd_typed(const BackwardArgs& b, const SeqGeometry& ge
                                     float* records, const SimtRecord& rec, float* states,
                                     float* dstates, float* dvp, cudaStream_t stream) {
   const PrefillArgs& a = b.fwd;
+  if (a.C != kBwdC || geo.C != kBwdC) return cudaErrorInvalidValue;
   cudaError_t err =
       launch_forward_for_backward(a, geo, max_chunks, records, rec, states, stream);
   if (err != cudaSuccess) return err;

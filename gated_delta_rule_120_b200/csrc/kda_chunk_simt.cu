@@ -307,17 +307,22 @@ constexpr int kSlice = 32;
 
 constexpr int kSimtRedFloats = 4096;  // split-contraction partial sums of the tiled step
 
-// One chunk of the state chain with register tiles (d_k, d_v multiples of 4; C in {16, 32, 64};
+// The state chain with register tiles (d_k, d_v multiples of 4; C in {16, 32, 64};
 // kSimtThreads threads). Shared memory as in chunk_state_simt_kernel plus kSimtRedFloats.
+// Per chunk:
 //   V' = U - W S and O_inter = Qt S: 2 x 4 output tiles, the d_k contraction split 64 / C ways;
 //   O = O_inter + Tril(A_qk) V' (Eq. 9): 2 x 4 tiles;  S = Diag(gamma_C) S + Kt^T V' (Eq. 8):
 //   4 x 4 tiles of the state slice, updated in place.
+// The record sections arrive by cp.async in two groups, each issued a phase ahead of its use:
+// group A (W, Qt, the U slice: the first phase) of chunk c + 1 while chunk c computes its output
+// and state update, group B (A_qk, Kt, gamma_C: the output and the update) of chunk c while chunk
+// c computes its first phase.
 template <typename Tin>
-__device__ __forceinline__ void state_step_tiled(const float* __restrict__ ws,
-                                                 const SimtRecord& rec, int c, int t0,
-                                                 int L, int C, int H, int h, int Dk, int Dv,
-                                                 int j0, int NV, float* smem, Tin* o,
-                                                 float* states_out) {
+__device__ __forceinline__ void state_chain_tiled(const float* __restrict__ ws,
+                                                  const SimtRecord& rec, int c_first, int nchunks,
+                                                  int tb, int te, int C, int H, int h, int Dk,
+                                                  int Dv, int j0, int NV, float* smem, Tin* o,
+                                                  float* states_out) {
   const int tid = threadIdx.x;
   const int dq = Dk >> 2;  // float4 columns of a d_k row
   float4* sS = reinterpret_cast<float4*>(smem);  // [Dk][8]
@@ -329,130 +334,161 @@ __device__ __forceinline__ void state_step_tiled(const float* __restrict__ ws,
   float* sAq = reinterpret_cast<float*>(sVp + C * 8);  // [C][C]
   float* sGam = sAq + C * C;                            // [Dk]
   float4* sRed = reinterpret_cast<float4*>(sGam + Dk);  // [split][2][C][8]
-  const float4* r4 = reinterpret_cast<const float4*>(ws + rec.record_floats * ((size_t)c * H + h));
-
-  __syncthreads();  // the previous chunk is done with the staging buffers
-  for (int i = tid; i < C * dq; i += kSimtThreads) {
-    sW[i] = r4[rec.off_w / 4 + i];
-    sKt[i] = r4[rec.off_kt / 4 + i];
-    if (o) sQt[i] = r4[rec.off_qt / 4 + i];
-  }
-  for (int i = tid; i < C * 8; i += kSimtThreads) {
-    const int r = i >> 3, q = i & 7;
-    sU[i] = 4 * q < NV ? r4[(rec.off_u + (size_t)r * Dv + j0) / 4 + q] : make_float4(0, 0, 0, 0);
-  }
-  for (int i = tid; i < C * C / 4; i += kSimtThreads)
-    reinterpret_cast<float4*>(sAq)[i] = r4[rec.off_aqk / 4 + i];
-  for (int i = tid; i < dq; i += kSimtThreads)
-    reinterpret_cast<float4*>(sGam)[i] = r4[rec.off_gam / 4 + i];
-  if (states_out) {  // the state entering this chunk, for the backward pass
-    float* so = states_out + ((size_t)c * H + h) * Dk * Dv;
-    for (int i = tid; i < Dk * 8; i += kSimtThreads) {
-      const int cc = i >> 3, q = i & 7;
-      if (4 * q < NV) *reinterpret_cast<float4*>(so + (size_t)cc * Dv + j0 + 4 * q) = sS[i];
+  // record sections are 16-byte aligned (d_k, d_v multiples of 4; C multiple of 16)
+  auto record = [&](int c) {
+    return reinterpret_cast<const float4*>(ws + rec.record_floats * ((size_t)c * H + h));
+  };
+  auto issue_a = [&](int c) {
+    const float4* r4 = record(c);
+    for (int i = tid; i < C * dq; i += kSimtThreads) {
+      cp_async_16B(sW + i, r4 + rec.off_w / 4 + i);
+      if (o) cp_async_16B(sQt + i, r4 + rec.off_qt / 4 + i);
     }
-  }
-  __syncthreads();
+    for (int i = tid; i < C * 8; i += kSimtThreads) {
+      const int r = i >> 3, q = i & 7;
+      if (4 * q < NV)
+        cp_async_16B(sU + i, r4 + (rec.off_u + (size_t)r * Dv + j0) / 4 + q);
+      else
+        sU[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_commit();
+  };
+  auto issue_b = [&](int c) {
+    const float4* r4 = record(c);
+    for (int i = tid; i < C * dq; i += kSimtThreads) cp_async_16B(sKt + i, r4 + rec.off_kt / 4 + i);
+    for (int i = tid; i < C * C / 4; i += kSimtThreads)
+      cp_async_16B(reinterpret_cast<float4*>(sAq) + i, r4 + rec.off_aqk / 4 + i);
+    for (int i = tid; i < dq; i += kSimtThreads)
+      cp_async_16B(reinterpret_cast<float4*>(sGam) + i, r4 + rec.off_gam / 4 + i);
+    cp_async_commit();
+  };
 
-  // V' and O_inter: tile (rows 2 rp, 2 rp + 1; columns 4 jq .. 4 jq + 3), d_k split `split` ways
   const int split = 64 / C;
   const int rp = (tid >> 3) % (C >> 1), jq = tid & 7, sp = tid / (4 * C);
   const int kq = (dq + split - 1) / split, q0 = sp * kq, q1 = min(dq, q0 + kq);
-  float aw[2][4] = {}, aq[2][4] = {};
   const int r0 = 2 * rp, r1 = r0 + 1;
-  // acc[a] += X[row a] S over this thread's share of d_k, for X = W and (with o) X = Qt
-  auto contract = [&](const float4* X, float (&acc)[2][4]) {
-    for (int q = q0; q < q1; ++q) {
-      const float4 x0 = X[r0 * dq + q], x1 = X[r1 * dq + q];
-      const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 sv = sS[(4 * q + k) * 8 + jq];
-        acc[0][0] = fmaf(xa[k], sv.x, acc[0][0]); acc[0][1] = fmaf(xa[k], sv.y, acc[0][1]);
-        acc[0][2] = fmaf(xa[k], sv.z, acc[0][2]); acc[0][3] = fmaf(xa[k], sv.w, acc[0][3]);
-        acc[1][0] = fmaf(xb[k], sv.x, acc[1][0]); acc[1][1] = fmaf(xb[k], sv.y, acc[1][1]);
-        acc[1][2] = fmaf(xb[k], sv.z, acc[1][2]); acc[1][3] = fmaf(xb[k], sv.w, acc[1][3]);
+
+  if (nchunks > 0) issue_a(c_first);
+  __syncthreads();  // the initial state slice is in place
+  for (int ci = 0; ci < nchunks; ++ci) {
+    const int c = c_first + ci;
+    const int t0 = tb + ci * C;
+    const int L = min(C, te - t0);
+    issue_b(c);
+    if (states_out) {  // the state entering this chunk, for the backward pass
+      float* so = states_out + ((size_t)c * H + h) * Dk * Dv;
+      for (int i = tid; i < Dk * 8; i += kSimtThreads) {
+        const int cc = i >> 3, q = i & 7;
+        if (4 * q < NV) *reinterpret_cast<float4*>(so + (size_t)cc * Dv + j0 + 4 * q) = sS[i];
       }
     }
-  };
-  contract(sW, aw);
-  if (o) contract(sQt, aq);
-  if (split > 1) {  // partial sums of the split contraction, summed by the sp == 0 threads
-    sRed[((sp * 2 + 0) * C + r0) * 8 + jq] = make_float4(aw[0][0], aw[0][1], aw[0][2], aw[0][3]);
-    sRed[((sp * 2 + 0) * C + r1) * 8 + jq] = make_float4(aw[1][0], aw[1][1], aw[1][2], aw[1][3]);
-    if (o) {
-      sRed[((sp * 2 + 1) * C + r0) * 8 + jq] =
-          make_float4(aq[0][0], aq[0][1], aq[0][2], aq[0][3]);
-      sRed[((sp * 2 + 1) * C + r1) * 8 + jq] =
-          make_float4(aq[1][0], aq[1][1], aq[1][2], aq[1][3]);
-    }
+    cp_async_wait<1>();  // group A of this chunk has landed (group B may be in flight)
     __syncthreads();
-    if (sp == 0) {
-      for (int s2 = 1; s2 < split; ++s2) {
+
+    // V' and O_inter: tile (rows 2 rp, 2 rp + 1; columns 4 jq .. 4 jq + 3), d_k split `split` ways
+    float aw[2][4] = {}, aq[2][4] = {};
+    // acc[a] += X[row a] S over this thread's share of d_k, for X = W and (with o) X = Qt
+    auto contract = [&](const float4* X, float (&acc)[2][4]) {
+      for (int q = q0; q < q1; ++q) {
+        const float4 x0 = X[r0 * dq + q], x1 = X[r1 * dq + q];
+        const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const float4 pw = sRed[((s2 * 2 + 0) * C + r0 + a) * 8 + jq];
-          aw[a][0] += pw.x; aw[a][1] += pw.y; aw[a][2] += pw.z; aw[a][3] += pw.w;
-          if (o) {
-            const float4 pq = sRed[((s2 * 2 + 1) * C + r0 + a) * 8 + jq];
-            aq[a][0] += pq.x; aq[a][1] += pq.y; aq[a][2] += pq.z; aq[a][3] += pq.w;
+        for (int k = 0; k < 4; ++k) {
+          const float4 sv = sS[(4 * q + k) * 8 + jq];
+          acc[0][0] = fmaf(xa[k], sv.x, acc[0][0]); acc[0][1] = fmaf(xa[k], sv.y, acc[0][1]);
+          acc[0][2] = fmaf(xa[k], sv.z, acc[0][2]); acc[0][3] = fmaf(xa[k], sv.w, acc[0][3]);
+          acc[1][0] = fmaf(xb[k], sv.x, acc[1][0]); acc[1][1] = fmaf(xb[k], sv.y, acc[1][1]);
+          acc[1][2] = fmaf(xb[k], sv.z, acc[1][2]); acc[1][3] = fmaf(xb[k], sv.w, acc[1][3]);
+        }
+      }
+    };
+    contract(sW, aw);
+    if (o) contract(sQt, aq);
+    if (split > 1) {  // partial sums of the split contraction, summed by the sp == 0 threads
+      sRed[((sp * 2 + 0) * C + r0) * 8 + jq] = make_float4(aw[0][0], aw[0][1], aw[0][2], aw[0][3]);
+      sRed[((sp * 2 + 0) * C + r1) * 8 + jq] = make_float4(aw[1][0], aw[1][1], aw[1][2], aw[1][3]);
+      if (o) {
+        sRed[((sp * 2 + 1) * C + r0) * 8 + jq] =
+            make_float4(aq[0][0], aq[0][1], aq[0][2], aq[0][3]);
+        sRed[((sp * 2 + 1) * C + r1) * 8 + jq] =
+            make_float4(aq[1][0], aq[1][1], aq[1][2], aq[1][3]);
+      }
+      __syncthreads();
+      if (sp == 0) {
+        for (int s2 = 1; s2 < split; ++s2) {
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const float4 pw = sRed[((s2 * 2 + 0) * C + r0 + a) * 8 + jq];
+            aw[a][0] += pw.x; aw[a][1] += pw.y; aw[a][2] += pw.z; aw[a][3] += pw.w;
+            if (o) {
+              const float4 pq = sRed[((s2 * 2 + 1) * C + r0 + a) * 8 + jq];
+              aq[a][0] += pq.x; aq[a][1] += pq.y; aq[a][2] += pq.z; aq[a][3] += pq.w;
+            }
           }
         }
       }
     }
-  }
-  if (sp == 0) {
+    if (sp == 0) {
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const float4 u = sU[(r0 + a) * 8 + jq];
-      sVp[(r0 + a) * 8 + jq] =
-          make_float4(u.x - aw[a][0], u.y - aw[a][1], u.z - aw[a][2], u.w - aw[a][3]);
-    }
-  }
-  __syncthreads();
-
-  // O = O_inter + Tril(A_qk) V' (Eq. 9)
-  if (o && sp == 0) {
-    for (int i = 0; i <= r1; ++i) {
-      const float4 v = sVp[i * 8 + jq];
-      const float a0 = i <= r0 ? sAq[r0 * C + i] : 0.f, a1 = sAq[r1 * C + i];
-      aq[0][0] = fmaf(a0, v.x, aq[0][0]); aq[0][1] = fmaf(a0, v.y, aq[0][1]);
-      aq[0][2] = fmaf(a0, v.z, aq[0][2]); aq[0][3] = fmaf(a0, v.w, aq[0][3]);
-      aq[1][0] = fmaf(a1, v.x, aq[1][0]); aq[1][1] = fmaf(a1, v.y, aq[1][1]);
-      aq[1][2] = fmaf(a1, v.z, aq[1][2]); aq[1][3] = fmaf(a1, v.w, aq[1][3]);
-    }
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      const int r = r0 + a;
-      if (r < L)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (4 * jq + e < NV)
-            o[((size_t)(t0 + r) * H + h) * Dv + j0 + 4 * jq + e] = from_f32<Tin>(aq[a][e]);
-    }
-  }
-  // S = Diag(gamma_C) S + Kt^T V' (Eq. 8): 4 x 4 tiles (rows 4 cq .. 4 cq + 3)
-  for (int t = tid; t < dq * 8; t += kSimtThreads) {
-    const int cq = t >> 3, jj = t & 7;
-    float acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float g = sGam[4 * cq + a];
-      const float4 sv = sS[(4 * cq + a) * 8 + jj];
-      acc[a][0] = g * sv.x; acc[a][1] = g * sv.y; acc[a][2] = g * sv.z; acc[a][3] = g * sv.w;
-    }
-    for (int i = 0; i < C; ++i) {
-      const float4 kv = sKt[i * dq + cq], v = sVp[i * 8 + jj];
-      const float kx[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        acc[a][0] = fmaf(kx[a], v.x, acc[a][0]); acc[a][1] = fmaf(kx[a], v.y, acc[a][1]);
-        acc[a][2] = fmaf(kx[a], v.z, acc[a][2]); acc[a][3] = fmaf(kx[a], v.w, acc[a][3]);
+      for (int a = 0; a < 2; ++a) {
+        const float4 u = sU[(r0 + a) * 8 + jq];
+        sVp[(r0 + a) * 8 + jq] =
+            make_float4(u.x - aw[a][0], u.y - aw[a][1], u.z - aw[a][2], u.w - aw[a][3]);
       }
     }
+    __syncthreads();  // V' complete; W, Qt and U are free for the next chunk
+    if (ci + 1 < nchunks) {
+      issue_a(c + 1);
+      cp_async_wait<1>();  // group B of this chunk has landed
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+
+    // O = O_inter + Tril(A_qk) V' (Eq. 9)
+    if (o && sp == 0) {
+      for (int i = 0; i <= r1; ++i) {
+        const float4 v = sVp[i * 8 + jq];
+        const float a0 = i <= r0 ? sAq[r0 * C + i] : 0.f, a1 = sAq[r1 * C + i];
+        aq[0][0] = fmaf(a0, v.x, aq[0][0]); aq[0][1] = fmaf(a0, v.y, aq[0][1]);
+        aq[0][2] = fmaf(a0, v.z, aq[0][2]); aq[0][3] = fmaf(a0, v.w, aq[0][3]);
+        aq[1][0] = fmaf(a1, v.x, aq[1][0]); aq[1][1] = fmaf(a1, v.y, aq[1][1]);
+        aq[1][2] = fmaf(a1, v.z, aq[1][2]); aq[1][3] = fmaf(a1, v.w, aq[1][3]);
+      }
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-      sS[(4 * cq + a) * 8 + jj] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+      for (int a = 0; a < 2; ++a) {
+        const int r = r0 + a;
+        if (r < L)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (4 * jq + e < NV)
+              o[((size_t)(t0 + r) * H + h) * Dv + j0 + 4 * jq + e] = from_f32<Tin>(aq[a][e]);
+      }
+    }
+    // S = Diag(gamma_C) S + Kt^T V' (Eq. 8): 4 x 4 tiles (rows 4 cq .. 4 cq + 3)
+    for (int t = tid; t < dq * 8; t += kSimtThreads) {
+      const int cq = t >> 3, jj = t & 7;
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float g = sGam[4 * cq + a];
+        const float4 sv = sS[(4 * cq + a) * 8 + jj];
+        acc[a][0] = g * sv.x; acc[a][1] = g * sv.y; acc[a][2] = g * sv.z; acc[a][3] = g * sv.w;
+      }
+      for (int i = 0; i < C; ++i) {
+        const float4 kv = sKt[i * dq + cq], v = sVp[i * 8 + jj];
+        const float kx[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          acc[a][0] = fmaf(kx[a], v.x, acc[a][0]); acc[a][1] = fmaf(kx[a], v.y, acc[a][1]);
+          acc[a][2] = fmaf(kx[a], v.z, acc[a][2]); acc[a][3] = fmaf(kx[a], v.w, acc[a][3]);
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        sS[(4 * cq + a) * 8 + jj] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    }
+    __syncthreads();  // the state update is complete; A_qk, Kt and gamma_C are free
   }
 }
 
@@ -492,9 +528,8 @@ __global__ void __launch_bounds__(kSimtThreads)
   const bool tiled = (Dk & 3) == 0 && (Dv & 3) == 0 && nt == kSimtThreads &&
                      (C == 16 || C == 32 || C == 64);
   if (tiled) {
-    for (int ci = 0; ci < nchunks; ++ci)
-      state_step_tiled<Tin>(ws, rec, c_first + ci, tb + ci * C, min(C, te - tb - ci * C), C, H,
-                            h, Dk, Dv, j0, NV, smem, o, states_out);
+    state_chain_tiled<Tin>(ws, rec, c_first, nchunks, tb, te, C, H, h, Dk, Dv, j0, NV, smem, o,
+                           states_out);
   } else {
     for (int ci = 0; ci < nchunks; ++ci) {
       const int c = c_first + ci;

@@ -146,6 +146,23 @@ struct SeqGeometry {
 };
 
 // ---------------------------------------------------------------------------------------------
+// Asynchronous 16-byte global -> shared copies (cp.async, L2 only) in commit groups: a thread
+// waits for its own groups; a barrier after the wait makes every thread's copies visible.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async_16B(void* dst_smem, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// waits until at most `pending` of this thread's most recent groups are still in flight
+template <int pending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(pending) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
 // Packed fp32 pairs (mov/fma/mul .f32x2, sm_100a): one issued instruction works on two values,
 // each rounded exactly as the scalar operation would round it.
 // ---------------------------------------------------------------------------------------------

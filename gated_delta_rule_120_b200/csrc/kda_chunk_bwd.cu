@@ -40,11 +40,12 @@ __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<floa
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
 }
+// acc += s b on packed pairs (each lane rounded as fmaf rounds it)
 __device__ __forceinline__ void fma4(float s, float4 b, float4& acc) {
-  acc.x = fmaf(s, b.x, acc.x);
-  acc.y = fmaf(s, b.y, acc.y);
-  acc.z = fmaf(s, b.z, acc.z);
-  acc.w = fmaf(s, b.w, acc.w);
+  const f32x2 ss = f2_pack(s, s);
+  const float2 lo = f2_unpack(f2_fma(ss, f2_pack(b.x, b.y), f2_pack(acc.x, acc.y)));
+  const float2 hi = f2_unpack(f2_fma(ss, f2_pack(b.z, b.w), f2_pack(acc.z, acc.w)));
+  acc = make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
 
@@ -332,20 +333,111 @@ struct RowVec {
   }
 };
 
-// acc[u][w] += sum_{k < K} X[(tm + 16u) * ldx + k] * Y[(tn + 16w) * ldy + k]  (K multiple of 4)
+// Factored ratio-form sums of one key channel over the rows r = kParity, kParity + 2, ... of the
+// chunk (i <= r; dA and dP are zero for i >= r and i > r, so whole float4 groups are read):
+//   row r:     s1 = sum_i dA_ri kF_i, s2 = sum_i dP_ri kF_i  ->  dk_r += beta_r E_r s1,
+//              dq_r += E_r s2, dg_r += beta_r k_r E_r s1 + q_r E_r s2
+//   column i:  cacc_i += dA_ri beta_r k_r E_r + dP_ri q_r E_r   (scaled by F_i by the caller)
+// with e_ri = E_r F_i, E_r = exp(g_r - m), F_i = exp(m - g_i), kF_i = k_i F_i.
+template <int kParity>
+__device__ __forceinline__ void ratio_rows(const float* sdA, const float* sdP, int ldc,
+                                           const float* sK, const float* sQ, const float* sG,
+                                           const float* sbeta, int ldk, int a, float m,
+                                           const float (&kF)[kBwdC], float (&cacc)[kBwdC],
+                                           float* dk, float* dq, float* dg) {
+#pragma unroll
+  for (int r = kParity; r < kBwdC; r += 2) {
+    const float Er = expf(sG[r * ldk + a] - m);
+    const float bE = sbeta[r] * Er;
+    const float bkE = bE * sK[r * ldk + a], qE = sQ[r * ldk + a] * Er;
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i4 = 0; i4 <= r / 4; ++i4) {
+      const float4 da = ld4(sdA + r * ldc + 4 * i4), dp = ld4(sdP + r * ldc + 4 * i4);
+      const float xa[4] = {da.x, da.y, da.z, da.w}, xp[4] = {dp.x, dp.y, dp.z, dp.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = 4 * i4 + u;
+        s1 = fmaf(xa[u], kF[i], s1);
+        s2 = fmaf(xp[u], kF[i], s2);
+        cacc[i] = fmaf(xa[u], bkE, fmaf(xp[u], qE, cacc[i]));
+      }
+    }
+    dk[r * ldk + a] += bE * s1;
+    dq[r * ldk + a] += Er * s2;
+    dg[r * ldk + a] += bkE * s1 + qE * s2;
+  }
+}
+
+// acc[u][w] += sum_{k < K} X[(tm + 16u) * ldx + k] * Y[(tn + 16w) * ldy + k]  (K multiple of 4),
+// on packed pairs: the even and the odd k are summed apart and added at the end
 __device__ __forceinline__ void abt_2x2(const float* X, int ldx, const float* Y, int ldy, int K,
                                         int tm, int tn, float (&acc)[2][2]) {
   const float* x0 = X + tm * ldx;
   const float* x1 = X + (tm + 16) * ldx;
   const float* y0 = Y + tn * ldy;
   const float* y1 = Y + (tn + 16) * ldy;
+  f32x2 p[2][2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) p[u][w] = f2_pack(0.f, 0.f);
   for (int k = 0; k < K; k += 4) {
     const float4 a0 = ld4(x0 + k), a1 = ld4(x1 + k), b0 = ld4(y0 + k), b1 = ld4(y1 + k);
-    acc[0][0] = dot4(a0, b0, acc[0][0]);
-    acc[0][1] = dot4(a0, b1, acc[0][1]);
-    acc[1][0] = dot4(a1, b0, acc[1][0]);
-    acc[1][1] = dot4(a1, b1, acc[1][1]);
+    const f32x2 al[2] = {f2_pack(a0.x, a0.y), f2_pack(a1.x, a1.y)};
+    const f32x2 ah[2] = {f2_pack(a0.z, a0.w), f2_pack(a1.z, a1.w)};
+    const f32x2 bl[2] = {f2_pack(b0.x, b0.y), f2_pack(b1.x, b1.y)};
+    const f32x2 bh[2] = {f2_pack(b0.z, b0.w), f2_pack(b1.z, b1.w)};
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int w = 0; w < 2; ++w) p[u][w] = f2_fma(ah[u], bh[w], f2_fma(al[u], bl[w], p[u][w]));
   }
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const float2 v = f2_unpack(p[u][w]);
+      acc[u][w] += v.x + v.y;
+    }
+}
+
+// Two products sharing the right operand: accA[u][w] += X1 row . Y row, accB[u][w] += X2 row .
+// Y row, with abt_2x2's tiles and packed pairs (each Y row read once for both).
+__device__ __forceinline__ void abt_2x2_dual(const float* XA, const float* XB, int ldx,
+                                             const float* Y, int ldy, int K, int tm, int tn,
+                                             float (&accA)[2][2], float (&accB)[2][2]) {
+  const float* y0 = Y + tn * ldy;
+  const float* y1 = Y + (tn + 16) * ldy;
+  f32x2 pa[2][2], pb[2][2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) pa[u][w] = pb[u][w] = f2_pack(0.f, 0.f);
+  for (int k = 0; k < K; k += 4) {
+    const float4 b0 = ld4(y0 + k), b1 = ld4(y1 + k);
+    const f32x2 bl[2] = {f2_pack(b0.x, b0.y), f2_pack(b1.x, b1.y)};
+    const f32x2 bh[2] = {f2_pack(b0.z, b0.w), f2_pack(b1.z, b1.w)};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float4 a = ld4(XA + (tm + 16 * u) * ldx + k), c = ld4(XB + (tm + 16 * u) * ldx + k);
+      const f32x2 al = f2_pack(a.x, a.y), ah = f2_pack(a.z, a.w);
+      const f32x2 cl = f2_pack(c.x, c.y), ch = f2_pack(c.z, c.w);
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        pa[u][w] = f2_fma(ah, bh[w], f2_fma(al, bl[w], pa[u][w]));
+        pb[u][w] = f2_fma(ch, bh[w], f2_fma(cl, bl[w], pb[u][w]));
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const float2 va = f2_unpack(pa[u][w]), vb = f2_unpack(pb[u][w]);
+      accA[u][w] += va.x + va.y;
+      accB[u][w] += vb.x + vb.y;
+    }
 }
 
 template <typename Tin>
@@ -473,7 +565,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
 
-  // ---- P1: products with the chunk-start state S (rows streamed 32 at a time)
+  // ---- P1: products with the chunk-start state S, its rows streamed in slices of 32: slice s of
+  // S in Y1 / Y2 alternately and of dS' in X1 (free until V' is stored), slice s + 1 fetched while
+  // slice s is used; the last step fetches P2's first slice of dS' instead.
   // V' = U - W S: this thread's rows {tm, tm + 16}, column groups {4 tn, 64 + 4 tn}
   float4 vp[2][2];
 #pragma unroll
@@ -484,33 +578,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       vp[u][w] = j < Dv ? ld4(r_ + rec.off_u + (tm + 16 * u) * Dv + j)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  for (int a0 = 0; a0 < Dk; a0 += 32) {
+  const int nsl = (Dk + 31) / 32;
+  auto sbuf = [&](int i) { return (i & 1) ? Y2 : Y1; };  // the two slice buffers
+  auto fetch_rows = [&](float* dst, const float* src, int a0) {  // (state rows: 16-byte aligned)
     const int na = min(32, Dk - a0);
-    __syncthreads();  // previous slice consumed (and, the first time, the cumsum done)
-    for (int idx = tid; idx < na * Dv4; idx += nt) {  // (state rows: 16-byte aligned)
+    for (int idx = tid; idx < na * Dv4; idx += nt) {
       const int aa = idx / Dv4, j4 = idx - aa * Dv4;
-      cp_async_16B(Y1 + aa * ldv + 4 * j4, S0 + (size_t)(a0 + aa) * Dv + 4 * j4);
-      cp_async_16B(Y2 + aa * ldv + 4 * j4, dS1 + (size_t)(a0 + aa) * Dv + 4 * j4);
+      cp_async_16B(dst + aa * ldv + 4 * j4, src + (size_t)(a0 + aa) * Dv + 4 * j4);
+    }
+  };
+  fetch_rows(Y1, S0, 0);
+  fetch_rows(X1, dS1, 0);
+  cp_async_commit();
+  for (int sl = 0; sl < nsl; ++sl) {
+    const int a0 = 32 * sl, na = min(32, Dk - a0);
+    const float* Ys = sbuf(sl);
+    cp_async_wait<0>();
+    __syncthreads();  // slice sl landed; slice sl - 1 consumed (the first time: the cumsum done)
+    {  // dgamma_C = rowsum(dS' . S): eight lanes per row, each over every eighth float4
+      const int aa = tid >> 3, part = tid & 7;
+      float s = 0.f;
+      if (aa < na)
+        for (int j = 4 * part; j < Dv; j += 32)
+          s = dot4(ld4(X1 + aa * ldv + j), ld4(Ys + aa * ldv + j), s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (aa < na && part == 0) sdgam[a0 + aa] = s;
+    }
+    __syncthreads();  // X1 and the other slice buffer are free
+    if (sl + 1 < nsl) {
+      fetch_rows(sbuf(sl + 1), S0, a0 + 32);
+      fetch_rows(X1, dS1, a0 + 32);
+    } else {
+      fetch_rows(sbuf(sl + 1), dS1, 0);
     }
     cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    for (int aa = 0; aa < na; ++aa) {
-      const float w0 = X4[tm * ldk + a0 + aa], w1 = X4[(tm + 16) * ldk + a0 + aa];
+    for (int a4 = 0; a4 < na; a4 += 4) {  // (na is a multiple of 4)
+      const float4 w04 = ld4(X4 + tm * ldk + a0 + a4), w14 = ld4(X4 + (tm + 16) * ldk + a0 + a4);
+      const float w0s[4] = {w04.x, w04.y, w04.z, w04.w}, w1s[4] = {w14.x, w14.y, w14.z, w14.w};
 #pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const int j = 4 * tn + 64 * w;
-        if (j < Dv) {
-          const float4 sv = ld4(Y1 + aa * ldv + j);
-          fma4(-w0, sv, vp[0][w]);
-          fma4(-w1, sv, vp[1][w]);
+      for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int j = 4 * tn + 64 * w;
+          if (j < Dv) {
+            const float4 sv = ld4(Ys + (a4 + e) * ldv + j);
+            fma4(-w0s[e], sv, vp[0][w]);
+            fma4(-w1s[e], sv, vp[1][w]);
+          }
         }
-      }
     }
     if (tn < na || tn + 16 < na) {  // dQt = dO S^T, dW = -dV' S^T over this slice's columns
       float a1[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, a2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-      abt_2x2(sdO, ldv, Y1, ldv, Dv, tm, tn, a1);
-      abt_2x2(sdV, ldv, Y1, ldv, Dv, tm, tn, a2);
+      abt_2x2_dual(sdO, sdV, ldv, Ys, ldv, Dv, tm, tn, a1, a2);
 #pragma unroll
       for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -522,19 +643,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
     }
-    {  // dgamma_C = rowsum(dS' . S): eight lanes per row, each over every eighth float4
-      const int aa = tid >> 3, part = tid & 7;
-      float s = 0.f;
-      if (aa < na)
-        for (int j = 4 * part; j < Dv; j += 32)
-          s = dot4(ld4(Y2 + aa * ldv + j), ld4(Y1 + aa * ldv + j), s);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      s += __shfl_xor_sync(0xffffffffu, s, 4);
-      if (aa < na && part == 0) sdgam[a0 + aa] = s;
-    }
   }
-  __syncthreads();
 #pragma unroll
   for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -542,20 +651,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int j = 4 * tn + 64 * w;
       if (j < Dv) st4(X1 + (tm + 16 * u) * ldv + j, vp[u][w]);
     }
-  // ---- P2: dKt = V' dS'^T (W is dead: its buffer takes dKt)
-  for (int a0 = 0; a0 < Dk; a0 += 32) {
-    const int na = min(32, Dk - a0);
-    __syncthreads();
-    for (int idx = tid; idx < na * Dv4; idx += nt) {
-      const int aa = idx / Dv4, j4 = idx - aa * Dv4;
-      cp_async_16B(Y2 + aa * ldv + 4 * j4, dS1 + (size_t)(a0 + aa) * Dv + 4 * j4);
-    }
-    cp_async_commit();
+  // ---- P2: dKt = V' dS'^T over slices of dS' rows in the same two buffers, slice s + 1 fetched
+  // while slice s is used (W is dead: its buffer takes dKt)
+  for (int sl = 0; sl < nsl; ++sl) {
+    const int a0 = 32 * sl, na = min(32, Dk - a0);
+    const float* Ys = sbuf(nsl + sl);
     cp_async_wait<0>();
-    __syncthreads();
+    __syncthreads();  // slice sl landed; V' stored; slice sl - 1 consumed
+    if (sl + 1 < nsl) {
+      fetch_rows(sbuf(nsl + sl + 1), dS1, a0 + 32);
+      cp_async_commit();
+    }
     if (tn < na || tn + 16 < na) {
       float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-      abt_2x2(X1, ldv, Y2, ldv, Dv, tm, tn, acc);
+      abt_2x2(X1, ldv, Ys, ldv, Dv, tm, tn, acc);
 #pragma unroll
       for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -687,10 +796,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     X3[x] = dkg * e + dkt * et;                                // dk
   }
   __syncthreads();
-  // ratio-form products through A and P: threads [0, Dk) accumulate along rows (row r over
-  // i <= r) into the dk / dq / dg buffers, threads [128, 128 + Dk) along columns (column i over
-  // r >= i) into the dead Gamma.K / d(Gamma.K) buffers; each thread owns one key channel
-  if (tid < Dk) {
+  // ratio-form products through A and P, per key channel, each pair (r >= i) weighed by
+  // e_ri = exp(g_r - g_i) <= 1. When every channel's cumulative decay spans at most 2 x 40 nats
+  // over the chunk, e_ri is taken as E_r F_i around the channel's midpoint m (every factor within
+  // e^+-40, so each product keeps fp32 relative precision): two threads per channel (even and odd
+  // rows), 64 exponentials per channel instead of one per pair, four FMAs per pair. Otherwise
+  // threads [0, Dk) accumulate along rows (row r over i <= r) into the dk / dq / dg buffers and
+  // threads [128, 128 + Dk) along columns (column i over r >= i), one exponential per pair.
+  // Column sums go to the dead Gamma.K / d(Gamma.K) buffers either way.
+  bool span_ok = true;
+  float gmid = 0.f;
+  if ((tid & 127) < Dk) {
+    const int a = tid & 127;
+    float gmin = sG[a], gmax = gmin;
+    for (int r = 1; r < C; ++r) {
+      const float g = sG[r * ldk + a];
+      gmin = fminf(gmin, g);
+      gmax = fmaxf(gmax, g);
+    }
+    span_ok = gmax - gmin <= 80.f;  // false for NaN or infinite decays
+    gmid = 0.5f * (gmax + gmin);
+  }
+  if (__syncthreads_and(span_ok)) {
+    const int a = tid & 127, half = tid >> 7;
+    float F[C], kF[C], cacc[C];
+    if (a < Dk) {
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        F[i] = expf(gmid - sG[i * ldk + a]);
+        kF[i] = sK[i * ldk + a] * F[i];
+        cacc[i] = 0.f;
+      }
+      if (half == 0)
+        ratio_rows<0>(sdM, sdP, ldc, sK, sQ, sG, sbeta, ldk, a, gmid, kF, cacc, X3, X2, X1);
+      else
+        ratio_rows<1>(sdM, sdP, ldc, sK, sQ, sG, sbeta, ldk, a, gmid, kF, cacc, X3, X2, X1);
+      if (half == 0) {
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+          Y1[i * ldk + a] = F[i] * cacc[i];
+          Y2[i * ldk + a] = -kF[i] * cacc[i];
+        }
+      }
+    }
+    __syncthreads();
+    if (a < Dk && half == 1) {
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        Y1[i * ldk + a] += F[i] * cacc[i];
+        Y2[i * ldk + a] -= kF[i] * cacc[i];
+      }
+    }
+  } else if (tid < Dk) {
     const int a = tid;
     for (int r = 0; r < C; ++r) {
       const float kr = sK[r * ldk + a], qr = sQ[r * ldk + a], gr = sG[r * ldk + a];

@@ -395,10 +395,8 @@ __device__ __forceinline__ void state_chain_tiled(const float* __restrict__ ws,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float4 sv = sS[(4 * q + k) * 8 + jq];
-          acc[0][0] = fmaf(xa[k], sv.x, acc[0][0]); acc[0][1] = fmaf(xa[k], sv.y, acc[0][1]);
-          acc[0][2] = fmaf(xa[k], sv.z, acc[0][2]); acc[0][3] = fmaf(xa[k], sv.w, acc[0][3]);
-          acc[1][0] = fmaf(xb[k], sv.x, acc[1][0]); acc[1][1] = fmaf(xb[k], sv.y, acc[1][1]);
-          acc[1][2] = fmaf(xb[k], sv.z, acc[1][2]); acc[1][3] = fmaf(xb[k], sv.w, acc[1][3]);
+          fma_s4(xa[k], sv, acc[0]);
+          fma_s4(xb[k], sv, acc[1]);
         }
       }
     };
@@ -450,10 +448,8 @@ __device__ __forceinline__ void state_chain_tiled(const float* __restrict__ ws,
       for (int i = 0; i <= r1; ++i) {
         const float4 v = sVp[i * 8 + jq];
         const float a0 = i <= r0 ? sAq[r0 * C + i] : 0.f, a1 = sAq[r1 * C + i];
-        aq[0][0] = fmaf(a0, v.x, aq[0][0]); aq[0][1] = fmaf(a0, v.y, aq[0][1]);
-        aq[0][2] = fmaf(a0, v.z, aq[0][2]); aq[0][3] = fmaf(a0, v.w, aq[0][3]);
-        aq[1][0] = fmaf(a1, v.x, aq[1][0]); aq[1][1] = fmaf(a1, v.y, aq[1][1]);
-        aq[1][2] = fmaf(a1, v.z, aq[1][2]); aq[1][3] = fmaf(a1, v.w, aq[1][3]);
+        fma_s4(a0, v, aq[0]);
+        fma_s4(a1, v, aq[1]);
       }
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
@@ -479,10 +475,7 @@ __device__ __forceinline__ void state_chain_tiled(const float* __restrict__ ws,
         const float4 kv = sKt[i * dq + cq], v = sVp[i * 8 + jj];
         const float kx[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          acc[a][0] = fmaf(kx[a], v.x, acc[a][0]); acc[a][1] = fmaf(kx[a], v.y, acc[a][1]);
-          acc[a][2] = fmaf(kx[a], v.z, acc[a][2]); acc[a][3] = fmaf(kx[a], v.w, acc[a][3]);
-        }
+        for (int a = 0; a < 4; ++a) fma_s4(kx[a], v, acc[a]);
       }
 #pragma unroll
       for (int a = 0; a < 4; ++a)

@@ -187,5 +187,15 @@ __device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// acc[0..3] += s * b on two packed pairs (each element rounded as fmaf rounds it)
+__device__ __forceinline__ void fma_s4(float s, float4 b, float (&acc)[4]) {
+  const f32x2 ss = f2_pack(s, s);
+  const float2 lo = f2_unpack(f2_fma(ss, f2_pack(b.x, b.y), f2_pack(acc[0], acc[1])));
+  const float2 hi = f2_unpack(f2_fma(ss, f2_pack(b.z, b.w), f2_pack(acc[2], acc[3])));
+  acc[0] = lo.x;
+  acc[1] = lo.y;
+  acc[2] = hi.x;
+  acc[3] = hi.y;
+}
 
 }  // namespace kda

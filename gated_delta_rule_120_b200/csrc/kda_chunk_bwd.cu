@@ -294,18 +294,6 @@ struct BwdSmem {  // float offsets of the chunk-local pass (C = 32)
   }
 };
 
-// A 16-byte vector of Tin into fp32 shared memory (4 floats, or 8 from bf16).
-__device__ __forceinline__ void store_vec(float* p, uint4 u, float) {
-  st4(p, make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
-                     __uint_as_float(u.w)));
-}
-__device__ __forceinline__ void store_vec(float* p, uint4 u, __nv_bfloat16) {
-  st4(p, make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u)));
-  st4(p + 4, make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
-                         __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u)));
-}
-
 // A [kBwdC][D] tile of Tin rows (row r at src + r * stride; rows >= L read as zeros; D <= 128 a
 // multiple of kPer; 16-byte aligned rows) moved into fp32 shared-memory rows as 16-byte vectors:
 // load() issues every load of the thread, store() converts them once they have been issued.

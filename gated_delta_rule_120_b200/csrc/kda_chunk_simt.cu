@@ -112,20 +112,22 @@ cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t
 // K1: chunk-local UT transform (fp32, CUDA cores)
 // ----------------------------------------------------------------------------------------------
 template <typename Tin>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, 3)
     chunk_local_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                             const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                             const float* __restrict__ beta, SeqGeometry geo, int H, int Dk, int Dv,
                             float* __restrict__ ws, SimtRecord rec, Fusion fz) {
   extern __shared__ __align__(16) float smem[];
   const int C = geo.C;
-  float* sk = smem;            // [C][Dk]  k, later Gamma.K
-  float* sq = sk + C * Dk;     // [C][Dk]
+  const int ldk = Dk + 4;      // row pitch of sk: rows of one float4 column hit distinct banks
+  float* sk = smem;            // [C][ldk] k (k F in the factored form), later Gamma.K
+  float* sq = sk + C * ldk;    // [C][Dk]
   float* sv = sq + C * Dk;     // [C][Dv]
-  float* sg = sv + C * Dv;     // [C][Dk]  cumulative log decay
+  float* sg = sv + C * Dv;     // [C][Dk]  cumulative log decay (E in the factored form)
   float* sA = sg + C * Dk;     // [C][C]   A_kk (strict lower), then M
   float* sT = sA + C * C;      // [C][C]   (I + A)^{-1}
   float* sb = sT + C * C;      // [C]
+  float* smid = sb + C;        // [Dk]     per-channel midpoint m of g (factored form)
 
   if (!geo.ok()) return;
   const ChunkItem item = chunk_item();
@@ -138,20 +140,41 @@ __global__ void __launch_bounds__(kSimtThreads)
   float* out = ws + rec.record_floats * ((size_t)c * H + h);
 
   const float neg_a = fz.A_log ? -expf(fz.A_log[h]) : 0.f;
-  for (int idx = tid; idx < C * Dk; idx += nt) {
-    const int r = idx / Dk, cc = idx - r * Dk;
-    const size_t gi = ((size_t)(t0 + r) * H + h) * Dk + cc;
-    const bool in = r < L;
-    sk[idx] = in ? to_f32(k[gi]) : 0.f;
-    sq[idx] = in ? to_f32(q[gi]) : 0.f;
-    float la = in ? log_alpha[gi] : 0.f;
-    if (fz.A_log && in)  // fused gate: raw gate -> log decay
-      la = neg_a * softplus_f(la + (fz.dt_bias ? fz.dt_bias[h * Dk + cc] : 0.f));
-    sg[idx] = la;
+  constexpr int kPer = 16 / sizeof(Tin);
+  const bool vec_in = ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                        reinterpret_cast<uintptr_t>(v)) & 15) == 0 &&
+                      Dk % kPer == 0 && Dv % kPer == 0;
+  const bool vec_la = !fz.A_log && (reinterpret_cast<uintptr_t>(log_alpha) & 15) == 0 &&
+                      Dk % 4 == 0;
+  const size_t bk = ((size_t)t0 * H + h) * Dk, bv = ((size_t)t0 * H + h) * Dv;
+  if (vec_in) {  // 16-byte vectors, several in flight per thread
+    stage_rows_f32<Tin>(sk, ldk, k + bk, (size_t)H * Dk, C, L, Dk, tid, nt);
+    stage_rows_f32<Tin>(sq, Dk, q + bk, (size_t)H * Dk, C, L, Dk, tid, nt);
+    stage_rows_f32<Tin>(sv, Dv, v + bv, (size_t)H * Dv, C, L, Dv, tid, nt);
+  } else {
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, cc = idx - r * Dk;
+      const size_t gi = bk + (size_t)r * H * Dk + cc;
+      const bool in = r < L;
+      sk[r * ldk + cc] = in ? to_f32(k[gi]) : 0.f;
+      sq[idx] = in ? to_f32(q[gi]) : 0.f;
+    }
+    for (int idx = tid; idx < C * Dv; idx += nt) {
+      const int r = idx / Dv, cc = idx - r * Dv;
+      sv[idx] = r < L ? to_f32(v[bv + (size_t)r * H * Dv + cc]) : 0.f;
+    }
   }
-  for (int idx = tid; idx < C * Dv; idx += nt) {
-    const int r = idx / Dv, cc = idx - r * Dv;
-    sv[idx] = r < L ? to_f32(v[((size_t)(t0 + r) * H + h) * Dv + cc]) : 0.f;
+  if (vec_la) {
+    stage_rows_f32<float>(sg, Dk, log_alpha + bk, (size_t)H * Dk, C, L, Dk, tid, nt);
+  } else {
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, cc = idx - r * Dk;
+      const bool in = r < L;
+      float la = in ? log_alpha[bk + (size_t)r * H * Dk + cc] : 0.f;
+      if (fz.A_log && in)  // fused gate: raw gate -> log decay
+        la = neg_a * softplus_f(la + (fz.dt_bias ? fz.dt_bias[h * Dk + cc] : 0.f));
+      sg[idx] = la;
+    }
   }
   for (int r = tid; r < C; r += nt) sb[r] = r < L ? beta[(size_t)(t0 + r) * H + h] : 0.f;
   __syncthreads();
@@ -159,7 +182,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     for (int r = warp; r < C; r += nt / 32) {
       float ssk = 0.f, ssq = 0.f;
       for (int cc = lane; cc < Dk; cc += 32) {
-        ssk += sk[r * Dk + cc] * sk[r * Dk + cc];
+        ssk += sk[r * ldk + cc] * sk[r * ldk + cc];
         ssq += sq[r * Dk + cc] * sq[r * Dk + cc];
       }
 #pragma unroll
@@ -169,7 +192,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       }
       const float ik = rsqrtf(ssk + fz.eps), iq = rsqrtf(ssq + fz.eps);
       for (int cc = lane; cc < Dk; cc += 32) {
-        sk[r * Dk + cc] *= ik;
+        sk[r * ldk + cc] *= ik;
         sq[r * Dk + cc] *= iq;
       }
     }
@@ -186,40 +209,115 @@ __global__ void __launch_bounds__(kSimtThreads)
   }
   __syncthreads();
 
-  // A_kk and A_qk: one warp per (r, i) pair with i <= r, lanes over key channels
+  // A_kk and A_qk. With d_k a multiple of 4 and every key channel's cumulative decay spanning at
+  // most 80 nats over the chunk, exp(g_r - g_i) = E_r F_i around the channel's midpoint m
+  // (E = exp(g - m), F = exp(m - g), each factor within e^+-40, so every term keeps fp32 relative
+  // precision): sk <- k F, sg <- E, and A_kk = (k F E^2)(k F)^T, A_qk = (q E)(k F)^T are
+  // register-tiled products over d_k (2 x 2 tiles: rows {rp, rp + C/2}, columns {ip, ip + C/2};
+  // sk's padded pitch spreads a warp's 16 columns over the banks). Otherwise one warp per (r, i)
+  // pair with lanes over key channels, one exponential per term.
   float* gAqk = out + rec.off_aqk;
-  const int npairs = C * (C + 1) / 2;
-  for (int p = warp; p < npairs; p += nt / 32) {
-    int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
-    while ((r + 1) * (r + 2) / 2 <= p) ++r;
-    while (r * (r + 1) / 2 > p) --r;
-    const int i = p - r * (r + 1) / 2;
-    float akk = 0.f, aqk = 0.f;
-    for (int cc = lane; cc < Dk; cc += 32) {
-      // gamma_r / gamma_i <= 1; the fast exponential's relative error (a few 1e-7 plus the
-      // argument's rounding, < 1e-5 for any argument above -87) is far below fp32 parity needs
-      const float f = __expf(sg[r * Dk + cc] - sg[i * Dk + cc]);
-      const float ki = sk[i * Dk + cc] * f;
-      akk += sk[r * Dk + cc] * ki;
-      aqk += sq[r * Dk + cc] * ki;
+  float* sgC = smid + Dk;  // [Dk] g of the chunk's last row (gamma_C), kept in the factored form
+  bool span_ok = (Dk & 3) == 0;
+  for (int cc = tid; cc < Dk; cc += nt) {
+    float gmin = sg[cc], gmax = gmin;
+    for (int r = 1; r < C; ++r) {
+      const float g = sg[r * Dk + cc];
+      gmin = fminf(gmin, g);
+      gmax = fmaxf(gmax, g);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      akk += __shfl_xor_sync(0xffffffffu, akk, off);
-      aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
-    }
-    if (lane == 0) {
-      sA[r * C + i] = (i < r) ? sb[r] * akk : 0.f;
-      gAqk[r * C + i] = aqk;
-      if (rec.off_b != SimtRecord::kNone) out[rec.off_b + r * C + i] = (i < r) ? akk : 0.f;
-    }
+    span_ok = span_ok && gmax - gmin <= 80.f;  // false for NaN or infinite decays
+    smid[cc] = 0.5f * (gmax + gmin);
+    sgC[cc] = sg[(C - 1) * Dk + cc];
   }
-  for (int idx = tid; idx < C * C; idx += nt) {  // upper triangles
-    const int r = idx / C, i = idx - r * C;
-    if (i > r) {
-      sA[idx] = 0.f;
-      gAqk[idx] = 0.f;
-      if (rec.off_b != SimtRecord::kNone) out[rec.off_b + idx] = 0.f;
+  const bool factored = __syncthreads_and(span_ok) != 0;
+  if (factored) {
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, cc = idx - r * Dk;
+      const float d = sg[idx] - smid[cc];
+      sk[r * ldk + cc] *= expf(-d);
+      sg[idx] = expf(d);
+    }
+    __syncthreads();
+    const int half = C >> 1, dq = Dk >> 2;
+    for (int t = tid; t < half * half; t += nt) {
+      const int rp = t / half, ip = t - rp * half;
+      const int rr[2] = {rp, rp + half}, ii[2] = {ip, ip + half};
+      f32x2 pk[2][2], pq[2][2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) pk[u][w] = pq[u][w] = f2_pack(0.f, 0.f);
+      for (int c4 = 0; c4 < dq; ++c4) {
+        f32x2 bl[2], bh[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const float4 b = *reinterpret_cast<const float4*>(sk + ii[w] * ldk + 4 * c4);
+          bl[w] = f2_pack(b.x, b.y);
+          bh[w] = f2_pack(b.z, b.w);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float4 kf = *reinterpret_cast<const float4*>(sk + rr[u] * ldk + 4 * c4);
+          const float4 e = *reinterpret_cast<const float4*>(sg + rr[u] * Dk + 4 * c4);
+          const float4 qv = *reinterpret_cast<const float4*>(sq + rr[u] * Dk + 4 * c4);
+          const f32x2 el = f2_pack(e.x, e.y), eh = f2_pack(e.z, e.w);
+          const f32x2 kel = f2_mul(f2_mul(f2_pack(kf.x, kf.y), el), el);
+          const f32x2 keh = f2_mul(f2_mul(f2_pack(kf.z, kf.w), eh), eh);
+          const f32x2 qel = f2_mul(f2_pack(qv.x, qv.y), el), qeh = f2_mul(f2_pack(qv.z, qv.w), eh);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            pk[u][w] = f2_fma(keh, bh[w], f2_fma(kel, bl[w], pk[u][w]));
+            pq[u][w] = f2_fma(qeh, bh[w], f2_fma(qel, bl[w], pq[u][w]));
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int r = rr[u], i = ii[w];
+          const float2 a2 = f2_unpack(pk[u][w]), q2 = f2_unpack(pq[u][w]);
+          const float akk = a2.x + a2.y, aqk = q2.x + q2.y;
+          sA[r * C + i] = (i < r) ? sb[r] * akk : 0.f;
+          gAqk[r * C + i] = (i <= r) ? aqk : 0.f;
+          if (rec.off_b != SimtRecord::kNone) out[rec.off_b + r * C + i] = (i < r) ? akk : 0.f;
+        }
+    }
+  } else {
+    const int npairs = C * (C + 1) / 2;
+    for (int p = warp; p < npairs; p += nt / 32) {
+      int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+      while ((r + 1) * (r + 2) / 2 <= p) ++r;
+      while (r * (r + 1) / 2 > p) --r;
+      const int i = p - r * (r + 1) / 2;
+      float akk = 0.f, aqk = 0.f;
+      for (int cc = lane; cc < Dk; cc += 32) {
+        // gamma_r / gamma_i <= 1; the fast exponential's relative error (a few 1e-7 plus the
+        // argument's rounding, < 1e-5 for any argument above -87) is far below fp32 parity needs
+        const float f = __expf(sg[r * Dk + cc] - sg[i * Dk + cc]);
+        const float ki = sk[i * ldk + cc] * f;
+        akk += sk[r * ldk + cc] * ki;
+        aqk += sq[r * Dk + cc] * ki;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        akk += __shfl_xor_sync(0xffffffffu, akk, off);
+        aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
+      }
+      if (lane == 0) {
+        sA[r * C + i] = (i < r) ? sb[r] * akk : 0.f;
+        gAqk[r * C + i] = aqk;
+        if (rec.off_b != SimtRecord::kNone) out[rec.off_b + r * C + i] = (i < r) ? akk : 0.f;
+      }
+    }
+    for (int idx = tid; idx < C * C; idx += nt) {  // upper triangles
+      const int r = idx / C, i = idx - r * C;
+      if (i > r) {
+        sA[idx] = 0.f;
+        gAqk[idx] = 0.f;
+        if (rec.off_b != SimtRecord::kNone) out[rec.off_b + idx] = 0.f;
+      }
     }
   }
   __syncthreads();
@@ -247,41 +345,51 @@ __global__ void __launch_bounds__(kSimtThreads)
     sT[idx] *= sb[idx % C];
   }
 
-  // Kt = (gamma_C/gamma_i) k_i, Qt = gamma_r q_r, gamma_C; then sk <- Gamma.K
-  const float* gC = sg + (C - 1) * Dk;
-  for (int idx = tid; idx < C * Dk; idx += nt) {
-    const int cc = idx % Dk;
-    const float g = sg[idx];
-    const float kk = sk[idx];
-    const float eg = __expf(g);  // operand scales (arguments <= 0); the carried gamma_C uses expf
-    out[rec.off_kt + idx] = kk * __expf(gC[cc] - g);
-    out[rec.off_qt + idx] = sq[idx] * eg;
-    sk[idx] = kk * eg;
+  // Kt = (gamma_C/gamma_i) k_i, Qt = gamma_r q_r, gamma_C; then sk <- Gamma.K. In the factored
+  // form (sk = k F, sg = E): Kt = k F E_C, Qt = q E e^m, Gamma.K = k F E^2 e^m.
+  if (factored) {
+    const float* EC = sg + (C - 1) * Dk;
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, cc = idx - r * Dk;
+      const float e = sg[idx], em = expf(smid[cc]), kf = sk[r * ldk + cc];
+      out[rec.off_kt + idx] = kf * EC[cc];
+      out[rec.off_qt + idx] = sq[idx] * e * em;
+      sk[r * ldk + cc] = kf * e * e * em;
+    }
+  } else {
+    const float* gC = sg + (C - 1) * Dk;
+    for (int idx = tid; idx < C * Dk; idx += nt) {
+      const int r = idx / Dk, cc = idx - r * Dk;
+      const float g = sg[idx];
+      const float kk = sk[r * ldk + cc];
+      const float eg = __expf(g);  // operand scales (arguments <= 0); gamma_C uses expf
+      out[rec.off_kt + idx] = kk * __expf(gC[cc] - g);
+      out[rec.off_qt + idx] = sq[idx] * eg;
+      sk[r * ldk + cc] = kk * eg;
+    }
   }
-  for (int cc = tid; cc < Dk; cc += nt) out[rec.off_gam + cc] = expf(gC[cc]);
+  for (int cc = tid; cc < Dk; cc += nt) out[rec.off_gam + cc] = expf(sgC[cc]);
   __syncthreads();
 
   // W = M (Gamma.K), U = M V
   if ((Dk & 3) == 0 && (Dv & 3) == 0) {  // 2 x 4 register tiles, float4 rows and record stores
     const int dq = Dk >> 2, vq = Dv >> 2;
-    const float4* k4 = reinterpret_cast<const float4*>(sk);
+    const float4* k4 = reinterpret_cast<const float4*>(sk);  // rows of ldk / 4 float4
     const float4* v4 = reinterpret_cast<const float4*>(sv);
     for (int t = tid; t < (C >> 1) * (dq + vq); t += nt) {
       const int rp = t / (dq + vq), cq = t - rp * (dq + vq);
       const int r0 = 2 * rp, r1 = r0 + 1;
-      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i <= r1; ++i) {  // M is lower triangular: M[r0][r1] = 0
         const float m0 = sT[r0 * C + i], m1 = sT[r1 * C + i];
-        const float4 x = cq < dq ? k4[i * dq + cq] : v4[i * vq + (cq - dq)];
-        a0.x = fmaf(m0, x.x, a0.x); a0.y = fmaf(m0, x.y, a0.y);
-        a0.z = fmaf(m0, x.z, a0.z); a0.w = fmaf(m0, x.w, a0.w);
-        a1.x = fmaf(m1, x.x, a1.x); a1.y = fmaf(m1, x.y, a1.y);
-        a1.z = fmaf(m1, x.z, a1.z); a1.w = fmaf(m1, x.w, a1.w);
+        const float4 x = cq < dq ? k4[i * (dq + 1) + cq] : v4[i * vq + (cq - dq)];
+        fma_s4(m0, x, a0);
+        fma_s4(m1, x, a1);
       }
       float* dst = cq < dq ? out + rec.off_w + 4 * cq : out + rec.off_u + 4 * (cq - dq);
       const int ld = cq < dq ? Dk : Dv;
-      *reinterpret_cast<float4*>(dst + r0 * ld) = a0;
-      *reinterpret_cast<float4*>(dst + r1 * ld) = a1;
+      *reinterpret_cast<float4*>(dst + r0 * ld) = make_float4(a0[0], a0[1], a0[2], a0[3]);
+      *reinterpret_cast<float4*>(dst + r1 * ld) = make_float4(a1[0], a1[1], a1[2], a1[3]);
     }
     return;
   }
@@ -290,7 +398,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     const int r = idx / wu, cc = idx - r * wu;
     float acc = 0.f;
     if (cc < Dk) {
-      for (int i = 0; i <= r; ++i) acc += sT[r * C + i] * sk[i * Dk + cc];
+      for (int i = 0; i <= r; ++i) acc += sT[r * C + i] * sk[i * ldk + cc];
       out[rec.off_w + r * Dk + cc] = acc;
     } else {
       const int cv = cc - Dk;
@@ -600,7 +708,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 }
 
 size_t simt_local_smem_bytes(int C, int Dk, int Dv) {
-  return sizeof(float) * ((size_t)3 * C * Dk + (size_t)C * Dv + 2 * (size_t)C * C + C);
+  return sizeof(float) * ((size_t)C * (Dk + 4) + 2 * (size_t)C * Dk + (size_t)C * Dv +
+                          2 * (size_t)C * C + C + 2 * (size_t)Dk);
 }
 size_t simt_state_smem_bytes(int C, int Dk) {
   return sizeof(float) * ((size_t)Dk * kSlice + 3 * (size_t)C * Dk + 2 * (size_t)C * kSlice +

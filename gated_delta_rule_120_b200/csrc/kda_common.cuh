@@ -163,6 +163,47 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ---------------------------------------------------------------------------------------------
+// 16-byte vectors of the input dtype into fp32 shared memory (4 floats, or 8 from bf16).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void store_vec(float* p, uint4 u, float) {
+  *reinterpret_cast<float4*>(p) = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                              __uint_as_float(u.z), __uint_as_float(u.w));
+}
+__device__ __forceinline__ void store_vec(float* p, uint4 u, __nv_bfloat16) {
+  *reinterpret_cast<float4*>(p) =
+      make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                  __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+  *reinterpret_cast<float4*>(p + 4) =
+      make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                  __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u));
+}
+
+// Rows of Tin (row r at src + r * stride; D a multiple of 16 / sizeof(Tin); 16-byte aligned
+// rows) into fp32 shared-memory rows of pitch ld (a multiple of 4), rows >= L as zeros: each
+// thread keeps four 16-byte loads in flight before converting them.
+template <typename Tin>
+__device__ __forceinline__ void stage_rows_f32(float* dst, int ld, const Tin* src, size_t stride,
+                                               int rows, int L, int D, int tid, int nt) {
+  constexpr int kPer = 16 / sizeof(Tin);
+  const int vpr = D / kPer, total = rows * vpr;
+  for (int base = 0; base < total; base += 4 * nt) {
+    uint4 x[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = base + m * nt + tid, r = idx / vpr, c = idx - r * vpr;
+      x[m] = (idx < total && r < L)
+                 ? __ldg(reinterpret_cast<const uint4*>(src + r * stride + c * kPer))
+                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = base + m * nt + tid, r = idx / vpr, c = idx - r * vpr;
+      if (idx < total) store_vec(dst + r * ld + c * kPer, x[m], Tin());
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Packed fp32 pairs (mov/fma/mul .f32x2, sm_100a): one issued instruction works on two values,
 // each rounded exactly as the scalar operation would round it.
 // ---------------------------------------------------------------------------------------------

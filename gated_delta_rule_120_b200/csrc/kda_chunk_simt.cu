@@ -111,6 +111,42 @@ cudaError_t launch_chunk_map(const int32_t* cu, int N, int total, int C, int32_t
 // ----------------------------------------------------------------------------------------------
 // K1: chunk-local UT transform (fp32, CUDA cores)
 // ----------------------------------------------------------------------------------------------
+
+// Column cc of T = (I + A)^{-1} (A strictly lower, C <= kMaxC rows), held in registers:
+// T[r][cc] = [r == cc] - sum_{cc <= j < r} A[r][j] T[j][cc] (col[j] = 0 for j < cc). Up to 32 rows
+// each row's sum runs as four partial sums (float4 groups of A's row, then the rest), so mostly
+// the newest column entries are on the dependency chain; 64 rows keep one sum (register budget).
+template <int kMaxC>
+__device__ __forceinline__ void forward_subst(const float* sA, float* sT, int C, int cc) {
+  float col[kMaxC];
+#pragma unroll
+  for (int r = 0; r < kMaxC; ++r) {
+    if (r < C) {
+      float val;
+      if (kMaxC <= 32) {
+        float acc[4] = {(r == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j4 = 0; j4 < r / 4; ++j4) {
+          const float4 a = *reinterpret_cast<const float4*>(sA + r * C + 4 * j4);
+          acc[0] = fmaf(-a.x, col[4 * j4], acc[0]);
+          acc[1] = fmaf(-a.y, col[4 * j4 + 1], acc[1]);
+          acc[2] = fmaf(-a.z, col[4 * j4 + 2], acc[2]);
+          acc[3] = fmaf(-a.w, col[4 * j4 + 3], acc[3]);
+        }
+#pragma unroll
+        for (int jj = 4 * (r / 4); jj < r; ++jj)
+          acc[jj & 3] = fmaf(-sA[r * C + jj], col[jj], acc[jj & 3]);
+        val = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      } else {
+        val = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < r; ++jj) val -= sA[r * C + jj] * col[jj];
+      }
+      col[r] = r >= cc ? val : 0.f;
+      sT[r * C + cc] = col[r];
+    }
+  }
+}
 template <typename Tin>
 __global__ void __launch_bounds__(kSimtThreads, 3)
     chunk_local_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
@@ -239,6 +275,7 @@ __global__ void __launch_bounds__(kSimtThreads, 3)
       sg[idx] = expf(d);
     }
     __syncthreads();
+    for (int cc = tid; cc < Dk; cc += nt) smid[cc] = expf(smid[cc]);  // e^m, read after the inverse
     const int half = C >> 1, dq = Dk >> 2;
     for (int t = tid; t < half * half; t += nt) {
       const int rp = t / half, ip = t - rp * half;
@@ -323,20 +360,12 @@ __global__ void __launch_bounds__(kSimtThreads, 3)
   __syncthreads();
 
   // (I + A)^{-1} by forward substitution, one lane per column of the inverse (warps 0 and 1
-  // for C = 64), the column held in registers: T[r][cc] = [r == cc] - sum_{cc<=j<r} A[r][j] T[j][cc]
+  // for C = 64)
   if (tid < C) {
-    const int cc = tid;
-    float col[64];
-#pragma unroll
-    for (int r = 0; r < 64; ++r) {
-      if (r < C) {
-        float val = (r == cc) ? 1.f : 0.f;
-#pragma unroll
-        for (int jj = 0; jj < r; ++jj) val -= sA[r * C + jj] * col[jj];  // col[j] = 0 for j < cc
-        col[r] = r >= cc ? val : 0.f;
-        sT[r * C + cc] = col[r];
-      }
-    }
+    if (C <= 32)
+      forward_subst<32>(sA, sT, C, tid);
+    else
+      forward_subst<64>(sA, sT, C, tid);
   }
   __syncthreads();
   // M = (I + A)^{-1} Diag(beta)  (the backward pass keeps (I + A)^{-1} itself)
@@ -346,12 +375,12 @@ __global__ void __launch_bounds__(kSimtThreads, 3)
   }
 
   // Kt = (gamma_C/gamma_i) k_i, Qt = gamma_r q_r, gamma_C; then sk <- Gamma.K. In the factored
-  // form (sk = k F, sg = E): Kt = k F E_C, Qt = q E e^m, Gamma.K = k F E^2 e^m.
+  // form (sk = k F, sg = E, smid = e^m): Kt = k F E_C, Qt = q E e^m, Gamma.K = k F E^2 e^m.
   if (factored) {
     const float* EC = sg + (C - 1) * Dk;
     for (int idx = tid; idx < C * Dk; idx += nt) {
       const int r = idx / Dk, cc = idx - r * Dk;
-      const float e = sg[idx], em = expf(smid[cc]), kf = sk[r * ldk + cc];
+      const float e = sg[idx], em = smid[cc], kf = sk[r * ldk + cc];
       out[rec.off_kt + idx] = kf * EC[cc];
       out[rec.off_qt + idx] = sq[idx] * e * em;
       sk[r * ldk + cc] = kf * e * e * em;

@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   const int t0 = geo.seq_begin(n) + (c - geo.first_chunk(n)) * kC;
   const int L = min(kC, geo.seq_end(n) - t0);
   uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)c * H + h);
+#ifdef KDA_BOUNDS_CHECK
   if (!KDA_IN_BOUNDS(kBufWork, rec, kRecBytes)) return;  // (uniform: the whole CTA leaves)
+#endif
 
   // ---- phase 1: raw k, q, v straight into their operand tiles; log decay into registers ------
   const int cg = tid & 15, rg = tid >> 4;  // thread = 8 channels (one 16-byte chunk) x 4 rows
@@ -194,11 +196,12 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   for (int i = 0; i < 4; ++i) {
     const int r = rg * 4 + i;
     const uint32_t off = tile_chunk_off(r, cg, 8192);
-    const size_t row = (size_t)(t0 + r) * H + h;
-    if (r < L && KDA_IN_BOUNDS(kBufK, k + row * kD + cg * 8, 16) &&
-        KDA_IN_BOUNDS(kBufQ, q + row * kD + cg * 8, 16) &&
-        KDA_IN_BOUNDS(kBufV, v + row * kD + cg * 8, 16) &&
-        KDA_IN_BOUNDS(kBufLogAlpha, log_alpha + row * kD + cg * 8, 32)) {
+    if (r < L KDA_AND_IN_BOUNDS(kBufK, k + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 16)
+              KDA_AND_IN_BOUNDS(kBufQ, q + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 16)
+              KDA_AND_IN_BOUNDS(kBufV, v + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 16)
+              KDA_AND_IN_BOUNDS(kBufLogAlpha,
+                                log_alpha + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 32)) {
+      const size_t row = (size_t)(t0 + r) * H + h;
       cp_async16(sb + kS1Kg + off, reinterpret_cast<const uint4*>(k + row * kD) + cg);
       cp_async16(sb + kS1Qg + off, reinterpret_cast<const uint4*>(q + row * kD) + cg);
       cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     }
   }
   if (tid < kC)
-    sBeta[tid] = (tid < L && KDA_IN_BOUNDS(kBufBeta, beta + (size_t)(t0 + tid) * H + h, 4))
+    sBeta[tid] = (tid < L KDA_AND_IN_BOUNDS(kBufBeta, beta + (size_t)(t0 + tid) * H + h, 4))
                      ? beta[(size_t)(t0 + tid) * H + h]
                      : 0.f;
   // the tensor memory and the barrier are first used in phase 3: set them up while the loads
@@ -231,10 +234,15 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     fence_mbar_init();
   }
   if (fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log decays
+#ifdef KDA_BOUNDS_CHECK
     const float neg_a = KDA_IN_BOUNDS(kBufALog, fz.A_log + h, 4) ? -expf(fz.A_log[h]) : 0.f;
-    float bias[8];
     const bool bias_ok =
         fz.dt_bias && KDA_IN_BOUNDS(kBufDtBias, fz.dt_bias + h * kD + cg * 8, 32);
+#else
+    const float neg_a = -expf(fz.A_log[h]);
+    const bool bias_ok = fz.dt_bias != nullptr;
+#endif
+    float bias[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) bias[j] = bias_ok ? fz.dt_bias[h * kD + cg * 8 + j] : 0.f;
 #pragma unroll
@@ -458,9 +466,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
         const int i = second ? t - 48 : t;
         if (i >= 16 * R + 16) continue;
         float kc[8];
-        const uint4* kci = reinterpret_cast<const uint4*>(k + ((size_t)(t0 + i) * H + h) * kD) + cg;
-        if (i < L && KDA_IN_BOUNDS(kBufK, kci, 16)) {
-          unpack8(*kci, kc);
+        if (i < L KDA_AND_IN_BOUNDS(kBufK, k + ((size_t)(t0 + i) * H + h) * kD + cg * 8, 16)) {
+          unpack8(*(reinterpret_cast<const uint4*>(k + ((size_t)(t0 + i) * H + h) * kD) + cg), kc);
           const float sc = fz.l2 ? sInv[i] : 1.f;
           const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i)) + cg * 8;
           const float4 ga = *reinterpret_cast<const float4*>(gi);
@@ -549,9 +556,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     for (int ii = 0; ii < 4; ++ii) {
       const int r = rg * 4 + ii;
       const uint32_t off = tile_chunk_off(r, cg, 8192);
-      const size_t row = (size_t)(t0 + r) * H + h;
-      if (r < L && KDA_IN_BOUNDS(kBufV, v + row * kD + cg * 8, 16) &&
-          KDA_IN_BOUNDS(kBufK, k + row * kD + cg * 8, 16)) {
+      if (r < L KDA_AND_IN_BOUNDS(kBufV, v + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 16)
+                KDA_AND_IN_BOUNDS(kBufK, k + ((size_t)(t0 + r) * H + h) * kD + cg * 8, 16)) {
+        const size_t row = (size_t)(t0 + r) * H + h;
         cp_async16(sb + kS1V + off, reinterpret_cast<const uint4*>(v + row * kD) + cg);
         float kf[8];
         unpack8(*(reinterpret_cast<const uint4*>(k + row * kD) + cg), kf);
@@ -577,9 +584,9 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       while (r * (r + 1) / 2 > p) --r;
       const int i = p - r * (r + 1) / 2;
       float akk = 0.f, aqk = 0.f;
-      const size_t rowr0 = (size_t)(t0 + r) * H + h, rowi0 = (size_t)(t0 + i) * H + h;
-      if (r < L && KDA_IN_BOUNDS(kBufK, k + rowr0 * kD, 256) &&
-          KDA_IN_BOUNDS(kBufK, k + rowi0 * kD, 256) && KDA_IN_BOUNDS(kBufQ, q + rowr0 * kD, 256)) {
+      if (r < L KDA_AND_IN_BOUNDS(kBufK, k + ((size_t)(t0 + r) * H + h) * kD, 256)
+                KDA_AND_IN_BOUNDS(kBufK, k + ((size_t)(t0 + i) * H + h) * kD, 256)
+                KDA_AND_IN_BOUNDS(kBufQ, q + ((size_t)(t0 + r) * H + h) * kD, 256)) {
         const float* gr = reinterpret_cast<const float*>(rec + g_scratch_off(r));
         const float* gi = reinterpret_cast<const float*>(rec + g_scratch_off(i));
         const size_t rowr = (size_t)(t0 + r) * H + h, rowi = (size_t)(t0 + i) * H + h;

@@ -55,9 +55,13 @@ __device__ __forceinline__ bool in_bounds(int role, const void* p, unsigned long
   return false;
 }
 #define KDA_IN_BOUNDS(role, p, n) (::kda::in_bounds((role), (p), (n)))
+// appends "&& the check" to a condition; nothing at all in the normal build, so that a kernel's
+// normal code is exactly what it is without the checks
+#define KDA_AND_IN_BOUNDS(role, p, n) && ::kda::in_bounds((role), (p), (n))
 constexpr bool kBoundsChecked = true;
 #else
 #define KDA_IN_BOUNDS(role, p, n) ((void)(p), true)
+#define KDA_AND_IN_BOUNDS(role, p, n)
 constexpr bool kBoundsChecked = false;
 #endif
 

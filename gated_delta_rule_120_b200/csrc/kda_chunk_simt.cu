@@ -30,7 +30,7 @@ constexpr int kSimtThreads = 256;
 
 // ----------------------------------------------------------------------------------------------
 // chunk map for packed variable-length batches: chunk_off[n] = sum_{m<n} ceil(len_m / C).
-// Validates cu_seqlens (cu[0] == 0, non-decreasing, cu[N] <= total) and records the verdict in
+// Validates cu_seqlens (cu[0] == 0, non-decreasing, cu[N] <= total) and records the outcome in
 // `valid`; the other kernels do nothing when it is 0 and the per-device status word is raised.
 // With `order` it also writes the sequences by decreasing chunk count (ties by index) for up to
 // blockDim.x sequences, the identity beyond that.

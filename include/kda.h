@@ -49,7 +49,7 @@ typedef struct CUstream_st* kda_stream_t; /* identical to cudaStream_t */
 typedef enum {
   KDA_OK = 0,
   KDA_ERR_INVALID_ARG = 1, /* null pointer, negative size, misalignment, bad cu_seqlens */
-  KDA_ERR_UNSUPPORTED = 2, /* a size or dtype combination this build has no kernel for */
+  KDA_ERR_UNSUPPORTED = 2, /* a size or dtype combination the library has no kernel for */
   KDA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch error, no device, ...) */
   KDA_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up */
   KDA_ERR_WORKSPACE = 5    /* workspace missing, too small or not 256-byte aligned */

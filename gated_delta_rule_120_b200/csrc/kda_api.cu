@@ -143,7 +143,8 @@ BwdLayout backward_layout(int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t D
 
 cudaError_t register_bounds(const BoundsTable& t, cudaStream_t stream) {
 #ifdef KDA_BOUNDS_CHECK
-  return cudaMemcpyToSymbolAsync(g_bounds, &t, sizeof(t), 0, cudaMemcpyHostToDevice, stream);
+  set_bounds_kernel<<<1, 1, 0, stream>>>(t);
+  return cudaGetLastError();
 #else
   (void)t;
   (void)stream;
@@ -225,8 +226,23 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, kda_dtyp
     return KDA_ERR_WORKSPACE;
 
   cudaStream_t stream = (cudaStream_t)stream_;
-  if (kBoundsChecked) {  // the varlen chunk map is the instrumented kernel of this call
+  if (kBoundsChecked) {
     BoundsTable t = {};
+    const size_t th = (size_t)tokens * H, states = (size_t)N * H * Dk * Dv * 4;
+    set_extent(t, kBufQ, q, th * Dk * es);
+    set_extent(t, kBufK, k, th * Dk * es);
+    set_extent(t, kBufV, v, th * Dv * es);
+    set_extent(t, kBufLogAlpha, log_alpha, th * Dk * 4);
+    set_extent(t, kBufBeta, beta, th * 4);
+    set_extent(t, kBufInitial, initial_state, initial_state ? states : 0);
+    set_extent(t, kBufDO, d_o, th * Dv * es);
+    set_extent(t, kBufDFinal, d_final_state, d_final_state ? states : 0);
+    set_extent(t, kBufDQ, dq, th * Dk * es);
+    set_extent(t, kBufDK, dk, th * Dk * es);
+    set_extent(t, kBufDV, dv, th * Dv * es);
+    set_extent(t, kBufDLogAlpha, dlog_alpha, th * Dk * 4);
+    set_extent(t, kBufDBeta, dbeta, th * 4);
+    set_extent(t, kBufDInitial, d_initial_state, d_initial_state ? states : 0);
     set_extent(t, kBufWork, workspace, workspace_bytes);
     set_extent(t, kBufCuSeqlens, cu_seqlens, varlen ? ((size_t)N + 1) * 4 : 0);
     st = from_cuda(register_bounds(t, stream));

@@ -86,6 +86,19 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
   const int tb = geo.seq_begin(n), te = geo.seq_end(n);
   const int c_first = geo.first_chunk(n);
   const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
+#ifdef KDA_BOUNDS_CHECK
+  {  // the chain's records, dO and dV' rows, cotangent slices and chunk-end cotangents
+    const size_t rf = rec.record_floats, st = (size_t)Dk * Dv, rv = (size_t)H * Dv;
+    const bool ok =
+        rows_in_bounds(kBufWork, ws + h * rf, c_first, c_first + nchunks, H * rf, rf) &&
+        rows_in_bounds(kBufDO, d_o + (size_t)h * Dv + j0, tb, te, rv, NV) &&
+        rows_in_bounds(kBufWork, dvp + (size_t)h * Dv + j0, tb, te, rv, NV) &&
+        rows_in_bounds(kBufWork, dstates + h * st, c_first, c_first + nchunks, H * st, st) &&
+        (!d_final || rows_in_bounds(kBufDFinal, d_final + sbase + j0, 0, Dk, Dv, NV)) &&
+        (!d_initial || rows_in_bounds(kBufDInitial, d_initial + sbase + j0, 0, Dk, Dv, NV));
+    if (!ok) return;  // (uniform: the whole CTA leaves)
+  }
+#endif
 
   // record sections are 16-byte aligned (d_k multiple of 4, C multiple of 16)
   auto record = [&](int c) { return ws + rec.record_floats * ((size_t)c * H + h); };
@@ -476,6 +489,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const float* S0 = states + ((size_t)c * H + h) * Dk * Dv;   // state entering the chunk
   const float* dS1 = dstates + ((size_t)c * H + h) * Dk * Dv; // cotangent of the state leaving it
   const int Dv4 = Dv >> 2;
+#ifdef KDA_BOUNDS_CHECK
+  {  // every access of the item lies in its record and states and in rows t0 .. t0 + L - 1
+    const size_t rk = (size_t)H * Dk, rv = (size_t)H * Dv, hk = (size_t)h * Dk, hv = (size_t)h * Dv;
+    const bool ok =
+        in_bounds(kBufWork, r_, rec.record_floats * sizeof(float)) &&
+        in_bounds(kBufWork, S0, (size_t)Dk * Dv * 4) && in_bounds(kBufWork, dS1, (size_t)Dk * Dv * 4) &&
+        rows_in_bounds(kBufWork, dvp + hv, t0, t0 + L, rv, Dv) &&
+        rows_in_bounds(kBufQ, q + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufK, k + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufV, v + hv, t0, t0 + L, rv, Dv) &&
+        rows_in_bounds(kBufLogAlpha, log_alpha + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufBeta, beta + h, t0, t0 + L, H, 1) &&
+        rows_in_bounds(kBufDO, d_o + hv, t0, t0 + L, rv, Dv) &&
+        rows_in_bounds(kBufDQ, dq + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufDK, dk + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufDV, dv + hv, t0, t0 + L, rv, Dv) &&
+        rows_in_bounds(kBufDLogAlpha, dla + hk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufDBeta, dbeta + h, t0, t0 + L, H, 1);
+    if (!ok) return;  // (uniform: the whole CTA leaves)
+  }
+#endif
 
   // ---- P0: inputs, record, cumulative decay. With 16-byte aligned input rows every copy is
   // issued before any is used: the record, dV' and log_alpha by cp.async, the Tin inputs as

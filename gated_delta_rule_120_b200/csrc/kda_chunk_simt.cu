@@ -174,6 +174,21 @@ __global__ void __launch_bounds__(kSimtThreads, 3)
   const int L = min(C, geo.seq_end(n) - t0);
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
   float* out = ws + rec.record_floats * ((size_t)c * H + h);
+#ifdef KDA_BOUNDS_CHECK
+  {  // every access of the item lies in its record and in rows t0 .. t0 + L - 1 of head h
+    const size_t rk = (size_t)H * Dk, rv = (size_t)H * Dv;
+    const bool ok =
+        in_bounds(kBufWork, out, rec.record_floats * sizeof(float)) &&
+        rows_in_bounds(kBufK, k + (size_t)h * Dk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufQ, q + (size_t)h * Dk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufV, v + (size_t)h * Dv, t0, t0 + L, rv, Dv) &&
+        rows_in_bounds(kBufLogAlpha, log_alpha + (size_t)h * Dk, t0, t0 + L, rk, Dk) &&
+        rows_in_bounds(kBufBeta, beta + h, t0, t0 + L, H, 1) &&
+        (!fz.A_log || in_bounds(kBufALog, fz.A_log + h, 4)) &&
+        (!fz.A_log || !fz.dt_bias || in_bounds(kBufDtBias, fz.dt_bias + (size_t)h * Dk, Dk * 4ull));
+    if (!ok) return;  // (uniform: the whole CTA leaves)
+  }
+#endif
 
   const float neg_a = fz.A_log ? -expf(fz.A_log[h]) : 0.f;
   constexpr int kPer = 16 / sizeof(Tin);
@@ -645,15 +660,28 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int tid = threadIdx.x, nt = blockDim.x, j = tid & 31, rg = tid >> 5;
   const int ng = nt >> 5;
   const size_t sbase = ((size_t)n * H + h) * Dk * Dv;
+  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
+  const int c_first = geo.first_chunk(n);
+  const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
+#ifdef KDA_BOUNDS_CHECK
+  {  // the chain's records, o rows, state slices and chunk-start states
+    const size_t rf = rec.record_floats, st = (size_t)Dk * Dv;
+    const bool ok =
+        rows_in_bounds(kBufWork, ws + h * rf, c_first, c_first + nchunks, H * rf, rf) &&
+        (!o || rows_in_bounds(kBufO, o + (size_t)h * Dv + j0, tb, te, (size_t)H * Dv, NV)) &&
+        (!initial_state || rows_in_bounds(kBufInitial, initial_state + sbase + j0, 0, Dk, Dv, NV)) &&
+        (!final_state || rows_in_bounds(kBufFinal, final_state + sbase + j0, 0, Dk, Dv, NV)) &&
+        (!states_out ||
+         rows_in_bounds(kBufWork, states_out + h * st, c_first, c_first + nchunks, H * st, st));
+    if (!ok) return;  // (uniform: the whole CTA leaves)
+  }
+#endif
 
   for (int idx = tid; idx < Dk * kSlice; idx += nt) {
     const int cc = idx / kSlice, jj = idx - cc * kSlice;
     sS[idx] = (initial_state && jj < NV) ? initial_state[sbase + (size_t)cc * Dv + j0 + jj] : 0.f;
   }
 
-  const int tb = geo.seq_begin(n), te = geo.seq_end(n);
-  const int c_first = geo.first_chunk(n);
-  const int nchunks = te > tb ? ceil_div(te - tb, C) : 0;
   // d_k and d_v multiples of 4: 16-byte record sections and float4 register tiles
   const bool tiled = (Dk & 3) == 0 && (Dv & 3) == 0 && nt == kSimtThreads &&
                      (C == 16 || C == 32 || C == 64);

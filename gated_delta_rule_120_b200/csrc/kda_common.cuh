@@ -38,7 +38,9 @@ __device__ __forceinline__ void raise_status(unsigned int bits) { atomicOr(&g_st
 // ---------------------------------------------------------------------------------------------
 enum BufRole : int {
   kBufQ = 0, kBufK, kBufV, kBufLogAlpha, kBufBeta, kBufInitial, kBufFinal, kBufO, kBufWork,
-  kBufCuSeqlens, kBufState, kBufIndices, kBufGate, kBufDtBias, kBufALog, kBufNormW, kBufRoles
+  kBufCuSeqlens, kBufState, kBufIndices, kBufGate, kBufDtBias, kBufALog, kBufNormW,
+  // the backward's cotangents in and gradients out
+  kBufDO, kBufDFinal, kBufDQ, kBufDK, kBufDV, kBufDLogAlpha, kBufDBeta, kBufDInitial, kBufRoles
 };
 struct BoundsTable {
   const void* base[kBufRoles];
@@ -46,6 +48,9 @@ struct BoundsTable {
 };
 #ifdef KDA_BOUNDS_CHECK
 __device__ BoundsTable g_bounds;
+// The table travels as a kernel parameter (captured by value when the call is recorded in a CUDA
+// graph, unlike a copy from the caller's stack).
+__global__ void set_bounds_kernel(BoundsTable t) { g_bounds = t; }
 __device__ __forceinline__ bool in_bounds(int role, const void* p, unsigned long long n) {
   const char* b = static_cast<const char*>(g_bounds.base[role]);
   const char* c = static_cast<const char*>(p);
@@ -55,6 +60,14 @@ __device__ __forceinline__ bool in_bounds(int role, const void* p, unsigned long
   return false;
 }
 #define KDA_IN_BOUNDS(role, p, n) (::kda::in_bounds((role), (p), (n)))
+// Rows r0 .. r1 - 1 of a row-strided array (row r at p + r * stride elements, D elements each) lie
+// in the buffer when its first and its last row do: the rows in between lie between them.
+template <typename T>
+__device__ __forceinline__ bool rows_in_bounds(int role, const T* p, long long r0, long long r1,
+                                               size_t stride, size_t D) {
+  return r1 <= r0 || (in_bounds(role, p + (size_t)r0 * stride, D * sizeof(T)) &&
+                      in_bounds(role, p + (size_t)(r1 - 1) * stride, D * sizeof(T)));
+}
 // appends "&& the check" to a condition; nothing at all in the normal build, so that a kernel's
 // normal code is exactly what it is without the checks
 #define KDA_AND_IN_BOUNDS(role, p, n) && ::kda::in_bounds((role), (p), (n))

@@ -20,9 +20,17 @@ __global__ void __launch_bounds__(32 * kEpiRowsPerBlock)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kEpiRowsPerBlock + warp;
   // varlen: tokens past the last sequence end are not the operator's output
-  const long long limit = cu_end ? min(rows, (long long)(*cu_end) * H) : rows;
+  const long long limit = (cu_end KDA_AND_IN_BOUNDS(kBufCuSeqlens, cu_end, 4))
+                              ? min(rows, (long long)(*cu_end) * H)
+                              : rows;
   if (row >= limit) return;
   T* orow = o + row * Dv;
+#ifdef KDA_BOUNDS_CHECK
+  if (!(in_bounds(kBufO, orow, Dv * sizeof(T)) &&
+        (!gate || in_bounds(kBufGate, gate + row * Dv, Dv * sizeof(T))) &&
+        (!weight || in_bounds(kBufNormW, weight, Dv * 4ull))))
+    return;  // (uniform in the warp that owns the row)
+#endif
   float x[4];
   float ss = 0.f;
 #pragma unroll

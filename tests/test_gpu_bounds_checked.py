@@ -1,11 +1,15 @@
 """The bounds-checked build of the library (libkda_checked.so, compiled with KDA_BOUNDS_CHECK):
-every global access of the prefill, decode and recurrent-mode kernels is tested against the extent
-of the buffer it belongs to, and an access outside is skipped and reported through the status word
-instead of faulting. These tests check that the check is really compiled in and fires (its
-self-test tests one access just past a registered buffer, without performing it), that the normal
-build has none, and that the checked build runs the operator's workloads with no report and with
-the normal build's results. The whole GPU suite can also run on it:
-KDA_LIBRARY=<repo>/gated_delta_rule_120_b200/libkda_checked.so python -m pytest tests -m gpu."""
+the kernels test their global accesses against the extent of the buffer each belongs to (the
+tensor-core prefill, decode and recurrent-mode kernels access by access; the fp32 chunk kernels,
+the output epilogue and the backward kernels by the first and last row of each work item), and an
+access outside is skipped and reported through the status word instead of faulting. These tests
+check that the check is really compiled in and fires (its self-test tests one access just past a
+registered buffer, without performing it), that the normal build has none, and that the checked
+build runs the operator's workloads with no report and with the normal build's results: the
+tensor-core prefill (plain, packed varlen, fused), the decode step, the recurrent mode, the fp32
+chunk kernels with the output epilogue, and the backward pass. The whole GPU suite can also run
+on it: KDA_LIBRARY=<repo>/gated_delta_rule_120_b200/libkda_checked.so python -m pytest tests -m gpu.
+"""
 import json
 import os
 import subprocess
@@ -70,9 +74,28 @@ idx = torch.tensor([7, 2, -1, 0, 5, 4], dtype=torch.int32, device=dev)
 o = kda.kda_recurrent_fwd(xr["q"], xr["k"], xr["v"], xr["log_alpha"], xr["beta"], pool, idx,
                           o=torch.zeros_like(xr["v"]))
 res["recurrent"] = (o, pool)
+# the fp32 path (CUDA-core chunk kernels) on a packed batch, with the output epilogue kernel
+fspec = PrefillSpec("e", B=1, T=150, H=2, Dk=64, Dv=64, chunk=32, dtype="f32", decay="fast",
+                    init_std=0.02, seqlens=(50, 0, 100))
+xf = kda_synth.prefill_inputs(fspec, 44, dev)
+res["f32_epilogue"] = kda.kda_chunk_fwd(
+    xf["q"], xf["k"], xf["v"], xf["log_alpha"], xf["beta"], initial_state=xf["initial_state"],
+    cu_seqlens=xf["cu_seqlens"], chunk=32,
+    fusion=dict(out_norm=True, out_norm_weight=torch.rand(64, generator=g, device=dev) + 0.5,
+                out_gate=torch.randn(xf["v"].shape, generator=g, device=dev)))
+# the backward pass (bf16, and fp32 on the packed batch)
+for name, bx in (("bwd_bf16", x), ("bwd_f32_varlen", xf)):
+    d_o = torch.randn(bx["v"].shape, generator=g, device=dev).to(bx["v"].dtype)
+    n_seq = bx["initial_state"].shape[0] if bx["initial_state"] is not None else \
+        bx["cu_seqlens"].numel() - 1
+    d_fin = torch.randn((n_seq,) + tuple(bx["v"].shape[2:3]) + (bx["q"].shape[-1], bx["v"].shape[-1]),
+                        generator=g, device=dev)
+    res[name] = kda.kda_chunk_bwd(bx["q"], bx["k"], bx["v"], bx["log_alpha"], bx["beta"], d_o,
+                                  initial_state=bx["initial_state"], d_final_state=d_fin,
+                                  cu_seqlens=bx["cu_seqlens"])
 torch.cuda.synchronize()
 out["status"] = kda.kda_last_device_error()
-torch.save({k: (a.float().cpu(), b.float().cpu()) for k, (a, b) in res.items()},
+torch.save({k: tuple(t.float().cpu() for t in v if t is not None) for k, v in res.items()},
            os.environ["KDA_OUT"])
 print(json.dumps(out))
 """

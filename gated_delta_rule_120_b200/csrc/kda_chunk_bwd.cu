@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
     cp_async_wait<1>();  // group B of this chunk has landed (group A may be in flight)
     __syncthreads();
     // dV'[i][j] = sum_r P[r][i] dO[r][j] + sum_a Kt[i][a] dS'[a][j] (P[r][i] = 0 for r < i):
-    // 2 x 4 tiles (rows i0, i0 + 1; columns 4 jq .. 4 jq + 3), the d_k part split 64 / C ways
+    // 2 x 4 tiles (rows i0, i0 + 1; columns 4 jq .. 4 jq + 3), the d_k part split between the two
+    // thread halves
     {
       const float4* Kt4 = reinterpret_cast<const float4*>(sKt);
       const float4* S4 = reinterpret_cast<const float4*>(sdS);  // [Dk][8]
@@ -167,7 +168,10 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
       const int dq = Dk >> 2;
       const int ip = (tid >> 3) % (C >> 1), jq = tid & 7, sp = tid / (4 * C);
       const int i0 = 2 * ip, i1 = i0 + 1;
-      const int kq = (dq + split - 1) / split, q0 = sp * kq, q1 = min(dq, q0 + kq);
+      static_assert(split == 2, "the dV' phase splits its d_k part between two thread halves");
+      // the first half also runs the A_qk part (about C / 5 float4 groups' worth of work), so it
+      // takes that many fewer d_k groups
+      const int qs = max(0, (dq - C / 5) / 2), q0 = sp == 0 ? 0 : qs, q1 = sp == 0 ? qs : dq;
       float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
       for (int q = q0; q < q1; ++q) {
         const float4 x0 = Kt4[i0 * dq + q], x1 = Kt4[i1 * dq + q];

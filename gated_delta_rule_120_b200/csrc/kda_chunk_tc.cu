@@ -157,6 +157,15 @@ __device__ __forceinline__ void readout_rows_bf16(uint32_t tmem, int warp, int l
   }
 }
 
+// The reference of a channel in the shifted fast mode: half its decay over the chunk when that
+// exceeds exp(-L), else the chunk start.
+__device__ __forceinline__ float shift_ref(float g_c, float limit) {
+  return g_c < -limit ? 0.5f * g_c : 0.f;
+}
+
+// kShift: the shifted fast mode is compiled in (the fused-gate calls, whose decays are strong);
+// plain calls run the kernel without it, whose common path it would slow by ~3 %.
+template <bool kShift>
 __global__ void __launch_bounds__(kK1Threads, 3)
     chunk_local_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                           const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
@@ -292,17 +301,28 @@ __global__ void __launch_bounds__(kK1Threads, 3)
 #pragma unroll
   for (int j = 0; j < 8; ++j) gmin = fminf(gmin, g[3][j]);
   const bool fast = __syncthreads_and(rg != 15 || gmin >= -decay_limit) != 0;
+  // Up to exp(-2L) over the chunk the fast evaluation still holds around a per-channel reference
+  // m = g_C / 2 (for the channels with g_C < -L): the factors k exp(g - m), k exp(m - g) then stay
+  // within e^+-L. Gamma.Q for the record and Gamma.K for W are rescaled by e^m.
+  bool shifted = false;
+  if constexpr (kShift)
+    shifted = !fast && __syncthreads_and(rg != 15 || gmin >= -2.f * decay_limit) != 0;
   float egc[8];
   {
     const float4* gcp = reinterpret_cast<const float4*>(sGC + cg * 8);
     const float4 a = gcp[0], b = gcp[1];
     const float gcv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    if constexpr (kShift) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      egc[j] = __expf(gcv[j]);  // only scales a bf16 operand; the carried gamma_C uses expf
+      for (int j = 0; j < 8; ++j) egc[j] = __expf(gcv[j] - shift_ref(sGC[cg * 8 + j], decay_limit));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        egc[j] = __expf(gcv[j]);  // only scales a bf16 operand; the carried gamma_C uses expf
+    }
   }
   int mode = kModeFast;
-  if (!fast) {
+  if (!fast && !shifted) {
     bool blocks_ok = true;  // every channel's decay within every 16-row block
     if (tid < kD) {
       float prev = 0.f;
@@ -349,6 +369,12 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       }
     }
     if (mode == kModeFast) {
+      if constexpr (kShift) {
+        if (shifted) {  // the factors around the reference m (the record's Q~ is rewritten below)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) g[i][j] -= shift_ref(sGC[cg * 8 + j], decay_limit);
+        }
+      }
       float kg[8], ki[8], kt[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -447,6 +473,27 @@ __global__ void __launch_bounds__(kK1Threads, 3)
             *reinterpret_cast<uint4*>(rec + kRecAqk + tile_chunk_off(r, part * 4 + c8, 8192)) =
                 pack8(f);
           }
+        }
+      }
+    }
+    if constexpr (kShift) {
+      if (shifted) {  // the A products have read their tiles: rescale this thread's chunks by
+        // e^m, Gamma.K in place for W and Gamma.Q into the record
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rg * 4 + i;
+          const uint32_t off = tile_chunk_off(r, cg, 8192);
+          float kg[8], qg[8];
+          unpack8(ld_shared_v4(sb + kS1Kg + off), kg);
+          unpack8(ld_shared_v4(sb + kS1Qg + off), qg);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float em = __expf(shift_ref(sGC[cg * 8 + j], decay_limit));
+            kg[j] *= em;
+            qg[j] *= em;
+          }
+          st_shared_v4(sb + kS1Kg + off, pack8(kg));
+          *reinterpret_cast<uint4*>(rec + kRecQW + qw_chunk_off(r, cg)) = pack8(qg);
         }
       }
     }
@@ -1178,8 +1225,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
   const bool norm = a.fz.onorm != 0;
   const int sm1 = (int)tc_local_smem_bytes();
   const int sm2 = (int)(norm ? tc::K2Smem<true>::bytes + 1024 : tc_state_smem_bytes());
-  cudaError_t err = cudaFuncSetAttribute(tc::chunk_local_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
+  auto* k1 = a.fz.A_log ? tc::chunk_local_tc_kernel<true> : tc::chunk_local_tc_kernel<false>;
+  cudaError_t err = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(norm ? tc::chunk_state_tc_kernel<true>
                                   : tc::chunk_state_tc_kernel<false>,
@@ -1187,7 +1234,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, const SeqGeometry& geo, int 
   if (err != cudaSuccess) return err;
   if (max_chunks > 0) {
     ProfileScope prof("chunk_local_tc", stream);
-    tc::chunk_local_tc_kernel<<<dim3(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
+    k1<<<dim3(max_chunks, a.H), tc::kK1Threads, sm1, stream>>>(
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
         a.log_alpha, a.beta, geo, a.H, records, a.fz);
     err = cudaGetLastError();

@@ -60,41 +60,63 @@ def chunk_reference(k, q, v, la, beta, L):
                 gam=np.exp(g[-1]))
 
 
-def chunk_mode(la_chunk: np.ndarray, limit: float = 60.0) -> str:
+def chunk_mode(la_chunk: np.ndarray, limit: float = 60.0, shifted: bool = False) -> str:
     """Which evaluation of A_kk / A_qk the kernel picks for one chunk of one head: "fast" when
-    every channel decays by at most exp(-limit) over the chunk, "blocks" when it does so within
-    every 16-row block, "exact" otherwise. The limit is 60 for caller-provided keys and 80 when
-    the kernel L2-normalises them."""
+    every channel decays by at most exp(-limit) over the chunk; with `shifted` (the kernel built
+    for the in-kernel gate) "shifted" — the fast evaluation around a per-channel reference at
+    half the channel's decay — when every channel decays by at most exp(-2 limit); "blocks" when
+    every channel decays by at most exp(-limit) within every 16-row block; "exact" otherwise. The
+    limit is 60 for caller-provided keys and 80 when the kernel L2-normalises them."""
     g = np.concatenate([np.zeros((1, la_chunk.shape[1])), np.cumsum(la_chunk, axis=0)])
     if g[-1].min() >= -limit:
         return "fast"
+    if shifted and g[-1].min() >= -2 * limit:
+        return "shifted"
     ends = [min(16 * (R + 1), la_chunk.shape[0]) for R in range(4)]
     starts = [min(16 * R, la_chunk.shape[0]) for R in range(4)]
     drops = [(g[s] - g[e]).max() for s, e in zip(starts, ends)]
     return "blocks" if max(drops) <= limit else "exact"
 
 
-# per-chunk decay scalings: (channels scaled, factor); 1 = the plain recipe
-MIXED_MODES = [(slice(None), 1.0), (slice(None), 4.0), (slice(None), 40.0), (slice(0, 32), 4.0)]
+# per-chunk decays: (channels, per-token level or None for the plain recipe, scale). A level
+# replaces the channels' log decays by level + 0.05 x the plain ones (a small per-token spread):
+# -1.4 decays a channel by 90-97 nats over a chunk (between 60 and 120), -2.2 by 141-148 nats
+# (beyond 120) but 35-37 nats per 16-row block (within 60).
+MIXED_MODES = [(slice(None), None, 1.0), (slice(None), -1.4, 1.0), (slice(None), -2.2, 1.0),
+               (slice(None), None, 40.0), (slice(0, 32), -2.2, 1.0)]
 
 
-@pytest.mark.parametrize("T,mixed", [(64, False), (150, False), (250, True)])
-def test_chunk_records_match_formulas(cuda_device, T, mixed):
+@pytest.mark.parametrize("T,mixed,gate", [(64, False, "given"), (150, False, "given"),
+                                          (314, True, "given"), (314, True, "in_kernel")])
+def test_chunk_records_match_formulas(cuda_device, T, mixed, gate):
     spec = PrefillSpec("t", B=1, T=T, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16", decay="fast",
                        init_std=0.02)
     inp = kda_synth.prefill_inputs(spec, 500 + T, cuda_device)
+    in_kernel = gate == "in_kernel"
     if mixed:  # one chunk in each mode, the block mode twice (all channels / 32 of them, ragged)
         la = inp["log_alpha"].clone()
-        for c, (chs, f) in enumerate(MIXED_MODES):
-            la[:, 64 * c:64 * c + 64, :, chs] *= f
+        for c, (chs, level, f) in enumerate(MIXED_MODES):
+            part = la[:, 64 * c:64 * c + 64, :, chs]
+            la[:, 64 * c:64 * c + 64, :, chs] = f * part if level is None else level + 0.05 * part
         inp["log_alpha"] = la
-        modes = [chunk_mode(to_np(la[0, 64 * c:64 * c + 64, h])) for c in range(4)
-                 for h in range(2)]
-        assert modes == ["fast"] * 2 + ["blocks"] * 2 + ["exact"] * 2 + ["blocks"] * 2, modes
+        modes = [chunk_mode(to_np(la[0, 64 * c:64 * c + 64, h]), shifted=in_kernel)
+                 for c in range(5) for h in range(2)]
+        assert modes == (["fast"] * 2 + ["shifted" if in_kernel else "blocks"] * 2 +
+                         ["blocks"] * 2 + ["exact"] * 2 + ["blocks"] * 2), modes
+    fusion, la_in = None, inp["log_alpha"]
+    if in_kernel:
+        # the kernel forms log alpha = -exp(A_log) softplus(g + dt_bias); with A_log = 0 and
+        # dt_bias = 0 the raw gate g = log(expm1(-log alpha)) gives back the decays above, and
+        # the formulas take -softplus(g) of the fp32 g the kernel reads
+        y = (-inp["log_alpha"].double()).clamp_min(1e-6)
+        la_in = torch.log(torch.expm1(y)).float()
+        inp["log_alpha"] = -torch.nn.functional.softplus(la_in.double())
+        fusion = dict(A_log=torch.zeros((2,), device=cuda_device),
+                      dt_bias=torch.zeros((2, 128), device=cuda_device))
     nbytes = kda.kda_chunk_fwd_workspace_size(1, T, 2, 128, 128, 64, 1, torch.bfloat16)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda_device)
-    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
-                      initial_state=inp["initial_state"], chunk=64, workspace=ws)
+    kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], la_in, inp["beta"],
+                      initial_state=inp["initial_state"], chunk=64, workspace=ws, fusion=fusion)
     torch.cuda.synchronize()
     assert kda.kda_last_device_error() == kda.KDA_OK
     buf = ws.cpu().numpy()

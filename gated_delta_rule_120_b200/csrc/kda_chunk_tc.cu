@@ -157,15 +157,23 @@ __device__ __forceinline__ void readout_rows_bf16(uint32_t tmem, int warp, int l
   }
 }
 
+// softplus for the in-kernel gate of this bf16 path: max(x, 0) + log(1 + exp(-|x|)) with the
+// hardware exp2/log2 approximations. Its absolute error (below 1e-6 per token) is far under what
+// the bf16 operands' rounding does to the decays; the fp32 paths keep the accurate form.
+__device__ __forceinline__ float softplus_approx(float x) {
+  return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
+}
+
 // The reference of a channel in the shifted fast mode: half its decay over the chunk when that
 // exceeds exp(-L), else the chunk start.
 __device__ __forceinline__ float shift_ref(float g_c, float limit) {
   return g_c < -limit ? 0.5f * g_c : 0.f;
 }
 
-// kShift: the shifted fast mode is compiled in (the fused-gate calls, whose decays are strong);
-// plain calls run the kernel without it, whose common path it would slow by ~3 %.
-template <bool kShift>
+// kGate: the instance for calls with the in-kernel decay gate (A_log given). It forms the log
+// decays from the raw gates and has the shifted fast mode for the strong decays such gates give;
+// the instance for caller-given log decays has neither (the extra code slowed its common path).
+template <bool kGate>
 __global__ void __launch_bounds__(kK1Threads, 3)
     chunk_local_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                           const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
@@ -242,7 +250,8 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     mbar_init(bar, 1);
     fence_mbar_init();
   }
-  if (fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log decays
+  if (kGate && fz.A_log) {  // fused gate: the loaded values are raw gates; valid rows become log
+                            // decays
 #ifdef KDA_BOUNDS_CHECK
     const float neg_a = KDA_IN_BOUNDS(kBufALog, fz.A_log + h, 4) ? -expf(fz.A_log[h]) : 0.f;
     const bool bias_ok =
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
     for (int i = 0; i < 4; ++i)
       if (rg * 4 + i < L)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) g[i][j] = neg_a * softplus_f(g[i][j] + bias[j]);
+        for (int j = 0; j < 8; ++j) g[i][j] = neg_a * softplus_approx(g[i][j] + bias[j]);
   }
 #pragma unroll
   for (int i = 1; i < 4; ++i)
@@ -305,14 +314,14 @@ __global__ void __launch_bounds__(kK1Threads, 3)
   // m = g_C / 2 (for the channels with g_C < -L): the factors k exp(g - m), k exp(m - g) then stay
   // within e^+-L. Gamma.Q for the record and Gamma.K for W are rescaled by e^m.
   bool shifted = false;
-  if constexpr (kShift)
+  if constexpr (kGate)
     shifted = !fast && __syncthreads_and(rg != 15 || gmin >= -2.f * decay_limit) != 0;
   float egc[8];
   {
     const float4* gcp = reinterpret_cast<const float4*>(sGC + cg * 8);
     const float4 a = gcp[0], b = gcp[1];
     const float gcv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    if constexpr (kShift) {
+    if constexpr (kGate) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) egc[j] = __expf(gcv[j] - shift_ref(sGC[cg * 8 + j], decay_limit));
     } else {
@@ -369,7 +378,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
       }
     }
     if (mode == kModeFast) {
-      if constexpr (kShift) {
+      if constexpr (kGate) {
         if (shifted) {  // the factors around the reference m (the record's Q~ is rewritten below)
 #pragma unroll
           for (int j = 0; j < 8; ++j) g[i][j] -= shift_ref(sGC[cg * 8 + j], decay_limit);
@@ -476,7 +485,7 @@ __global__ void __launch_bounds__(kK1Threads, 3)
         }
       }
     }
-    if constexpr (kShift) {
+    if constexpr (kGate) {
       if (shifted) {  // the A products have read their tiles: rescale this thread's chunks by
         // e^m, Gamma.K in place for W and Gamma.Q into the record
 #pragma unroll

@@ -848,23 +848,19 @@ constexpr int kEpiWarps = 8;                       // two per TMEM sub-partition
 constexpr int kK2Threads = 64 + 32 * kEpiWarps;    // warp 0 producer, warp 1 MMA, then epilogue
 // stage: QW [128 x 128] | AZ [128 x 64] = A_qk rows 0..63, zero rows 64..127 | Kt [64 x 128] |
 //        U (this CTA's 64-column block) [64 x 64] | gamma_C fp32 [128]
-//        (+ with the output epilogue: the output-gate rows of this CTA's columns [64 x 64] bf16,
-//        row-major)
 constexpr uint32_t kStQW = 0, kStAZ = 32768, kStKt = 49152, kStU = 65536, kStGam = 73728;
-constexpr uint32_t kStGate = 74752;
 constexpr uint32_t kStageTx = 32768 + 8192 + 16384 + 8192 + 512;
 constexpr int kStages = 2;
 constexpr uint32_t kS2Stage0 = 0;
 constexpr int kNumBars2 = 2 * kStages + 5;
 constexpr int kOutWarps = 4;
 
-// shared-memory map of K2; the output epilogue (head-wise RMSNorm x sigmoid gate) adds a gate
-// tile to every stage, and, because the two column halves of one (sequence, head) run as a
-// cluster of two CTAs that exchange per-row sums of squares of their 64 columns, the exchange
-// buffers
+// shared-memory map of K2; the output epilogue (head-wise RMSNorm x sigmoid gate) adds, because
+// the two column halves of one (sequence, head) run as a cluster of two CTAs that exchange per-row
+// sums of squares of their 64 columns, the exchange buffers
 template <bool kNorm>
 struct K2Smem {
-  static constexpr uint32_t stage = kNorm ? 74752 + 8192 : 74752;  // 1024-aligned stages
+  static constexpr uint32_t stage = 74752;         // 1024-aligned stages
   static constexpr uint32_t S = kStages * stage;   // [128 x 64] bf16 state tile (B operand)
   static constexpr uint32_t Vp = S + 16384;        // [64 x 64] bf16 pseudo-value tile
   static constexpr uint32_t Bar = Vp + 8192;
@@ -946,51 +942,30 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     // launched as a programmatic dependent of the chunk-local kernel: the records are complete
     // and visible only after this wait (the set-up above overlapped that kernel's tail)
     if (lane == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-    // lane 0 copies the record; with the gated output epilogue the whole warp also copies the
-    // chunk's gate rows (128 bytes of this CTA's columns per row)
-    const bool gate_rows = kNorm && fz.og != nullptr;
-    if (lane == 0 || gate_rows) {
+    if (lane == 0) {
       for (int ci = 0; ci < nchunks; ++ci) {
         const int st = ci % kStages;
-        bool ok = (ci < kStages || mbar_wait(empty + st, ((ci / kStages) - 1) & 1)) &&
-                  !*abort_flag;
-        if (gate_rows) ok = __all_sync(0xffffffffu, ok);
-        if (!ok) {
+        if (!((ci < kStages || mbar_wait(empty + st, ((ci / kStages) - 1) & 1)) &&
+              !*abort_flag)) {
           *abort_flag = 1;
           break;
         }
         uint8_t* stage = sm + kS2Stage0 + st * kStageBytes;
-        const int t0 = tb + ci * kC;
-        const int L = min(kC, te - t0);
         const uint8_t* rec = ws_records + (size_t)kRecBytes * ((size_t)(c_first + ci) * H + h);
-        const __nv_bfloat16* g0 = reinterpret_cast<const __nv_bfloat16*>(fz.og);
-        // the gate rows of this chunk lie between its first and last row's 128 bytes
-        const bool gates_in =
-            !gate_rows ||
-            (KDA_IN_BOUNDS(kBufGate, g0 + ((size_t)t0 * H + h) * kD + j0, 128) &&
-             KDA_IN_BOUNDS(kBufGate, g0 + ((size_t)(t0 + L - 1) * H + h) * kD + j0, 128));
-        if (lane == 0 && !KDA_IN_BOUNDS(kBufWork, rec, kRecBytes)) {
+        if (!KDA_IN_BOUNDS(kBufWork, rec, kRecBytes)) {
           mbar_arrive(full + st);  // nothing copied: the phase completes on the stale stage
-        } else if (lane == 0) {
-          mbar_arrive_expect_tx(full + st,
-                                kStageTx + (gate_rows && gates_in ? (uint32_t)L * 128u : 0u));
+        } else {
+          mbar_arrive_expect_tx(full + st, kStageTx);
           bulk_g2s(stage + kStQW, rec + kRecQW, 32768, full + st);
           bulk_g2s(stage + kStAZ, rec + kRecAqk, 8192, full + st);
           bulk_g2s(stage + kStKt, rec + kRecKt, 16384, full + st);
           bulk_g2s(stage + kStU, rec + kRecU + (j0 >> 6) * 8192, 8192, full + st);
           bulk_g2s(stage + kStGam, rec + kRecGam, 512, full + st);
         }
-        if (gate_rows && gates_in && (!kBoundsChecked || __shfl_sync(0xffffffffu,
-                                                                      (int)KDA_IN_BOUNDS(kBufWork, rec, kRecBytes), 0))) {
-          for (int rr = lane; rr < L; rr += 32)
-            bulk_g2s(stage + kStGate + rr * 128, g0 + ((size_t)(t0 + rr) * H + h) * kD + j0, 128,
-                     full + st);
-        }
       }
       // the last copies must land before the CTA may exit
-      if (lane == 0)
-        for (int ci = nchunks > kStages ? nchunks - kStages : 0; ci < nchunks; ++ci)
-          mbar_wait(full + ci % kStages, (ci / kStages) & 1);
+      for (int ci = nchunks > kStages ? nchunks - kStages : 0; ci < nchunks; ++ci)
+        mbar_wait(full + ci % kStages, (ci / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -1080,6 +1055,20 @@ __global__ void __launch_bounds__(kK2Threads, 1)
     };
     write_state_tile();
 
+    // the output-gate row of this thread's chunk row (its 32 columns, 64 bytes), loaded from
+    // global memory a chunk ahead of its use
+    uint4 graw[4] = {};
+    const __nv_bfloat16* g0 = reinterpret_cast<const __nv_bfloat16*>(fz.og);
+    auto load_gate = [&](int ci) {
+      if (kNorm && out_warp && g0 && ci < nchunks && tb + ci * kC + r < te) {
+        const __nv_bfloat16* gp = g0 + ((size_t)(tb + ci * kC + r) * H + h) * kD + j0 + 32 * chalf;
+        if (KDA_IN_BOUNDS(kBufGate, gp, 64)) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) graw[q8] = __ldg(reinterpret_cast<const uint4*>(gp) + q8);
+        }
+      }
+    };
+    load_gate(0);
     float va[32];
     for (int ci = 0; ci < nchunks; ++ci) {
       const int st = ci % kStages;
@@ -1093,13 +1082,6 @@ __global__ void __launch_bounds__(kK2Threads, 1)
         break;
       }
       const float gam = reinterpret_cast<const float*>(sm + st * kStageBytes + kStGam)[row];
-      // the output gate row leaves the stage now: the stage is released once V' is in
-      uint4 graw[4];
-      if (kNorm && out_warp && fz.og && r < L) {
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          graw[q8] = ld_shared_v4(stage + kStGate + r * 128 + chalf * 64 + q8 * 16);
-      }
       if (!out_warp) {  // V' = U - W S for chunk row r, this warp's 32 columns
         float u[32];
 #pragma unroll
@@ -1178,7 +1160,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
               rsqrtf((sPart[r] + sPart[64 + r] + sPeer[r]) * (1.f / kD) + fz.oeps);
           const float* sW = reinterpret_cast<const float*>(sm + SM::W) + 32 * chalf;
           float gt[32];
-          if (gated) {  // the gate row staged by the producer: 32 columns of row r
+          if (gated) {  // the gate row loaded a chunk ahead: 32 columns of row r
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
               float f[8];
@@ -1191,6 +1173,7 @@ __global__ void __launch_bounds__(kK2Threads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) gt[j] = 1.f;
           }
+          load_gate(ci + 1);
 #pragma unroll
           for (int j = 0; j < 32; ++j) va[j] = va[j] * inv * sW[j] * gt[j];
         }

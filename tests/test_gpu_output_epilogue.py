@@ -75,19 +75,24 @@ def test_chunk_bf16_output_epilogue(cuda_device, T):
     assert rel_err(y, y_from_plain) <= 1e-2
 
 
-def test_chunk_bf16_output_epilogue_varlen_no_gate(cuda_device):
+@pytest.mark.parametrize("gated", [False, True], ids=["no_gate", "gate_and_weight"])
+def test_chunk_bf16_output_epilogue_varlen(cuda_device, gated):
+    """Packed sequences with ragged last chunks: the gate rows of a chunk's padding rows belong to
+    the next sequence (or lie past the batch) and must not be read into the output."""
     lens = [130, 0, 64, 1, 257]
     T = sum(lens)
     spec = PrefillSpec("t", B=1, T=T, H=2, Dk=128, Dv=128, chunk=64, dtype="bf16", decay="fast",
                        init_std=0.0, seqlens=tuple(lens))
     inp = kda_synth.prefill_inputs(spec, 810, cuda_device)
-    fz = _epilogue(cuda_device, inp["v"].shape, torch.bfloat16, 811, gate=False, weight=False)
+    fz = _epilogue(cuda_device, inp["v"].shape, torch.bfloat16, 811, gate=gated, weight=gated)
     y, _ = kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
                              cu_seqlens=inp["cu_seqlens"], chunk=64, fusion=fz)
     torch.cuda.synchronize()
     assert kda.kda_last_device_error() == kda.KDA_OK
     y_ref, _, o_ref = _oracle_y(inp, fz, inp["cu_seqlens"].cpu().numpy(), 2)
     assert epilogue_err(y, y_ref, o_ref, fz, 2) <= TOL_BF16_O
+    if gated:
+        return
     # ungated, unweighted rows have RMS sqrt(ms / (ms + eps)) for the mean square ms of o: ~1 for
     # every row well above eps
     ms = np.mean(o_ref * o_ref, axis=-1)

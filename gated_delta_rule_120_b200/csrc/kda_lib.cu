@@ -3,6 +3,7 @@
 // relocatable device code.
 #include "kda_api.cu"
 #include "kda_profile.cu"
+#include "kda_recurrent_chunk.cu"
 #include "kda_decode.cu"
 #include "kda_chunk_simt.cu"
 #include "kda_chunk_tc.cu"

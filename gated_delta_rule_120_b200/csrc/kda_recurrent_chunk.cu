@@ -1,0 +1,435 @@
+// kda_recurrent_chunk.cu — the recurrent mode (a few tokens per sequence against pooled states) in
+// the chunk form, fp32, one CTA per (sequence, head).
+//
+// For T <= 16 tokens the whole call is one chunk of the chunkwise form ("Kimi Linear: An
+// Expressive, Efficient Attention Architecture", paper-graph-ui walkthrough, §3.4 "Chunkwise
+// Parallelization"): with g_t the cumulative log decay of token t from the item's start and S the
+// pooled state,
+//   A_kk[r][i] = sum_c k_r[c] k_i[c] exp(g_r[c] - g_i[c])  (i < r),  A_qk likewise with q_r (i <= r)
+//   M  = (I + StrictTril(Diag(beta) A_kk))^{-1} Diag(beta)
+//   W  = M (exp(g) . K),  U = M V,  V' = U - W S
+//   O  = (exp(g) . Q) S + A_qk V'
+//   S' = Diag(exp(g_T)) S + (K . exp(g_T - g))^T V'
+// The token-by-token kernels spend most of an item in per-token reductions across the state's
+// rows; here the state is read once into shared memory and enters two products, [W; Q~] S and
+// K~^T V', evaluated as register-tiled fp32 products on packed pairs. Every ratio exp(g_r - g_i)
+// is formed exactly per term (no factoring around a reference), so any finite decay is safe.
+// The state is read from and written back to its pool row; everything else stays on chip.
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "kda_sm100.cuh"
+
+namespace kda {
+namespace rchunk {
+
+constexpr int kT = 16;         // tokens per item at most
+constexpr int kD = 128;        // d_k = d_v
+constexpr int kThreads = 256;  // 8 warps
+constexpr float kLog2e = 1.4426950408889634f;
+
+// shared memory (fp32 words)
+constexpr int kOffS = 0;                   // S [128][128], row-major
+constexpr int kOffK = kOffS + kD * kD;     // k [16][128], then K~
+constexpr int kOffQ = kOffK + kT * kD;     // q [16][128]   } later [W; Q~]^T [128][32] (swizzled)
+constexpr int kOffG = kOffQ + kT * kD;     // g log2e [16][128] }
+constexpr int kOffV = kOffG + kT * kD;     // v, then U, then V' [16][128]
+constexpr int kOffKG = kOffV + kT * kD;    // exp(g) . k [16][128]
+constexpr int kOffAkk = kOffKG + kT * kD;  // Diag(beta) A_kk strict lower [16][16]
+constexpr int kOffAqk = kOffAkk + kT * kT; // A_qk lower [16][16]
+constexpr int kOffM = kOffAqk + kT * kT;   // M [16][16]
+constexpr int kOffBeta = kOffM + kT * kT;  // beta [16]
+constexpr int kOffGam = kOffBeta + kT;     // exp(g_T) [128]
+constexpr int kWords = kOffGam + kD;
+constexpr size_t kSmemBytes = (size_t)kWords * 4;
+static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+
+// [W; Q~]^T: row = key channel (128), 32 columns (W rows 0..15, Q~ rows 16..31) in groups of four,
+// the group index XOR-ed by (row % 8) so that a column of rows spreads over the banks
+__device__ __forceinline__ int at_idx(int row, int col) {
+  return row * 32 + ((((col >> 2) ^ (row & 7)) << 2) | (col & 3));
+}
+
+template <typename Tin>
+__device__ __forceinline__ void load_row8(float* dst, const Tin* src);
+template <>
+__device__ __forceinline__ void load_row8<__nv_bfloat16>(float* dst, const __nv_bfloat16* src) {
+  store_vec(dst, __ldg(reinterpret_cast<const uint4*>(src)), __nv_bfloat16());
+}
+template <>
+__device__ __forceinline__ void load_row8<float>(float* dst, const float* src) {
+  store_vec(dst, __ldg(reinterpret_cast<const uint4*>(src)), float());
+  store_vec(dst + 4, __ldg(reinterpret_cast<const uint4*>(src) + 1), float());
+}
+
+template <typename Tin>
+__device__ __forceinline__ void store4(Tin* dst, const float (&v)[4]);
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(dst) = make_uint2(sm100::pack_bf16(v[0], v[1]), sm100::pack_bf16(v[2], v[3]));
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 2)
+    recurrent_chunk_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                           const Tin* __restrict__ v, const float* __restrict__ log_alpha,
+                           const float* __restrict__ beta, float* __restrict__ pool,
+                           const int32_t* __restrict__ state_indices, Tin* __restrict__ o, int T,
+                           int H, int P) {
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  float* sS = sm + kOffS;
+  float* sK = sm + kOffK;
+  float* sQ = sm + kOffQ;
+  float* sG = sm + kOffG;
+  float* sAT = sm + kOffQ;  // aliases q and g once the A products have read them
+  float* sV = sm + kOffV;
+  float* sKG = sm + kOffKG;
+  float* sAkk = sm + kOffAkk;
+  float* sAqk = sm + kOffAqk;
+  float* sM = sm + kOffM;
+  float* sBeta = sm + kOffBeta;
+  float* sGam = sm + kOffGam;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item = blockIdx.x, n = item / H, h = item - n * H;
+  const int slot = state_indices ? (KDA_IN_BOUNDS(kBufIndices, state_indices + n, 4)
+                                        ? state_indices[n]
+                                        : -1)
+                                 : n;
+  if (slot < 0) return;  // a skipped sequence: no state update, o untouched
+  if (slot >= P) {
+    if (tid == 0) raise_status(kStatusBadSeqlens);
+    return;
+  }
+  float* state = pool + ((size_t)slot * H + h) * kD * kD;
+  const size_t row0 = ((size_t)n * T) * H + h;  // token t's row: row0 + t * H
+#ifdef KDA_BOUNDS_CHECK
+  {
+    const size_t rs = (size_t)H;
+    bool ok = in_bounds(kBufState, state, (size_t)kD * kD * 4) &&
+              rows_in_bounds(kBufQ, q + row0 * kD, 0, T, rs * kD, kD) &&
+              rows_in_bounds(kBufK, k + row0 * kD, 0, T, rs * kD, kD) &&
+              rows_in_bounds(kBufV, v + row0 * kD, 0, T, rs * kD, kD) &&
+              rows_in_bounds(kBufLogAlpha, log_alpha + row0 * kD, 0, T, rs * kD, kD) &&
+              rows_in_bounds(kBufBeta, beta + row0, 0, T, rs, 1) &&
+              rows_in_bounds(kBufO, o + row0 * kD, 0, T, rs * kD, kD);
+    if (__syncthreads_or(!ok)) return;
+  }
+#endif
+
+  // ---- phase 1: the state by cp.async (needed from phase 5 on), the token rows as fp32 --------
+#pragma unroll
+  for (int j = 0; j < (kD * kD / 4) / kThreads; ++j) {
+    const int i4 = tid + j * kThreads;
+    cp_async_16B(sS + 4 * i4, reinterpret_cast<const float4*>(state) + i4);
+  }
+  cp_async_commit();
+  {
+    const int t = tid >> 4, c8 = (tid & 15) * 8;  // token row t, channels c8 .. c8 + 7
+    if (t < T) {
+      const size_t r = (row0 + (size_t)t * H) * kD + c8;
+      load_row8<Tin>(sK + t * kD + c8, k + r);
+      load_row8<Tin>(sQ + t * kD + c8, q + r);
+      load_row8<Tin>(sV + t * kD + c8, v + r);
+      load_row8<float>(sG + t * kD + c8, log_alpha + r);
+    } else {  // padding rows: no key, no decay
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sK[t * kD + c8 + j] = 0.f;
+        sQ[t * kD + c8 + j] = 0.f;
+        sV[t * kD + c8 + j] = 0.f;
+        sG[t * kD + c8 + j] = 0.f;
+      }
+    }
+    if (tid < kT) sBeta[tid] = tid < T ? beta[row0 + (size_t)tid * H] : 0.f;
+    for (int i = tid; i < 2 * kT * kT; i += kThreads) sAkk[i] = 0.f;  // A_kk and A_qk
+  }
+  __syncthreads();
+
+  // ---- phase 2: cumulative decay per channel; exp(g) . k; Q~ and K~ kept in registers ---------
+  // The A products take each channel's ratios exp(g_r - g_i) as k_r exp(g_r - m) times
+  // k_i exp(m - g_i) around the channel's midpoint m, both factors within 2^(span / 2) (span in
+  // log2 units over the item). An item with a channel spanning more than kSpanMax takes every
+  // ratio exactly instead (slower).
+  constexpr float kSpanMax = 200.f;
+  // thread = channel c and half of the tokens (8 half .. + 7); both halves run the channel's scan
+  const int c = tid & (kD - 1), th0 = 8 * (tid >> 7);
+  float qt[8], kt[8], gl[kT];
+  bool wide;
+  {
+    float run = 0.f;
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+      run += sG[t * kD + c];
+      gl[t] = run * kLog2e;
+    }
+    if (th0 == 0) sGam[c] = exp2f(gl[kT - 1]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int t = th0 + j;
+      const float gt = th0 ? gl[8 + j] : gl[j];  // (constant indices: gl stays in registers)
+      const float e = exp2f(gt), kv = sK[t * kD + c];
+      sKG[t * kD + c] = kv * e;
+      qt[j] = sQ[t * kD + c] * e;
+      kt[j] = kv * exp2f(gl[kT - 1] - gt);
+    }
+    wide = gl[0] - gl[kT - 1] > kSpanMax;
+  }
+  wide = __syncthreads_or(wide) != 0;  // the item's form, known to every thread
+  if (wide) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sG[(th0 + j) * kD + c] = th0 ? gl[8 + j] : gl[j];
+  } else {  // k exp(g - m), q exp(g - m) in place of k, q; k exp(m - g) in place of g
+    const float m = 0.5f * (gl[0] + gl[kT - 1]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int t = th0 + j;
+      const float gt = th0 ? gl[8 + j] : gl[j];
+      const float ep = exp2f(gt - m), em = exp2f(m - gt);
+      const float kv = sK[t * kD + c];
+      sK[t * kD + c] = kv * ep;
+      sQ[t * kD + c] = sQ[t * kD + c] * ep;
+      sG[t * kD + c] = kv * em;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 3: A_kk, A_qk ---------------------------------------------------------------
+  if (!wide) {  // thread = pair (r, i); channels rotated by i so the 16 rows i spread over banks
+    const int r = tid >> 4, i = tid & 15;
+    float akk = 0.f, aqk = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < kD / 4; ++j) {
+      const int c4 = 4 * ((j + i) & (kD / 4 - 1));
+      const float4 kr = *reinterpret_cast<const float4*>(sK + r * kD + c4);
+      const float4 qr = *reinterpret_cast<const float4*>(sQ + r * kD + c4);
+      const float4 ki = *reinterpret_cast<const float4*>(sG + i * kD + c4);
+      akk = fmaf(kr.x, ki.x, fmaf(kr.y, ki.y, fmaf(kr.z, ki.z, fmaf(kr.w, ki.w, akk))));
+      aqk = fmaf(qr.x, ki.x, fmaf(qr.y, ki.y, fmaf(qr.z, ki.z, fmaf(qr.w, ki.w, aqk))));
+    }
+    if (r < T) {
+      if (i < r) sAkk[r * kT + i] = sBeta[r] * akk;
+      if (i <= r) sAqk[r * kT + i] = aqk;
+    }
+  } else {  // exact ratios: warp = pairs (r, i), lane = four channels
+    const int c4 = 4 * lane;
+    for (int p = warp; p < kT * (kT + 1) / 2; p += kThreads / 32) {
+      int r = 0;
+      while ((r + 1) * (r + 2) / 2 <= p) ++r;
+      const int i = p - r * (r + 1) / 2;
+      if (r >= T) continue;  // warp-uniform: padding rows stay zero
+      const float4 kr = *reinterpret_cast<const float4*>(sK + r * kD + c4);
+      const float4 ki = *reinterpret_cast<const float4*>(sK + i * kD + c4);
+      const float4 qr = *reinterpret_cast<const float4*>(sQ + r * kD + c4);
+      const float4 gr = *reinterpret_cast<const float4*>(sG + r * kD + c4);
+      const float4 gi = *reinterpret_cast<const float4*>(sG + i * kD + c4);
+      const float e0 = exp2f(gr.x - gi.x), e1 = exp2f(gr.y - gi.y);
+      const float e2 = exp2f(gr.z - gi.z), e3 = exp2f(gr.w - gi.w);
+      const float b0 = ki.x * e0, b1 = ki.y * e1, b2 = ki.z * e2, b3 = ki.w * e3;
+      float akk = kr.x * b0 + kr.y * b1 + kr.z * b2 + kr.w * b3;
+      float aqk = qr.x * b0 + qr.y * b1 + qr.z * b2 + qr.w * b3;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        akk += __shfl_xor_sync(0xffffffffu, akk, off);
+        aqk += __shfl_xor_sync(0xffffffffu, aqk, off);
+      }
+      if (lane == 0) {
+        if (i < r) sAkk[r * kT + i] = sBeta[r] * akk;
+        sAqk[r * kT + i] = aqk;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 4: Q~ and K~ out of the registers (q and g are dead); M by forward substitution --
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    sAT[at_idx(c, kT + th0 + j)] = qt[j];
+    sK[(th0 + j) * kD + c] = kt[j];
+  }
+  if (warp == 0 && lane < kT) {  // column `lane` of (I + A)^{-1}, then M = T Diag(beta)
+    float col[kT];
+#pragma unroll
+    for (int i = 0; i < kT; ++i) {
+      float val = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+      for (int m = 0; m < i; ++m) val -= sAkk[i * kT + m] * col[m];
+      col[i] = val;
+    }
+    const float bj = sBeta[lane];
+#pragma unroll
+    for (int i = 0; i < kT; ++i) sM[i * kT + lane] = col[i] * bj;
+  }
+  __syncthreads();
+
+  // ---- phase 5: W = M (exp(g) . K) into [W; Q~]^T, U = M V over V (rows 8 half .. + 7) ---------
+  {
+    const int c = tid & (kD - 1), half = tid >> 7;
+    float w[8], u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = u[j] = 0.f;
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+      const float kg = sKG[t * kD + c], vv = sV[t * kD + c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float m = sM[(8 * half + j) * kT + t];  // zero for t > row
+        w[j] = fmaf(m, kg, w[j]);
+        u[j] = fmaf(m, vv, u[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sAT[at_idx(c, 8 * half + j)] = w[j];
+    __syncthreads();  // every thread has read V
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sV[(8 * half + j) * kD + c] = u[j];
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---- phase 6: [W; Q~] S; V' = U - W S; O = Q~ S + A_qk V' -----------------------------------
+  // warp = 16 state columns, lane = 4 rows (mg) x 4 columns (cg) of the 32 x 128 product; the
+  // accumulators stay packed pairs of adjacent columns
+  {
+    const int mg = lane >> 2, cg = lane & 3, col = 16 * warp + 4 * cg;
+    f32x2 acc[4][2];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = f2_pack(0.f, 0.f);
+#pragma unroll 8
+    for (int kk = 0; kk < kD; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(sAT + kk * 32 + ((mg ^ (kk & 7)) << 2));
+      const float4 sv = *reinterpret_cast<const float4*>(sS + kk * kD + col);
+      const f32x2 s01 = f2_pack(sv.x, sv.y), s23 = f2_pack(sv.z, sv.w);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const f32x2 ar = f2_pack(av[r], av[r]);
+        acc[r][0] = f2_fma(ar, s01, acc[r][0]);
+        acc[r][1] = f2_fma(ar, s23, acc[r][1]);
+      }
+    }
+    if (mg < 4) {  // rows 4 mg .. + 3 of W S: V' in place of U
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float4* up = reinterpret_cast<float4*>(sV + (4 * mg + r) * kD + col);
+        const float4 uu = *up;
+        const float2 lo = f2_unpack(acc[r][0]), hi = f2_unpack(acc[r][1]);
+        *up = make_float4(uu.x - lo.x, uu.y - lo.y, uu.z - hi.x, uu.w - hi.y);
+      }
+    }
+    __syncwarp();  // this warp's 16 columns of V' are complete
+    if (mg >= 4) {  // output rows t = 4 (mg - 4) .. + 3
+      const int t0 = 4 * (mg - 4);
+#pragma unroll
+      for (int tau = 0; tau < kT; ++tau) {
+        const float4 vp = *reinterpret_cast<const float4*>(sV + tau * kD + col);
+        const f32x2 v01 = f2_pack(vp.x, vp.y), v23 = f2_pack(vp.z, vp.w);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float aq = sAqk[(t0 + r) * kT + tau];
+          const f32x2 ar = f2_pack(aq, aq);
+          acc[r][0] = f2_fma(ar, v01, acc[r][0]);
+          acc[r][1] = f2_fma(ar, v23, acc[r][1]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int t = t0 + r;
+        const float2 lo = f2_unpack(acc[r][0]), hi = f2_unpack(acc[r][1]);
+        const float y[4] = {lo.x, lo.y, hi.x, hi.y};
+        if (t < T) store4<Tin>(o + (row0 + (size_t)t * H) * kD + col, y);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 7: S' = Diag(exp(g_T)) S + K~^T V' into the pool row --------------------------
+  // warp = 16 state rows, lane = 4 columns (two packed pairs)
+  {
+    const int r0 = 16 * warp, c4 = 4 * lane;
+    f32x2 acc[16][2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float4 sv = *reinterpret_cast<const float4*>(sS + (r0 + i) * kD + c4);
+      const float g = sGam[r0 + i];
+      const f32x2 gg = f2_pack(g, g);
+      acc[i][0] = f2_mul(gg, f2_pack(sv.x, sv.y));
+      acc[i][1] = f2_mul(gg, f2_pack(sv.z, sv.w));
+    }
+    for (int t = 0; t < T; ++t) {
+      const float4 vp = *reinterpret_cast<const float4*>(sV + t * kD + c4);
+      const f32x2 v01 = f2_pack(vp.x, vp.y), v23 = f2_pack(vp.z, vp.w);
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const float4 kk = *reinterpret_cast<const float4*>(sK + t * kD + r0 + 4 * i4);
+        const float kv[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const f32x2 kr = f2_pack(kv[e], kv[e]);
+          acc[4 * i4 + e][0] = f2_fma(kr, v01, acc[4 * i4 + e][0]);
+          acc[4 * i4 + e][1] = f2_fma(kr, v23, acc[4 * i4 + e][1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 lo = f2_unpack(acc[i][0]), hi = f2_unpack(acc[i][1]);
+      *reinterpret_cast<float4*>(state + (size_t)(r0 + i) * kD + c4) =
+          make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+  }
+}
+
+}  // namespace rchunk
+
+// The recurrent mode through the chunk-form kernel: 2 <= T <= 16, d_k = d_v = 128, no fusion, 16-byte
+// aligned rows. Returns false (nothing launched) when the call does not qualify.
+static bool recurrent_chunk_applies(kda_dtype_t dt, int T, int Dk, int Dv, const void* q,
+                                    const void* k, const void* v, const float* log_alpha,
+                                    const float* pool, const void* o, const Fusion& fz) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
+  const bool fused = fz.l2 || fz.A_log || fz.onorm;
+  return !fused && T >= 2 && T <= rchunk::kT && Dk == rchunk::kD && Dv == rchunk::kD &&
+         (dt == KDA_DTYPE_BF16 || dt == KDA_DTYPE_F32) && al16(q) && al16(k) && al16(v) &&
+         al16(log_alpha) && al16(pool) && ((uintptr_t)o & (dt == KDA_DTYPE_BF16 ? 7u : 15u)) == 0;
+}
+
+static cudaError_t launch_recurrent_chunk(const void* q, const void* k, const void* v,
+                                          kda_dtype_t dt, const float* log_alpha,
+                                          const float* beta, float* pool, const int32_t* idx,
+                                          void* o, long long heads, int T, int H, int P,
+                                          cudaStream_t stream) {
+  if (heads > INT32_MAX) return cudaErrorInvalidConfiguration;
+  const int smem = (int)rchunk::kSmemBytes;
+  ProfileScope prof("recurrent_chunk", stream);
+  if (dt == KDA_DTYPE_BF16) {
+    cudaError_t err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err == cudaSuccess)  // two CTAs per SM: the whole unified array as shared memory
+      err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (err != cudaSuccess) return err;
+    rchunk::recurrent_chunk_kernel<__nv_bfloat16><<<(unsigned)heads, rchunk::kThreads, smem,
+                                                    stream>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha, beta,
+        pool, idx, (__nv_bfloat16*)o, T, H, P);
+  } else {
+    cudaError_t err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<float>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<float>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (err != cudaSuccess) return err;
+    rchunk::recurrent_chunk_kernel<float><<<(unsigned)heads, rchunk::kThreads, smem, stream>>>(
+        (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, pool, idx, (float*)o,
+        T, H, P);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -153,13 +153,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // ---- phase 2: cumulative decay per channel; exp(g) . k; Q~ and K~ kept in registers ---------
   // The A products take each channel's ratios exp(g_r - g_i) as k_r exp(g_r - m) times
-  // k_i exp(m - g_i) around the channel's midpoint m, both factors within 2^(span / 2) (span in
-  // log2 units over the item). An item with a channel spanning more than kSpanMax takes every
-  // ratio exactly instead (slower).
+  // k_i exp(m - g_i) around the midpoint m of the channel's range of g, both factors within
+  // 2^(span / 2) (span = that range in log2 units). An item with a channel spanning more than
+  // kSpanMax takes every ratio exactly instead (slower).
   constexpr float kSpanMax = 200.f;
   // thread = channel c and half of the tokens (8 half .. + 7); both halves run the channel's scan
   const int c = tid & (kD - 1), th0 = 8 * (tid >> 7);
-  float qt[8], kt[8], gl[kT];
+  float qt[8], kt[8], gl[kT], gmid;
   bool wide;
   {
     float run = 0.f;
@@ -178,14 +178,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       qt[j] = sQ[t * kD + c] * e;
       kt[j] = kv * exp2f(gl[kT - 1] - gt);
     }
-    wide = gl[0] - gl[kT - 1] > kSpanMax;
+    float lo = gl[0], hi = gl[0];  // (log decays are <= 0, so g falls; any sign is handled)
+#pragma unroll
+    for (int t = 1; t < kT; ++t) {
+      lo = fminf(lo, gl[t]);
+      hi = fmaxf(hi, gl[t]);
+    }
+    wide = !(hi - lo <= kSpanMax);  // (a NaN decay takes the exact form too)
+    gmid = 0.5f * (lo + hi);
   }
   wide = __syncthreads_or(wide) != 0;  // the item's form, known to every thread
   if (wide) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) sG[(th0 + j) * kD + c] = th0 ? gl[8 + j] : gl[j];
   } else {  // k exp(g - m), q exp(g - m) in place of k, q; k exp(m - g) in place of g
-    const float m = 0.5f * (gl[0] + gl[kT - 1]);
+    const float m = gmid;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int t = th0 + j;

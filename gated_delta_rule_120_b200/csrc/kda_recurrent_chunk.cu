@@ -63,6 +63,26 @@ __device__ __forceinline__ void load_row8<float>(float* dst, const float* src) {
 }
 
 template <typename Tin>
+__device__ __forceinline__ void load8(const Tin* src, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* src, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f[2 * j] = __uint_as_float(w[j] << 16);
+    f[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* src, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <typename Tin>
 __device__ __forceinline__ void store4(Tin* dst, const float (&v)[4]);
 template <>
 __device__ __forceinline__ void store4<float>(float* dst, const float (&v)[4]) {
@@ -73,13 +93,15 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, const 
   *reinterpret_cast<uint2*>(dst) = make_uint2(sm100::pack_bf16(v[0], v[1]), sm100::pack_bf16(v[2], v[3]));
 }
 
-template <typename Tin>
+// kFused: the prologue and epilogue of kda_fusion_t — q and k L2-normalised per token, the log
+// decay formed from the raw gate, the output rows normalised and gated before the store.
+template <typename Tin, bool kFused>
 __global__ void __launch_bounds__(kThreads, 2)
     recurrent_chunk_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                            const Tin* __restrict__ v, const float* __restrict__ log_alpha,
                            const float* __restrict__ beta, float* __restrict__ pool,
                            const int32_t* __restrict__ state_indices, Tin* __restrict__ o, int T,
-                           int H, int P) {
+                           int H, int P, Fusion fz) {
   extern __shared__ float4 smem4[];
   float* sm = reinterpret_cast<float*>(smem4);
   float* sS = sm + kOffS;
@@ -118,6 +140,14 @@ __global__ void __launch_bounds__(kThreads, 2)
               rows_in_bounds(kBufLogAlpha, log_alpha + row0 * kD, 0, T, rs * kD, kD) &&
               rows_in_bounds(kBufBeta, beta + row0, 0, T, rs, 1) &&
               rows_in_bounds(kBufO, o + row0 * kD, 0, T, rs * kD, kD);
+    if (kFused) {
+      const Tin* og = reinterpret_cast<const Tin*>(fz.og);
+      ok = ok && (!fz.A_log || in_bounds(kBufALog, fz.A_log + h, 4)) &&
+           (!(fz.A_log && fz.dt_bias) ||
+            in_bounds(kBufDtBias, fz.dt_bias + (size_t)h * kD, kD * 4)) &&
+           (!(fz.onorm && fz.ow) || in_bounds(kBufNormW, fz.ow, kD * 4)) &&
+           (!(fz.onorm && og) || rows_in_bounds(kBufGate, og + row0 * kD, 0, T, rs * kD, kD));
+    }
     if (__syncthreads_or(!ok)) return;
   }
 #endif
@@ -131,7 +161,52 @@ __global__ void __launch_bounds__(kThreads, 2)
   cp_async_commit();
   {
     const int t = tid >> 4, c8 = (tid & 15) * 8;  // token row t, channels c8 .. c8 + 7
-    if (t < T) {
+    if (kFused) {  // rows through registers: L2 norms over the row's 16 lanes, the gate per channel
+      float kx[8], qx[8], gx[8];
+      const size_t r = (row0 + (size_t)t * H) * kD + c8;
+      if (t < T) {
+        load8<Tin>(k + r, kx);
+        load8<Tin>(q + r, qx);
+        load8<float>(log_alpha + r, gx);
+        load_row8<Tin>(sV + t * kD + c8, v + r);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kx[j] = qx[j] = gx[j] = sV[t * kD + c8 + j] = 0.f;
+      }
+      if (fz.l2) {
+        float ssk = 0.f, ssq = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          ssk = fmaf(kx[j], kx[j], ssk);
+          ssq = fmaf(qx[j], qx[j], ssq);
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) {  // the 16 lanes of this row
+          ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+          ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+        }
+        const float ik = rsqrtf(ssk + fz.eps), iq = rsqrtf(ssq + fz.eps);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          kx[j] *= ik;
+          qx[j] *= iq;
+        }
+      }
+      if (fz.A_log && t < T) {  // log alpha = -exp(A_log[h]) softplus(g + dt_bias[h])
+        const float neg_a = -expf(fz.A_log[h]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float bias = fz.dt_bias ? fz.dt_bias[(size_t)h * kD + c8 + j] : 0.f;
+          gx[j] = neg_a * softplus_f(gx[j] + bias);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sK[t * kD + c8 + j] = kx[j];
+        sQ[t * kD + c8 + j] = qx[j];
+        sG[t * kD + c8 + j] = gx[j];
+      }
+    } else if (t < T) {
       const size_t r = (row0 + (size_t)t * H) * kD + c8;
       load_row8<Tin>(sK + t * kD + c8, k + r);
       load_row8<Tin>(sQ + t * kD + c8, q + r);
@@ -330,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     __syncwarp();  // this warp's 16 columns of V' are complete
-    if (mg >= 4) {  // output rows t = 4 (mg - 4) .. + 3
-      const int t0 = 4 * (mg - 4);
+    const int t0 = 4 * (mg - 4);  // output rows t0 .. t0 + 3 (lanes with mg >= 4)
+    if (mg >= 4) {
 #pragma unroll
       for (int tau = 0; tau < kT; ++tau) {
         const float4 vp = *reinterpret_cast<const float4*>(sV + tau * kD + col);
@@ -344,12 +419,49 @@ __global__ void __launch_bounds__(kThreads, 2)
           acc[r][1] = f2_fma(ar, v23, acc[r][1]);
         }
       }
+    }
+    float y[4][4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float2 lo = f2_unpack(acc[r][0]), hi = f2_unpack(acc[r][1]);
+      y[r][0] = lo.x;
+      y[r][1] = lo.y;
+      y[r][2] = hi.x;
+      y[r][3] = hi.y;
+    }
+    if (kFused && fz.onorm) {  // y = sigmoid(gate) weight o / RMS over the row's 128 columns
+      float* sPart = sAkk;     // [8 warps][16 rows] partial sums of squares (A_kk is dead)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float ss = y[r][0] * y[r][0] + y[r][1] * y[r][1] + y[r][2] * y[r][2] + y[r][3] * y[r][3];
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);  // the four lanes of this row's 16 columns
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        if (mg >= 4 && cg == 0) sPart[warp * kT + t0 + r] = ss;
+      }
+      __syncthreads();
+      if (mg >= 4) {
+        const Tin* og = reinterpret_cast<const Tin*>(fz.og);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int t = t0 + r;
+          float tot = 0.f;
+#pragma unroll
+          for (int w = 0; w < kThreads / 32; ++w) tot += sPart[w * kT + t];
+          const float inv = rsqrtf(tot * (1.f / kD) + fz.oeps);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float f = inv * (fz.ow ? fz.ow[col + c] : 1.f);
+            if (og && t < T) f *= sigmoid_f(to_f32(og[(row0 + (size_t)t * H) * kD + col + c]));
+            y[r][c] *= f;
+          }
+        }
+      }
+    }
+    if (mg >= 4) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int t = t0 + r;
-        const float2 lo = f2_unpack(acc[r][0]), hi = f2_unpack(acc[r][1]);
-        const float y[4] = {lo.x, lo.y, hi.x, hi.y};
-        if (t < T) store4<Tin>(o + (row0 + (size_t)t * H) * kD + col, y);
+        if (t < T) store4<Tin>(o + (row0 + (size_t)t * H) * kD + col, y[r]);
       }
     }
   }
@@ -394,49 +506,52 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 }  // namespace rchunk
 
-// The recurrent mode through the chunk-form kernel: 2 <= T <= 16, d_k = d_v = 128, no fusion, 16-byte
-// aligned rows. Returns false (nothing launched) when the call does not qualify.
+// The recurrent mode through the chunk-form kernel: 2 <= T <= 16, d_k = d_v = 128, 16-byte aligned
+// rows. Returns false (nothing launched) when the call does not qualify.
 static bool recurrent_chunk_applies(kda_dtype_t dt, int T, int Dk, int Dv, const void* q,
                                     const void* k, const void* v, const float* log_alpha,
-                                    const float* pool, const void* o, const Fusion& fz) {
+                                    const float* pool, const void* o) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
-  const bool fused = fz.l2 || fz.A_log || fz.onorm;
-  return !fused && T >= 2 && T <= rchunk::kT && Dk == rchunk::kD && Dv == rchunk::kD &&
+  return T >= 2 && T <= rchunk::kT && Dk == rchunk::kD && Dv == rchunk::kD &&
          (dt == KDA_DTYPE_BF16 || dt == KDA_DTYPE_F32) && al16(q) && al16(k) && al16(v) &&
          al16(log_alpha) && al16(pool) && ((uintptr_t)o & (dt == KDA_DTYPE_BF16 ? 7u : 15u)) == 0;
+}
+
+template <typename Tin, bool kFused>
+static cudaError_t launch_rchunk_typed(const void* q, const void* k, const void* v,
+                                       const float* log_alpha, const float* beta, float* pool,
+                                       const int32_t* idx, void* o, long long heads, int T, int H,
+                                       int P, const Fusion& fz, cudaStream_t stream) {
+  const int smem = (int)rchunk::kSmemBytes;
+  cudaError_t err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<Tin, kFused>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err == cudaSuccess)  // two CTAs per SM: the whole unified array as shared memory
+    err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<Tin, kFused>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (err != cudaSuccess) return err;
+  rchunk::recurrent_chunk_kernel<Tin, kFused><<<(unsigned)heads, rchunk::kThreads, smem, stream>>>(
+      (const Tin*)q, (const Tin*)k, (const Tin*)v, log_alpha, beta, pool, idx, (Tin*)o, T, H, P,
+      fz);
+  return cudaGetLastError();
 }
 
 static cudaError_t launch_recurrent_chunk(const void* q, const void* k, const void* v,
                                           kda_dtype_t dt, const float* log_alpha,
                                           const float* beta, float* pool, const int32_t* idx,
                                           void* o, long long heads, int T, int H, int P,
-                                          cudaStream_t stream) {
+                                          const Fusion& fz, cudaStream_t stream) {
   if (heads > INT32_MAX) return cudaErrorInvalidConfiguration;
-  const int smem = (int)rchunk::kSmemBytes;
-  ProfileScope prof("recurrent_chunk", stream);
-  if (dt == KDA_DTYPE_BF16) {
-    cudaError_t err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<__nv_bfloat16>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err == cudaSuccess)  // two CTAs per SM: the whole unified array as shared memory
-      err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (err != cudaSuccess) return err;
-    rchunk::recurrent_chunk_kernel<__nv_bfloat16><<<(unsigned)heads, rchunk::kThreads, smem,
-                                                    stream>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, log_alpha, beta,
-        pool, idx, (__nv_bfloat16*)o, T, H, P);
-  } else {
-    cudaError_t err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<float>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(rchunk::recurrent_chunk_kernel<float>,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (err != cudaSuccess) return err;
-    rchunk::recurrent_chunk_kernel<float><<<(unsigned)heads, rchunk::kThreads, smem, stream>>>(
-        (const float*)q, (const float*)k, (const float*)v, log_alpha, beta, pool, idx, (float*)o,
-        T, H, P);
-  }
-  return cudaGetLastError();
+  const bool fused = fz.l2 || fz.A_log || fz.onorm;
+  ProfileScope prof(fused ? "recurrent_chunk_fused" : "recurrent_chunk", stream);
+  if (dt == KDA_DTYPE_BF16)
+    return fused ? launch_rchunk_typed<__nv_bfloat16, true>(q, k, v, log_alpha, beta, pool, idx,
+                                                             o, heads, T, H, P, fz, stream)
+                 : launch_rchunk_typed<__nv_bfloat16, false>(q, k, v, log_alpha, beta, pool, idx,
+                                                              o, heads, T, H, P, fz, stream);
+  return fused ? launch_rchunk_typed<float, true>(q, k, v, log_alpha, beta, pool, idx, o, heads,
+                                                  T, H, P, fz, stream)
+               : launch_rchunk_typed<float, false>(q, k, v, log_alpha, beta, pool, idx, o, heads,
+                                                   T, H, P, fz, stream);
 }
 
 }  // namespace kda

@@ -20,7 +20,7 @@ def _inputs(N, T, H, Dk, Dv, dtype, seed, dev):
 
 @pytest.mark.parametrize("dtype,dims", [("bf16", (128, 128)), ("f32", (40, 12)),
                                         ("bf16", (64, 128)), ("f32", (128, 128))])
-@pytest.mark.parametrize("T", [1, 2, 7, 16, 64])
+@pytest.mark.parametrize("T", [1, 2, 7, 16, 37, 64])
 def test_recurrent_fwd_with_state_pool(cuda_device, dtype, dims, T):
     Dk, Dv = dims
     N, H, P = 6, 3, 10

@@ -76,9 +76,10 @@ def test_recurrent_fwd_index_beyond_pool_is_reported(cuda_device):
 
 
 def test_recurrent_fwd_strong_and_mild_decays_in_one_launch(cuda_device):
-    """Items whose decay over the call stays mild and items whose rows decay below e^-60 within
-    the call (the kernel keeps the second kind on its token-by-token form) in one launch, against
-    the oracle at the recurrent mode's tolerances."""
+    """Items whose decay over the call stays mild and items whose channels decay by hundreds of
+    nats within the call in one launch (the chunk-form kernel factors the first kind's ratios
+    around each channel's midpoint and forms the second kind's exactly), against the oracle at
+    the recurrent mode's tolerances."""
     N, T, H = 8, 12, 3
     x = _inputs(N, T, H, 128, 128, "bf16", 670, cuda_device)
     la = x["log_alpha"].clone()

@@ -405,9 +405,11 @@ def run_fused_prefill(spec, seed, dev, steps, warmup, world, epilogue=False):
     return timed(step, steps, warmup, world, dev)
 
 
-def run_recurrent_mode(N, T, H, D, dev, steps, warmup, world, seed):
+def run_recurrent_mode(N, T, H, D, dev, steps, warmup, world, seed, fused=False):
     """Multi-token recurrent mode (kda_recurrent_fwd): N sequences x T tokens applied to states
-    gathered from a pool by index (serving-cache layout); bf16 q/k/v, fp32 gates and states."""
+    gathered from a pool by index (serving-cache layout); bf16 q/k/v, fp32 gates and states. With
+    ``fused`` the layer's prologue and epilogue run in the kernel: raw q/k L2-normalised, the log
+    decay formed from a raw gate (A_log, dt_bias), the output RMS-normalised, weighted and gated."""
     import torch
 
     import gated_delta_rule_120_b200 as kda
@@ -421,9 +423,21 @@ def run_recurrent_mode(N, T, H, D, dev, steps, warmup, world, seed):
     pool = torch.randn((P, H, D, D), generator=g, device=dev) * 0.02
     idx = torch.randperm(P, generator=g, device=dev)[:N].to(torch.int32)
     o = torch.empty_like(x["v"])
+    fusion = None
+    if fused:
+        x["q"] = (x["q"].float() * 3.0).to(x["q"].dtype)
+        x["k"] = (x["k"].float() * 3.0).to(x["k"].dtype)
+        x["log_alpha"] = torch.randn(x["log_alpha"].shape, generator=g, device=dev) - 1.0
+        fusion = dict(qk_l2norm=True, eps=1e-6,
+                      A_log=torch.log(torch.rand((H,), generator=g, device=dev) * 15 + 1) - 2.0,
+                      dt_bias=torch.randn((H, D), generator=g, device=dev) * 0.5,
+                      out_norm=True, out_norm_eps=1e-5,
+                      out_norm_weight=torch.rand((D,), generator=g, device=dev) + 0.5,
+                      out_gate=torch.randn(x["v"].shape, generator=g, device=dev).to(x["v"].dtype))
 
     def step(i):
-        kda.kda_recurrent_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool, idx, o=o)
+        kda.kda_recurrent_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool, idx, o=o,
+                              fusion=fusion)
 
     return timed(step, steps, warmup, world, dev)
 
@@ -707,6 +721,15 @@ def main():
         "ms_per_call": per,
         "achieved_gbs": rtotal / (per / 1e3) / 1e9,
         "frac_hbm": rtotal / (per / 1e3) / 1e9 / hbm_peak}
+    fms = run_recurrent_mode(rN, rT, 32, 128, dev, rsteps, 2, world, 2015 + 10 * rank, fused=True)
+    fper = fms / rsteps
+    ftotal = rtotal + rN * 32 * rT * 128 * 2  # + the output-gate rows
+    extra["recurrent_mode"]["fused"] = {
+        "workload": f"recurrent_N{rN}_T{rT}_H32_d128_pool_fused_prologue_epilogue",
+        "tokens_per_s": whole_job_rate(rN * rT, world, fper),
+        "ms_per_call": fper,
+        "achieved_gbs": ftotal / (fper / 1e3) / 1e9,
+        "frac_hbm": ftotal / (fper / 1e3) / 1e9 / hbm_peak}
     torch.cuda.empty_cache()
     # the backward pass of the standard prefill
     bsteps = max(3, args.steps // 4)

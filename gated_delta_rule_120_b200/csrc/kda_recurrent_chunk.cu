@@ -25,16 +25,16 @@
 namespace kda {
 namespace rchunk {
 
-constexpr int kT = 16;         // tokens per item at most
+constexpr int kT = 16;         // tokens per chunk
 constexpr int kD = 128;        // d_k = d_v
 constexpr int kThreads = 256;  // 8 warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory (fp32 words)
 constexpr int kOffS = 0;                   // S [128][128], row-major
-constexpr int kOffK = kOffS + kD * kD;     // k [16][128], then K~
-constexpr int kOffQ = kOffK + kT * kD;     // q [16][128]   } later [W; Q~]^T [128][32] (swizzled)
-constexpr int kOffG = kOffQ + kT * kD;     // g log2e [16][128] }
+constexpr int kOffK = kOffS + kD * kD;     // k [16][128], k exp(g - m), then K~
+constexpr int kOffQ = kOffK + kT * kD;     // q, q exp(g - m) } later [W; Q~]^T [128][32]
+constexpr int kOffG = kOffQ + kT * kD;     // g log2e or k exp(m - g) }  (swizzled)
 constexpr int kOffV = kOffG + kT * kD;     // v, then U, then V' [16][128]
 constexpr int kOffKG = kOffV + kT * kD;    // exp(g) . k [16][128]
 constexpr int kOffAkk = kOffKG + kT * kD;  // Diag(beta) A_kk strict lower [16][16]

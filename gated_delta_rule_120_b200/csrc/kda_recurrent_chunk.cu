@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       f32x2 acc[4][2];
 #pragma unroll
       for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = f2_pack(0.f, 0.f);
-#pragma unroll 16
+#pragma unroll 32
       for (int kk = 0; kk < kD; ++kk) {
         const float4 a = *reinterpret_cast<const float4*>(sAT + kk * 32 + ((mg ^ (kk & 7)) << 2));
         const float4 sv = *reinterpret_cast<const float4*>(sS + kk * kD + col);

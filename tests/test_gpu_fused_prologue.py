@@ -101,9 +101,10 @@ def test_chunk_fused_f32_varlen(cuda_device):
 
 
 @pytest.mark.parametrize("dtype,dims", [("bf16", (128, 128)), ("f32", (40, 12))])
-def test_recurrent_fused(cuda_device, dtype, dims):
+@pytest.mark.parametrize("T", [9, 37])
+def test_recurrent_fused(cuda_device, dtype, dims, T):
     Dk, Dv = dims
-    N, T, H = 4, 9, 3
+    N, H = 4, 3
     x = _raw_inputs(N, T, H, Dk, Dv, dtype, 720, cuda_device)
     fusion = dict(qk_l2norm=True, eps=1e-6, A_log=x["A_log"], dt_bias=x["dt_bias"])
     pool = torch.randn((N, H, Dk, Dv), device=cuda_device) * 0.05

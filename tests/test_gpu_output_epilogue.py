@@ -127,9 +127,11 @@ def test_chunk_f32_output_epilogue_varlen(cuda_device):
 
 
 @pytest.mark.parametrize("dtype,dims", [("bf16", (128, 128)), ("f32", (40, 12))])
-def test_recurrent_output_epilogue(cuda_device, dtype, dims):
+@pytest.mark.parametrize("T", [9, 37])
+def test_recurrent_output_epilogue(cuda_device, dtype, dims, T):
+    """T = 37 runs three chunks of the chunk-form kernel (d = 128), the last one ragged."""
     Dk, Dv = dims
-    N, T, H = 4, 9, 3
+    N, H = 4, 3
     spec = PrefillSpec("r", B=N, T=T, H=H, Dk=Dk, Dv=Dv, chunk=64, dtype=dtype, decay="fast",
                        init_std=0.0)
     inp = kda_synth.prefill_inputs(spec, 830, cuda_device)

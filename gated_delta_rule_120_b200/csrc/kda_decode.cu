@@ -1405,7 +1405,7 @@ cudaError_t launch_recurrent_multi(const void* q, const void* k, const void* v, 
                                    int Dv, int P, const Fusion& fz, cudaStream_t stream) {
   const long long heads = (long long)N * H;
   if (heads == 0 || T == 0) return cudaSuccess;
-  if (recurrent_chunk_applies(dt, T, Dk, Dv, q, k, v, log_alpha, pool, o))
+  if (recurrent_chunk_applies(dt, T, Dk, Dv, q, k, v, log_alpha, pool, o, fz))
     return launch_recurrent_chunk(q, k, v, dt, log_alpha, beta, pool, idx, o, heads, T, H, P, fz,
                                   stream);
   const int es = dt == KDA_DTYPE_BF16 ? 2 : 4;

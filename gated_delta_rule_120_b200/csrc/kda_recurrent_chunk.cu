@@ -383,6 +383,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     cp_async_wait<0>();
     __syncthreads();
+    if (kFused && fz.onorm && fz.og) {  // the chunk's output-gate rows into the dead exp(g) . k
+      // buffer, in flight under the [W; Q~] S product
+      constexpr int kPerRow = kD * (int)sizeof(Tin) / 16;  // 16-byte words per row
+      const Tin* og = reinterpret_cast<const Tin*>(fz.og);
+      for (int w = tid; w < kT * kPerRow; w += kThreads) {
+        const int t = w / kPerRow, c16 = w - t * kPerRow;
+        if (t < T)
+          cp_async_16B(reinterpret_cast<Tin*>(sKG) + t * kD + c16 * (16 / (int)sizeof(Tin)),
+                       og + (rowc + (size_t)t * H) * kD + c16 * (16 / (int)sizeof(Tin)));
+      }
+      cp_async_commit();
+    }
 
     // ---- phase 6: [W; Q~] S; V' = U - W S; O = Q~ S + A_qk V' -----------------------------------
     // warp = 16 state columns, lane = 4 rows (mg) x 4 columns (cg) of the 32 x 128 product; the
@@ -448,9 +460,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           ss += __shfl_xor_sync(0xffffffffu, ss, 2);
           if (mg >= 4 && cg == 0) sPart[warp * kT + t0 + r] = ss;
         }
+        cp_async_wait<0>();  // this thread's gate-row copies
         __syncthreads();
         if (mg >= 4) {
-          const Tin* og = reinterpret_cast<const Tin*>(fz.og);
+          const Tin* sOg = reinterpret_cast<const Tin*>(sKG);  // the staged gate rows
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int t = t0 + r;
@@ -461,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               float f = inv * (fz.ow ? fz.ow[col + c] : 1.f);
-              if (og && t < T) f *= sigmoid_f(to_f32(og[(rowc + (size_t)t * H) * kD + col + c]));
+              if (fz.og && t < T) f *= sigmoid_f(to_f32(sOg[t * kD + col + c]));
               y[r][c] *= f;
             }
           }
@@ -525,11 +538,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Returns false (nothing launched) when the call does not qualify.
 static bool recurrent_chunk_applies(kda_dtype_t dt, int T, int Dk, int Dv, const void* q,
                                     const void* k, const void* v, const float* log_alpha,
-                                    const float* pool, const void* o) {
+                                    const float* pool, const void* o, const Fusion& fz) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15u) == 0; };
   return T >= 2 && Dk == rchunk::kD && Dv == rchunk::kD &&
          (dt == KDA_DTYPE_BF16 || dt == KDA_DTYPE_F32) && al16(q) && al16(k) && al16(v) &&
-         al16(log_alpha) && al16(pool) && ((uintptr_t)o & (dt == KDA_DTYPE_BF16 ? 7u : 15u)) == 0;
+         al16(log_alpha) && al16(pool) && ((uintptr_t)o & (dt == KDA_DTYPE_BF16 ? 7u : 15u)) == 0 &&
+         (!(fz.onorm && fz.og) || al16(fz.og));
 }
 
 template <typename Tin, bool kFused>
